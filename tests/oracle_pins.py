@@ -1,0 +1,257 @@
+"""Pins of the oracle to facts fixed by the SP-KV page and by mathematics.
+
+Each ``pin_*`` function raises AssertionError when the oracle disagrees with a
+closed form, a library special case, a hand-derived fixture or a brute-force
+enumeration.  ``test_oracle_pins.py`` runs them all; ``test_oracle_mutations.py``
+plants plausible mistakes in the oracle and checks that some pin catches each.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+from scipy.special import expit
+
+from oracle import spkv_oracle as O
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _golden(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+def _close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert a.shape == b.shape, f"{what}: shape {a.shape} vs {b.shape}"
+    assert err <= tol, f"{what}: max abs error {err:.3e} > {tol:.1e}"
+
+
+def _sdpa(Q, K, V, mask):
+    """torch scaled_dot_product_attention in fp64 on CPU.  Q [n][Hq][d] queries at
+    positions 0..n-1, K/V [T][Hkv][d]; key heads are repeated for GQA (query head
+    h uses key head h // G).  ``mask``: None for plain causal, else a bool [n][T]."""
+    Hq, Hkv = Q.shape[1], K.shape[1]
+    G = Hq // Hkv
+    q = torch.from_numpy(np.ascontiguousarray(Q.transpose(1, 0, 2))).double()
+    k = torch.from_numpy(np.ascontiguousarray(K.transpose(1, 0, 2))).double().repeat_interleave(G, 0)
+    v = torch.from_numpy(np.ascontiguousarray(V.transpose(1, 0, 2))).double().repeat_interleave(G, 0)
+    if mask is None:
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, is_causal=True)
+    else:
+        o = torch.nn.functional.scaled_dot_product_attention(q, k, v, attn_mask=torch.from_numpy(mask))
+    return o.numpy().transpose(1, 0, 2)
+
+
+def _rand_qkv(rng, T, Hq, Hkv, d):
+    Q = rng.standard_normal((T, Hq, d))
+    K = rng.standard_normal((T, Hkv, d))
+    V = rng.standard_normal((T, Hkv, d))
+    return Q, K, V
+
+
+def _mlp(rng, N, D, hid, Hkv, scale=0.3):
+    h = rng.standard_normal((N, D))
+    W1 = rng.standard_normal((hid, D)) * scale
+    b1 = rng.standard_normal(hid) * scale
+    W2 = rng.standard_normal((Hkv, hid)) * scale
+    b2 = rng.standard_normal(Hkv) * scale
+    return h, W1, b1, W2, b2
+
+
+# ---------------------------------------------------------------- Eq. (1) ----
+
+def pin_gelu_textbook():
+    g = _golden("gelu_sigmoid_values.json")
+    for a, want in g["gelu"]:
+        _close(O.gelu(np.array([a])), [want], 1e-15, f"GELU({a})")
+    for x, want in g["sigmoid"]:
+        _close(O.sigmoid(np.array([x])), [want], 1e-15, f"sigmoid({x})")
+
+
+def pin_gelu_library():
+    x = np.linspace(-8, 8, 1001)
+    ref = torch.nn.functional.gelu(torch.from_numpy(x), approximate="none").numpy()
+    _close(O.gelu(x), ref, 1e-14, "GELU vs torch (exact erf form)")
+
+
+def pin_utility_zero_weights():
+    """W1 = W2 = 0 leaves u = sigmoid(b2) for every token (closed form)."""
+    rng = np.random.default_rng(1)
+    N, D, hid, Hkv = 7, 12, 5, 3
+    h = rng.standard_normal((N, D))
+    b2 = np.array([-3.0, 0.0, 2.5])
+    u = O.utility(h, np.zeros((hid, D)), rng.standard_normal(hid), np.zeros((Hkv, hid)), b2)
+    _close(u, np.broadcast_to(expit(b2), (N, Hkv)), 1e-15, "u with zero weights")
+
+
+def pin_utility_hand_example():
+    """One token, one hidden unit: a = 1 -> GELU = Phi(1); W2 = 2, b2 = -1 ->
+    logit = 2 Phi(1) - 1."""
+    phi1 = 0.8413447460685429
+    u = O.utility(np.array([[1.0, 5.0]]), np.array([[1.0, 0.0]]), np.array([0.0]),
+                  np.array([[2.0]]), np.array([-1.0]))
+    _close(u, [[expit(2 * phi1 - 1)]], 1e-15, "hand example")
+
+
+def pin_utility_library():
+    """The perceptron equals torch Linear -> GELU -> Linear -> sigmoid in fp64."""
+    rng = np.random.default_rng(2)
+    h, W1, b1, W2, b2 = _mlp(rng, 33, 24, 16, 4)
+    l1 = torch.nn.Linear(24, 16).double()
+    l2 = torch.nn.Linear(16, 4).double()
+    with torch.no_grad():
+        l1.weight.copy_(torch.from_numpy(W1)); l1.bias.copy_(torch.from_numpy(b1))
+        l2.weight.copy_(torch.from_numpy(W2)); l2.bias.copy_(torch.from_numpy(b2))
+        ref = torch.sigmoid(l2(torch.nn.functional.gelu(l1(torch.from_numpy(h))))).numpy()
+    _close(O.utility(h, W1, b1, W2, b2), ref, 1e-14, "utility vs torch MLP")
+
+
+# ---------------------------------------------------------------- Eq. (2) ----
+
+def pin_gate_threshold():
+    """z = 1[u >= tau]: equality keeps the token; the next double above tau drops it."""
+    u = O.utility(np.zeros((1, 3)), np.zeros((2, 3)), np.zeros(2), np.zeros((1, 2)), np.zeros(1))
+    assert float(u[0, 0]) == 0.5
+    assert O.gate(u, 0.5)[0, 0] == 1, "u == tau must be kept"
+    assert O.gate(u, np.nextafter(0.5, 1.0))[0, 0] == 0
+    assert O.gate(u, np.nextafter(0.5, 0.0))[0, 0] == 1
+    uu = np.array([0.1, 0.2, 0.3, 0.7])
+    assert list(O.gate(uu, 0.3)) == [0, 0, 1, 1]
+
+
+def pin_gate_extremes():
+    """tau = 0 keeps every token (u > 0); tau > 1 keeps none (u < 1)."""
+    rng = np.random.default_rng(3)
+    h, W1, b1, W2, b2 = _mlp(rng, 50, 10, 8, 2, scale=3.0)
+    u = O.utility(h, W1, b1, W2, b2)
+    assert O.gate(u, 0.0).all()
+    assert not O.gate(u, 1.5).any()
+
+
+# ----------------------------------------------------------- Eqs. (3)-(4) ----
+
+def pin_keysets_golden():
+    """With q = 0 every visible key gets the same weight, so with one-hot values the
+    output is the indicator of the visible set divided by its size, and lse = ln|S|.
+    The visible sets are hand-derived from Eq. (4)."""
+    for case in _golden("keysets_eq4.json")["cases"]:
+        T, w, z = case["T"], case["w"], np.array(case["z"], dtype=np.uint8)
+        d = T
+        Q = np.zeros((T, 1, d))
+        K = np.random.default_rng(4).standard_normal((T, 1, d))
+        V = np.eye(T).reshape(T, 1, d)
+        o, lse = O.gated_attention(Q, K, V, z.reshape(T, 1), w, np.arange(T))
+        for t in range(T):
+            want = np.zeros(T)
+            want[case["S"][t]] = 1.0 / len(case["S"][t])
+            _close(o[t, 0], want, 1e-15, f"key set T={T} w={w} t={t}")
+            _close([lse[t, 0]], [math.log(len(case["S"][t]))], 1e-15, "lse")
+
+
+def pin_two_key_softmax():
+    """Two visible keys with scaled logits 1 and 0 (d_k = 4, so q.k = 2 and 0):
+    weights e/(e+1) and 1/(e+1); lse = ln(e + 1)."""
+    q = np.array([2.0, 0.0, 0.0, 0.0])
+    K = np.array([[1.0, 0, 0, 0], [0.0, 0, 0, 0]])
+    V = np.array([[1.0, 0, 0, 0], [0.0, 1, 0, 0]])
+    o, lse = O.attend(q, K, V, np.array([True, True]))
+    p = math.e / (math.e + 1)
+    _close(o, [p, 1 - p, 0, 0], 1e-15, "two-key softmax")
+    _close([lse], [math.log(math.e + 1)], 1e-15, "two-key lse")
+
+
+def pin_tau0_is_causal():
+    """tau = 0 gates every key in (u > 0), so Eqs. (3)-(4) reduce to causal
+    attention: torch SDPA (is_causal) in fp64."""
+    rng = np.random.default_rng(5)
+    T, Hq, Hkv, d, w = 40, 4, 2, 8, 5
+    Q, K, V = _rand_qkv(rng, T, Hq, Hkv, d)
+    h, W1, b1, W2, b2 = _mlp(rng, T, 6, 5, Hkv)
+    z = O.gate(O.utility(h, W1, b1, W2, b2), 0.0)
+    o, _ = O.gated_attention(Q, K, V, z, w, np.arange(T))
+    _close(o, _sdpa(Q, K, V, None), 1e-12, "tau=0 vs causal SDPA")
+
+
+def pin_tau_gt1_is_sliding_window():
+    """tau > 1 gates every key out (u < 1), leaving sliding-window-w attention:
+    torch SDPA with a band mask built from tril."""
+    rng = np.random.default_rng(6)
+    T, Hq, Hkv, d, w = 40, 4, 2, 8, 6
+    Q, K, V = _rand_qkv(rng, T, Hq, Hkv, d)
+    h, W1, b1, W2, b2 = _mlp(rng, T, 6, 5, Hkv)
+    z = O.gate(O.utility(h, W1, b1, W2, b2), 1.5)
+    o, _ = O.gated_attention(Q, K, V, z, w, np.arange(T))
+    ones = torch.ones(T, T, dtype=torch.bool)
+    band = (ones.tril(0) & ~ones.tril(-w)).numpy()
+    _close(o, _sdpa(Q, K, V, band), 1e-12, "tau>1 vs sliding-window SDPA")
+
+
+def pin_wide_window_is_causal():
+    """w >= T puts every earlier key in the window whatever z is."""
+    rng = np.random.default_rng(7)
+    T, Hq, Hkv, d = 30, 2, 1, 8
+    Q, K, V = _rand_qkv(rng, T, Hq, Hkv, d)
+    z = (rng.random((T, Hkv)) < 0.3).astype(np.uint8)
+    o, _ = O.gated_attention(Q, K, V, z, T, np.arange(T))
+    _close(o, _sdpa(Q, K, V, None), 1e-12, "w>=T vs causal SDPA")
+
+
+def pin_dense_brute_force(seeds=200):
+    """Tiny inputs: enumerate Eq. (4) with explicit loops into a dense T x T mask and
+    compute the masked softmax densely (whole matrices); compare per query."""
+    for seed in range(seeds):
+        rng = np.random.default_rng(1000 + seed)
+        T = int(rng.integers(1, 20))
+        w = int(rng.choice([1, 2, 4, 8]))
+        Hkv, G, d = 1 + seed % 2, 1 + (seed // 2) % 2, 4
+        Hq = Hkv * G
+        Q, K, V = _rand_qkv(rng, T, Hq, Hkv, d)
+        z = (rng.random((T, Hkv)) < 0.4).astype(np.uint8)
+        o, _ = O.gated_attention(Q, K, V, z, w, np.arange(T))
+        for hk in range(Hkv):
+            M = np.full((T, T), -np.inf)
+            for t in range(T):
+                for s in range(T):
+                    if (0 <= t - s < w) or (z[s, hk] == 1 and s <= t):
+                        M[t, s] = 0.0
+            for g in range(G):
+                hq = hk * G + g
+                S = Q[:, hq] @ K[:, hk].T / math.sqrt(d) + M
+                P = np.exp(S - S.max(axis=1, keepdims=True))
+                P /= P.sum(axis=1, keepdims=True)
+                _close(o[:, hq], P @ V[:, hk], 1e-12, f"brute force seed {seed}")
+
+
+def pin_cache_rows():
+    """The persistent cache is the increasing list of gated-in positions; its length
+    is the kept count sum(z); together with the window it is exactly the visible set
+    of Eq. (4) for every query."""
+    rng = np.random.default_rng(8)
+    for w in (1, 3, 16):
+        T = 60
+        z = (rng.random(T) < 0.35).astype(np.uint8)
+        for upto in (0, 1, 17, T):
+            rows = O.cache_rows(z, upto)
+            assert len(rows) == int(z[:upto].sum())
+            assert list(rows) == [s for s in range(upto) if z[s] == 1]
+            assert np.all(np.diff(rows) > 0)
+        s = np.arange(T)
+        for t in range(T):
+            window = set(range(max(0, t - w + 1), t + 1))
+            cached = set(O.cache_rows(z, max(0, t - w + 1)).tolist())
+            assert set(np.nonzero(O.visible(t, s, z, w))[0].tolist()) == window | cached
+
+
+ALL_PINS = [
+    pin_gelu_textbook, pin_gelu_library, pin_utility_zero_weights, pin_utility_hand_example,
+    pin_utility_library, pin_gate_threshold, pin_gate_extremes, pin_keysets_golden,
+    pin_two_key_softmax, pin_tau0_is_causal, pin_tau_gt1_is_sliding_window,
+    pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows,
+]

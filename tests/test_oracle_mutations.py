@@ -1,0 +1,96 @@
+"""Plant plausible mistakes in the oracle (on the CPU) and check that some pin
+catches each one: the pins are strong enough to trust the oracle."""
+import numpy as np
+import pytest
+from scipy.special import erf
+
+from oracle import spkv_oracle as O
+from tests import oracle_pins as P
+
+
+def _gelu_tanh(a):
+    a = np.asarray(a, dtype=np.float64)
+    return 0.5 * a * (1 + np.tanh(np.sqrt(2 / np.pi) * (a + 0.044715 * a ** 3)))
+
+
+def _visible_window_off_by_one(t, s, z, w):
+    s = np.asarray(s)
+    return ((t - s >= 0) & (t - s <= w)) | ((np.asarray(z) == 1) & (s <= t))
+
+
+def _visible_ignores_z(t, s, z, w):
+    s = np.asarray(s)
+    return (t - s >= 0) & (t - s < w)
+
+
+def _visible_acausal(t, s, z, w):
+    s = np.asarray(s)
+    return ((t - s >= 0) & (t - s < w)) | (np.asarray(z) == 1)
+
+
+def _gate_strict(u, tau):
+    return (np.asarray(u, dtype=np.float64) > tau).astype(np.uint8)
+
+
+def _attend_no_scale(q, K, V, mask):
+    return _ORIG_ATTEND(np.asarray(q) * np.sqrt(np.asarray(q).shape[-1]), K, V, mask)
+
+
+def _utility_no_b1(h, W1, b1, W2, b2):
+    return _ORIG_LOGITS(h, W1, np.zeros_like(np.asarray(b1, dtype=np.float64)), W2, b2)
+
+
+def _sigmoid_flipped(x):
+    return 1.0 / (1.0 + np.exp(np.asarray(x, dtype=np.float64)))
+
+
+def _gqa_modulo(Q, K, V, z, w, q_pos):
+    # query head h reads key head h % Hkv instead of h // G
+    Q = np.asarray(Q, dtype=np.float64)
+    n_q, Hq, d = Q.shape
+    T, Hkv, _ = np.asarray(K).shape
+    o = np.zeros((n_q, Hq, d)); lse = np.zeros((n_q, Hq))
+    for i, t in enumerate(q_pos):
+        for h in range(Hq):
+            hk = h % Hkv
+            m = O.visible(int(t), np.arange(T), z[:, hk], w)
+            o[i, h], lse[i, h] = O.attend(Q[i, h], np.asarray(K)[:, hk], np.asarray(V)[:, hk], m)
+    return o, lse
+
+
+def _gelu_wrong_scale(a):
+    a = np.asarray(a, dtype=np.float64)
+    return 0.5 * a * (1 + erf(a))
+
+
+_ORIG_ATTEND = O.attend
+_ORIG_LOGITS = O.utility_logits
+
+MUTANTS = {
+    "gelu_tanh_approximation": ("gelu", _gelu_tanh),
+    "gelu_missing_sqrt2": ("gelu", _gelu_wrong_scale),
+    "window_off_by_one": ("visible", _visible_window_off_by_one),
+    "gate_ignored": ("visible", _visible_ignores_z),
+    "gated_keys_not_causal": ("visible", _visible_acausal),
+    "gate_strict_inequality": ("gate", _gate_strict),
+    "missing_inv_sqrt_dk": ("attend", _attend_no_scale),
+    "dropped_b1": ("utility_logits", _utility_no_b1),
+    "sigmoid_sign": ("sigmoid", _sigmoid_flipped),
+    "gqa_modulo_mapping": ("gated_attention", _gqa_modulo),
+}
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name, monkeypatch):
+    attr, fn = MUTANTS[name]
+    monkeypatch.setattr(O, attr, fn)
+    caught = []
+    for pin in P.ALL_PINS:
+        try:
+            if pin is P.pin_dense_brute_force:
+                pin(seeds=40)
+            else:
+                pin()
+        except AssertionError:
+            caught.append(pin.__name__)
+    assert caught, f"no pin catches the planted mistake {name}"
