@@ -1,0 +1,525 @@
+#!/usr/bin/env python
+"""Gated decode throughput of SP-KV on B200: tokens/s and effective KV GB/s at 32K context.
+
+Workload (decode32k): batch 8, 32 query / 8 key-value heads, head_dim 128,
+d_model 4096, utility perceptron 4096 -> 128 -> 8, window 128, tau 0.5, 32 layers,
+32768 tokens already processed per row (per-head keep rates drawn in [5%, 50%]).
+One step = one decode token for every batch row through all 32 layers: per layer
+score the new token (a1), retire token t-128 into the gated cache if its gate is 1
+and store the new token in the ring (a2, a3), then gated decode attention with the
+split merge (a4, a5).  Steps are real consecutive decode steps (positions 32768,
+32769, ...), each captured once in a CUDA graph; every step reads ~9.5 GB of K/V,
+far more than the 126 MB L2, so no flush is needed between steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spkv|reference]
+
+Under torchrun every rank runs its own replica (batch rows and key heads are
+independent: no collective on the data path); the elapsed time is the max over
+ranks and ``value`` counts every rank's tokens.  ``--impl reference`` times the
+fp64 CPU oracle on bounded samples of the same workload on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gated decode tokens/s and effective KV GB/s (% HBM peak) at 32K ctx"
+WORKLOAD = "decode32k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+# ----------------------------------------------------------------- distributed ----
+
+def _dist_init():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def _barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def _max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device: int):
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not self.uuid.startswith("GPU-"):
+                self.uuid = "GPU-" + self.uuid
+        except Exception:
+            pass
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if self.uuid:
+            cmd += ["-i", self.uuid]
+        try:
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        rows = []
+        with open(self.out.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.out.name)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        power = [num(r[3]) for r in rows if num(r[3]) is not None]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------------- GPU arm -------
+
+def _kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for name in ("decode.cu", "common.cuh"):
+        with open(os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _profiled_traffic():
+    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
+    on the current kernel source (else None)."""
+    path = os.path.join(ROOT, "profiles", "decode_attn_decode32k.md")
+    if not os.path.exists(path):
+        return None
+    want = _kernel_source_hash()
+    vals = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("bench-key "):
+                k, _, v = line[len("bench-key "):].strip().partition("=")
+                vals[k.strip()] = v.strip()
+    if vals.get("source_hash") != want or "traffic_bytes_per_launch" not in vals:
+        return None
+    return float(vals["traffic_bytes_per_launch"])
+
+
+def build_state(wl, layers, steps_total, device):
+    """All layers' gated caches at 32K context, built through the library (score and
+    compact the prefix; the last 128 tokens go to the ring with their gates), plus
+    per-step decode inputs resident in HBM."""
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.inputs import device as D
+    from sparse_decode_attention_spkv_b200.inputs import gen
+
+    B, Hq, Hkv, d, Dm, w = wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.window
+    T0 = wl.ctx[0]
+    Tt = wl.T_total
+    p = S.make_params(B, Hq, Hkv, d, Dm, wl.hid, w, wl.tau, S.BF16)
+    bf = torch.bfloat16
+    chunk = 4096
+    h_c = torch.empty((B, chunk, Dm), dtype=bf, device=device)
+    k_c = torch.empty((B, chunk, Hkv, d), dtype=bf, device=device)
+    v_c = torch.empty_like(k_c)
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    keep_table = W.load_biases()[wl.name]["keep_target"]
+    Ls = []
+    for l in range(layers):
+        W1 = torch.from_numpy(wl.w1(l)).to(bf).to(device)
+        b1 = torch.from_numpy(wl.b1(l)).to(device)
+        W2 = torch.from_numpy(wl.w2(l)).to(device)
+        b2 = torch.from_numpy(wl.b2(l)).to(device)
+        rows_head = [min(T0 + steps_total, int(keep_table[l][kh] * 1.15 * T0) + steps_total + 256)
+                     for kh in range(Hkv)]
+        max_pages = R.pages_for(max(rows_head))
+        num_pages = B * sum(R.pages_for(r) for r in rows_head)
+        L = R.Layer.create(p, W1, b1, W2, b2, num_pages, max_pages, device)
+        kh_, kk_, kv_ = wl.key(l, gen.T_H), wl.key(l, gen.T_K), wl.key(l, gen.T_V)
+        for c0 in range(0, T0, chunk):
+            n = min(chunk, T0 - c0)
+            for b in range(B):
+                D.fill_normal(h_c[b, :n], kh_, 1.0, offset=(b * Tt + c0) * Dm)
+                D.fill_normal(k_c[b, :n], kk_, wl.qkv_scale, offset=(b * Tt + c0) * Hkv * d)
+                D.fill_normal(v_c[b, :n], kv_, wl.qkv_scale, offset=(b * Tt + c0) * Hkv * d)
+            hc = h_c[:, :n].contiguous() if n < chunk else h_c
+            kc = k_c[:, :n].contiguous() if n < chunk else k_c
+            vc = v_c[:, :n].contiguous() if n < chunk else v_c
+            _, z = R.score(L, hc, B * n)
+            n_compact = max(0, min(c0 + n, T0 - w) - c0)
+            src = torch.full((B,), c0, dtype=torch.int32, device=device)
+            if n_compact:
+                S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, src, n_compact, n)
+            S.spkv_ring_write(p, L.ring, kc, vc, z, n_compact, src, n, n)
+        Ls.append(L)
+    del h_c, k_c, v_c
+    # per-step inputs [steps][layers][B][...] for positions T0, T0+1, ...
+    S_ = steps_total
+    h_s = torch.empty((layers, B, S_, Dm), dtype=bf, device=device)
+    q_s = torch.empty((layers, B, S_, Hq, d), dtype=bf, device=device)
+    k_s = torch.empty((layers, B, S_, Hkv, d), dtype=bf, device=device)
+    v_s = torch.empty_like(k_s)
+    for l in range(layers):
+        for b in range(B):
+            D.fill_normal(h_s[l, b], wl.key(l, gen.T_H), 1.0, offset=(b * Tt + T0) * Dm)
+            D.fill_normal(q_s[l, b], wl.key(l, gen.T_Q), wl.qkv_scale, offset=(b * Tt + T0) * Hq * d)
+            D.fill_normal(k_s[l, b], wl.key(l, gen.T_K), wl.qkv_scale, offset=(b * Tt + T0) * Hkv * d)
+            D.fill_normal(v_s[l, b], wl.key(l, gen.T_V), wl.qkv_scale, offset=(b * Tt + T0) * Hkv * d)
+    inputs = {
+        "h": h_s.permute(2, 0, 1, 3).contiguous(),
+        "q": q_s.permute(2, 0, 1, 3, 4).contiguous(),
+        "k": k_s.permute(2, 0, 1, 3, 4).contiguous(),
+        "v": v_s.permute(2, 0, 1, 3, 4).contiguous(),
+        "t": (torch.arange(S_, dtype=torch.int32, device=device) + T0).view(S_, 1).repeat(1, B).contiguous(),
+    }
+    del h_s, q_s, k_s, v_s
+    torch.cuda.synchronize()
+    for L in Ls:
+        status, flags = S.spkv_cache_check(L.cache)
+        if status != S.OK:
+            raise RuntimeError(f"cache setup failed: {S.status_str(status)} flags={flags}")
+    return p, Ls, inputs
+
+
+class Step:
+    """Launch sequence of one decode step (all layers) on fixed buffers."""
+
+    def __init__(self, p, layers, device):
+        from sparse_decode_attention_spkv_b200 import spkv as S
+        self.S, self.p, self.layers = S, p, layers
+        n = len(layers)
+        self.o = torch.empty((n, p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((n, p.B, p.Hq), dtype=torch.float32, device=device)
+        self.u = torch.empty((n, p.B, p.Hkv), dtype=torch.float32, device=device)
+        self.z = torch.empty((n, p.B, p.Hkv), dtype=torch.uint8, device=device)
+
+    def launch(self, h, q, k, v, t, ev=None):
+        """h [L][B][D], q [L][B][Hq][d], k, v [L][B][Hkv][d], t [B]; ev: per-layer
+        (start, end) timing events around the decode-attention launch."""
+        S, p = self.S, self.p
+        for l, L in enumerate(self.layers):
+            S.spkv_score(p, h[l], p.B, L.W1, L.b1, L.W2, L.b2, self.u[l], self.z[l])
+            S.spkv_decode_append(p, L.cache, L.ring, t, k[l], v[l], self.z[l], 1)
+            if ev is not None:
+                ev[l][0].record()
+            S.spkv_decode_attn(p, L.cache, L.ring, q[l], t, self.o[l], self.lse[l], L.ws)
+            if ev is not None:
+                ev[l][1].record()
+
+    LAUNCHES_PER_LAYER = 3
+
+
+def kv_bytes(p, layers, t):
+    """Algorithmic K/V bytes of one decode step at query position t: every head reads
+    its live cache rows and its window rows once (K and V, bf16)."""
+    total = 0
+    n_win = min(p.window, t + 1)
+    for L in layers:
+        total += int((L.cache.count.to(torch.int64) + n_win).sum().item())
+    return total * 2 * p.head_dim * 2
+
+
+def run_gpu(args, world, rank, local):
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+
+    device = torch.device("cuda", local)
+    wl = W.WORKLOADS[WORKLOAD]
+    layers = wl.layers
+    K, Wm, E = args.steps, args.warmup, args.e2e_steps
+    steps_total = Wm + K + E
+    if steps_total > wl.decode_steps:
+        raise SystemExit(f"warmup+steps+e2e-steps must be <= {wl.decode_steps}")
+    p, Ls, inp = build_state(wl, layers, steps_total, device)
+    T0 = wl.ctx[0]
+    step = Step(p, Ls, device)
+
+    # one eager decode-attention call per layer sets kernel attributes before capture
+    for l, L in enumerate(Ls):
+        S.spkv_decode_attn(p, L.cache, L.ring, inp["q"][0, l], inp["t"][0], step.o[l], step.lse[l], L.ws)
+    torch.cuda.synchronize()
+
+    graphs, events = [], []
+    for i in range(Wm + K):
+        ev = [(torch.cuda.Event(enable_timing=True, external=True),
+               torch.cuda.Event(enable_timing=True, external=True)) for _ in range(layers)]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i], ev)
+        graphs.append(g)
+        events.append(ev)
+    torch.cuda.synchronize()
+
+    for i in range(Wm):
+        graphs[i].replay()
+    torch.cuda.synchronize()
+    bytes_before = kv_bytes(p, Ls, T0 + Wm)
+
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    with clocks:
+        _barrier(world)
+        torch.cuda.synchronize()
+        start.record()
+        for i in range(Wm, Wm + K):
+            graphs[i].replay()
+        end.record()
+        torch.cuda.synchronize()
+        _barrier(world)
+    elapsed_ms = start.elapsed_time(end)
+    bytes_after = kv_bytes(p, Ls, T0 + Wm + K - 1)
+    step_bytes = 0.5 * (bytes_before + bytes_after)
+    attn_ms = [events[i][l][0].elapsed_time(events[i][l][1]) for i in range(Wm, Wm + K)
+               for l in range(layers)]
+    attn_avg_ms = sum(attn_ms) / len(attn_ms)
+    launch_bytes = step_bytes / layers
+    elapsed_max = _max_over_ranks(elapsed_ms, world)
+    for L in Ls:
+        status, flags = S.spkv_cache_check(L.cache)
+        if status != S.OK:
+            raise RuntimeError(f"device error after timing: {S.status_str(status)} flags={flags}")
+    if not torch.isfinite(step.o.float()).all():
+        raise RuntimeError("non-finite decode output")
+
+    # ---- end to end: host inputs in, host outputs back, every step -------------------
+    e2e = None
+    if E > 0:
+        st = {k: torch.empty_like(inp[k][0]) for k in ("h", "q", "k", "v", "t")}
+        host = {k: inp[k][Wm + K:].cpu().pin_memory() for k in ("h", "q", "k", "v", "t")}
+        o_host = torch.empty((E,) + tuple(step.o.shape), dtype=step.o.dtype).pin_memory()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.launch(st["h"], st["q"], st["k"], st["v"], st["t"])
+        torch.cuda.synchronize()
+        s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        _barrier(world)
+        torch.cuda.synchronize()
+        s0.record()
+        for j in range(E):
+            for k_ in st:
+                st[k_].copy_(host[k_][j], non_blocking=True)
+            g.replay()
+            o_host[j].copy_(step.o, non_blocking=True)
+        s1.record()
+        torch.cuda.synchronize()
+        _barrier(world)
+        e2e_ms = _max_over_ranks(s0.elapsed_time(s1), world)
+        h2d = sum(host[k_][0].numel() * host[k_][0].element_size() for k_ in host)
+        d2h = step.o.numel() * step.o.element_size()
+        e2e = {"value": world * p.B * E / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E}
+        del g
+    del graphs
+
+    peak, peak_kind = _peaks()
+    achieved = launch_bytes / (attn_avg_ms / 1e3) / 1e9
+    traffic = _profiled_traffic()
+    tokens_s = world * p.B * K / (elapsed_max / 1e3)
+    ms_step = elapsed_max / K
+    live = sum(int(L.cache.count.sum().item()) for L in Ls)
+    heads = layers * p.B * p.Hkv
+    out = {
+        "metric": METRIC, "value": tokens_s, "unit": "tokens/s", "n_gpus": world, "steps": K,
+        "warmup": Wm, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode32k: batch 8 x 32 layers, 32q/8kv heads, head_dim 128, "
+                               "d_model 4096, utility MLP 4096->128->8, w=128, tau=0.5, 32768-token "
+                               "context, per-head keep U[5%,50%], per-token retirement",
+                   "global_batch": world * p.B, "seq_len": T0, "layers": layers,
+                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "l2": "inputs larger than L2 (every step reads all live K/V, ~GBs)"},
+        "kv_gbs_effective": step_bytes / (ms_step / 1e3) / 1e9,
+        "kv_bytes_per_step": step_bytes,
+        "kv_density_nonlocal": (live / heads) / (T0 - p.window),
+        "decode_attn_ms_avg": attn_avg_ms,
+        "roofline": {"bound": "hbm", "kernel": "decode_attn", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_kind": peak_kind,
+                     "traffic": traffic, "algorithmic_bytes_per_launch": launch_bytes},
+        "gpu_launches": Step.LAUNCHES_PER_LAYER * layers * K,
+        "clocks": clocks.summary(),
+        "e2e": e2e,
+    }
+    return out
+
+
+# -------------------------------------------------------------- CPU oracle arm -----
+
+def oracle_decode_sample(units: int, seed: int = 0):
+    """Time the fp64 oracle on `units` (layer, batch row) units of the decode32k step
+    at t = 32768: the utility of the row's new token and Eqs. (3)-(4) for its 32 query
+    heads over 32769 keys.  Inputs are random numbers of the workload's shapes and
+    keep rates (their values do not change the work).  Returns (seconds per unit,
+    threads used)."""
+    from oracle import spkv_oracle as O
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = 1
+    wl = W.WORKLOADS[WORKLOAD]
+    rng = np.random.default_rng(seed)
+    t = wl.ctx[0]
+    T = t + 1
+    W1 = rng.standard_normal((wl.hid, wl.d_model)) * 0.02
+    b1 = rng.standard_normal(wl.hid) * 0.02
+    W2 = rng.standard_normal((wl.Hkv, wl.hid)) * 0.02
+    b2 = np.zeros(wl.Hkv)
+    Q = rng.standard_normal((1, wl.Hq, wl.head_dim)) / math.sqrt(wl.head_dim)
+    K = rng.standard_normal((T, wl.Hkv, wl.head_dim)) / math.sqrt(wl.head_dim)
+    V = rng.standard_normal((T, wl.Hkv, wl.head_dim)) / math.sqrt(wl.head_dim)
+    z = (rng.random((T, wl.Hkv)) < 0.275).astype(np.uint8)
+    h = rng.standard_normal((1, wl.d_model))
+    t0 = time.perf_counter()
+    for _ in range(units):
+        O.gate(O.utility(h, W1, b1, W2, b2), wl.tau)
+        O.gated_attention(Q, K, V, z, wl.window, [t])
+    dt = time.perf_counter() - t0
+    return dt / units, threads
+
+
+def cpu_baseline(units: int):
+    per_unit, threads = oracle_decode_sample(units)
+    wl_units = 32 * 8  # (layer, batch row) units in one decode32k step
+    step_s = per_unit * wl_units
+    return {"value": 8 / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"{units} of the 256 (layer, batch row) units of one decode32k step at "
+                      f"t=32768 (fp64 numpy oracle: utility + Eqs. (3)-(4) for 32 query heads "
+                      f"over 32769 keys), {per_unit * 1e3:.1f} ms per unit, extrapolated to the "
+                      f"full step"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    units = args.cpu_units
+    for _ in range(args.warmup):
+        oracle_decode_sample(1)
+    times = []
+    for _ in range(args.steps):
+        per_unit, threads = oracle_decode_sample(units)
+        times.append(per_unit * 256)
+    step_s = sum(times) / len(times)
+    value = 8 / step_s
+    cb = cpu_baseline_desc = {
+        "value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+        "sample": f"each step: {units} of the 256 (layer, batch row) units of one decode32k "
+                  f"step, extrapolated to the full step"}
+    return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "decode32k (see the spkv arm)", "global_batch": 8,
+                       "seq_len": 32768, "layers": 32, "parallelism": "host cores"},
+            "cpu_baseline": cb,
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="spkv", choices=["spkv", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--cpu-units", type=int, default=48)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = _dist_init()
+    out = run_gpu(args, world, rank, local)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            out["cpu_baseline"] = cpu_baseline(args.cpu_units)
+        else:
+            out["cpu_baseline"] = None
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

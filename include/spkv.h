@@ -1,0 +1,206 @@
+/*
+ * spkv.h -- C ABI of libspkv.so: the hot path of Self-Pruned Key-Value attention
+ * (SP-KV) on NVIDIA B200 (sm_100a).
+ *
+ * Source of the method: "Self-Pruned Key-Value Attention: Learning When to Write
+ * by Predicting Future Utility" (arXiv 2605.14037), §2.1:
+ *   Eq. (1)  u_s = sigmoid(f(h_s)), f a small two-layer perceptron per layer,
+ *            one output per key head;
+ *   Eq. (2)  z_s = 1[u_s >= tau];
+ *   Eq. (3)  a_{t,s} = softmax(q_t k_s^T / sqrt(d_k) + M_{t,s});
+ *   Eq. (4)  M_{t,s} = 0 if 0 <= t-s < w, or z_s = 1 and s <= t; else -inf;
+ *   "efficient implementation at deployment": only pairs with z_s = 1 are kept in
+ *   a persistent cache; each query attends to that cache plus the local window.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *   allocates nothing; the caller provides every buffer (the decode workspace
+ *   included) and must keep it alive until the stream work that uses it ends.
+ * - Every call enqueues work on `stream` (a cudaStream_t; NULL means the legacy
+ *   default stream) and returns without synchronising, except spkv_cache_check.
+ * - Return value: SPKV_OK, or an error code.  Arguments are validated on the host
+ *   before anything is enqueued; on SPKV_ERR_ARG nothing was enqueued.  Conditions
+ *   only the device can see (cache pool exhausted, page table full, a bounded wait
+ *   that gave up) set bits of cache->err_flag, read by spkv_cache_check.
+ *   No entry point aborts, throws or traps.
+ * - Element types: `dtype` SPKV_F32 or SPKV_BF16 applies to h, W1, q, k, v, the
+ *   cache pool, the ring and the attention output.  b1, W2, b2, u and lse are fp32
+ *   in both cases.  Arithmetic is fp32 (bf16 inputs are widened exactly).
+ * - Layouts are dense row-major with the shapes given below.  head_dim must be
+ *   64 or 128, Hq a multiple of Hkv with Hq/Hkv in {1,2,4,8}, window in [1, 1024],
+ *   page_rows 64.  Pointers to tensors must be 16-byte aligned.
+ * - Positions are absolute token indices (int32).  Query head h reads key head
+ *   h / (Hq/Hkv) (grouped-query attention).
+ */
+#ifndef SPKV_H
+#define SPKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef void* spkv_stream_t; /* cudaStream_t */
+
+enum spkv_status {
+  SPKV_OK = 0,
+  SPKV_ERR_ARG = 1,         /* invalid argument: nothing enqueued */
+  SPKV_ERR_CAPACITY = 2,    /* device-detected: pool or page table exhausted */
+  SPKV_ERR_CUDA = 3,        /* a CUDA runtime call or a launch failed */
+  SPKV_ERR_UNSUPPORTED = 4, /* valid but not built (shape/dtype combination) */
+  SPKV_ERR_TIMEOUT = 5      /* device-detected: a bounded wait gave up */
+};
+
+enum spkv_dtype { SPKV_F32 = 0, SPKV_BF16 = 1 };
+
+enum spkv_src_kind {
+  SPKV_SRC_CHUNK = 0, /* rows come from a chunk tensor [B][src_batch_rows][Hkv][head_dim] */
+  SPKV_SRC_RING = 1   /* rows come from the ring: position p lives in slot p mod window */
+};
+
+/* err_flag bits */
+#define SPKV_FLAG_POOL_FULL 1u  /* no free page was left for an append */
+#define SPKV_FLAG_TABLE_FULL 2u /* a key head reached max_pages_per_head */
+#define SPKV_FLAG_TIMEOUT 4u    /* a bounded wait inside a kernel gave up */
+
+/* Shapes of one attention layer. */
+typedef struct spkv_params {
+  int B;        /* batch rows */
+  int Hq;       /* query heads */
+  int Hkv;      /* key/value heads */
+  int head_dim; /* d_k */
+  int d_model;  /* width of h */
+  int hid;      /* hidden width of the utility perceptron, <= 128 */
+  int window;   /* w of Eq. (4) */
+  float tau;    /* threshold of Eq. (2) */
+  int dtype;    /* enum spkv_dtype */
+} spkv_params;
+
+/* Persistent gated cache of one layer (§2.1, deployment).  Storage is paged:
+ * key head kh of batch row b (index bh = b*Hkv + kh) owns the pages listed in
+ * page_table[bh][0..], assigned on demand by the device from a bump allocator
+ * (pool_top).  Cache row i of head bh is row i % page_rows of page
+ * page_table[bh][i / page_rows]; its absolute position is pos_pool at the same
+ * place.  Rows are appended in increasing position order. */
+typedef struct spkv_cache {
+  void* K_pool;        /* [num_pages][page_rows][head_dim] dtype */
+  void* V_pool;        /* [num_pages][page_rows][head_dim] dtype */
+  int32_t* pos_pool;   /* [num_pages][page_rows] absolute positions */
+  int32_t* page_table; /* [B*Hkv][max_pages_per_head], -1 = none */
+  int32_t* count;      /* [B*Hkv] rows stored per key head */
+  int32_t* count_prev; /* [B*Hkv] value of count before the last chunk append */
+  int32_t* pool_top;   /* [1] next free page */
+  uint32_t* err_flag;  /* [1] SPKV_FLAG_* bits, sticky until spkv_cache_reset */
+  int num_pages;
+  int page_rows; /* must be 64 */
+  int max_pages_per_head;
+} spkv_cache;
+
+/* Local window (Eq. (4), 1_win): the last `window` keys/values of every
+ * (batch row, key head), position p in slot p % window; z_win holds the gate of
+ * the token in each slot (for retirement into the cache). */
+typedef struct spkv_ring {
+  void* K_win;    /* [B][Hkv][window][head_dim] dtype */
+  void* V_win;    /* [B][Hkv][window][head_dim] dtype */
+  uint8_t* z_win; /* [B][window][Hkv] */
+} spkv_ring;
+
+/* Static text for a status code. */
+const char* spkv_status_str(int status);
+
+/* Library version (major*10000 + minor*100 + patch). */
+int spkv_version(void);
+
+/* Zero the cache (count, count_prev, pool_top, err_flag), set page_table to -1
+ * and, if ring is not NULL, zero its z_win. */
+int spkv_cache_reset(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                     spkv_stream_t stream);
+
+/* Synchronise `stream`, copy err_flag to *flags_out (if not NULL) and return
+ * SPKV_ERR_CAPACITY if a pool/table bit is set, SPKV_ERR_TIMEOUT if the timeout
+ * bit is set, else SPKV_OK. */
+int spkv_cache_check(const spkv_cache* cache, spkv_stream_t stream, uint32_t* flags_out);
+
+/* a1 -- utility score and gate, Eqs. (1)-(2), fused:
+ *   a = h W1^T + b1;  x = GELU(a) (exact erf form);  l = x W2^T + b2;
+ *   u = sigmoid(l);   z = 1[u >= tau]   for every token and key head.
+ * h [n_tok][d_model] dtype; W1 [hid][d_model] dtype; b1 [hid] f32;
+ * W2 [Hkv][hid] f32; b2 [Hkv] f32.  Outputs u_out [n_tok][Hkv] f32 (may be
+ * NULL) and z_out [n_tok][Hkv] uint8.  n_tok >= 0 (0 enqueues nothing). */
+int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, const float* b1,
+               const float* W2, const float* b2, float* u_out, uint8_t* z_out,
+               spkv_stream_t stream);
+
+/* a2 -- stream compaction (§2.1 deployment): for every (b, key head), append the
+ * rows i in [0, n_rows) with z = 1, in increasing i, to the cache, recording
+ * position src_pos[b] + i.
+ *   src_kind SPKV_SRC_CHUNK: K_src/V_src [B][src_batch_rows][Hkv][head_dim];
+ *   src_kind SPKV_SRC_RING: rows are read from ring->K_win/V_win (K_src/V_src
+ *     ignored), row i of batch b from slot (src_pos[b] + i) % window; requires
+ *     n_rows <= window.
+ * z [B][src_batch_rows][Hkv] uint8 (device); src_pos [B] int32 (device).
+ * Positions must exceed those already stored for that head.  Rows that do not fit
+ * are dropped and flagged in err_flag.  Two kernels: plan (page allocation), then
+ * scatter. */
+int spkv_write_compact(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                       int src_kind, const void* K_src, const void* V_src, const uint8_t* z,
+                       const int32_t* src_pos, int n_rows, int src_batch_rows,
+                       spkv_stream_t stream);
+
+/* a2 + a3 for one decode step per batch row (per-token retirement): with
+ * t = t_pos[b], if retire != 0 and t - window >= 0, the token s = t - window
+ * leaves the window; it is appended to the cache if its gate (ring->z_win of its
+ * slot) is 1.  Then k_new, v_new (and z_new, if not NULL; else 0) are stored in
+ * slot t % window.  k_new, v_new [B][Hkv][head_dim] dtype; z_new [B][Hkv] uint8;
+ * t_pos [B] int32, all device. */
+int spkv_decode_append(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                       const int32_t* t_pos, const void* k_new, const void* v_new,
+                       const uint8_t* z_new, int retire, spkv_stream_t stream);
+
+/* a3 -- store the last min(n_rows, window) rows of a chunk in the ring: row i of
+ * batch b (position src_pos[b] + i) goes to slot (src_pos[b] + i) % window.  The
+ * slot's gate is 0 for rows i < gated_from (already in the cache, so retiring them
+ * appends nothing) and z_src[b][i][kh] for the others (z_src may be NULL when
+ * gated_from >= n_rows).  K_src/V_src [B][src_batch_rows][Hkv][head_dim],
+ * z_src [B][src_batch_rows][Hkv]. */
+int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
+                    const void* V_src, const uint8_t* z_src, int gated_from,
+                    const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream);
+
+/* Bytes of decode workspace spkv_decode_attn needs for this cache geometry.  The
+ * workspace must be zero-filled once before its first use; the library leaves
+ * its counters at zero after every call.  Calls that share a workspace must not
+ * overlap on the device. */
+size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* cache);
+
+/* a4 + a5 -- gated decode attention, Eqs. (3)-(4), one query per batch row:
+ * query t = t_pos[b] attends to the window slots holding positions
+ * max(0, t-window+1)..t and to the cache rows with position <= t - window.
+ * Split-K over balanced chunks of rows, with the log-sum-exp merge of the chunk
+ * partials done by the last chunk of each key head to finish.
+ * q [B][Hq][head_dim] dtype; o [B][Hq][head_dim] dtype; lse [B][Hq] f32 natural
+ * log (may be NULL).  The token t itself must already be in the ring. */
+int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                     const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
+                     size_t ws_bytes, spkv_stream_t stream);
+
+/* a6 -- gated prefill attention, Eqs. (3)-(4), for the chunk of queries at
+ * positions chunk_start .. chunk_start+chunk_len-1 of every batch row.  Keys:
+ * the window, from K_chunk/V_chunk (positions >= chunk_start) and from the ring
+ * (earlier positions, which must hold the previous chunk's last rows), and the
+ * cache rows with position <= t - window (the cache may already hold rows of
+ * this chunk; those are used only by queries they have left the window of).
+ * q [B][chunk_len][Hq][head_dim]; K_chunk, V_chunk [B][chunk_len][Hkv][head_dim];
+ * o [B][chunk_len][Hq][head_dim]; lse [B][chunk_len][Hq] f32 (may be NULL). */
+int spkv_prefill_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                      const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
+                      int chunk_len, void* o, float* lse, spkv_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPKV_H */

@@ -1,0 +1,194 @@
+// api.cu -- the C ABI (include/spkv.h): host-side validation, then launches.
+// Validation touches no CUDA API, so argument errors are reported without a GPU.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+
+#include "../../include/spkv.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace {
+
+using spkv::kPageRows;
+
+int status_of(cudaError_t e) { return e == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool params_ok(const spkv_params* p) {
+  if (!p) return false;
+  if (p->B < 1 || p->Hkv < 1 || p->Hq < p->Hkv || p->Hq % p->Hkv) return false;
+  const int G = p->Hq / p->Hkv;
+  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+  if (p->head_dim != 64 && p->head_dim != 128) return false;
+  if (p->window < 1 || p->window > 1024) return false;
+  if (p->dtype != SPKV_F32 && p->dtype != SPKV_BF16) return false;
+  if (!(p->tau == p->tau)) return false;  // NaN threshold
+  return true;
+}
+
+bool cache_ok(const spkv_params* p, const spkv_cache* c) {
+  if (!c) return false;
+  if (!c->K_pool || !c->V_pool || !c->pos_pool || !c->page_table || !c->count ||
+      !c->count_prev || !c->pool_top || !c->err_flag)
+    return false;
+  if (c->page_rows != kPageRows || c->num_pages < 1 || c->max_pages_per_head < 1) return false;
+  if (!aligned16(c->K_pool) || !aligned16(c->V_pool)) return false;
+  (void)p;
+  return true;
+}
+
+bool ring_ok(const spkv_ring* r) {
+  return r && r->K_win && r->V_win && r->z_win && aligned16(r->K_win) && aligned16(r->V_win);
+}
+
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  static std::mutex mu;
+  static int cached[64] = {0};
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev < 0 || dev >= 64) return -1;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spkv_status_str(int status) {
+  switch (status) {
+    case SPKV_OK: return "ok";
+    case SPKV_ERR_ARG: return "invalid argument";
+    case SPKV_ERR_CAPACITY: return "cache capacity exhausted";
+    case SPKV_ERR_CUDA: return "CUDA error";
+    case SPKV_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case SPKV_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+int spkv_version(void) { return 100; }
+
+int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                     spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c)) return SPKV_ERR_ARG;
+  if (ring && !ring_ok(ring)) return SPKV_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t heads = (size_t)p->B * p->Hkv;
+  cudaError_t e = cudaMemsetAsync(c->page_table, 0xff, heads * c->max_pages_per_head * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->count, 0, heads * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->count_prev, 0, heads * 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->pool_top, 0, 4, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(c->err_flag, 0, 4, s);
+  if (e == cudaSuccess && ring) e = cudaMemsetAsync(ring->z_win, 0, (size_t)p->B * p->window * p->Hkv, s);
+  return status_of(e);
+}
+
+int spkv_cache_check(const spkv_cache* c, spkv_stream_t stream, uint32_t* flags_out) {
+  if (!c || !c->err_flag) return SPKV_ERR_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t flags = 0;
+  cudaError_t e = cudaMemcpyAsync(&flags, c->err_flag, 4, cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return SPKV_ERR_CUDA;
+  if (flags_out) *flags_out = flags;
+  if (flags & (SPKV_FLAG_POOL_FULL | SPKV_FLAG_TABLE_FULL)) return SPKV_ERR_CAPACITY;
+  if (flags & SPKV_FLAG_TIMEOUT) return SPKV_ERR_TIMEOUT;
+  return SPKV_OK;
+}
+
+int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, const float* b1,
+               const float* W2, const float* b2, float* u_out, uint8_t* z_out,
+               spkv_stream_t stream) {
+  if (!params_ok(p) || n_tok < 0) return SPKV_ERR_ARG;
+  if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
+  if (n_tok == 0) return SPKV_OK;
+  if (!h || !W1 || !b1 || !W2 || !b2 || !z_out) return SPKV_ERR_ARG;
+  if (!spkv::score_supported(*p)) return SPKV_ERR_UNSUPPORTED;
+  return status_of(spkv::launch_score(*p, h, n_tok, W1, b1, W2, b2, u_out, z_out,
+                                      static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_write_compact(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                       int src_kind, const void* K_src, const void* V_src, const uint8_t* z,
+                       const int32_t* src_pos, int n_rows, int src_batch_rows,
+                       spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
+  if (n_rows == 0) return SPKV_OK;
+  if (!z || !src_pos) return SPKV_ERR_ARG;
+  if (src_kind == SPKV_SRC_CHUNK) {
+    if (!K_src || !V_src || !aligned16(K_src) || !aligned16(V_src)) return SPKV_ERR_ARG;
+  } else if (src_kind == SPKV_SRC_RING) {
+    if (!ring_ok(ring) || n_rows > p->window) return SPKV_ERR_ARG;
+  } else {
+    return SPKV_ERR_ARG;
+  }
+  return status_of(spkv::launch_write_compact(*p, *c, ring, src_kind, K_src, V_src, z, src_pos,
+                                              n_rows, src_batch_rows,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_decode_append(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                       const int32_t* t_pos, const void* k_new, const void* v_new,
+                       const uint8_t* z_new, int retire, spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!t_pos || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_decode_append(*p, *c, *ring, t_pos, k_new, v_new, z_new, retire,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
+                    const void* V_src, const uint8_t* z_src, int gated_from,
+                    const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream) {
+  if (!params_ok(p) || !ring_ok(ring) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
+  if (n_rows == 0) return SPKV_OK;
+  if (!K_src || !V_src || !src_pos || !aligned16(K_src) || !aligned16(V_src)) return SPKV_ERR_ARG;
+  if (gated_from < 0) return SPKV_ERR_ARG;
+  if (!z_src && gated_from < n_rows) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_ring_write(*p, *ring, K_src, V_src, z_src, gated_from, src_pos,
+                                           n_rows, src_batch_rows,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* c) {
+  (void)c;
+  if (!params_ok(p)) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return spkv::decode_workspace_bytes(*p, sms);
+}
+
+int spkv_decode_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                     const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
+                     size_t ws_bytes, spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
+  if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_decode(*p, *c, *ring, q, t_pos, o, lse, workspace, ws_bytes, sms,
+                                       static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_prefill_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                      const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
+                      int chunk_len, void* o, float* lse, spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (chunk_start < 0 || chunk_len < 0) return SPKV_ERR_ARG;
+  if (chunk_len == 0) return SPKV_OK;
+  if (!q || !K_chunk || !V_chunk || !o) return SPKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(K_chunk) || !aligned16(V_chunk) || !aligned16(o)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_prefill(*p, *c, *ring, q, K_chunk, V_chunk, chunk_start,
+                                        chunk_len, o, lse, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

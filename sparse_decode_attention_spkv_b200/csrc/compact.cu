@@ -1,0 +1,302 @@
+// compact.cu -- a2/a3: writes into the persistent gated cache and the window ring.
+//
+// "Self-Pruned Key-Value Attention" (arXiv 2605.14037), §2.1, efficient
+// implementation at deployment: the persistent cache stores only the KV pairs
+// with z_s = 1; the most recent w tokens stay reachable through the local window
+// (Eq. (4), 1_win).  These kernels move rows between those two stores:
+//   compact_plan / compact_scatter  stable stream compaction of gated rows (a2),
+//   decode_append                   per-token retirement t-w -> cache, then the
+//                                   new token into its ring slot (a2 + a3),
+//   ring_write                      last rows of a prefill chunk into the ring (a3).
+// Rows are moved as 16-byte vectors by the lanes of one warp (a 256-byte row is
+// 16 lanes), so every copy is coalesced.
+#include "common.cuh"
+#include "launch.h"
+
+namespace spkv {
+namespace {
+
+struct CacheMut {
+  char* K;
+  char* V;
+  int32_t* pos;
+  int32_t* page_table;
+  int32_t* count;
+  int32_t* count_prev;
+  int32_t* pool_top;
+  uint32_t* err;
+  int num_pages;
+  int max_pages;
+};
+
+CacheMut mut(const spkv_cache& c) {
+  return CacheMut{static_cast<char*>(c.K_pool), static_cast<char*>(c.V_pool), c.pos_pool,
+                  c.page_table, c.count, c.count_prev, c.pool_top, c.err_flag, c.num_pages,
+                  c.max_pages_per_head};
+}
+
+__device__ __forceinline__ int block_sum(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+#pragma unroll
+  for (int m = 16; m > 0; m >>= 1) v += __shfl_xor_sync(0xffffffffu, v, m);
+  __syncthreads();
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  int total = 0;
+  for (int w = 0; w < (int)(blockDim.x >> 5); ++w) total += red[w];
+  return total;
+}
+
+// One CTA per (batch row, key head): count this call's gated rows, extend the
+// head's page list from the bump allocator, and publish count_prev / count.
+__global__ void __launch_bounds__(256)
+    compact_plan(CacheMut c, const uint8_t* __restrict__ z, int n_rows, int src_batch_rows,
+                 int hkv) {
+  __shared__ int red[8];
+  __shared__ int s_first, s_have, s_grant;
+  const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
+  const uint8_t* zb = z + (size_t)b * src_batch_rows * hkv + kh;
+  int kept = 0;
+  for (int i = threadIdx.x; i < n_rows; i += blockDim.x) kept += zb[(size_t)i * hkv];
+  const int total = block_sum(kept, red);
+  if (threadIdx.x == 0) {
+    const int old = c.count[bh];
+    const int cap = c.max_pages * kPageRows;
+    int want = old + total;
+    if (want > cap) {
+      atomicOr(c.err, SPKV_FLAG_TABLE_FULL);
+      want = cap;
+    }
+    const int have = (old + kPageRows - 1) / kPageRows;
+    int need = (want + kPageRows - 1) / kPageRows;
+    int first = 0, grant = 0;
+    if (need > have) {
+      first = atomicAdd(c.pool_top, need - have);
+      grant = need - have;
+      if (first + grant > c.num_pages) {
+        grant = c.num_pages - first > 0 ? c.num_pages - first : 0;
+        atomicOr(c.err, SPKV_FLAG_POOL_FULL);
+        need = have + grant;
+        if (want > need * kPageRows) want = need * kPageRows;
+      }
+    }
+    c.count_prev[bh] = old;
+    c.count[bh] = want;
+    s_first = first;
+    s_have = have;
+    s_grant = grant;
+  }
+  __syncthreads();
+  for (int j = threadIdx.x; j < s_grant; j += blockDim.x)
+    c.page_table[(size_t)bh * c.max_pages + s_have + j] = s_first + j;
+}
+
+constexpr int kScatterTile = 1024;
+constexpr int kScatterThreads = 256;
+
+// grid (B*Hkv, tiles of 1024 rows).  Each CTA counts the gated rows before its
+// tile (z is tiny), so tiles need no inter-CTA ordering; inside a tile, 256-row
+// rounds are ranked with a warp-ballot prefix sum and copied by lane groups.
+__global__ void __launch_bounds__(kScatterThreads)
+    compact_scatter(CacheMut c, const char* __restrict__ Ksrc, const char* __restrict__ Vsrc,
+                    const uint8_t* __restrict__ z, const int32_t* __restrict__ src_pos,
+                    int n_rows, int src_batch_rows, int hkv, int row_bytes, int from_ring,
+                    int window) {
+  __shared__ int red[8];
+  __shared__ int warp_tot[8];
+  __shared__ int list_src[kScatterThreads];
+  __shared__ int list_dst[kScatterThreads];
+  const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
+  const int tile0 = blockIdx.y * kScatterTile;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const uint8_t* zb = z + (size_t)b * src_batch_rows * hkv + kh;
+
+  int before = 0;
+  for (int i = threadIdx.x; i < tile0; i += blockDim.x) before += zb[(size_t)i * hkv];
+  const int prefix = block_sum(before, red);
+  const int base = c.count_prev[bh];
+  const int limit = c.count[bh];
+  const int p0 = src_pos[b];
+  int running = base + prefix;
+
+  const int lpr = row_bytes >> 4;      // lanes per row
+  const int rpw = 32 / lpr;            // rows per warp pass
+  const int sub = lane / lpr, col = lane % lpr;
+
+  for (int r0 = tile0; r0 < tile0 + kScatterTile && r0 < n_rows; r0 += kScatterThreads) {
+    const int i = r0 + threadIdx.x;
+    const int flag = (i < n_rows) ? zb[(size_t)i * hkv] : 0;
+    const unsigned ball = __ballot_sync(0xffffffffu, flag);
+    const int in_warp = __popc(ball & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(ball);
+    __syncthreads();
+    int warp_off = 0, round_total = 0;
+    for (int w = 0; w < kScatterThreads / 32; ++w) {
+      if (w < warp) warp_off += warp_tot[w];
+      round_total += warp_tot[w];
+    }
+    const int rank = warp_off + in_warp;
+    if (flag) {
+      list_src[rank] = i;
+      list_dst[rank] = running + rank;
+    }
+    __syncthreads();
+    for (int e = warp * rpw + sub; e < round_total; e += (kScatterThreads / 32) * rpw) {
+      const int src_i = list_src[e];
+      const int dst = list_dst[e];
+      if (dst >= limit) continue;  // dropped: capacity (flag already raised by the plan)
+      const int page = c.page_table[(size_t)bh * c.max_pages + (dst >> 6)];
+      const size_t drow = (size_t)page * kPageRows + (dst & 63);
+      size_t srow;
+      if (from_ring) {
+        const int slot = (p0 + src_i) % window;
+        srow = ((size_t)bh * window + slot);
+      } else {
+        srow = ((size_t)b * src_batch_rows + src_i) * hkv + kh;
+      }
+      const uint4 kv = *reinterpret_cast<const uint4*>(Ksrc + srow * row_bytes + col * 16);
+      const uint4 vv = *reinterpret_cast<const uint4*>(Vsrc + srow * row_bytes + col * 16);
+      *reinterpret_cast<uint4*>(c.K + drow * row_bytes + col * 16) = kv;
+      *reinterpret_cast<uint4*>(c.V + drow * row_bytes + col * 16) = vv;
+      if (col == 0) c.pos[drow] = p0 + src_i;
+    }
+    running += round_total;
+    __syncthreads();
+  }
+}
+
+// One warp per (batch row, key head).
+__global__ void __launch_bounds__(128)
+    decode_append_kernel(CacheMut c, char* __restrict__ Kwin, char* __restrict__ Vwin,
+                         uint8_t* __restrict__ zwin, const int32_t* __restrict__ t_pos,
+                         const char* __restrict__ k_new, const char* __restrict__ v_new,
+                         const uint8_t* __restrict__ z_new, int retire, int n_heads, int hkv,
+                         int window, int row_bytes) {
+  const int lane = threadIdx.x & 31;
+  const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
+  if (bh >= n_heads) return;
+  const int b = bh / hkv, kh = bh % hkv;
+  const int t = t_pos[b];
+  if (t < 0) return;  // positions are non-negative by contract
+  const int slot = t % window;
+  const int s = t - window;
+  const int lpr = row_bytes >> 4;
+  const size_t ring_row = (size_t)bh * window + slot;
+  uint8_t* zslot = zwin + ((size_t)b * window + slot) * hkv + kh;
+  if (retire && s >= 0 && *zslot) {
+    const int i = c.count[bh];
+    int page = -1;
+    if ((i & 63) == 0) {
+      if (lane == 0) {
+        if ((i >> 6) >= c.max_pages) {
+          atomicOr(c.err, SPKV_FLAG_TABLE_FULL);
+        } else {
+          const int pg = atomicAdd(c.pool_top, 1);
+          if (pg >= c.num_pages) {
+            atomicOr(c.err, SPKV_FLAG_POOL_FULL);
+          } else {
+            page = pg;
+            c.page_table[(size_t)bh * c.max_pages + (i >> 6)] = pg;
+          }
+        }
+      }
+      page = __shfl_sync(0xffffffffu, page, 0);
+    } else {
+      page = c.page_table[(size_t)bh * c.max_pages + (i >> 6)];
+    }
+    if (page >= 0) {
+      const size_t drow = (size_t)page * kPageRows + (i & 63);
+      if (lane < lpr) {
+        const uint4 kv = *reinterpret_cast<const uint4*>(Kwin + ring_row * row_bytes + lane * 16);
+        const uint4 vv = *reinterpret_cast<const uint4*>(Vwin + ring_row * row_bytes + lane * 16);
+        *reinterpret_cast<uint4*>(c.K + drow * row_bytes + lane * 16) = kv;
+        *reinterpret_cast<uint4*>(c.V + drow * row_bytes + lane * 16) = vv;
+      }
+      if (lane == 0) {
+        c.pos[drow] = s;
+        c.count[bh] = i + 1;
+      }
+    }
+  }
+  __syncwarp();
+  if (lane < lpr) {
+    const uint4 kv = *reinterpret_cast<const uint4*>(k_new + (size_t)bh * row_bytes + lane * 16);
+    const uint4 vv = *reinterpret_cast<const uint4*>(v_new + (size_t)bh * row_bytes + lane * 16);
+    *reinterpret_cast<uint4*>(Kwin + ring_row * row_bytes + lane * 16) = kv;
+    *reinterpret_cast<uint4*>(Vwin + ring_row * row_bytes + lane * 16) = vv;
+  }
+  if (lane == 0) *zslot = z_new ? z_new[bh] : 0;
+}
+
+// grid (B*Hkv); the last min(n_rows, window) rows of a chunk go to their slots.
+__global__ void __launch_bounds__(256)
+    ring_write_kernel(char* __restrict__ Kwin, char* __restrict__ Vwin, uint8_t* __restrict__ zwin,
+                      const char* __restrict__ Ksrc, const char* __restrict__ Vsrc,
+                      const uint8_t* __restrict__ z_src, int gated_from,
+                      const int32_t* __restrict__ src_pos, int n_rows, int src_batch_rows, int hkv,
+                      int window, int row_bytes) {
+  const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int lpr = row_bytes >> 4, rpw = 32 / lpr, sub = lane / lpr, col = lane % lpr;
+  const int n_w = n_rows < window ? n_rows : window;
+  const int first = n_rows - n_w;
+  const int p0 = src_pos[b];
+  for (int r = warp * rpw + sub; r < n_w; r += (blockDim.x >> 5) * rpw) {
+    const int i = first + r;
+    const int slot = (p0 + i) % window;
+    const size_t srow = ((size_t)b * src_batch_rows + i) * hkv + kh;
+    const size_t drow = (size_t)bh * window + slot;
+    const uint4 kv = *reinterpret_cast<const uint4*>(Ksrc + srow * row_bytes + col * 16);
+    const uint4 vv = *reinterpret_cast<const uint4*>(Vsrc + srow * row_bytes + col * 16);
+    *reinterpret_cast<uint4*>(Kwin + drow * row_bytes + col * 16) = kv;
+    *reinterpret_cast<uint4*>(Vwin + drow * row_bytes + col * 16) = vv;
+    if (col == 0) zwin[((size_t)b * window + slot) * hkv + kh] = (i >= gated_from) ? z_src[srow] : 0;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
+                                 int src_kind, const void* K_src, const void* V_src,
+                                 const uint8_t* z, const int32_t* src_pos, int n_rows,
+                                 int src_batch_rows, cudaStream_t stream) {
+  const int n_heads = p.B * p.Hkv;
+  const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
+  const int row_bytes = p.head_dim * esize;
+  CacheMut m = mut(c);
+  compact_plan<<<n_heads, 256, 0, stream>>>(m, z, n_rows, src_batch_rows, p.Hkv);
+  const char* Ks = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->K_win : K_src);
+  const char* Vs = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->V_win : V_src);
+  dim3 grid(n_heads, (n_rows + kScatterTile - 1) / kScatterTile);
+  compact_scatter<<<grid, kScatterThreads, 0, stream>>>(m, Ks, Vs, z, src_pos, n_rows,
+                                                        src_batch_rows, p.Hkv, row_bytes,
+                                                        src_kind == SPKV_SRC_RING, p.window);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                                 const int32_t* t_pos, const void* k_new, const void* v_new,
+                                 const uint8_t* z_new, int retire, cudaStream_t stream) {
+  const int n_heads = p.B * p.Hkv;
+  const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
+  decode_append_kernel<<<(n_heads + 3) / 4, 128, 0, stream>>>(
+      mut(c), static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win, t_pos,
+      static_cast<const char*>(k_new), static_cast<const char*>(v_new), z_new, retire, n_heads,
+      p.Hkv, p.window, p.head_dim * esize);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const void* K_src,
+                              const void* V_src, const uint8_t* z_src, int gated_from,
+                              const int32_t* src_pos, int n_rows, int src_batch_rows,
+                              cudaStream_t stream) {
+  const int n_heads = p.B * p.Hkv;
+  const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
+  ring_write_kernel<<<n_heads, 256, 0, stream>>>(
+      static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win,
+      static_cast<const char*>(K_src), static_cast<const char*>(V_src), z_src, gated_from, src_pos,
+      n_rows, src_batch_rows, p.Hkv, p.window, p.head_dim * esize);
+  return cudaGetLastError();
+}
+
+}  // namespace spkv

@@ -1,0 +1,41 @@
+// launch.h -- internal launchers behind the C ABI (host side).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/spkv.h"
+
+namespace spkv {
+
+cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const void* W1,
+                         const float* b1, const float* W2, const float* b2, float* u_out,
+                         uint8_t* z_out, cudaStream_t stream);
+bool score_supported(const spkv_params& p);
+
+cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
+                                 int src_kind, const void* K_src, const void* V_src,
+                                 const uint8_t* z, const int32_t* src_pos, int n_rows,
+                                 int src_batch_rows, cudaStream_t stream);
+
+cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                                 const int32_t* t_pos, const void* k_new, const void* v_new,
+                                 const uint8_t* z_new, int retire, cudaStream_t stream);
+
+cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const void* K_src,
+                              const void* V_src, const uint8_t* z_src, int gated_from,
+                              const int32_t* src_pos, int n_rows, int src_batch_rows,
+                              cudaStream_t stream);
+
+size_t decode_workspace_bytes(const spkv_params& p, int num_sms);
+cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                          const void* q, const int32_t* t_pos, void* o, float* lse,
+                          void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream);
+
+cudaError_t launch_prefill(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                           const void* q, const void* K_chunk, const void* V_chunk,
+                           int chunk_start, int chunk_len, void* o, float* lse,
+                           cudaStream_t stream);
+
+}  // namespace spkv

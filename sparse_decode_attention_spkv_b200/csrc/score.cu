@@ -1,0 +1,151 @@
+// score.cu -- a1: utility score and gate (Eqs. (1)-(2) of "Self-Pruned Key-Value
+// Attention", arXiv 2605.14037, §2.1), fused in one kernel:
+//   a = h W1^T + b1, x = GELU(a), l = x W2^T + b2, u = sigmoid(l), z = [u >= tau].
+//
+// Work split: a cluster of 8 CTAs owns a tile of 32 tokens; CTA rank r computes the
+// partial first-layer sums over its eighth of d_model (split-K, so that a handful
+// of decode tokens still spreads the W1 read over 8 SMs), the partials are summed
+// through distributed shared memory, and each rank finishes 4 of the 32 tokens
+// (bias, GELU, second layer in fp32, sigmoid, threshold).
+#include <cooperative_groups.h>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace cg = cooperative_groups;
+
+namespace spkv {
+namespace {
+
+constexpr int kTok = 32;     // tokens per cluster
+constexpr int kKS = 8;       // cluster size (split of d_model)
+constexpr int kKT = 32;      // K step staged in shared memory
+constexpr int kThreads = 256;
+constexpr int kMaxHid = 128;
+
+template <typename E>
+__global__ void __cluster_dims__(1, kKS, 1) __launch_bounds__(kThreads)
+    score_kernel(const typename E::T* __restrict__ h, int n_tok, int d_model,
+                 const typename E::T* __restrict__ W1, const float* __restrict__ b1,
+                 const float* __restrict__ W2, const float* __restrict__ b2, int hid, int hkv,
+                 float tau, float* __restrict__ u_out, uint8_t* __restrict__ z_out) {
+  using T = typename E::T;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x;
+  const int tok0 = blockIdx.x * kTok;
+
+  __shared__ float hs[kTok][kKT + 1];
+  __shared__ float ws[kMaxHid][kKT + 1];
+  __shared__ float part[kTok][kMaxHid];
+  __shared__ float xs[kTok / kKS][kMaxHid];
+
+  const int ty = tid >> 5;  // tokens ty*4 .. ty*4+3
+  const int tx = tid & 31;  // hidden units tx + 32*j
+  const int nj = (hid + 31) >> 5;
+  float acc[4][kMaxHid / 32];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < kMaxHid / 32; ++j) acc[i][j] = 0.f;
+
+  const int steps = d_model / kKT;
+  const int s_begin = rank * steps / kKS;
+  const int s_end = (rank + 1) * steps / kKS;
+  for (int s = s_begin; s < s_end; ++s) {
+    const int k0 = s * kKT;
+    for (int e = tid; e < kTok * kKT; e += kThreads) {
+      const int r = e / kKT, c = e % kKT;
+      const int tok = tok0 + r;
+      hs[r][c] = tok < n_tok ? to_f32(h[(size_t)tok * d_model + k0 + c]) : 0.f;
+    }
+    for (int e = tid; e < hid * kKT; e += kThreads) {
+      const int r = e / kKT, c = e % kKT;
+      ws[r][c] = to_f32(W1[(size_t)r * d_model + k0 + c]);
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < kKT; ++k) {
+      float hv[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) hv[i] = hs[ty * 4 + i][k];
+#pragma unroll
+      for (int j = 0; j < kMaxHid / 32; ++j) {
+        if (j < nj) {
+          const int unit = tx + 32 * j;
+          const float wv = unit < hid ? ws[unit][k] : 0.f;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) acc[i][j] = fmaf(hv[i], wv, acc[i][j]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < kMaxHid / 32; ++j) {
+      const int unit = tx + 32 * j;
+      if (j < nj && unit < hid) part[ty * 4 + i][unit] = acc[i][j];
+    }
+  cluster.sync();
+
+  // Rank r finishes tokens r*4 .. r*4+3 of the tile.
+  constexpr int kMine = kTok / kKS;
+  for (int e = tid; e < kMine * hid; e += kThreads) {
+    const int r = e / hid, unit = e % hid;
+    const int row = rank * kMine + r;
+    float a = 0.f;
+#pragma unroll
+    for (int q = 0; q < kKS; ++q) {
+      const float* remote = cluster.map_shared_rank(&part[0][0], q);
+      a += remote[row * kMaxHid + unit];
+    }
+    a += b1[unit];
+    xs[r][unit] = 0.5f * a * (1.f + erff(a * 0.70710678118654752440f));
+  }
+  __syncthreads();
+
+  // Second layer: one warp per (token, key head) pair, lanes over hidden units.
+  const int warp = tid >> 5, lane = tid & 31;
+  for (int pair = warp; pair < kMine * hkv; pair += kThreads / 32) {
+    const int r = pair / hkv, kh = pair % hkv;
+    const int tok = tok0 + rank * kMine + r;
+    float sum = 0.f;
+    for (int unit = lane; unit < hid; unit += 32) sum = fmaf(xs[r][unit], W2[kh * hid + unit], sum);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+    if (lane == 0 && tok < n_tok) {
+      const float logit = sum + b2[kh];
+      const float u = 1.f / (1.f + expf(-logit));
+      if (u_out) u_out[(size_t)tok * hkv + kh] = u;
+      z_out[(size_t)tok * hkv + kh] = (u >= tau) ? 1 : 0;
+    }
+  }
+  cluster.sync();  // keep this CTA's partials alive until every rank has read them
+}
+
+}  // namespace
+
+cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const void* W1,
+                         const float* b1, const float* W2, const float* b2, float* u_out,
+                         uint8_t* z_out, cudaStream_t stream) {
+  dim3 grid((n_tok + kTok - 1) / kTok, kKS);
+  if (p.dtype == SPKV_BF16) {
+    score_kernel<BF16><<<grid, kThreads, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(h), n_tok, p.d_model,
+        static_cast<const __nv_bfloat16*>(W1), b1, W2, b2, p.hid, p.Hkv, p.tau, u_out, z_out);
+  } else {
+    score_kernel<F32><<<grid, kThreads, 0, stream>>>(
+        static_cast<const float*>(h), n_tok, p.d_model, static_cast<const float*>(W1), b1, W2,
+        b2, p.hid, p.Hkv, p.tau, u_out, z_out);
+  }
+  return cudaGetLastError();
+}
+
+bool score_supported(const spkv_params& p) {
+  return p.hid >= 1 && p.hid <= kMaxHid && p.d_model % kKT == 0 && p.Hkv <= 64;
+}
+
+}  // namespace spkv

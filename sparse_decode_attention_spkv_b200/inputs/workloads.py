@@ -150,7 +150,7 @@ WORKLOADS = {
                      keep="fixed25"),
     "decode32k": Workload("decode32k", 1, B=8, Hq=32, Hkv=8, head_dim=128, d_model=4096, hid=128,
                           window=128, tau=0.5, dtype="bf16", layers=32, ctx=[32768] * 8,
-                          decode_steps=64, keep="u05_50"),
+                          decode_steps=256, keep="u05_50"),
     "prefill16k": Workload("prefill16k", 2, B=1, Hq=32, Hkv=8, head_dim=128, d_model=4096,
                            hid=128, window=128, tau=0.5, dtype="bf16", layers=1, ctx=[16384],
                            decode_steps=0, chunk=4096, rope_base=1e4, keep="fixed20"),

@@ -1,0 +1,144 @@
+"""Schedules of the SP-KV hot path, driven through the C ABI.
+
+A ``Layer`` holds one attention layer's utility-perceptron weights, gated cache,
+window ring and decode workspace on the device.  The functions below sequence the
+library calls for the three schedules the workloads use:
+
+* chunked prefill, compacting each chunk right after scoring it (the chunk's
+  gated rows are in the cache before its attention runs; queries only use cache
+  rows that have left their window);
+* per-token decode: score the new token, retire the token leaving the window into
+  the cache if gated in, store the new token in the ring, attend;
+* buffered decode: tokens go to the ring ungated; every ``bulk`` steps the
+  buffered hidden states are scored together and their gated rows compacted from
+  the ring, before the oldest of them leaves the window.
+
+Every step runs in the library's kernels; this module only allocates buffers and
+orders calls.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+from . import spkv as S
+
+
+@dataclass
+class Layer:
+    p: S.spkv_params
+    W1: torch.Tensor
+    b1: torch.Tensor
+    W2: torch.Tensor
+    b2: torch.Tensor
+    cache: S.Cache
+    ring: S.Ring
+    ws: torch.Tensor
+
+    @staticmethod
+    def create(p: S.spkv_params, W1, b1, W2, b2, num_pages: int, max_pages_per_head: int,
+               device="cuda") -> "Layer":
+        cache = S.Cache.allocate(p, num_pages, max_pages_per_head, device)
+        ring = S.Ring.allocate(p, device)
+        ws = S.alloc_decode_workspace(p, cache, device)
+        layer = Layer(p, W1, b1, W2, b2, cache, ring, ws)
+        S.spkv_cache_reset(p, cache, ring)
+        return layer
+
+    @property
+    def dtype(self) -> torch.dtype:
+        return S.torch_dtype(self.p.dtype)
+
+
+def pages_for(rows_per_head, window: int = 0, slack: int = 2) -> int:
+    """Pages a head needs to hold ``rows_per_head`` rows (plus slack)."""
+    return (int(rows_per_head) + S.PAGE_ROWS - 1) // S.PAGE_ROWS + slack
+
+
+def score(layer: Layer, h: torch.Tensor, n_tok: int, u: Optional[torch.Tensor] = None):
+    """a1: u, z for n_tok tokens of h [n_tok][d_model]."""
+    dev = h.device
+    z = torch.empty((n_tok, layer.p.Hkv), dtype=torch.uint8, device=dev)
+    if u is None:
+        u = torch.empty((n_tok, layer.p.Hkv), dtype=torch.float32, device=dev)
+    S.spkv_score(layer.p, h, n_tok, layer.W1, layer.b1, layer.W2, layer.b2, u, z)
+    return u, z
+
+
+def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optional[int] = None,
+                  src_pos: Optional[torch.Tensor] = None):
+    """One chunk of chunked prefill for all batch rows.
+
+    h [B][Tc][d_model], q [B][Tc][Hq][d], k, v [B][Tc][Hkv][d] (contiguous).  The
+    first ``n_compact`` rows (default: all) are compacted after scoring; the rest
+    stay only in the ring with their gates, to be retired by per-token decode.
+    Returns (o [B][Tc][Hq][d], lse [B][Tc][Hq], u, z [B][Tc][Hkv])."""
+    p = layer.p
+    B, Tc = h.shape[0], h.shape[1]
+    dev = h.device
+    if n_compact is None:
+        n_compact = Tc
+    if src_pos is None:
+        src_pos = torch.full((B,), chunk_start, dtype=torch.int32, device=dev)
+    u, z = score(layer, h, B * Tc)
+    if n_compact > 0:
+        S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, k, v, z, src_pos, n_compact, Tc)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Tc, p.Hq), dtype=torch.float32, device=dev)
+    S.spkv_prefill_attn(p, layer.cache, layer.ring, q, k, v, chunk_start, Tc, o, lse)
+    S.spkv_ring_write(p, layer.ring, k, v, z, n_compact, src_pos, Tc, Tc)
+    return o, lse, u.view(B, Tc, p.Hkv), z.view(B, Tc, p.Hkv)
+
+
+def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: bool = True,
+                o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+    """One decode step for every batch row at positions t_pos [B] (device int32).
+
+    h_t [B][d_model] (ignored when retire is False: buffered scoring), q_t [B][Hq][d],
+    k_t, v_t [B][Hkv][d].  Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
+    p = layer.p
+    z_t = None
+    if retire:
+        _, z_t = score(layer, h_t, p.B)
+    S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, z_t, retire)
+    if o is None:
+        o = torch.empty_like(q_t)
+    if lse is None:
+        lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
+    S.spkv_decode_attn(p, layer.cache, layer.ring, q_t, t_pos, o, lse, layer.ws)
+    return o, lse, z_t
+
+
+def bulk_compact(layer: Layer, h_buf: torch.Tensor, start_pos: torch.Tensor):
+    """Buffered decode: score the ``n`` buffered tokens h_buf [B][n][d_model] whose
+    positions start at start_pos [B] and compact their gated rows from the ring."""
+    p = layer.p
+    B, n = h_buf.shape[0], h_buf.shape[1]
+    u, z = score(layer, h_buf, B * n)
+    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_RING, None, None, z, start_pos, n, n)
+    return u.view(B, n, p.Hkv), z.view(B, n, p.Hkv)
+
+
+def cache_lists(layer: Layer):
+    """Host copy of every head's cache positions, as a list of int32 arrays."""
+    count = layer.cache.count.cpu().numpy()
+    table = layer.cache.page_table.cpu().numpy()
+    pos = layer.cache.pos_pool.cpu().numpy()
+    out = []
+    for bh, n in enumerate(count):
+        rows = [pos[table[bh, i // S.PAGE_ROWS], i % S.PAGE_ROWS] for i in range(int(n))]
+        out.append(torch.tensor(rows, dtype=torch.int32).numpy())
+    return out
+
+
+def cache_rows_kv(layer: Layer, bh: int):
+    """Host copies (K, V) [count][d] of one head's cache rows, in cache order."""
+    n = int(layer.cache.count[bh].item())
+    table = layer.cache.page_table[bh].cpu()
+    idx = torch.arange(n)
+    pages = table[idx // S.PAGE_ROWS].long()
+    K = layer.cache.K_pool.cpu()[pages, idx % S.PAGE_ROWS]
+    V = layer.cache.V_pool.cpu()[pages, idx % S.PAGE_ROWS]
+    return K, V

@@ -1,0 +1,217 @@
+"""Thin ctypes binding of ``libspkv.so`` (C ABI in include/spkv.h).
+
+Argument marshalling only: every step of the SP-KV path runs in the CUDA kernels
+of the library.  PyTorch tensors provide device memory, their ``data_ptr()`` is
+passed through, and the stream is the caller's current torch CUDA stream unless
+one is given.  There is no fallback: if the library is missing, importing this
+module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspkv.so")
+if not os.path.exists(_LIB_PATH):
+    raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                      "`python -m sparse_decode_attention_spkv_b200.build`")
+lib = ctypes.CDLL(_LIB_PATH)
+
+OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT = range(6)
+F32, BF16 = 0, 1
+SRC_CHUNK, SRC_RING = 0, 1
+FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT = 1, 2, 4
+PAGE_ROWS = 64
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int
+
+
+class spkv_params(ctypes.Structure):
+    _fields_ = [("B", _i32), ("Hq", _i32), ("Hkv", _i32), ("head_dim", _i32), ("d_model", _i32),
+                ("hid", _i32), ("window", _i32), ("tau", ctypes.c_float), ("dtype", _i32)]
+
+
+class spkv_cache(ctypes.Structure):
+    _fields_ = [("K_pool", _vp), ("V_pool", _vp), ("pos_pool", _vp), ("page_table", _vp),
+                ("count", _vp), ("count_prev", _vp), ("pool_top", _vp), ("err_flag", _vp),
+                ("num_pages", _i32), ("page_rows", _i32), ("max_pages_per_head", _i32)]
+
+
+class spkv_ring(ctypes.Structure):
+    _fields_ = [("K_win", _vp), ("V_win", _vp), ("z_win", _vp)]
+
+
+_P = ctypes.POINTER
+_sigs = {
+    "spkv_status_str": (ctypes.c_char_p, [_i32]),
+    "spkv_version": (_i32, []),
+    "spkv_cache_reset": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp]),
+    "spkv_cache_check": (_i32, [_P(spkv_cache), _vp, _P(ctypes.c_uint32)]),
+    "spkv_score": (_i32, [_P(spkv_params), _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "spkv_write_compact": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _i32, _vp, _vp,
+                                  _vp, _vp, _i32, _i32, _vp]),
+    "spkv_decode_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp,
+                                  _vp, _i32, _vp]),
+    "spkv_ring_write": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _i32, _vp, _i32, _i32,
+                                _vp]),
+    "spkv_decode_workspace_bytes": (ctypes.c_size_t, [_P(spkv_params), _P(spkv_cache)]),
+    "spkv_decode_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _vp,
+                                _vp, ctypes.c_size_t, _vp]),
+    "spkv_prefill_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _i32,
+                                 _i32, _vp, _vp, _vp]),
+}
+for _name, (_res, _args) in _sigs.items():
+    _fn = getattr(lib, _name)
+    _fn.restype = _res
+    _fn.argtypes = _args
+
+
+class SpkvError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        super().__init__(f"{fn}: {status_str(status)} ({status})")
+        self.status = status
+
+
+def status_str(status: int) -> str:
+    return lib.spkv_status_str(status).decode()
+
+
+def _check(fn: str, status: int) -> int:
+    if status != OK:
+        raise SpkvError(fn, status)
+    return status
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def torch_dtype(dtype: int) -> torch.dtype:
+    return torch.bfloat16 if dtype == BF16 else torch.float32
+
+
+def make_params(B, Hq, Hkv, head_dim, d_model, hid, window, tau, dtype) -> spkv_params:
+    return spkv_params(B, Hq, Hkv, head_dim, d_model, hid, window, float(tau), dtype)
+
+
+@dataclass
+class Cache:
+    """Device tensors of one layer's gated cache and the ctypes view of them."""
+    K_pool: torch.Tensor
+    V_pool: torch.Tensor
+    pos_pool: torch.Tensor
+    page_table: torch.Tensor
+    count: torch.Tensor
+    count_prev: torch.Tensor
+    pool_top: torch.Tensor
+    err_flag: torch.Tensor
+    c: spkv_cache
+
+    @staticmethod
+    def allocate(p: spkv_params, num_pages: int, max_pages_per_head: int, device="cuda") -> "Cache":
+        dt = torch_dtype(p.dtype)
+        heads = p.B * p.Hkv
+        K = torch.empty((num_pages, PAGE_ROWS, p.head_dim), dtype=dt, device=device)
+        V = torch.empty_like(K)
+        pos = torch.empty((num_pages, PAGE_ROWS), dtype=torch.int32, device=device)
+        table = torch.full((heads, max_pages_per_head), -1, dtype=torch.int32, device=device)
+        count = torch.zeros(heads, dtype=torch.int32, device=device)
+        count_prev = torch.zeros(heads, dtype=torch.int32, device=device)
+        top = torch.zeros(1, dtype=torch.int32, device=device)
+        err = torch.zeros(1, dtype=torch.int32, device=device)
+        c = spkv_cache(K.data_ptr(), V.data_ptr(), pos.data_ptr(), table.data_ptr(),
+                       count.data_ptr(), count_prev.data_ptr(), top.data_ptr(), err.data_ptr(),
+                       num_pages, PAGE_ROWS, max_pages_per_head)
+        return Cache(K, V, pos, table, count, count_prev, top, err, c)
+
+
+@dataclass
+class Ring:
+    K_win: torch.Tensor
+    V_win: torch.Tensor
+    z_win: torch.Tensor
+    r: spkv_ring
+
+    @staticmethod
+    def allocate(p: spkv_params, device="cuda") -> "Ring":
+        dt = torch_dtype(p.dtype)
+        K = torch.zeros((p.B, p.Hkv, p.window, p.head_dim), dtype=dt, device=device)
+        V = torch.zeros_like(K)
+        z = torch.zeros((p.B, p.window, p.Hkv), dtype=torch.uint8, device=device)
+        return Ring(K, V, z, spkv_ring(K.data_ptr(), V.data_ptr(), z.data_ptr()))
+
+
+# ---- entry points (same names as the C ABI) -------------------------------------------
+
+def spkv_cache_reset(p, cache: Cache, ring: Optional[Ring] = None, stream=None):
+    return _check("spkv_cache_reset", lib.spkv_cache_reset(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r) if ring else None,
+        _stream(stream)))
+
+
+def spkv_cache_check(cache: Cache, stream=None):
+    flags = ctypes.c_uint32(0)
+    status = lib.spkv_cache_check(ctypes.byref(cache.c), _stream(stream), ctypes.byref(flags))
+    return status, int(flags.value)
+
+
+def spkv_score(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream=None):
+    return _check("spkv_score", lib.spkv_score(
+        ctypes.byref(p), _ptr(h), n_tok, _ptr(W1), _ptr(b1), _ptr(W2), _ptr(b2), _ptr(u_out),
+        _ptr(z_out), _stream(stream)))
+
+
+def spkv_write_compact(p, cache: Cache, ring: Optional[Ring], src_kind, K_src, V_src, z, src_pos,
+                       n_rows, src_batch_rows, stream=None):
+    return _check("spkv_write_compact", lib.spkv_write_compact(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r) if ring else None, src_kind,
+        _ptr(K_src), _ptr(V_src), _ptr(z), _ptr(src_pos), n_rows, src_batch_rows, _stream(stream)))
+
+
+def spkv_decode_append(p, cache: Cache, ring: Ring, t_pos, k_new, v_new, z_new, retire,
+                       stream=None):
+    return _check("spkv_decode_append", lib.spkv_decode_append(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(t_pos), _ptr(k_new),
+        _ptr(v_new), _ptr(z_new), int(retire), _stream(stream)))
+
+
+def spkv_ring_write(p, ring: Ring, K_src, V_src, z_src, gated_from, src_pos, n_rows,
+                    src_batch_rows, stream=None):
+    return _check("spkv_ring_write", lib.spkv_ring_write(
+        ctypes.byref(p), ctypes.byref(ring.r), _ptr(K_src), _ptr(V_src), _ptr(z_src),
+        int(gated_from), _ptr(src_pos), n_rows, src_batch_rows, _stream(stream)))
+
+
+def spkv_decode_workspace_bytes(p, cache: Cache) -> int:
+    return int(lib.spkv_decode_workspace_bytes(ctypes.byref(p), ctypes.byref(cache.c)))
+
+
+def alloc_decode_workspace(p, cache: Cache, device="cuda") -> torch.Tensor:
+    n = spkv_decode_workspace_bytes(p, cache)
+    if n == 0:
+        raise SpkvError("spkv_decode_workspace_bytes", ERR_ARG)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def spkv_decode_attn(p, cache: Cache, ring: Ring, q, t_pos, o, lse, workspace, stream=None):
+    return _check("spkv_decode_attn", lib.spkv_decode_attn(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
+        _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def spkv_prefill_attn(p, cache: Cache, ring: Ring, q, K_chunk, V_chunk, chunk_start, chunk_len,
+                      o, lse, stream=None):
+    return _check("spkv_prefill_attn", lib.spkv_prefill_attn(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(K_chunk),
+        _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _stream(stream)))

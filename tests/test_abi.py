@@ -1,0 +1,76 @@
+"""The C-ABI library loads and exports every entry point the header declares;
+host-side argument validation rejects bad calls before touching the GPU."""
+import ctypes
+import glob
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+LIB = os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "libspkv.so")
+
+
+def _declared():
+    names = []
+    for hdr in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(hdr).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^[A-Za-z_][\w \*]*?\b(spkv_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_hot_path():
+    names = _declared()
+    for required in ["spkv_score", "spkv_write_compact", "spkv_decode_attn", "spkv_prefill_attn",
+                     "spkv_decode_append", "spkv_ring_write"]:
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol():
+    assert os.path.exists(LIB), "build the library first"
+    lib = ctypes.CDLL(LIB)
+    missing = [n for n in _declared() if not hasattr(lib, n)]
+    assert not missing, missing
+
+
+def test_argument_validation_without_gpu():
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    assert S.lib.spkv_version() >= 100
+    assert S.status_str(S.ERR_CAPACITY) == "cache capacity exhausted"
+    # NULL params, bad head_dim, bad group size, NaN threshold: rejected on the host
+    assert S.lib.spkv_score(None, None, 4, None, None, None, None, None, None, None) == S.ERR_ARG
+    bad = [S.make_params(1, 4, 2, 96, 256, 64, 128, 0.5, S.F32),
+           S.make_params(1, 6, 2, 64, 256, 64, 128, 0.5, S.F32),
+           S.make_params(1, 4, 2, 64, 256, 64, 128, float("nan"), S.F32),
+           S.make_params(1, 4, 2, 64, 256, 64, 0, 0.5, S.F32),
+           S.make_params(0, 4, 2, 64, 256, 64, 128, 0.5, S.BF16)]
+    for p in bad:
+        assert S.lib.spkv_score(ctypes.byref(p), None, 4, None, None, None, None, None, None,
+                                None) == S.ERR_ARG
+    good = S.make_params(1, 4, 2, 64, 256, 64, 128, 0.5, S.F32)
+    # zero tokens is a no-op that needs no pointers
+    assert S.lib.spkv_score(ctypes.byref(good), None, 0, None, None, None, None, None, None,
+                            None) == S.OK
+    # missing cache buffers
+    cache = S.spkv_cache()
+    ring = S.spkv_ring()
+    assert S.lib.spkv_decode_attn(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
+                                  None, None, None, None, None, 0, None) == S.ERR_ARG
+    assert S.lib.spkv_prefill_attn(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
+                                   None, None, None, 0, 16, None, None, None) == S.ERR_ARG
+    # misaligned pool pointer
+    cache = S.spkv_cache(8, 16, 16, 16, 16, 16, 16, 16, 4, 64, 4)
+    assert S.lib.spkv_cache_reset(ctypes.byref(good), ctypes.byref(cache), None, None) == S.ERR_ARG
+    # page_rows other than 64
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, 4, 32, 4)
+    assert S.lib.spkv_cache_reset(ctypes.byref(good), ctypes.byref(cache), None, None) == S.ERR_ARG
+    # ring compaction longer than the window, negative gated_from
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, 4, 64, 4)
+    ring = S.spkv_ring(16, 16, 16)
+    assert S.lib.spkv_write_compact(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
+                                    S.SRC_RING, None, None, 16, 16, 129, 129, None) == S.ERR_ARG
+    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, 16, -1, 16, 4, 4,
+                                 None) == S.ERR_ARG
+    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, None, 0, 16, 4, 4,
+                                 None) == S.ERR_ARG

@@ -1,0 +1,259 @@
+"""CUDA path vs the oracle, element by element, at sizes the oracle finishes in
+seconds that still span several tiles and a ragged tail (GPU required)."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import spkv_oracle as O
+from sparse_decode_attention_spkv_b200.inputs import workloads as W
+from tests import cases as C
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import spkv as S
+
+
+def _params(wl):
+    return S.make_params(wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau,
+                         S.BF16 if wl.dtype == "bf16" else S.F32)
+
+
+def _layer(wl, rows_per_head, layer=0):
+    W1, b1, W2, b2 = C.weights(wl, layer)
+    p = _params(wl)
+    mp = R.pages_for(rows_per_head)
+    return R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                          num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp), (W1, b1, W2, b2)
+
+
+def _rows(wl, T, layer=0):
+    """Host h, q, k, v [B][T][...] for positions 0..T-1."""
+    hs, qs, ks, vs = [], [], [], []
+    for b in range(wl.B):
+        h, q, k, v = C.host_rows(wl, layer, b, np.arange(T))
+        hs.append(h); qs.append(q); ks.append(k); vs.append(v)
+    return np.stack(hs), np.stack(qs), np.stack(ks), np.stack(vs)
+
+
+SCORE_CASES = {
+    "tiny_f32_528": (W.small_case("tiny", ctx=[528], decode_steps=0), 528),
+    "llama_bf16_300": (W.small_case("decode32k", B=1, ctx=[300], decode_steps=0, layers=1), 300),
+    "llama_bf16_1": (W.small_case("decode32k", B=1, ctx=[1], decode_steps=0, layers=1), 1),
+    "llama_bf16_33": (W.small_case("decode32k", B=1, ctx=[33], decode_steps=0, layers=1), 33),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SCORE_CASES))
+def test_score_matches_oracle(name):
+    wl, n = SCORE_CASES[name]
+    layer, (W1, b1, W2, b2) = _layer(wl, 64)
+    h = wl.h_rows(0, 0, np.arange(n))
+    u, z = R.score(layer, C.dev(h, wl.dtype), n)
+    u_ref, z_ref = C.oracle_gates(h, W1, b1, W2, b2, wl.tau)
+    C.check_gates(C.to_np(u), z.cpu().numpy(), u_ref, z_ref, wl.tau)
+
+
+def test_score_empty_is_noop():
+    wl, _ = SCORE_CASES["tiny_f32_528"]
+    layer, _ = _layer(wl, 64)
+    z = torch.full((4, wl.Hkv), 7, dtype=torch.uint8, device="cuda")
+    S.spkv_score(layer.p, C.dev(np.zeros((1, wl.d_model)), wl.dtype), 0, layer.W1, layer.b1,
+                 layer.W2, layer.b2, None, z)
+    assert int(z.min()) == 7
+
+
+def _lists_equal(layer, z_ref, upto, positions_offset=0):
+    lists = R.cache_lists(layer)
+    B, _, Hkv = z_ref.shape
+    for b in range(B):
+        for kh in range(Hkv):
+            want = O.cache_rows(z_ref[b, :, kh], upto) + positions_offset
+            got = lists[b * Hkv + kh]
+            assert np.array_equal(got, want), f"cache list of head ({b},{kh}) differs"
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_compact_chunks_and_ring(dtype):
+    """Chunk compaction over several calls (ragged sizes), then ring compaction:
+    index lists and stored rows are exact."""
+    wl = W.small_case("decode32k", cid=40, B=2, Hq=8, Hkv=2, d_model=128, hid=64, dtype=dtype,
+                      ctx=[3000], decode_steps=0, layers=1, keep="fixed25")
+    T = 2500
+    layer, (W1, b1, W2, b2) = _layer(wl, T)
+    h, q, k, v = _rows(wl, T)
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    zd = torch.from_numpy(z_ref).cuda()
+    kd, vd = C.dev(k, dtype), C.dev(v, dtype)
+    # chunks [0,1000), [1000,1777), [1777,2372) from the chunk tensors
+    for c0, c1 in [(0, 1000), (1000, 1777), (1777, 2372)]:
+        src_pos = torch.full((wl.B,), c0, dtype=torch.int32, device="cuda")
+        S.spkv_write_compact(layer.p, layer.cache, layer.ring, S.SRC_CHUNK,
+                             kd[:, c0:].contiguous(), vd[:, c0:].contiguous(),
+                             zd[:, c0:].contiguous(), src_pos, c1 - c0, T - c0)
+    # the last 128 rows through the ring
+    w = wl.window
+    src_pos = torch.full((wl.B,), 2372, dtype=torch.int32, device="cuda")
+    S.spkv_ring_write(layer.p, layer.ring, kd[:, 2372:].contiguous(), vd[:, 2372:].contiguous(),
+                      zd[:, 2372:].contiguous(), 0, src_pos, T - 2372, T - 2372)
+    S.spkv_write_compact(layer.p, layer.cache, layer.ring, S.SRC_RING, None, None,
+                         zd[:, 2372:].contiguous(), src_pos, T - 2372, T - 2372)
+    assert T - 2372 == w
+    status, flags = S.spkv_cache_check(layer.cache)
+    assert status == S.OK and flags == 0
+    _lists_equal(layer, z_ref, T)
+    for b in range(wl.B):
+        for kh in range(wl.Hkv):
+            rows = O.cache_rows(z_ref[b, :, kh], T)
+            K, V = R.cache_rows_kv(layer, b * wl.Hkv + kh)
+            assert np.array_equal(K.float().numpy(), k[b, rows, kh])
+            assert np.array_equal(V.float().numpy(), v[b, rows, kh])
+
+
+def test_compact_capacity_is_flagged():
+    wl = W.small_case("decode32k", cid=41, B=1, Hq=4, Hkv=1, d_model=128, hid=32, dtype="bf16",
+                      ctx=[1000], decode_steps=0, layers=1, keep="fixed25")
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    layer = R.Layer.create(p, C.dev(W1, "bf16"), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                           num_pages=2, max_pages_per_head=8)
+    z = torch.ones((1, 1000, 1), dtype=torch.uint8, device="cuda")
+    kv = torch.randn((1, 1000, 1, 128), device="cuda").to(torch.bfloat16)
+    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, kv, kv, z,
+                         torch.zeros(1, dtype=torch.int32, device="cuda"), 1000, 1000)
+    status, flags = S.spkv_cache_check(layer.cache)
+    assert status == S.ERR_CAPACITY and flags & S.FLAG_POOL_FULL
+    assert int(layer.cache.count[0]) == 2 * S.PAGE_ROWS
+    assert np.array_equal(R.cache_lists(layer)[0], np.arange(128))
+
+
+PREFILL_CASES = {
+    # name: (workload, T, chunk)
+    "tiny_f32_one_chunk": (W.small_case("tiny", ctx=[512], decode_steps=0), 512, 512),
+    "bf16_g4_chunks": (W.small_case("decode32k", cid=42, B=2, Hq=8, Hkv=2, d_model=256, hid=64,
+                                    ctx=[1000], decode_steps=0, layers=1, keep="fixed20"), 1000, 256),
+    "bf16_g1_d64": (W.small_case("decode32k", cid=43, B=1, Hq=2, Hkv=2, head_dim=64, d_model=128,
+                                 hid=32, ctx=[700], decode_steps=0, layers=1, keep="fixed25"), 700, 300),
+    "f32_g8_d128": (W.small_case("tiny", cid=44, B=1, Hq=8, Hkv=1, head_dim=128, ctx=[400],
+                                 decode_steps=0), 400, 160),
+}
+
+
+@pytest.mark.parametrize("name", sorted(PREFILL_CASES))
+def test_chunked_prefill_matches_oracle(name):
+    wl, T, chunk = PREFILL_CASES[name]
+    layer, (W1, b1, W2, b2) = _layer(wl, T)
+    h, q, k, v = _rows(wl, T)
+    u_ref, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    u_ref = u_ref.reshape(wl.B, T, wl.Hkv)
+    outs, zs, us = [], [], []
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        o, lse, u, z = R.prefill_chunk(layer, C.dev(h[:, c0:c1], wl.dtype),
+                                       C.dev(q[:, c0:c1], wl.dtype), C.dev(k[:, c0:c1], wl.dtype),
+                                       C.dev(v[:, c0:c1], wl.dtype), c0)
+        outs.append(C.to_np(o)); zs.append(z.cpu().numpy()); us.append(C.to_np(u))
+    o_gpu = np.concatenate(outs, axis=1)
+    C.check_gates(np.concatenate(us, 1), np.concatenate(zs, 1), u_ref, z_ref, wl.tau)
+    for b in range(wl.B):
+        o_ref, _ = O.gated_attention(q[b], k[b], v[b], z_ref[b], wl.window, np.arange(T))
+        C.check_attn(o_gpu[b], o_ref, wl.dtype, f"{name} b={b}")
+    _lists_equal(layer, z_ref, T)
+
+
+def _decode_run(wl, T0, steps, layer_rows, retire=True, bulk=0):
+    """Prefill T0 tokens (per-token-ready state when retire) then decode `steps`
+    tokens; returns gpu outputs [steps][B][Hq][d], z per step and the layer."""
+    layer, (W1, b1, W2, b2) = _layer(wl, layer_rows)
+    T = T0 + steps
+    h, q, k, v = _rows(wl, T)
+    w = wl.window
+    chunk = 512
+    for c0 in range(0, T0, chunk):
+        c1 = min(T0, c0 + chunk)
+        n_compact = max(0, min(c1, T0 - w) - c0) if retire else c1 - c0
+        R.prefill_chunk(layer, C.dev(h[:, c0:c1], wl.dtype), C.dev(q[:, c0:c1], wl.dtype),
+                        C.dev(k[:, c0:c1], wl.dtype), C.dev(v[:, c0:c1], wl.dtype), c0,
+                        n_compact=n_compact)
+    outs, zs = [], []
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        o, lse, z = R.decode_step(layer, t_pos, C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype),
+                                  C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype), retire=retire)
+        outs.append(C.to_np(o))
+        zs.append(None if z is None else z.cpu().numpy())
+        if bulk and (i + 1) % bulk == 0:
+            start = torch.full((wl.B,), t - bulk + 1, dtype=torch.int32, device="cuda")
+            R.bulk_compact(layer, C.dev(h[:, t - bulk + 1:t + 1], wl.dtype), start)
+    return layer, outs, zs, (h, q, k, v), (W1, b1, W2, b2)
+
+
+DECODE_CASES = {
+    "tiny_f32_c0": W.small_case("tiny"),
+    "bf16_g4": W.small_case("decode32k", cid=45, B=3, Hq=8, Hkv=2, d_model=256, hid=64,
+                            ctx=[2000], decode_steps=8, layers=1, keep="u05_50"),
+    "bf16_g8_d64": W.small_case("decode32k", cid=46, B=2, Hq=8, Hkv=1, head_dim=64, d_model=128,
+                                hid=32, ctx=[900], decode_steps=6, layers=1, keep="fixed25"),
+    "bf16_g2": W.small_case("decode32k", cid=47, B=2, Hq=4, Hkv=2, d_model=128, hid=32,
+                            ctx=[1500], decode_steps=6, layers=1, keep="fixed25"),
+    "f32_g1_d128": W.small_case("tiny", cid=48, B=2, Hq=2, Hkv=2, head_dim=128, ctx=[700],
+                                decode_steps=5),
+    "bf16_short_ctx": W.small_case("decode32k", cid=49, B=2, Hq=8, Hkv=2, d_model=128, hid=32,
+                                   ctx=[40], decode_steps=100, layers=1, keep="fixed25"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(DECODE_CASES))
+def test_per_token_decode_matches_oracle(name):
+    wl = DECODE_CASES[name]
+    T0, steps = wl.ctx[0], wl.decode_steps
+    T = T0 + steps
+    layer, outs, zs, (h, q, k, v), (W1, b1, W2, b2) = _decode_run(wl, T0, steps, T)
+    u_ref, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    u_ref = u_ref.reshape(wl.B, T, wl.Hkv)
+    for i in range(steps):
+        t = T0 + i
+        near = np.abs(u_ref[:, t] - wl.tau) < C.EXCLUDE
+        assert np.all((zs[i] == z_ref[:, t]) | near), f"gate of token {t}"
+        for b in range(wl.B):
+            o_ref, _ = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
+                                         z_ref[b, :t + 1], wl.window, [t])
+            C.check_attn(outs[i][b], o_ref[0], wl.dtype, f"{name} step {i} b={b}")
+    # cache holds exactly the gated tokens that have left the window of the last query
+    _lists_equal(layer, z_ref, max(0, T - wl.window))
+
+
+def test_buffered_decode_matches_oracle():
+    """Buffered schedule: tokens enter the ring ungated; every 128 steps the buffer
+    is scored and compacted from the ring.  Same outputs as Eq. (3)-(4)."""
+    wl = W.small_case("decode32k", cid=50, B=2, Hq=8, Hkv=2, d_model=128, hid=32, ctx=[1000],
+                      decode_steps=256, layers=1, keep="fixed25")
+    T0, steps = 1000, 256
+    T = T0 + steps
+    layer, outs, _, (h, q, k, v), (W1, b1, W2, b2) = _decode_run(wl, T0, steps, T, retire=False,
+                                                                 bulk=128)
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    for i in list(range(0, steps, 17)) + [127, 128, 255]:
+        t = T0 + i
+        for b in range(wl.B):
+            o_ref, _ = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
+                                         z_ref[b, :t + 1], wl.window, [t])
+            C.check_attn(outs[i][b], o_ref[0], wl.dtype, f"bulk step {i} b={b}")
+    _lists_equal(layer, z_ref, T)
+
+
+def test_schedules_agree():
+    """Per-token and buffered schedules give the same decode outputs (the key set
+    of Eq. (4) does not depend on when a token was compacted)."""
+    wl = W.small_case("decode32k", cid=51, B=2, Hq=8, Hkv=2, d_model=128, hid=32, ctx=[700],
+                      decode_steps=128, layers=1, keep="fixed25")
+    _, a, _, _, _ = _decode_run(wl, 700, 128, 900, retire=True)
+    _, b, _, _, _ = _decode_run(wl, 700, 128, 900, retire=False, bulk=128)
+    for i in range(128):
+        C.check_attn(a[i], b[i], "bf16", f"step {i}")
