@@ -559,7 +559,8 @@ size_t decode_workspace_bytes(const spkv_params& p, int num_sms) {
   const size_t max_chunks = (size_t)num_sms * kUnitsPerCta + n_heads;
   const size_t ml_bytes = (max_chunks * G * 2 * 4 + 255) / 256 * 256;
   const size_t o_bytes = max_chunks * G * p.head_dim * 4;
-  return ctrl_bytes + ml_bytes + o_bytes;
+  const size_t tc = decode_tc_workspace_bytes(p, num_sms);
+  return ctrl_bytes + ml_bytes + o_bytes > tc ? ctrl_bytes + ml_bytes + o_bytes : tc;
 }
 
 cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
@@ -567,6 +568,8 @@ cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_
                           void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream) {
   if (p.B * p.Hkv > kMaxHeads) return cudaErrorInvalidValue;
   if (ws_bytes < decode_workspace_bytes(p, num_sms)) return cudaErrorInvalidValue;
+  if (decode_tc_supported(p))
+    return launch_decode_tc(p, c, ring, q, t_pos, o, lse, workspace, num_sms, stream);
   if (p.dtype == SPKV_BF16) {
     if (p.head_dim == 128) return dispatch_g<BF16, 128>(p, c, ring, q, t_pos, o, lse, workspace, num_sms, stream);
     if (p.head_dim == 64) return dispatch_g<BF16, 64>(p, c, ring, q, t_pos, o, lse, workspace, num_sms, stream);

@@ -29,10 +29,20 @@ cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const
                               cudaStream_t stream);
 
 size_t decode_workspace_bytes(const spkv_params& p, int num_sms);
+bool decode_tc_supported(const spkv_params& p);
+size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms);
+cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                             const void* q, const int32_t* t_pos, void* o, float* lse,
+                             void* workspace, int num_sms, cudaStream_t stream);
 cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                           const void* q, const int32_t* t_pos, void* o, float* lse,
                           void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream);
 
+bool prefill_tc_supported(const spkv_params& p, const spkv_cache& c, int chunk_start, int chunk_len);
+cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                              const void* q, const void* K_chunk, const void* V_chunk,
+                              int chunk_start, int chunk_len, void* o, float* lse,
+                              cudaStream_t stream);
 cudaError_t launch_prefill(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                            const void* q, const void* K_chunk, const void* V_chunk,
                            int chunk_start, int chunk_len, void* o, float* lse,

@@ -1,0 +1,507 @@
+// prefill_tc.cu -- a6 on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
+//
+// "Self-Pruned Key-Value Attention" (arXiv 2605.14037), §2.1, Eqs. (3)-(4), for a
+// chunk of queries.  One CTA owns 128 consecutive query positions of two query
+// heads of one key head.  Its key set is, in 64-key blocks:
+//   * the compacted cache pages holding rows with pos <= t_last - w (gated-in keys
+//     of Eq. (4)); pages whose rows all have pos <= t_first - w need no mask, the
+//     last one or two are masked per query (pos <= t - w), and pages beyond are
+//     never touched: the dead key blocks of the causal mask are simply absent;
+//   * the causal window band, positions t_first-128 .. t_first+127 (four blocks,
+//     from the ring for positions before the chunk, else from the chunk's K/V),
+//     masked per query by 0 <= t - s < 128.
+// Both contractions are dense tensor-core tiles: S = Q K^T (M=128 queries, N=64
+// keys, K=128) and O += P V (M=128, N=128, K=64 keys), bf16 operands, fp32
+// accumulators in TMEM.  P is written back into TMEM over S and fed to the second
+// MMA as its A operand.
+//
+// Warp roles (384 threads):
+//   warp 0      TMA producer: Q once, then K/V (+ positions) per block, 3 stages;
+//   warp 1      TMEM allocation and the single MMA-issuing thread;
+//   warps 4-7   softmax of head 0 (one query row per thread, TMEM lanes 0..127);
+//   warps 8-11  softmax of head 1.
+// Softmax runs in the log2 domain; the running max is raised only when a score
+// exceeds it by more than 8, and only then is the O row in TMEM rescaled.
+// Every mbarrier wait is bounded (a stuck wait raises SPKV_FLAG_TIMEOUT).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace spkv {
+namespace {
+
+constexpr int kQT = 128;          // queries per CTA and head
+constexpr int kKB = 64;           // keys per block
+constexpr int kHD = 128;          // head_dim
+constexpr int kWin = 128;         // window of this path
+constexpr int kStg = 3;
+constexpr int kThr = 384;
+constexpr int kMaxPages = 4096;   // pages per key head scanned in shared memory
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kSlack = 8.f;
+
+constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS0 = 256, kColS1 = 320;
+
+struct __align__(1024) TcSmem {
+  char q[2][2][kQT * 128];        // [head][d half] 128 rows x 128 B, 128B-swizzled
+  char k[kStg][2][kKB * 128];     // [stage][d half] 64 rows x 128 B
+  char v[kStg][2][kKB * 128];
+  int pos[kStg][kKB];
+  int first_pos[kMaxPages];
+  uint64_t q_full;
+  uint64_t kv_full[kStg];
+  uint64_t kv_empty[kStg];
+  uint64_t s_ready[2];
+  uint64_t p_ready[2];
+  uint64_t o_ready[2];
+  uint32_t tmem_base;
+  int cnt[4];
+};
+
+__device__ __forceinline__ uint64_t smem_desc(const void* p, uint32_t lbo, uint32_t sbo) {
+  const uint32_t a = smem_u32(p);
+  return (uint64_t)((a & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+         ((uint64_t)(sbo >> 4) << 32) | (1ull << 46) | (2ull << 61);
+}
+
+__device__ __forceinline__ void mma_ss(uint32_t d, uint64_t a, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_ts(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t idesc,
+                                       uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),
+      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                   smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t* r) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,"
+      "%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+      "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
+      "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
+      "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
+      "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+__device__ __forceinline__ void tma_2d(void* dst, const CUtensorMap* map, int c0, int c1, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* map, int c0, int c1, int c2,
+                                       int c3, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+struct Blocks {
+  int nc;      // cache blocks (pages 0..nc-1)
+  int nfull;   // rows visible to every query of the tile
+  int nrows;   // cache rows (count)
+  int wfirst;  // position of the first window block
+  int nw;      // window blocks
+};
+
+__global__ void __launch_bounds__(kThr, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
+                      const __grid_constant__ CUtensorMap tm_kc,
+                      const __grid_constant__ CUtensorMap tm_vc,
+                      const __grid_constant__ CUtensorMap tm_kp,
+                      const __grid_constant__ CUtensorMap tm_vp,
+                      const __grid_constant__ CUtensorMap tm_kr,
+                      const __grid_constant__ CUtensorMap tm_vr, CacheView cache,
+                      __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
+                      int chunk_start, int chunk_len, int hkv, int G, uint32_t* err) {
+  extern __shared__ __align__(1024) char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;  // 128B-swizzle atoms
+  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw + pad);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int n_qt = gridDim.x;
+  const int qt = n_qt - 1 - (int)blockIdx.x;  // later tiles (more cache) first
+  const int hp = blockIdx.y;
+  const int bh = blockIdx.z, b = bh / hkv, kh = bh % hkv;
+  const int Hq = hkv * G;
+  const int t0 = chunk_start + qt * kQT;
+  const int h0 = kh * G + 2 * hp;  // first of the two query heads
+
+  // ---- set-up: barriers, TMEM, cache extents -------------------------------------
+  if (tid == 0) {
+    mbar_init(&sm.q_full, 1);
+    for (int s = 0; s < kStg; ++s) {
+      mbar_init(&sm.kv_full[s], 1);
+      mbar_init(&sm.kv_empty[s], 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(&sm.s_ready[h], 1);
+      mbar_init(&sm.p_ready[h], 128);
+      mbar_init(&sm.o_ready[h], 1);
+    }
+    sm.cnt[0] = sm.cnt[1] = sm.cnt[2] = sm.cnt[3] = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(
+                     smem_u32(&sm.tmem_base))
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  const int n = __ldg(cache.count + bh);
+  const int npages = (n + kPageRows - 1) / kPageRows;
+  const int lim_full = t0 - kWin, lim_any = t0 + kQT - 1 - kWin;
+  for (int pg = tid; pg < npages; pg += kThr) sm.first_pos[pg] = cache_pos(cache, bh, pg * kPageRows);
+  __syncthreads();
+  {
+    int pf = 0, pa = 0;
+    for (int pg = tid; pg < npages; pg += kThr) {
+      pf += sm.first_pos[pg] <= lim_full;
+      pa += sm.first_pos[pg] <= lim_any;
+    }
+    if (pf) atomicAdd(&sm.cnt[0], pf);
+    if (pa) atomicAdd(&sm.cnt[1], pa);
+  }
+  __syncthreads();
+  {
+    const int Pf = sm.cnt[0], Pa = sm.cnt[1];
+    if (tid < 64 && Pf > 0) {
+      const int row = (Pf - 1) * kPageRows + tid;
+      if (row < n && cache_pos(cache, bh, row) <= lim_full) atomicAdd(&sm.cnt[2], 1);
+    } else if (tid >= 64 && tid < 128 && Pa > 0) {
+      const int row = (Pa - 1) * kPageRows + (tid - 64);
+      if (row < n && cache_pos(cache, bh, row) <= lim_any) atomicAdd(&sm.cnt[3], 1);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  Blocks bl;
+  {
+    const int Pf = sm.cnt[0], Pa = sm.cnt[1];
+    bl.nfull = Pf > 0 ? (Pf - 1) * kPageRows + sm.cnt[2] : 0;
+    const int n_any = Pa > 0 ? (Pa - 1) * kPageRows + sm.cnt[3] : 0;
+    bl.nc = (n_any + kKB - 1) / kKB;
+    bl.nrows = n;
+    bl.wfirst = t0 >= kWin ? t0 - kWin : t0;
+    bl.nw = (t0 + kQT - bl.wfirst) / kKB;
+  }
+  const int J = bl.nc + bl.nw;
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer --------------------------------
+    if (lane == 0) {
+      mbar_arrive_expect_tx(&sm.q_full, 2 * 2 * kQT * 128);
+      for (int hh = 0; hh < 2; ++hh)
+        for (int half = 0; half < 2; ++half)
+          tma_4d(sm.q[hh][half], &tm_q, half * 64, h0 + hh, t0 - chunk_start, b, &sm.q_full);
+      for (int j = 0; j < J; ++j) {
+        const int s = j % kStg;
+        mbar_wait(&sm.kv_empty[s], ((j / kStg) & 1) ^ 1, err);
+        if (j < bl.nc) {
+          const int page = __ldg(cache.page_table + (size_t)bh * cache.max_pages + j);
+          mbar_arrive_expect_tx(&sm.kv_full[s], 4 * kKB * 128 + kKB * 4);
+          for (int half = 0; half < 2; ++half) {
+            tma_2d(sm.k[s][half], &tm_kp, half * 64, page * kPageRows, &sm.kv_full[s]);
+            tma_2d(sm.v[s][half], &tm_vp, half * 64, page * kPageRows, &sm.kv_full[s]);
+          }
+          bulk_g2s(sm.pos[s], cache.pos + (size_t)page * kPageRows, kKB * 4, &sm.kv_full[s]);
+        } else {
+          const int pb = bl.wfirst + (j - bl.nc) * kKB;
+          mbar_arrive_expect_tx(&sm.kv_full[s], 4 * kKB * 128);
+          for (int half = 0; half < 2; ++half) {
+            if (pb >= chunk_start) {
+              tma_4d(sm.k[s][half], &tm_kc, half * 64, kh, pb - chunk_start, b, &sm.kv_full[s]);
+              tma_4d(sm.v[s][half], &tm_vc, half * 64, kh, pb - chunk_start, b, &sm.kv_full[s]);
+            } else {
+              tma_4d(sm.k[s][half], &tm_kr, half * 64, pb & (kWin - 1), kh, b, &sm.kv_full[s]);
+              tma_4d(sm.v[s][half], &tm_vr, half * 64, pb & (kWin - 1), kh, b, &sm.kv_full[s]);
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer -----------------------------------
+    if (lane == 0) {
+      constexpr uint32_t idesc_s = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKB >> 3) << 17) |
+                                   ((uint32_t)(kQT >> 4) << 24);
+      constexpr uint32_t idesc_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
+                                    ((uint32_t)(kHD >> 3) << 17) | ((uint32_t)(kQT >> 4) << 24);
+      const uint32_t colS[2] = {kColS0, kColS1}, colO[2] = {kColO0, kColO1};
+      mbar_wait(&sm.q_full, 0, err);
+      tc_fence_after();
+      for (int j = 0; j <= J; ++j) {
+        const int s = j % kStg, sp = (j + kStg - 1) % kStg;
+        if (j < J) {
+          mbar_wait(&sm.kv_full[s], (j / kStg) & 1, err);
+          tc_fence_after();
+        }
+        for (int hh = 0; hh < 2; ++hh) {
+          if (j > 0) {  // O_h += P_h(j-1) V(j-1)
+            mbar_wait(&sm.p_ready[hh], (j - 1) & 1, err);
+            tc_fence_after();
+#pragma unroll
+            for (int kk = 0; kk < kKB / 16; ++kk) {
+              const uint64_t bd = smem_desc(sm.v[sp][0] + kk * 16 * 128, 8192, 1024);
+              mma_ts(tmem + colO[hh], tmem + colS[hh] + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
+            }
+            if (j == J) mma_commit(&sm.o_ready[hh]);
+          }
+          if (j < J) {  // S_h = Q_h K(j)^T
+#pragma unroll
+            for (int kk = 0; kk < kHD / 16; ++kk) {
+              const uint64_t ad = smem_desc(sm.q[hh][kk >> 2] + (kk & 3) * 32, 16, 1024);
+              const uint64_t bd = smem_desc(sm.k[s][kk >> 2] + (kk & 3) * 32, 16, 1024);
+              mma_ss(tmem + colS[hh], ad, bd, idesc_s, kk > 0 ? 1u : 0u);
+            }
+            mma_commit(&sm.s_ready[hh]);
+          }
+        }
+        if (j > 0) mma_commit(&sm.kv_empty[sp]);
+      }
+    }
+  } else if (warp >= 4) {
+    // ------------------------------ softmax --------------------------------------
+    const int hh = (warp - 4) >> 2;
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;
+    const int t = t0 + r;
+    const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
+    const uint32_t colS = hh ? kColS1 : kColS0, colO = hh ? kColO1 : kColO0;
+    const float c = kLog2e * rsqrtf((float)kHD);
+    float m = -INFINITY, l = 0.f;
+    for (int j = 0; j < J; ++j) {
+      const int s = j % kStg;
+      mbar_wait(&sm.s_ready[hh], j & 1, err);
+      mbar_wait(&sm.kv_full[s], (j / kStg) & 1, err);
+      tc_fence_after();
+      uint32_t raw[64];
+      tmem_ld32(lane_addr + colS, raw);
+      tmem_ld32(lane_addr + colS + 32, raw + 32);
+      tmem_wait_ld();
+      float x[64];
+      float rmax = -INFINITY;
+      if (j < bl.nc) {
+        const bool dense = (j + 1) * kKB <= bl.nfull;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int row = j * kKB + i;
+          const bool vis = dense || (row < bl.nrows && sm.pos[s][i] <= t - kWin);
+          x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
+          rmax = fmaxf(rmax, x[i]);
+        }
+      } else {
+        const int pb = bl.wfirst + (j - bl.nc) * kKB;
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const int dlt = t - (pb + i);
+          const bool vis = dlt >= 0 && dlt < kWin;
+          x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
+          rmax = fmaxf(rmax, x[i]);
+        }
+      }
+      const bool need = rmax > m + kSlack;
+      if (__any_sync(0xffffffffu, need)) {
+        const float mnew = need ? fmaxf(m, rmax) : m;
+        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mnew);
+        if (j > 0) {  // O holds P V of earlier blocks: rescale it in TMEM
+#pragma unroll
+          for (int cc = 0; cc < kHD; cc += 32) {
+            uint32_t o[32];
+            tmem_ld32(lane_addr + colO + cc, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(lane_addr + colO + cc, o);
+          }
+          tmem_wait_st();
+        }
+        l *= alpha;
+        m = mnew;
+      }
+      uint32_t pk[32];
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = x[2 * i] == -INFINITY ? 0.f : exp2f(x[2 * i] - m);
+        const float p1 = x[2 * i + 1] == -INFINITY ? 0.f : exp2f(x[2 * i + 1] - m);
+        ps += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      l += ps;
+      tmem_st32(lane_addr + colS, pk);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(&sm.p_ready[hh]);
+    }
+    // epilogue: O / l
+    mbar_wait(&sm.o_ready[hh], 0, err);
+    tc_fence_after();
+    const int hg = h0 + hh;
+    const size_t row_out = ((size_t)b * chunk_len + (t - chunk_start)) * Hq + hg;
+    __nv_bfloat16* dst = out + row_out * kHD;
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+    for (int cc = 0; cc < kHD; cc += 32) {
+      uint32_t o[32];
+      tmem_ld32(lane_addr + colO + cc, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int v4 = 0; v4 < 4; ++v4) {
+        uint4 pkt;
+        pkt.x = pack_bf16(__uint_as_float(o[v4 * 8 + 0]) * inv, __uint_as_float(o[v4 * 8 + 1]) * inv);
+        pkt.y = pack_bf16(__uint_as_float(o[v4 * 8 + 2]) * inv, __uint_as_float(o[v4 * 8 + 3]) * inv);
+        pkt.z = pack_bf16(__uint_as_float(o[v4 * 8 + 4]) * inv, __uint_as_float(o[v4 * 8 + 5]) * inv);
+        pkt.w = pack_bf16(__uint_as_float(o[v4 * 8 + 6]) * inv, __uint_as_float(o[v4 * 8 + 7]) * inv);
+        *reinterpret_cast<uint4*>(dst + cc + v4 * 8) = pkt;
+      }
+    }
+    if (lse_out) lse_out[row_out] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem) : "memory");
+  }
+}
+
+// ---- host: tensor maps -------------------------------------------------------------------
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+              const cuuint64_t* strides, const cuuint32_t* box) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool prefill_tc_supported(const spkv_params& p, const spkv_cache& c, int chunk_start, int chunk_len) {
+  const int G = p.Hq / p.Hkv;
+  return p.dtype == SPKV_BF16 && p.head_dim == kHD && p.window == kWin && G % 2 == 0 &&
+         chunk_start % kQT == 0 && chunk_len % kQT == 0 && chunk_len > 0 &&
+         c.max_pages_per_head <= kMaxPages && encode_fn() != nullptr;
+}
+
+cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                              const void* q, const void* K_chunk, const void* V_chunk,
+                              int chunk_start, int chunk_len, void* o, float* lse,
+                              cudaStream_t stream) {
+  const int G = p.Hq / p.Hkv;
+  const cuuint64_t e = 2;  // bytes per element
+  CUtensorMap tq, tkc, tvc, tkp, tvp, tkr, tvr;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)p.Hq, (cuuint64_t)chunk_len, (cuuint64_t)p.B};
+    const cuuint64_t str[3] = {kHD * e, (cuuint64_t)p.Hq * kHD * e, (cuuint64_t)chunk_len * p.Hq * kHD * e};
+    const cuuint32_t box[4] = {64, 1, kQT, 1};
+    if (!make_map(&tq, q, 4, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)p.Hkv, (cuuint64_t)chunk_len, (cuuint64_t)p.B};
+    const cuuint64_t str[3] = {kHD * e, (cuuint64_t)p.Hkv * kHD * e, (cuuint64_t)chunk_len * p.Hkv * kHD * e};
+    const cuuint32_t box[4] = {64, 1, kKB, 1};
+    if (!make_map(&tkc, K_chunk, 4, dims, str, box) || !make_map(&tvc, V_chunk, 4, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[2] = {(cuuint64_t)kHD, (cuuint64_t)c.num_pages * kPageRows};
+    const cuuint64_t str[1] = {kHD * e};
+    const cuuint32_t box[2] = {64, kKB};
+    if (!make_map(&tkp, c.K_pool, 2, dims, str, box) || !make_map(&tvp, c.V_pool, 2, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)kWin, (cuuint64_t)p.Hkv, (cuuint64_t)p.B};
+    const cuuint64_t str[3] = {kHD * e, (cuuint64_t)kWin * kHD * e, (cuuint64_t)p.Hkv * kWin * kHD * e};
+    const cuuint32_t box[4] = {64, kKB, 1, 1};
+    if (!make_map(&tkr, ring.K_win, 4, dims, str, box) || !make_map(&tvr, ring.V_win, 4, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (err != cudaSuccess) return err;
+    configured = true;
+  }
+  CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
+               c.page_table, c.count, c.max_pages_per_head};
+  dim3 grid(chunk_len / kQT, G / 2, p.B * p.Hkv);
+  prefill_tc_kernel<<<grid, kThr, smem, stream>>>(tq, tkc, tvc, tkp, tvp, tkr, tvr, cv,
+                                                  static_cast<__nv_bfloat16*>(o), lse, chunk_start,
+                                                  chunk_len, p.Hkv, G, c.err_flag);
+  return cudaGetLastError();
+}
+
+}  // namespace spkv

@@ -126,11 +126,157 @@ __global__ void __cluster_dims__(1, kKS, 1) __launch_bounds__(kThreads)
   cluster.sync();  // keep this CTA's partials alive until every rank has read them
 }
 
+// ---- few tokens (decode): W1 streamed once, hidden units split over the cluster ----------
+//
+// With a handful of tokens the first layer is a matrix-vector product bound by the
+// W1 read (d_model x hid).  A cluster of 8 CTAs splits the hidden units; every
+// CTA stages the tokens' h in shared memory, each warp streams its W1 rows with
+// 16-byte loads (lanes along d_model) against all tokens at once, then the GELU
+// outputs are exchanged through distributed shared memory for the second layer.
+constexpr int kSmallRanks = 8;
+constexpr int kSmallThreads = 512;   // one warp per hidden unit of the rank (<= 16 units)
+constexpr int kSmallMaxVec = 16;     // 16-byte W1 vectors per lane (d_model <= 512 x per-lane elems)
+
+template <typename E, int NT>
+__global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThreads, 1)
+    score_small_kernel(const typename E::T* __restrict__ h, int n_tok, int d_model,
+                       const typename E::T* __restrict__ W1, const float* __restrict__ b1,
+                       const float* __restrict__ W2, const float* __restrict__ b2, int hid,
+                       int hkv, float tau, float* __restrict__ u_out, uint8_t* __restrict__ z_out) {
+  using T = typename E::T;
+  constexpr int EPL = 16 / E::kSize;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tok0 = (blockIdx.x / kSmallRanks) * NT;
+  const int nt = min(NT, n_tok - tok0);
+  extern __shared__ __align__(16) char smem_raw[];
+  T* hs = reinterpret_cast<T*>(smem_raw);                           // [NT][d_model]
+  float* xs = reinterpret_cast<float*>(hs + (size_t)NT * d_model);  // [units][NT]
+  const int units = (hid + kSmallRanks - 1) / kSmallRanks;
+  const int j = rank * units + warp;  // this warp's hidden unit
+  const bool active = warp < units && j < hid;
+  const int vec_per_row = d_model / EPL;
+  const int nv = vec_per_row / 32;    // vectors per lane
+
+  // W1 row first, all of it in flight at once; then the tokens into shared memory
+  uint4 wv[kSmallMaxVec];
+  if (active) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(W1 + (size_t)j * d_model);
+#pragma unroll
+    for (int i = 0; i < kSmallMaxVec; ++i)
+      if (i < nv) wv[i] = __ldg(wrow + lane + 32 * i);
+  }
+  for (int e = tid; e < nt * vec_per_row; e += kSmallThreads) {
+    const int n = e / vec_per_row, c = e % vec_per_row;
+    reinterpret_cast<uint4*>(hs)[(size_t)n * vec_per_row + c] =
+        __ldg(reinterpret_cast<const uint4*>(h + (size_t)(tok0 + n) * d_model) + c);
+  }
+  __syncthreads();
+
+  if (active) {
+    float acc[NT];
+#pragma unroll
+    for (int n = 0; n < NT; ++n) acc[n] = 0.f;
+#pragma unroll
+    for (int i = 0; i < kSmallMaxVec; ++i) {
+      if (i < nv) {
+        float wf[EPL];
+        Vec<E>::widen(wv[i], wf);
+#pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          if (n < nt) {
+            float hf[EPL];
+            Vec<E>::widen(reinterpret_cast<const uint4*>(hs)[(size_t)n * vec_per_row + lane + 32 * i], hf);
+#pragma unroll
+            for (int e = 0; e < EPL; ++e) acc[n] = fmaf(wf[e], hf[e], acc[n]);
+          }
+        }
+      }
+    }
+#pragma unroll
+    for (int n = 0; n < NT; ++n) {
+#pragma unroll
+      for (int m = 16; m > 0; m >>= 1) acc[n] += __shfl_xor_sync(0xffffffffu, acc[n], m);
+    }
+    if (lane == 0) {
+      const float bias = b1[j];
+#pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const float a = acc[n] + bias;
+        xs[warp * NT + n] = 0.5f * a * (1.f + erff(a * 0.70710678118654752440f));
+      }
+    }
+  }
+  cluster.sync();
+
+  // second layer: token n is finished by rank n % 8, one warp per (token, key head)
+  for (int pair = warp; pair < NT * hkv; pair += kSmallThreads / 32) {
+    const int n = pair / hkv, kh = pair % hkv;
+    if (n % kSmallRanks != rank || n >= nt) continue;
+    float sum = 0.f;
+    for (int jj = lane; jj < hid; jj += 32) {
+      const float* remote = cluster.map_shared_rank(xs, jj / units);
+      sum = fmaf(remote[(jj % units) * NT + n], W2[kh * hid + jj], sum);
+    }
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+    if (lane == 0) {
+      const float logit = sum + b2[kh];
+      const float uval = 1.f / (1.f + expf(-logit));
+      const size_t o = (size_t)(tok0 + n) * hkv + kh;
+      if (u_out) u_out[o] = uval;
+      z_out[o] = (uval >= tau) ? 1 : 0;
+    }
+  }
+  cluster.sync();
+}
+
+template <typename E, int NT>
+cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const void* W1,
+                         const float* b1, const float* W2, const float* b2, float* u_out,
+                         uint8_t* z_out, cudaStream_t stream) {
+  using T = typename E::T;
+  const int units = (p.hid + kSmallRanks - 1) / kSmallRanks;
+  const size_t smem = (size_t)NT * p.d_model * E::kSize + (size_t)units * NT * 4;
+  static int configured_smem = 0;
+  if ((int)smem > configured_smem) {
+    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    configured_smem = (int)smem;
+  }
+  const int groups = (n_tok + NT - 1) / NT;
+  score_small_kernel<E, NT><<<groups * kSmallRanks, kSmallThreads, smem, stream>>>(
+      static_cast<const T*>(h), n_tok, p.d_model, static_cast<const T*>(W1), b1, W2, b2, p.hid,
+      p.Hkv, p.tau, u_out, z_out);
+  return cudaGetLastError();
+}
+
+// The few-token kernel applies when the tokens fit in shared memory, every lane
+// holds whole 16-byte W1 vectors, and one warp per hidden unit covers a rank.
+bool small_ok(const spkv_params& p, int n_tok) {
+  const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
+  const int epl = 16 / esize;
+  const int units = (p.hid + kSmallRanks - 1) / kSmallRanks;
+  return n_tok <= 16 && p.d_model % (32 * epl) == 0 && p.d_model / (32 * epl) <= kSmallMaxVec &&
+         units <= kSmallThreads / 32 &&
+         (size_t)16 * p.d_model * esize + (size_t)units * 16 * 4 <= 160 * 1024;
+}
+
 }  // namespace
 
 cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const void* W1,
                          const float* b1, const float* W2, const float* b2, float* u_out,
                          uint8_t* z_out, cudaStream_t stream) {
+  if (small_ok(p, n_tok)) {
+    if (p.dtype == SPKV_BF16) {
+      return n_tok <= 8 ? launch_small<BF16, 8>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream)
+                        : launch_small<BF16, 16>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream);
+    }
+    return n_tok <= 8 ? launch_small<F32, 8>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream)
+                      : launch_small<F32, 16>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream);
+  }
   dim3 grid((n_tok + kTok - 1) / kTok, kKS);
   if (p.dtype == SPKV_BF16) {
     score_kernel<BF16><<<grid, kThreads, 0, stream>>>(

@@ -1,0 +1,109 @@
+"""Run one kernel of the SP-KV path on a small, fixed configuration (for profilers).
+
+    python -m sparse_decode_attention_spkv_b200.kernel_driver decode  [--layers 1] [--steps 3]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver score   [--tokens 8]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver prefill [--chunk 4096]
+
+``decode`` builds the decode32k state (batch 8, 32K context, ~300 MB of live K/V per
+layer, more than L2) for a few layers and runs eager decode steps; the others run
+their kernel a few times on decode32k / prefill16k shapes.  Prints nothing but a
+completion line: timings come from the profiler.
+"""
+from __future__ import annotations
+
+import argparse
+
+import torch
+
+from . import runner as R
+from . import spkv as S
+from .inputs import device as D
+from .inputs import gen
+from .inputs import workloads as W
+
+
+def _layer(wl, rows_per_head, device="cuda"):
+    p = S.make_params(wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau,
+                      S.BF16)
+    W1 = torch.from_numpy(wl.w1(0)).to(torch.bfloat16).to(device)
+    b1 = torch.from_numpy(wl.b1(0)).to(device)
+    W2 = torch.from_numpy(wl.w2(0)).to(device)
+    b2 = torch.from_numpy(wl.b2(0)).to(device)
+    mp = R.pages_for(rows_per_head)
+    return R.Layer.create(p, W1, b1, W2, b2, wl.B * wl.Hkv * mp, mp, device)
+
+
+def run_decode(args):
+    from .states import DecodeStep, build_decode_state
+    wl = W.WORKLOADS["decode32k"]
+    p, Ls, inp = build_decode_state(wl, args.layers, args.steps, torch.device("cuda"))
+    step = DecodeStep(p, Ls, "cuda")
+    for i in range(args.steps):
+        step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
+    torch.cuda.synchronize()
+
+
+def run_score(args):
+    wl = W.WORKLOADS["decode32k"]
+    L = _layer(wl, 64)
+    h = torch.empty((args.tokens, wl.d_model), dtype=torch.bfloat16, device="cuda")
+    D.fill_normal(h, wl.key(0, gen.T_H), 1.0)
+    for _ in range(args.steps):
+        R.score(L, h, args.tokens)
+    torch.cuda.synchronize()
+
+
+def run_compact(args):
+    wl = W.WORKLOADS["prefill16k"]
+    n = args.rows
+    L = _layer(wl, 4 * n)
+    k = torch.empty((1, n, wl.Hkv, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    h = torch.empty((n, wl.d_model), dtype=torch.bfloat16, device="cuda")
+    D.fill_normal(k, wl.key(0, gen.T_K), wl.qkv_scale)
+    D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale)
+    D.fill_normal(h, wl.key(0, gen.T_H), 1.0)
+    _, z = R.score(L, h, n)
+    for i in range(args.steps):
+        src = torch.full((1,), i * n, dtype=torch.int32, device="cuda")
+        S.spkv_write_compact(L.p, L.cache, L.ring, S.SRC_CHUNK, k, v, z, src, n, n)
+    torch.cuda.synchronize()
+
+
+def run_prefill(args):
+    wl = W.WORKLOADS["prefill16k"]
+    T = wl.ctx[0]
+    c = args.chunk
+    L = _layer(wl, T)
+    Tt = wl.T_total
+    for c0 in range(0, min(T, c * args.steps), c):
+        h = torch.empty((1, c, wl.d_model), dtype=torch.bfloat16, device="cuda")
+        q = torch.empty((1, c, wl.Hq, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+        k = torch.empty((1, c, wl.Hkv, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        D.fill_normal(h, wl.key(0, gen.T_H), 1.0, offset=c0 * wl.d_model)
+        D.fill_rope(q, wl.key(0, gen.T_Q), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_rope(k, wl.key(0, gen.T_K), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale, offset=c0 * wl.Hkv * wl.head_dim)
+        R.prefill_chunk(L, h, q, k, v, c0)
+    torch.cuda.synchronize()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("kernel", choices=["decode", "score", "compact", "prefill"])
+    ap.add_argument("--layers", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=3)
+    ap.add_argument("--tokens", type=int, default=8)
+    ap.add_argument("--rows", type=int, default=4096)
+    ap.add_argument("--chunk", type=int, default=4096)
+    args = ap.parse_args()
+    torch.cuda.set_device(0)
+    {"decode": run_decode, "score": run_score, "compact": run_compact, "prefill": run_prefill}[args.kernel](args)
+    st, flags = (S.OK, 0)
+    print(f"kernel_driver {args.kernel} done")
+
+
+if __name__ == "__main__":
+    main()

@@ -122,9 +122,9 @@ class Cache:
     def allocate(p: spkv_params, num_pages: int, max_pages_per_head: int, device="cuda") -> "Cache":
         dt = torch_dtype(p.dtype)
         heads = p.B * p.Hkv
-        K = torch.empty((num_pages, PAGE_ROWS, p.head_dim), dtype=dt, device=device)
-        V = torch.empty_like(K)
-        pos = torch.empty((num_pages, PAGE_ROWS), dtype=torch.int32, device=device)
+        K = torch.zeros((num_pages, PAGE_ROWS, p.head_dim), dtype=dt, device=device)
+        V = torch.zeros_like(K)
+        pos = torch.zeros((num_pages, PAGE_ROWS), dtype=torch.int32, device=device)
         table = torch.full((heads, max_pages_per_head), -1, dtype=torch.int32, device=device)
         count = torch.zeros(heads, dtype=torch.int32, device=device)
         count_prev = torch.zeros(heads, dtype=torch.int32, device=device)

@@ -138,6 +138,14 @@ PREFILL_CASES = {
                                  hid=32, ctx=[700], decode_steps=0, layers=1, keep="fixed25"), 700, 300),
     "f32_g8_d128": (W.small_case("tiny", cid=44, B=1, Hq=8, Hkv=1, head_dim=128, ctx=[400],
                                  decode_steps=0), 400, 160),
+    # tensor-core path (bf16, head_dim 128, window 128, chunks of multiples of 128)
+    "tc_g2_two_chunks": (W.small_case("decode32k", cid=52, B=2, Hq=4, Hkv=2, d_model=128, hid=32,
+                                      ctx=[1024], decode_steps=0, layers=1, keep="fixed25"), 1024, 512),
+    "tc_g8_three_chunks": (W.small_case("decode32k", cid=53, B=1, Hq=16, Hkv=2, d_model=128,
+                                        hid=32, ctx=[1152], decode_steps=0, layers=1,
+                                        keep="u05_50"), 1152, 384),
+    "tc_g4_dense_pages": (W.small_case("decode32k", cid=54, B=1, Hq=8, Hkv=2, d_model=128, hid=32,
+                                       ctx=[1536], decode_steps=0, layers=1, keep="spread"), 1536, 768),
 }
 
 
