@@ -187,6 +187,34 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_r
                      const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
                      size_t ws_bytes, spkv_stream_t stream);
 
+/* Size of the fixed device scratch used by spkv_decode_attn_noalloc (8 MiB).  Every
+ * GPU on which the library is loaded keeps this much memory until the process exits. */
+#define SPKV_NOALLOC_SCRATCH_BYTES (8u << 20)
+
+/* Gated decode attention without a caller-provided workspace.  The SP-KV paper has
+ * no counterpart: this is a deployment convenience of this library.
+ *
+ * spkv_decode_attn needs scratch memory for its split partials and counters, which
+ * the caller must allocate.  Some callers cannot: code running inside a host that
+ * owns all device memory through its own pool, a serving path that must not call
+ * cudaMalloc after start-up, or a runtime with no allocator to borrow from.  This
+ * entry point computes exactly what spkv_decode_attn computes (same arguments minus
+ * the workspace, same kernels) but takes its scratch from a fixed array of
+ * SPKV_NOALLOC_SCRATCH_BYTES inside the library.  It allocates and frees nothing.
+ *
+ * - Shapes whose scratch need (spkv_decode_workspace_bytes) exceeds the fixed size
+ *   are rejected with SPKV_ERR_UNSUPPORTED before anything is enqueued.
+ * - The first call on a device looks up the array's device address (set-up, once
+ *   per device, with that device current); make that first call before any stream
+ *   capture.
+ * - Every call shares the one array: the counters it needs at zero are cleared on
+ *   `stream` at the start of each call, but calls whose work overlaps on the device
+ *   (other streams, concurrent graph branches) race on the scratch and must not be
+ *   issued. */
+int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* cache,
+                             const spkv_ring* ring, const void* q, const int32_t* t_pos,
+                             void* o, float* lse, spkv_stream_t stream);
+
 /* a6 -- gated prefill attention, Eqs. (3)-(4), for the chunk of queries at
  * positions chunk_start .. chunk_start+chunk_len-1 of every batch row.  Keys:
  * the window, from K_chunk/V_chunk (positions >= chunk_start) and from the ring

@@ -64,7 +64,10 @@ _sigs = {
                                 _vp, ctypes.c_size_t, _vp]),
     "spkv_prefill_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _i32,
                                  _i32, _vp, _vp, _vp]),
+    "spkv_decode_attn_noalloc": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
+                                        _vp, _vp, _vp]),
 }
+NOALLOC_SCRATCH_BYTES = 8 << 20
 for _name, (_res, _args) in _sigs.items():
     _fn = getattr(lib, _name)
     _fn.restype = _res
@@ -215,3 +218,11 @@ def spkv_prefill_attn(p, cache: Cache, ring: Ring, q, K_chunk, V_chunk, chunk_st
     return _check("spkv_prefill_attn", lib.spkv_prefill_attn(
         ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(K_chunk),
         _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _stream(stream)))
+
+
+def spkv_decode_attn_noalloc(p, cache: Cache, ring: Ring, q, t_pos, o, lse, stream=None):
+    """spkv_decode_attn for callers that cannot allocate a workspace: the scratch is a
+    fixed array inside the library (see include/spkv.h)."""
+    return _check("spkv_decode_attn_noalloc", lib.spkv_decode_attn_noalloc(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
+        _ptr(lse), _stream(stream)))

@@ -1,0 +1,90 @@
+"""Decode attention through the no-allocation entry point (GPU required).
+
+Some callers cannot allocate the decode workspace themselves (a host that owns all
+device memory through its own pool, a path that may not call cudaMalloc after
+start-up).  spkv_decode_attn_noalloc serves them from a fixed scratch array inside
+the library.  Here it must give what spkv_decode_attn gives, on two calls in a row
+(the shared scratch keeps the previous call's contents), within the tolerance the
+parity tests use.  This file is collected last on purpose.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from sparse_decode_attention_spkv_b200.inputs import workloads as W
+from tests import cases as C
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import spkv as S
+
+
+def _state(wl, T0):
+    """A layer whose cache and ring hold T0 tokens (per-token-ready), built through the
+    library, and the inputs of the decode step at position T0."""
+    W1, b1, W2, b2 = C.weights(wl)
+    p = S.make_params(wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau,
+                      S.BF16 if wl.dtype == "bf16" else S.F32)
+    mp = R.pages_for(T0 + 8)
+    layer = R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                           num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp)
+    hs, qs, ks, vs = [], [], [], []
+    for b in range(wl.B):
+        h, q, k, v = C.host_rows(wl, 0, b, np.arange(T0 + 1))
+        hs.append(h); qs.append(q); ks.append(k); vs.append(v)
+    h, q, k, v = (np.stack(x) for x in (hs, qs, ks, vs))
+    w = wl.window
+    R.prefill_chunk(layer, C.dev(h[:, :T0], wl.dtype), C.dev(q[:, :T0], wl.dtype),
+                    C.dev(k[:, :T0], wl.dtype), C.dev(v[:, :T0], wl.dtype), 0,
+                    n_compact=max(0, T0 - w))
+    t_pos = torch.full((wl.B,), T0, dtype=torch.int32, device="cuda")
+    _, z_t = R.score(layer, C.dev(h[:, T0], wl.dtype), wl.B)
+    S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, C.dev(k[:, T0], wl.dtype),
+                         C.dev(v[:, T0], wl.dtype), z_t, 1)
+    return p, layer, C.dev(q[:, T0], wl.dtype), t_pos
+
+
+CASES = {
+    "bf16_g4_d128": W.small_case("decode32k", cid=60, B=2, Hq=8, Hkv=2, d_model=128, hid=32,
+                                 ctx=[3000], decode_steps=1, layers=1, keep="u05_50"),
+    "f32_g2_d64": W.small_case("tiny", cid=61, ctx=[700], decode_steps=1),
+}
+
+
+@pytest.mark.parametrize("name", sorted(CASES))
+def test_noalloc_matches_workspace_entry_point(name):
+    wl = CASES[name]
+    p, layer, q, t_pos = _state(wl, wl.ctx[0])
+    o_ref = torch.empty_like(q)
+    lse_ref = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+    S.spkv_decode_attn(p, layer.cache, layer.ring, q, t_pos, o_ref, lse_ref, layer.ws)
+    for call in range(2):
+        o = torch.full_like(q, float("nan"))
+        lse = torch.full((wl.B, wl.Hq), float("nan"), dtype=torch.float32, device="cuda")
+        S.spkv_decode_attn_noalloc(p, layer.cache, layer.ring, q, t_pos, o, lse)
+        torch.cuda.synchronize()
+        C.check_attn(C.to_np(o), C.to_np(o_ref), wl.dtype, f"{name} call {call}")
+        assert np.allclose(lse.cpu().numpy(), lse_ref.cpu().numpy(), atol=1e-4), f"lse, call {call}"
+    status, flags = S.spkv_cache_check(layer.cache)
+    assert status == S.OK, flags
+
+
+def test_noalloc_rejects_shapes_beyond_the_scratch():
+    """2048 key heads with 8 query heads each need more split scratch than the fixed
+    array holds: the call is refused before anything is enqueued."""
+    p = S.make_params(256, 64, 8, 128, 4096, 128, 128, 0.5, S.BF16)
+    need = S.lib.spkv_decode_workspace_bytes(ctypes.byref(p), None)
+    assert need > S.NOALLOC_SCRATCH_BYTES
+    buf = torch.zeros(1024, dtype=torch.uint8, device="cuda")
+    a = buf.data_ptr()
+    cache = S.spkv_cache(a, a, a, a, a, a, a, a, 1, S.PAGE_ROWS, 1)
+    ring = S.spkv_ring(a, a, a)
+    st = S.lib.spkv_decode_attn_noalloc(ctypes.byref(p), ctypes.byref(cache), ctypes.byref(ring),
+                                        a, a, a, None, None)
+    assert st == S.ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert int(buf.sum()) == 0
