@@ -283,7 +283,103 @@ def run_gpu(args, world, rank, local):
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
+    del Ls, inp, step
+    torch.cuda.empty_cache()
+    if not args.no_aux:
+        out["aux"] = {"prefill16k": measure_prefill(device, reps=3)}
     return out
+
+
+def measure_prefill(device, reps=3):
+    """Secondary measurement: the prefill16k chunked prefill (4 chunks of 4096: score,
+    compact, gated prefill attention, ring update) timed end to end with CUDA events,
+    and the prefill-attention kernel alone.  FLOPs are the live (query, key) pairs of
+    Eq. (4): 4 * head_dim * Hq * sum_t |S(t)| (QK^T and PV, multiply-add = 2)."""
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.inputs import device as D
+    from sparse_decode_attention_spkv_b200.inputs import gen
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+
+    wl = W.WORKLOADS["prefill16k"]
+    T, chunk = wl.ctx[0], wl.chunk
+    bf = torch.bfloat16
+    p = S.make_params(1, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau, S.BF16)
+    L = R.Layer.create(p, torch.from_numpy(wl.w1(0)).to(bf).to(device),
+                       torch.from_numpy(wl.b1(0)).to(device), torch.from_numpy(wl.w2(0)).to(device),
+                       torch.from_numpy(wl.b2(0)).to(device), num_pages=wl.Hkv * R.pages_for(T),
+                       max_pages_per_head=R.pages_for(T), device=device)
+    Tt = wl.T_total
+    n_ch = T // chunk
+    hs = [torch.empty((1, chunk, wl.d_model), dtype=bf, device=device) for _ in range(n_ch)]
+    qs = [torch.empty((1, chunk, wl.Hq, wl.head_dim), dtype=bf, device=device) for _ in range(n_ch)]
+    ks = [torch.empty((1, chunk, wl.Hkv, wl.head_dim), dtype=bf, device=device) for _ in range(n_ch)]
+    vs = [torch.empty_like(k) for k in ks]
+    for i in range(n_ch):
+        c0 = i * chunk
+        D.fill_normal(hs[i], wl.key(0, gen.T_H), 1.0, offset=c0 * wl.d_model)
+        D.fill_rope(qs[i], wl.key(0, gen.T_Q), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_rope(ks[i], wl.key(0, gen.T_K), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_normal(vs[i], wl.key(0, gen.T_V), wl.qkv_scale, offset=c0 * wl.Hkv * wl.head_dim)
+    o = torch.empty((1, chunk, wl.Hq, wl.head_dim), dtype=bf, device=device)
+    lse = torch.empty((1, chunk, wl.Hq), dtype=torch.float32, device=device)
+    u = torch.empty((chunk, wl.Hkv), dtype=torch.float32, device=device)
+    z = torch.empty((chunk, wl.Hkv), dtype=torch.uint8, device=device)
+    src = [torch.full((1,), i * chunk, dtype=torch.int32, device=device) for i in range(n_ch)]
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+
+    def run(evs=None):
+        for i in range(n_ch):
+            S.spkv_score(p, hs[i], chunk, L.W1, L.b1, L.W2, L.b2, u, z)
+            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, ks[i], vs[i], z, src[i], chunk, chunk)
+            if evs:
+                evs[i][0].record()
+            S.spkv_prefill_attn(p, L.cache, L.ring, qs[i], ks[i], vs[i], i * chunk, chunk, o, lse)
+            if evs:
+                evs[i][1].record()
+            S.spkv_ring_write(p, L.ring, ks[i], vs[i], z, chunk, src[i], chunk, chunk)
+
+    totals, attn = [], []
+    for r in range(reps + 1):
+        S.spkv_cache_reset(p, L.cache, L.ring)
+        flush.zero_()  # L2 flush: the chunk working set fits in L2
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(n_ch)]
+        a, bE = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        run(evs)
+        bE.record()
+        torch.cuda.synchronize()
+        if r:  # the first pass is a warm-up
+            totals.append(a.elapsed_time(bE))
+            attn.append(sum(e0.elapsed_time(e1) for e0, e1 in evs))
+    status, flags = S.spkv_cache_check(L.cache)
+    if status != S.OK:
+        raise RuntimeError(f"prefill measurement: {S.status_str(status)} flags={flags}")
+    # live pairs: every query sees min(w, t+1) window keys and the cached keys with pos <= t-w
+    pos = []
+    for lst in R.cache_lists(L):
+        pos.append(lst.astype("int64"))
+    w = wl.window
+    pairs_win = sum(min(w, t + 1) for t in range(T))
+    pairs_cache = sum(int(np.maximum(0, T - (pp + w)).sum()) for pp in pos)
+    flops = 4.0 * wl.head_dim * wl.G * (pairs_win * wl.Hkv + pairs_cache)
+    t_total = statistics.median(totals) / 1e3
+    t_attn = statistics.median(attn) / 1e3
+    import json as _json
+    with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) if os.path.exists(
+            os.path.join(ROOT, "MEASURED_PEAKS.json")) else open(os.devnull) as f:
+        txt = f.read()
+    peak_tf = float(_json.loads(txt)["bf16_tflops"]) if txt else 1590.0
+    return {"unit": "TFLOP/s", "live_pair_flops": flops, "ms_total": t_total * 1e3,
+            "ms_prefill_attn": t_attn * 1e3, "tflops_total": flops / t_total / 1e12,
+            "tflops_prefill_attn": flops / t_attn / 1e12,
+            "roofline": {"bound": "tensor", "kernel": "prefill_attn",
+                         "achieved": flops / t_attn / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": flops / t_attn / 1e12 / peak_tf,
+                         "peak_kind": "measured (burst)" if txt else "fallback"},
+            "density_nonlocal": float(sum(len(pp) for pp in pos)) / (wl.Hkv * T),
+            "l2": "512 MB buffer written before each repetition"}
 
 
 # -------------------------------------------------------------- CPU oracle arm -----
@@ -369,6 +465,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-units", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-aux", action="store_true", help="skip the secondary prefill measurement")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -160,6 +160,18 @@ int spkv_decode_append(const spkv_params* p, const spkv_cache* cache, const spkv
                        const int32_t* t_pos, const void* k_new, const void* v_new,
                        const uint8_t* z_new, int retire, spkv_stream_t stream);
 
+/* a1 + a2 + a3 fused for one per-token decode step: the same result as spkv_score on
+ * the B new tokens (h [B][d_model], one per batch row, at positions t_pos) followed by
+ * spkv_decode_append(..., z_new = z_out, retire = 1).  The warp that finishes the gate
+ * of (batch row b, key head kh) also retires token t-window of (b, kh) and stores the
+ * new token, so the step costs one launch.  u_out [B][Hkv] (may be NULL), z_out
+ * [B][Hkv] as in spkv_score; k_new, v_new [B][Hkv][head_dim]. */
+int spkv_decode_score_append(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                             const int32_t* t_pos, const void* h, const void* W1, const float* b1,
+                             const float* W2, const float* b2, const void* k_new,
+                             const void* v_new, float* u_out, uint8_t* z_out,
+                             spkv_stream_t stream);
+
 /* a3 -- store the last min(n_rows, window) rows of a chunk in the ring: row i of
  * batch b (position src_pos[b] + i) goes to slot (src_pos[b] + i) % window.  The
  * slot's gate is 0 for rows i < gated_from (already in the cache, so retiring them

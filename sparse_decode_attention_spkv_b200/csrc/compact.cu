@@ -10,30 +10,14 @@
 //   ring_write                      last rows of a prefill chunk into the ring (a3).
 // Rows are moved as 16-byte vectors by the lanes of one warp (a 256-byte row is
 // 16 lanes), so every copy is coalesced.
+#include "append.cuh"
 #include "common.cuh"
 #include "launch.h"
 
 namespace spkv {
 namespace {
 
-struct CacheMut {
-  char* K;
-  char* V;
-  int32_t* pos;
-  int32_t* page_table;
-  int32_t* count;
-  int32_t* count_prev;
-  int32_t* pool_top;
-  uint32_t* err;
-  int num_pages;
-  int max_pages;
-};
-
-CacheMut mut(const spkv_cache& c) {
-  return CacheMut{static_cast<char*>(c.K_pool), static_cast<char*>(c.V_pool), c.pos_pool,
-                  c.page_table, c.count, c.count_prev, c.pool_top, c.err_flag, c.num_pages,
-                  c.max_pages_per_head};
-}
+CacheMut mut(const spkv_cache& c) { return cache_mut(c); }
 
 __device__ __forceinline__ int block_sum(int v, int* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -178,54 +162,8 @@ __global__ void __launch_bounds__(128)
   const int b = bh / hkv, kh = bh % hkv;
   const int t = t_pos[b];
   if (t < 0) return;  // positions are non-negative by contract
-  const int slot = t % window;
-  const int s = t - window;
-  const int lpr = row_bytes >> 4;
-  const size_t ring_row = (size_t)bh * window + slot;
-  uint8_t* zslot = zwin + ((size_t)b * window + slot) * hkv + kh;
-  if (retire && s >= 0 && *zslot) {
-    const int i = c.count[bh];
-    int page = -1;
-    if ((i & 63) == 0) {
-      if (lane == 0) {
-        if ((i >> 6) >= c.max_pages) {
-          atomicOr(c.err, SPKV_FLAG_TABLE_FULL);
-        } else {
-          const int pg = atomicAdd(c.pool_top, 1);
-          if (pg >= c.num_pages) {
-            atomicOr(c.err, SPKV_FLAG_POOL_FULL);
-          } else {
-            page = pg;
-            c.page_table[(size_t)bh * c.max_pages + (i >> 6)] = pg;
-          }
-        }
-      }
-      page = __shfl_sync(0xffffffffu, page, 0);
-    } else {
-      page = c.page_table[(size_t)bh * c.max_pages + (i >> 6)];
-    }
-    if (page >= 0) {
-      const size_t drow = (size_t)page * kPageRows + (i & 63);
-      if (lane < lpr) {
-        const uint4 kv = *reinterpret_cast<const uint4*>(Kwin + ring_row * row_bytes + lane * 16);
-        const uint4 vv = *reinterpret_cast<const uint4*>(Vwin + ring_row * row_bytes + lane * 16);
-        *reinterpret_cast<uint4*>(c.K + drow * row_bytes + lane * 16) = kv;
-        *reinterpret_cast<uint4*>(c.V + drow * row_bytes + lane * 16) = vv;
-      }
-      if (lane == 0) {
-        c.pos[drow] = s;
-        c.count[bh] = i + 1;
-      }
-    }
-  }
-  __syncwarp();
-  if (lane < lpr) {
-    const uint4 kv = *reinterpret_cast<const uint4*>(k_new + (size_t)bh * row_bytes + lane * 16);
-    const uint4 vv = *reinterpret_cast<const uint4*>(v_new + (size_t)bh * row_bytes + lane * 16);
-    *reinterpret_cast<uint4*>(Kwin + ring_row * row_bytes + lane * 16) = kv;
-    *reinterpret_cast<uint4*>(Vwin + ring_row * row_bytes + lane * 16) = vv;
-  }
-  if (lane == 0) *zslot = z_new ? z_new[bh] : 0;
+  decode_append_warp(c, RingMut{Kwin, Vwin, zwin}, bh, b, kh, t, k_new, v_new,
+                     z_new ? z_new[bh] : (uint8_t)0, retire, hkv, window, row_bytes, lane);
 }
 
 // grid (B*Hkv); the last min(n_rows, window) rows of a chunk go to their slots.

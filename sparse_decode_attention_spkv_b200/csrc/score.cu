@@ -9,6 +9,7 @@
 // (bias, GELU, second layer in fp32, sigmoid, threshold).
 #include <cooperative_groups.h>
 
+#include "append.cuh"
 #include "common.cuh"
 #include "launch.h"
 
@@ -129,20 +130,34 @@ __global__ void __cluster_dims__(1, kKS, 1) __launch_bounds__(kThreads)
 // ---- few tokens (decode): W1 streamed once, hidden units split over the cluster ----------
 //
 // With a handful of tokens the first layer is a matrix-vector product bound by the
-// W1 read (d_model x hid).  A cluster of 8 CTAs splits the hidden units; every
-// CTA stages the tokens' h in shared memory, each warp streams its W1 rows with
-// 16-byte loads (lanes along d_model) against all tokens at once, then the GELU
-// outputs are exchanged through distributed shared memory for the second layer.
+// W1 read (d_model x hid).  A cluster of 8 CTAs splits the hidden units, one warp per
+// unit: the warp's W1 row is loaded into registers all at once while one bulk copy
+// brings the tokens' h into shared memory, the dot products use packed fp32 FMAs,
+// and the GELU outputs are exchanged through distributed shared memory for the
+// second layer.  With APPEND the warp that finishes (token b, key head kh) of a
+// per-token decode step also does that step's ring/cache update for (b, kh).
 constexpr int kSmallRanks = 8;
 constexpr int kSmallThreads = 512;   // one warp per hidden unit of the rank (<= 16 units)
-constexpr int kSmallMaxVec = 16;     // 16-byte W1 vectors per lane (d_model <= 512 x per-lane elems)
+constexpr int kSmallMaxVec = 16;     // 16-byte W1 vectors per lane
+constexpr uint32_t kBulkPiece = 32768;
 
-template <typename E, int NT>
+struct SmallAppend {
+  CacheMut c;
+  RingMut r;
+  const int32_t* t_pos;
+  const char* k_new;
+  const char* v_new;
+  int window;
+  int row_bytes;
+};
+
+template <typename E, int NT, bool APPEND>
 __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThreads, 1)
     score_small_kernel(const typename E::T* __restrict__ h, int n_tok, int d_model,
                        const typename E::T* __restrict__ W1, const float* __restrict__ b1,
                        const float* __restrict__ W2, const float* __restrict__ b2, int hid,
-                       int hkv, float tau, float* __restrict__ u_out, uint8_t* __restrict__ z_out) {
+                       int hkv, float tau, float* __restrict__ u_out, uint8_t* __restrict__ z_out,
+                       SmallAppend ap) {
   using T = typename E::T;
   constexpr int EPL = 16 / E::kSize;
   cg::cluster_group cluster = cg::this_cluster();
@@ -151,6 +166,7 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
   const int tok0 = (blockIdx.x / kSmallRanks) * NT;
   const int nt = min(NT, n_tok - tok0);
   extern __shared__ __align__(16) char smem_raw[];
+  __shared__ uint64_t hbar;
   T* hs = reinterpret_cast<T*>(smem_raw);                           // [NT][d_model]
   float* xs = reinterpret_cast<float*>(hs + (size_t)NT * d_model);  // [units][NT]
   const int units = (hid + kSmallRanks - 1) / kSmallRanks;
@@ -159,7 +175,18 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
   const int vec_per_row = d_model / EPL;
   const int nv = vec_per_row / 32;    // vectors per lane
 
-  // W1 row first, all of it in flight at once; then the tokens into shared memory
+  if (tid == 0) {
+    mbar_init(&hbar, 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (tid == 0) {  // the tokens' hidden states: one contiguous block
+    const uint32_t bytes = (uint32_t)nt * d_model * E::kSize;
+    mbar_arrive_expect_tx(&hbar, bytes);
+    const char* src = reinterpret_cast<const char*>(h + (size_t)tok0 * d_model);
+    for (uint32_t off = 0; off < bytes; off += kBulkPiece)
+      bulk_g2s(reinterpret_cast<char*>(hs) + off, src + off, min(kBulkPiece, bytes - off), &hbar);
+  }
   uint4 wv[kSmallMaxVec];
   if (active) {
     const uint4* wrow = reinterpret_cast<const uint4*>(W1 + (size_t)j * d_model);
@@ -167,17 +194,12 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
     for (int i = 0; i < kSmallMaxVec; ++i)
       if (i < nv) wv[i] = __ldg(wrow + lane + 32 * i);
   }
-  for (int e = tid; e < nt * vec_per_row; e += kSmallThreads) {
-    const int n = e / vec_per_row, c = e % vec_per_row;
-    reinterpret_cast<uint4*>(hs)[(size_t)n * vec_per_row + c] =
-        __ldg(reinterpret_cast<const uint4*>(h + (size_t)(tok0 + n) * d_model) + c);
-  }
-  __syncthreads();
+  mbar_wait(&hbar, 0, nullptr);
 
   if (active) {
-    float acc[NT];
+    float2 acc[NT];
 #pragma unroll
-    for (int n = 0; n < NT; ++n) acc[n] = 0.f;
+    for (int n = 0; n < NT; ++n) acc[n] = make_float2(0.f, 0.f);
 #pragma unroll
     for (int i = 0; i < kSmallMaxVec; ++i) {
       if (i < nv) {
@@ -189,21 +211,24 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
             float hf[EPL];
             Vec<E>::widen(reinterpret_cast<const uint4*>(hs)[(size_t)n * vec_per_row + lane + 32 * i], hf);
 #pragma unroll
-            for (int e = 0; e < EPL; ++e) acc[n] = fmaf(wf[e], hf[e], acc[n]);
+            for (int e = 0; e < EPL / 2; ++e)
+              acc[n] = fma2(make_float2(wf[2 * e], wf[2 * e + 1]), make_float2(hf[2 * e], hf[2 * e + 1]), acc[n]);
           }
         }
       }
     }
+    float sum[NT];
 #pragma unroll
     for (int n = 0; n < NT; ++n) {
+      sum[n] = acc[n].x + acc[n].y;
 #pragma unroll
-      for (int m = 16; m > 0; m >>= 1) acc[n] += __shfl_xor_sync(0xffffffffu, acc[n], m);
+      for (int m = 16; m > 0; m >>= 1) sum[n] += __shfl_xor_sync(0xffffffffu, sum[n], m);
     }
     if (lane == 0) {
       const float bias = b1[j];
 #pragma unroll
       for (int n = 0; n < NT; ++n) {
-        const float a = acc[n] + bias;
+        const float a = sum[n] + bias;
         xs[warp * NT + n] = 0.5f * a * (1.f + erff(a * 0.70710678118654752440f));
       }
     }
@@ -221,36 +246,58 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
     }
 #pragma unroll
     for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+    const float logit = sum + b2[kh];
+    const float uval = 1.f / (1.f + expf(-logit));
+    const uint8_t z = (uval >= tau) ? 1 : 0;
+    const size_t o = (size_t)(tok0 + n) * hkv + kh;
     if (lane == 0) {
-      const float logit = sum + b2[kh];
-      const float uval = 1.f / (1.f + expf(-logit));
-      const size_t o = (size_t)(tok0 + n) * hkv + kh;
       if (u_out) u_out[o] = uval;
-      z_out[o] = (uval >= tau) ? 1 : 0;
+      z_out[o] = z;
+    }
+    if constexpr (APPEND) {
+      const int b = tok0 + n;  // one new token per batch row
+      const int t = ap.t_pos[b];
+      if (t >= 0)
+        decode_append_warp(ap.c, ap.r, b * hkv + kh, b, kh, t, ap.k_new, ap.v_new, z, 1, hkv,
+                           ap.window, ap.row_bytes, lane);
     }
   }
   cluster.sync();
 }
 
-template <typename E, int NT>
+template <typename E, int NT, bool APPEND>
 cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const void* W1,
                          const float* b1, const float* W2, const float* b2, float* u_out,
-                         uint8_t* z_out, cudaStream_t stream) {
+                         uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
   using T = typename E::T;
   const int units = (p.hid + kSmallRanks - 1) / kSmallRanks;
   const size_t smem = (size_t)NT * p.d_model * E::kSize + (size_t)units * NT * 4;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT>,
+    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT, APPEND>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured_smem = (int)smem;
   }
   const int groups = (n_tok + NT - 1) / NT;
-  score_small_kernel<E, NT><<<groups * kSmallRanks, kSmallThreads, smem, stream>>>(
+  score_small_kernel<E, NT, APPEND><<<groups * kSmallRanks, kSmallThreads, smem, stream>>>(
       static_cast<const T*>(h), n_tok, p.d_model, static_cast<const T*>(W1), b1, W2, b2, p.hid,
-      p.Hkv, p.tau, u_out, z_out);
+      p.Hkv, p.tau, u_out, z_out, ap);
   return cudaGetLastError();
+}
+
+template <bool APPEND>
+cudaError_t dispatch_small(const spkv_params& p, const void* h, int n_tok, const void* W1,
+                           const float* b1, const float* W2, const float* b2, float* u_out,
+                           uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
+  if (p.dtype == SPKV_BF16) {
+    return n_tok <= 8
+               ? launch_small<BF16, 8, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
+               : launch_small<BF16, 16, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
+  }
+  return n_tok <= 8
+             ? launch_small<F32, 8, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
+             : launch_small<F32, 16, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }
 
 // The few-token kernel applies when the tokens fit in shared memory, every lane
@@ -269,14 +316,8 @@ bool small_ok(const spkv_params& p, int n_tok) {
 cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const void* W1,
                          const float* b1, const float* W2, const float* b2, float* u_out,
                          uint8_t* z_out, cudaStream_t stream) {
-  if (small_ok(p, n_tok)) {
-    if (p.dtype == SPKV_BF16) {
-      return n_tok <= 8 ? launch_small<BF16, 8>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream)
-                        : launch_small<BF16, 16>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream);
-    }
-    return n_tok <= 8 ? launch_small<F32, 8>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream)
-                      : launch_small<F32, 16>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream);
-  }
+  if (small_ok(p, n_tok))
+    return dispatch_small<false>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   dim3 grid((n_tok + kTok - 1) / kTok, kKS);
   if (p.dtype == SPKV_BF16) {
     score_kernel<BF16><<<grid, kThreads, 0, stream>>>(
@@ -288,6 +329,24 @@ cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const v
         b2, p.hid, p.Hkv, p.tau, u_out, z_out);
   }
   return cudaGetLastError();
+}
+
+cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                                const int32_t* t_pos, const void* h, const void* W1,
+                                const float* b1, const float* W2, const float* b2,
+                                const void* k_new, const void* v_new, float* u_out,
+                                uint8_t* z_out, cudaStream_t stream) {
+  if (!small_ok(p, p.B)) {  // many rows: the two steps as separate launches
+    cudaError_t e = launch_score(p, h, p.B, W1, b1, W2, b2, u_out, z_out, stream);
+    if (e != cudaSuccess) return e;
+    return launch_decode_append(p, c, ring, t_pos, k_new, v_new, z_out, 1, stream);
+  }
+  const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
+  SmallAppend ap{cache_mut(c),
+                 RingMut{static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win},
+                 t_pos, static_cast<const char*>(k_new), static_cast<const char*>(v_new), p.window,
+                 p.head_dim * esize};
+  return dispatch_small<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }
 
 bool score_supported(const spkv_params& p) {

@@ -93,16 +93,24 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
 
 
 def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: bool = True,
-                o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None):
+                o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                fused: bool = True):
     """One decode step for every batch row at positions t_pos [B] (device int32).
 
     h_t [B][d_model] (ignored when retire is False: buffered scoring), q_t [B][Hq][d],
-    k_t, v_t [B][Hkv][d].  Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
+    k_t, v_t [B][Hkv][d].  With ``fused`` the score and the ring/cache update are one
+    launch (spkv_decode_score_append), else spkv_score then spkv_decode_append.
+    Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
     p = layer.p
     z_t = None
-    if retire:
-        _, z_t = score(layer, h_t, p.B)
-    S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, z_t, retire)
+    if retire and fused:
+        z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
+        S.spkv_decode_score_append(p, layer.cache, layer.ring, t_pos, h_t, layer.W1, layer.b1,
+                                   layer.W2, layer.b2, k_t, v_t, None, z_t)
+    else:
+        if retire:
+            _, z_t = score(layer, h_t, p.B)
+        S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, z_t, retire)
     if o is None:
         o = torch.empty_like(q_t)
     if lse is None:

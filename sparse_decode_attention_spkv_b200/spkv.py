@@ -66,6 +66,8 @@ _sigs = {
                                  _i32, _vp, _vp, _vp]),
     "spkv_decode_attn_noalloc": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
                                         _vp, _vp, _vp]),
+    "spkv_decode_score_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
+                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
 }
 NOALLOC_SCRATCH_BYTES = 8 << 20
 for _name, (_res, _args) in _sigs.items():
@@ -226,3 +228,11 @@ def spkv_decode_attn_noalloc(p, cache: Cache, ring: Ring, q, t_pos, o, lse, stre
     return _check("spkv_decode_attn_noalloc", lib.spkv_decode_attn_noalloc(
         ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
         _ptr(lse), _stream(stream)))
+
+
+def spkv_decode_score_append(p, cache: Cache, ring: Ring, t_pos, h, W1, b1, W2, b2, k_new, v_new,
+                             u_out, z_out, stream=None):
+    return _check("spkv_decode_score_append", lib.spkv_decode_score_append(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(t_pos), _ptr(h), _ptr(W1),
+        _ptr(b1), _ptr(W2), _ptr(b2), _ptr(k_new), _ptr(v_new), _ptr(u_out), _ptr(z_out),
+        _stream(stream)))

@@ -1,34 +1,49 @@
 """Device state of the decode workloads, built through the library.
 
-``build_decode_state`` gives every layer of a per-token-retirement decode workload
-its gated cache at the full context (the prefix is scored and compacted chunk by
-chunk; the last ``window`` tokens go to the ring with their gates), plus the
-per-step decode inputs resident in HBM.  ``DecodeStep`` is the launch sequence of
-one decode step over all layers.  Used by ``bench.py`` and ``kernel_driver``.
+``build_decode_state`` gives every layer of a decode workload its gated cache at the
+workload's context (each batch row may have its own context length): the prefix is
+scored and compacted chunk by chunk, and the last ``window`` tokens of every row go
+to the ring.  Two end states:
+
+* per-token retirement (default): the cache holds the gated tokens that have left
+  the window, the ring holds the last ``window`` tokens with their gates;
+* buffered (``compact_window=True``): every gated token of the context is already in
+  the cache and the ring's gates are 0 ("already cached").
+
+It also draws the per-step decode inputs into HBM.  ``DecodeStep`` is the launch
+sequence of one per-token decode step over all layers.  Used by ``bench.py``,
+``kernel_driver`` and the full-size GPU tests.
 """
 from __future__ import annotations
 
 import torch
 
-def build_decode_state(wl, layers, steps_total, device):
-    """All layers' gated caches at 32K context, built through the library (score and
-    compact the prefix; the last 128 tokens go to the ring with their gates), plus
-    per-step decode inputs resident in HBM."""
+
+def build_decode_state(wl, layers, steps_total, device, compact_window: bool = False,
+                       chunk: int = 0):
+    """Returns (params, [Layer], inputs) where inputs["h"|"q"|"k"|"v"][i][l] are step i's
+    tensors of layer l and inputs["t"][i] the positions [B] of step i."""
     from sparse_decode_attention_spkv_b200 import runner as R
     from sparse_decode_attention_spkv_b200 import spkv as S
     from sparse_decode_attention_spkv_b200.inputs import device as D
     from sparse_decode_attention_spkv_b200.inputs import gen
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
 
     B, Hq, Hkv, d, Dm, w = wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.window
-    T0 = wl.ctx[0]
+    ctx = [int(c) for c in wl.ctx]
+    assert len(ctx) == B and min(ctx) >= w
+    Tmax = max(ctx)
     Tt = wl.T_total
     p = S.make_params(B, Hq, Hkv, d, Dm, wl.hid, w, wl.tau, S.BF16)
     bf = torch.bfloat16
-    chunk = 4096
+    if not chunk:
+        chunk = 4096 if B <= 8 else 1024
     h_c = torch.empty((B, chunk, Dm), dtype=bf, device=device)
     k_c = torch.empty((B, chunk, Hkv, d), dtype=bf, device=device)
     v_c = torch.empty_like(k_c)
-    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    # per row: positions below `limit` are compacted from the chunks
+    limit = torch.tensor([c if compact_window else c - w for c in ctx], dtype=torch.int32,
+                         device=device)
     keep_table = W.load_biases()[wl.name]["keep_target"]
     Ls = []
     for l in range(layers):
@@ -36,14 +51,15 @@ def build_decode_state(wl, layers, steps_total, device):
         b1 = torch.from_numpy(wl.b1(l)).to(device)
         W2 = torch.from_numpy(wl.w2(l)).to(device)
         b2 = torch.from_numpy(wl.b2(l)).to(device)
-        rows_head = [min(T0 + steps_total, int(keep_table[l][kh] * 1.15 * T0) + steps_total + 256)
-                     for kh in range(Hkv)]
+        rows_head = [min(Tmax + steps_total,
+                         int(keep_table[l][kh] * 1.15 * Tmax) + steps_total + 512) for kh in range(Hkv)]
         max_pages = R.pages_for(max(rows_head))
         num_pages = B * sum(R.pages_for(r) for r in rows_head)
         L = R.Layer.create(p, W1, b1, W2, b2, num_pages, max_pages, device)
         kh_, kk_, kv_ = wl.key(l, gen.T_H), wl.key(l, gen.T_K), wl.key(l, gen.T_V)
-        for c0 in range(0, T0, chunk):
-            n = min(chunk, T0 - c0)
+        n_lim = max(limit.tolist())
+        for c0 in range(0, n_lim, chunk):
+            n = min(chunk, n_lim - c0)
             for b in range(B):
                 D.fill_normal(h_c[b, :n], kh_, 1.0, offset=(b * Tt + c0) * Dm)
                 D.fill_normal(k_c[b, :n], kk_, wl.qkv_scale, offset=(b * Tt + c0) * Hkv * d)
@@ -52,14 +68,26 @@ def build_decode_state(wl, layers, steps_total, device):
             kc = k_c[:, :n].contiguous() if n < chunk else k_c
             vc = v_c[:, :n].contiguous() if n < chunk else v_c
             _, z = R.score(L, hc, B * n)
-            n_compact = max(0, min(c0 + n, T0 - w) - c0)
+            z = z.view(B, n, Hkv)
+            pos = torch.arange(c0, c0 + n, dtype=torch.int32, device=device)
+            z.mul_((pos[None, :] < limit[:, None]).to(torch.uint8)[:, :, None])  # beyond a row's prefix
             src = torch.full((B,), c0, dtype=torch.int32, device=device)
-            if n_compact:
-                S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, src, n_compact, n)
-            S.spkv_ring_write(p, L.ring, kc, vc, z, n_compact, src, n, n)
+            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, src, n, n)
+        # the ring: each row's last w tokens, gated (per-token) or marked as cached
+        kr = torch.empty((B, w, Hkv, d), dtype=bf, device=device)
+        vr = torch.empty_like(kr)
+        hr = torch.empty((B, w, Dm), dtype=bf, device=device)
+        for b in range(B):
+            s0 = ctx[b] - w
+            D.fill_normal(hr[b], kh_, 1.0, offset=(b * Tt + s0) * Dm)
+            D.fill_normal(kr[b], kk_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
+            D.fill_normal(vr[b], kv_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
+        _, zr = R.score(L, hr, B * w)
+        src = torch.tensor([c - w for c in ctx], dtype=torch.int32, device=device)
+        S.spkv_ring_write(p, L.ring, kr, vr, zr, w if compact_window else 0, src, w, w)
         Ls.append(L)
     del h_c, k_c, v_c
-    # per-step inputs [steps][layers][B][...] for positions T0, T0+1, ...
+    # per-step inputs [steps][layers][B][...]; row b's step i is position ctx[b] + i
     S_ = steps_total
     h_s = torch.empty((layers, B, S_, Dm), dtype=bf, device=device)
     q_s = torch.empty((layers, B, S_, Hq, d), dtype=bf, device=device)
@@ -67,18 +95,21 @@ def build_decode_state(wl, layers, steps_total, device):
     v_s = torch.empty_like(k_s)
     for l in range(layers):
         for b in range(B):
-            D.fill_normal(h_s[l, b], wl.key(l, gen.T_H), 1.0, offset=(b * Tt + T0) * Dm)
-            D.fill_normal(q_s[l, b], wl.key(l, gen.T_Q), wl.qkv_scale, offset=(b * Tt + T0) * Hq * d)
-            D.fill_normal(k_s[l, b], wl.key(l, gen.T_K), wl.qkv_scale, offset=(b * Tt + T0) * Hkv * d)
-            D.fill_normal(v_s[l, b], wl.key(l, gen.T_V), wl.qkv_scale, offset=(b * Tt + T0) * Hkv * d)
+            t0 = ctx[b]
+            D.fill_normal(h_s[l, b], wl.key(l, gen.T_H), 1.0, offset=(b * Tt + t0) * Dm)
+            D.fill_normal(q_s[l, b], wl.key(l, gen.T_Q), wl.qkv_scale, offset=(b * Tt + t0) * Hq * d)
+            D.fill_normal(k_s[l, b], wl.key(l, gen.T_K), wl.qkv_scale, offset=(b * Tt + t0) * Hkv * d)
+            D.fill_normal(v_s[l, b], wl.key(l, gen.T_V), wl.qkv_scale, offset=(b * Tt + t0) * Hkv * d)
+    ctx_t = torch.tensor(ctx, dtype=torch.int32, device=device)
     inputs = {
         "h": h_s.permute(2, 0, 1, 3).contiguous(),
         "q": q_s.permute(2, 0, 1, 3, 4).contiguous(),
         "k": k_s.permute(2, 0, 1, 3, 4).contiguous(),
         "v": v_s.permute(2, 0, 1, 3, 4).contiguous(),
-        "t": (torch.arange(S_, dtype=torch.int32, device=device) + T0).view(S_, 1).repeat(1, B).contiguous(),
+        "t": (torch.arange(S_, dtype=torch.int32, device=device)[:, None] + ctx_t[None, :]).contiguous(),
+        "h_layer_row": h_s,   # [layers][B][steps][d_model] (buffered scoring reads windows of it)
     }
-    del h_s, q_s, k_s, v_s
+    del q_s, k_s, v_s
     torch.cuda.synchronize()
     for L in Ls:
         status, flags = S.spkv_cache_check(L.cache)
@@ -104,22 +135,24 @@ class DecodeStep:
         (start, end) timing events around the decode-attention launch."""
         S, p = self.S, self.p
         for l, L in enumerate(self.layers):
-            S.spkv_score(p, h[l], p.B, L.W1, L.b1, L.W2, L.b2, self.u[l], self.z[l])
-            S.spkv_decode_append(p, L.cache, L.ring, t, k[l], v[l], self.z[l], 1)
+            # score the new token, retire t - w, store the new token: one launch
+            S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2, k[l],
+                                       v[l], self.u[l], self.z[l])
             if ev is not None:
                 ev[l][0].record()
             S.spkv_decode_attn(p, L.cache, L.ring, q[l], t, self.o[l], self.lse[l], L.ws)
             if ev is not None:
                 ev[l][1].record()
 
-    LAUNCHES_PER_LAYER = 3
+    LAUNCHES_PER_LAYER = 2
 
 
-def kv_bytes(p, layers, t):
-    """Algorithmic K/V bytes of one decode step at query position t: every head reads
-    its live cache rows and its window rows once (K and V, bf16)."""
+def kv_bytes(p, layers, t_min):
+    """Algorithmic K/V bytes of one decode step: every head reads its live cache rows and
+    its window rows once (K and V, bf16).  (The cache holds only rows <= t - w in the
+    per-token schedule, so count is the live row count.)"""
     total = 0
-    n_win = min(p.window, t + 1)
+    n_win = min(p.window, t_min + 1)
     for L in layers:
         total += int((L.cache.count.to(torch.int64) + n_win).sum().item())
     return total * 2 * p.head_dim * 2

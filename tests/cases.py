@@ -80,3 +80,35 @@ def check_attn(o_gpu, o_ref, dtype: str, what: str = ""):
 
 def to_np(t: torch.Tensor) -> np.ndarray:
     return t.float().cpu().numpy()
+
+
+def oracle_gates_rows(wl: W.Workload, layer: int, b: int, T: int, W1, b1, W2, b2, block: int = 2048):
+    """Oracle u, z [T][Hkv] of batch row b, positions 0..T-1 (hidden states regenerated on
+    the host in blocks)."""
+    us = []
+    for s0 in range(0, T, block):
+        h = wl.h_rows(layer, b, np.arange(s0, min(T, s0 + block)))
+        us.append(O.utility(h, W1, b1, W2, b2))
+    u = np.concatenate(us, axis=0)
+    return u, O.gate(u, wl.tau)
+
+
+def kv_rows(wl: W.Workload, layer: int, b: int, T: int, block: int = 4096):
+    """Host K, V [T][Hkv][d] of batch row b, positions 0..T-1."""
+    ks, vs = [], []
+    for s0 in range(0, T, block):
+        pos = np.arange(s0, min(T, s0 + block))
+        ks.append(wl.k_rows(layer, b, pos))
+        vs.append(wl.v_rows(layer, b, pos))
+    return np.concatenate(ks), np.concatenate(vs)
+
+
+def check_list(got, z_col, upto, u_col, tau):
+    """Cache index list against the oracle's, where tokens within EXCLUDE of tau may go
+    either way."""
+    want = O.cache_rows(z_col, upto)
+    near = set(np.nonzero(np.abs(u_col[:upto] - tau) < EXCLUDE)[0].tolist())
+    a = [int(x) for x in got if int(x) not in near]
+    c = [int(x) for x in want if int(x) not in near]
+    assert a == c, f"cache list differs away from the threshold ({len(a)} vs {len(c)} rows)"
+    return len(near)

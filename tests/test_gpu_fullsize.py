@@ -1,0 +1,140 @@
+"""CUDA path vs the oracle at the workloads' full sizes, in the launch configuration
+the benchmark times, on sampled outputs the oracle computes one by one (GPU required).
+
+* decode32k: one layer at 32768-token context, batch 8, one per-token decode step
+  (the benchmark's per-layer launches);
+* prefill16k: the whole 16384-token chunked prefill, sampled query positions;
+* ragged128k: contexts {128K, 96K, 64K, 32K}, one decode step, sampled rows;
+* serving: batch 32, contexts in [8K, 64K], 130 buffered decode steps with a bulk
+  score + compaction after step 128, sampled rows and steps.
+Gates outside the exclusion band, cache index lists and attention outputs are checked.
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import spkv_oracle as O
+from sparse_decode_attention_spkv_b200.inputs import workloads as W
+from tests import cases as C
+
+pytestmark = pytest.mark.gpu
+
+if torch.cuda.is_available():
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.states import DecodeStep, build_decode_state
+    from sparse_decode_attention_spkv_b200.inputs import device as D
+    from sparse_decode_attention_spkv_b200.inputs import gen
+
+
+def _one_layer(name, **kw):
+    return W.small_case(name, layers=1, **kw)
+
+
+def _check_row(wl, L, b, t, o_gpu_b, z_new_b, nrows_retired):
+    """Oracle for batch row b at query position t (token t already in the ring)."""
+    W1, b1, W2, b2 = C.weights(wl)
+    u, z = C.oracle_gates_rows(wl, 0, b, t + 1, W1, b1, W2, b2)
+    if z_new_b is not None:
+        near = np.abs(u[t] - wl.tau) < C.EXCLUDE
+        assert np.all((z_new_b == z[t]) | near), "gate of the new token"
+    lists = R.cache_lists(L)
+    for kh in range(wl.Hkv):
+        C.check_list(lists[b * wl.Hkv + kh], z[:, kh], nrows_retired, u[:, kh], wl.tau)
+    K, V = C.kv_rows(wl, 0, b, t + 1)
+    q = wl.q_rows(0, b, [t])
+    o_ref, _ = O.gated_attention(q, K, V, z, wl.window, [t])
+    C.check_attn(o_gpu_b, o_ref[0], "bf16", f"{wl.name} row {b}")
+
+
+def _decode_one_step(wl, rows):
+    p, Ls, inp = build_decode_state(wl, 1, 2, torch.device("cuda"))
+    step = DecodeStep(p, Ls, "cuda")
+    step.launch(inp["h"][0], inp["q"][0], inp["k"][0], inp["v"][0], inp["t"][0])
+    torch.cuda.synchronize()
+    status, flags = S.spkv_cache_check(Ls[0].cache)
+    assert status == S.OK, flags
+    o = step.o[0].float().cpu().numpy()
+    z = step.z[0].cpu().numpy()
+    t = inp["t"][0].cpu().numpy()
+    for b in rows:
+        _check_row(wl, Ls[0], b, int(t[b]), o[b], z[b], int(t[b]) - wl.window + 1)
+
+
+def test_decode32k_one_layer_full_size():
+    _decode_one_step(_one_layer("decode32k"), rows=[5])
+
+
+def test_ragged128k_full_size():
+    _decode_one_step(_one_layer("ragged128k"), rows=[3, 0])
+
+
+def test_serving_buffered_full_size():
+    wl = _one_layer("serving")
+    steps = 130
+    p, Ls, inp = build_decode_state(wl, 1, steps, torch.device("cuda"), compact_window=True)
+    L = Ls[0]
+    sample = {5: [], 127: [], 129: []}
+    for i in range(steps):
+        o, _, _ = R.decode_step(L, inp["t"][i], None, inp["q"][i][0], inp["k"][i][0],
+                                inp["v"][i][0], retire=False)
+        if i in sample:
+            sample[i] = o.float().cpu().numpy()
+        if i == 127:  # the 128-token buffer is full: score it and compact it from the ring
+            start = inp["t"][0].clone()
+            R.bulk_compact(L, inp["h_layer_row"][0][:, 0:128].contiguous(), start)
+    torch.cuda.synchronize()
+    status, flags = S.spkv_cache_check(L.cache)
+    assert status == S.OK, flags
+    t0 = inp["t"][0].cpu().numpy()
+    W1, b1, W2, b2 = C.weights(wl)
+    for b in (0, 17):
+        T_end = int(t0[b]) + steps
+        u, z = C.oracle_gates_rows(wl, 0, b, T_end, W1, b1, W2, b2)
+        K, V = C.kv_rows(wl, 0, b, T_end)
+        for i, o in sample.items():
+            t = int(t0[b]) + i
+            q = wl.q_rows(0, b, [t])
+            o_ref, _ = O.gated_attention(q, K[:t + 1], V[:t + 1], z[:t + 1], wl.window, [t])
+            C.check_attn(o[b], o_ref[0], "bf16", f"serving row {b} step {i}")
+        lists = R.cache_lists(L)
+        for kh in range(wl.Hkv):  # everything up to the end of the first buffer is cached
+            C.check_list(lists[b * wl.Hkv + kh], z[:, kh], int(t0[b]) + 128, u[:, kh], wl.tau)
+
+
+def test_prefill16k_full_size():
+    wl = W.WORKLOADS["prefill16k"]
+    T, chunk = wl.ctx[0], wl.chunk
+    W1, b1, W2, b2 = C.weights(wl)
+    p = S.make_params(1, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau, S.BF16)
+    mp = R.pages_for(T)
+    L = R.Layer.create(p, C.dev(W1, "bf16"), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                       num_pages=wl.Hkv * mp, max_pages_per_head=mp)
+    Tt = wl.T_total
+    outs = []
+    for c0 in range(0, T, chunk):
+        h = torch.empty((1, chunk, wl.d_model), dtype=torch.bfloat16, device="cuda")
+        q = torch.empty((1, chunk, wl.Hq, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+        k = torch.empty((1, chunk, wl.Hkv, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+        v = torch.empty_like(k)
+        D.fill_normal(h, wl.key(0, gen.T_H), 1.0, offset=c0 * wl.d_model)
+        D.fill_rope(q, wl.key(0, gen.T_Q), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_rope(k, wl.key(0, gen.T_K), c0, Tt, wl.qkv_scale, wl.rope_base)
+        D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale, offset=c0 * wl.Hkv * wl.head_dim)
+        o, _, _, _ = R.prefill_chunk(L, h, q, k, v, c0)
+        outs.append(o[0].float().cpu().numpy())
+    o_gpu = np.concatenate(outs)
+    status, flags = S.spkv_cache_check(L.cache)
+    assert status == S.OK, flags
+    u, z = C.oracle_gates_rows(wl, 0, 0, T, W1, b1, W2, b2)
+    lists = R.cache_lists(L)
+    for kh in range(wl.Hkv):
+        C.check_list(lists[kh], z[:, kh], T, u[:, kh], wl.tau)
+    K, V = C.kv_rows(wl, 0, 0, T)
+    rng = np.random.default_rng(0)
+    ts = sorted(set([0, 1, 127, 128, 129, 4095, 4096, 4097, 8191, 8192, 12287, 16383] +
+                    rng.integers(0, T, 20).tolist()))
+    Q = wl.q_rows(0, 0, ts)
+    for i, t in enumerate(ts):
+        o_ref, _ = O.gated_attention(Q[i:i + 1], K[:t + 1], V[:t + 1], z[:t + 1], wl.window, [t])
+        C.check_attn(o_gpu[t], o_ref[0], "bf16", f"prefill16k query {t}")

@@ -172,7 +172,7 @@ def test_chunked_prefill_matches_oracle(name):
     _lists_equal(layer, z_ref, T)
 
 
-def _decode_run(wl, T0, steps, layer_rows, retire=True, bulk=0):
+def _decode_run(wl, T0, steps, layer_rows, retire=True, bulk=0, fused=True):
     """Prefill T0 tokens (per-token-ready state when retire) then decode `steps`
     tokens; returns gpu outputs [steps][B][Hq][d], z per step and the layer."""
     layer, (W1, b1, W2, b2) = _layer(wl, layer_rows)
@@ -191,7 +191,8 @@ def _decode_run(wl, T0, steps, layer_rows, retire=True, bulk=0):
         t = T0 + i
         t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
         o, lse, z = R.decode_step(layer, t_pos, C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype),
-                                  C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype), retire=retire)
+                                  C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype), retire=retire,
+                                  fused=fused)
         outs.append(C.to_np(o))
         zs.append(None if z is None else z.cpu().numpy())
         if bulk and (i + 1) % bulk == 0:
@@ -265,3 +266,17 @@ def test_schedules_agree():
     _, b, _, _, _ = _decode_run(wl, 700, 128, 900, retire=False, bulk=128)
     for i in range(128):
         C.check_attn(a[i], b[i], "bf16", f"step {i}")
+
+
+def test_fused_and_separate_decode_steps_agree():
+    """spkv_decode_score_append (one launch) against spkv_score + spkv_decode_append:
+    identical gates, cache lists and outputs."""
+    wl = W.small_case("decode32k", cid=55, B=3, Hq=8, Hkv=2, d_model=256, hid=64, ctx=[600],
+                      decode_steps=150, layers=1, keep="u05_50")
+    la, a, za, _, _ = _decode_run(wl, 600, 150, 800, fused=True)
+    lb, b, zb, _, _ = _decode_run(wl, 600, 150, 800, fused=False)
+    for i in range(150):
+        assert np.array_equal(za[i], zb[i])
+        assert np.array_equal(a[i], b[i]), f"step {i}"
+    for x, y in zip(R.cache_lists(la), R.cache_lists(lb)):
+        assert np.array_equal(x, y)
