@@ -138,7 +138,7 @@ class ClockSampler:
 
 def _kernel_source_hash() -> str:
     h = hashlib.sha256()
-    for name in ("decode.cu", "common.cuh"):
+    for name in ("decode.cu", "decode_tc.cu", "common.cuh"):
         with open(os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]

@@ -191,8 +191,8 @@ size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* cache
 /* a4 + a5 -- gated decode attention, Eqs. (3)-(4), one query per batch row:
  * query t = t_pos[b] attends to the window slots holding positions
  * max(0, t-window+1)..t and to the cache rows with position <= t - window.
- * Split-K over balanced chunks of rows, with the log-sum-exp merge of the chunk
- * partials done by the last chunk of each key head to finish.
+ * Split-K over balanced chunks of rows (a5: the chunk partials of a head are
+ * combined by their log-sum-exp weights in a second kernel on the same stream).
  * q [B][Hq][head_dim] dtype; o [B][Hq][head_dim] dtype; lse [B][Hq] f32 natural
  * log (may be NULL).  The token t itself must already be in the ring. */
 int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,

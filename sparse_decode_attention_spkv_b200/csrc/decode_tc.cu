@@ -9,23 +9,26 @@
 // G query heads of a group are the rows of a 16-row MMA tile, so the same bytes cost
 // a few instructions and the kernel is left bound by HBM.
 //
-// Structure (one CTA per SM, 10 warps):
-//  * Plan (every CTA, same result): live cache rows per head, rows rounded to
-//    128-row tiles (two cache pages), chunk size so that all heads give ~8 chunks per
-//    CTA, chunk prefix.  The producer pulls chunks from a global atomic counter, so
-//    ragged heads balance.
-//  * Producer warp: per tile, TMA boxes (64 rows x 64 bf16, 128B-swizzled) of K and V
-//    from two cache pages or the ring into a ring of shared-memory stages; with a
-//    chunk's first tile it also copies the chunk's G query rows (bulk copy).
-//  * 8 consumer warps, 16 rows of each tile apiece: S = Q K^T with mma.m16n8k16 (Q rows
+// Structure (one CTA per SM, 5 warps):
+//  * Plan (every CTA, same result): live cache rows per head, rows rounded to 64-row
+//    tiles (cache pages), chunk size so that all heads give a few chunks per CTA,
+//    chunk prefix.  The producer pulls chunks from a global atomic counter, so ragged
+//    heads balance.
+//  * Producer warp: per chunk, its lanes fetch all the chunk's page-table entries at
+//    once into shared memory; then one lane streams 64-row tiles (TMA boxes of
+//    64 rows x 64 bf16, 128B-swizzled) of K and V from the cache pages or the ring
+//    into a 4-stage ring of shared memory, the chunk's G query rows riding along with
+//    its first tile (bulk copy).  Four queued tiles cover the next chunk's fetches.
+//  * 4 consumer warps, 16 rows of each tile apiece: S = Q K^T with mma.m16n8k16 (Q rows
 //    = the G heads, zero-padded to 16), fp32 softmax in the log2 domain (running max
 //    raised only when exceeded by > 8), P re-packed in registers as the A operand of
-//    O += P V (V via ldmatrix.trans).  When a chunk ends they leave their (o, m, l) in
-//    shared memory for the finisher and go straight on with the next chunk.
-//  * Finisher warp: combines the 8 warps' states; a head with one chunk gets o and lse
-//    written, otherwise the chunk's partial goes to the workspace, and the finisher
-//    that completes a head's last chunk (atomic count) merges all of them:
-//    o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i.
+//    O += P V (V via ldmatrix.trans).
+//  * Chunk end: the warps combine through shared memory; a head with one chunk writes
+//    o and lse, otherwise the chunk's (o, m, l) partial goes to the workspace.
+//  * decode_merge_kernel (one CTA per head with several chunks, launched next on the
+//    same stream) combines the partials: o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i,
+//    and resets the work counter for the next call.  A second launch costs less than
+//    the decode CTAs waiting on an arrival count at the end of every head.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -38,16 +41,16 @@
 namespace spkv {
 namespace {
 
-constexpr int kTileR = 128;          // rows per tile: two cache pages, or the whole window
-constexpr int kCons = 8;             // consumer warps, 16 rows each
-constexpr int kProducer = kCons;     // warp index of the producer
-constexpr int kFinisher = kCons + 1; // warp index of the finisher
-constexpr int kThreadsT = (kCons + 2) * 32;
+constexpr int kTileR = 64;           // rows per tile (one cache page)
+constexpr int kCons = 4;             // consumer warps, 16 rows each
+constexpr int kThreadsT = (kCons + 1) * 32;   // + producer
+constexpr int kMergeThreads = 128;
 constexpr int kConsThreads = kCons * 32;
-constexpr int kUnitsPerCta = 8;      // target chunks per CTA
+constexpr int kStagesT = 4;
+constexpr int kUnitsPerCta = 4;      // target chunks per CTA
 constexpr int kMaxHeadsT = 2048;
-constexpr int kMergeBatch = 128;     // partials whose weights the finisher stages at once
-constexpr int kSegTiles = 64;        // tiles whose page numbers the producer fetches at once
+constexpr int kChunkPages = 256;     // page numbers staged per fetch
+constexpr int kMergeBatch = 128;     // partials whose weights are staged at once
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kLn2T = 0.6931471805599453f;
 constexpr float kSlackT = 8.f;
@@ -55,7 +58,7 @@ constexpr float kSlackT = 8.f;
 template <int D>
 struct TileBuf {
   static constexpr int kHalves = D / 64;
-  static constexpr int kHalfBytes = kTileR * 128;       // 128 rows x 128 B
+  static constexpr int kHalfBytes = kTileR * 128;       // 64 rows x 128 B
   static constexpr int kBytes = kHalves * kHalfBytes;   // K (or V) of one tile
   alignas(1024) char k[kHalves][kHalfBytes];
   alignas(1024) char v[kHalves][kHalfBytes];
@@ -65,25 +68,22 @@ struct TileRef {
   int chunk;  // -1: no more work
   int bh;
   int valid;  // valid rows
+  int last;   // last tile of its chunk
   int qslot;  // query staging slot of the chunk
 };
 
-template <int D, int G, int NST>
+template <int D, int G>
 struct TcDecSmem {
-  TileBuf<D> st[NST];
+  TileBuf<D> st[kStagesT];
   alignas(16) __nv_bfloat16 qbuf[2][G * D];
   float red_o[kCons][G][D];
   float red_m[kCons][G];
   float red_l[kCons][G];
-  float fin_w[kMergeBatch * G];   // finisher: weights of a batch of partials
-  int pages[2 * kSegTiles];       // producer: page numbers of a stretch of tiles
-  uint64_t full[NST];
-  uint64_t empty[NST];
+  int pages[kChunkPages];
+  uint64_t full[kStagesT];
+  uint64_t empty[kStagesT];
   uint64_t q_free[2];
-  uint64_t chunk_done;
-  uint64_t red_free;
-  TileRef info[NST];
-  int red_chunk, red_bh;
+  TileRef info[kStagesT];
   int red[kThreadsT];
   int misc[4];
   // followed (dynamic) by rows[n_heads], live[n_heads], base[n_heads + 1]
@@ -140,7 +140,7 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
-template <int D, int G, int NST>
+template <int D, int G>
 __global__ void __launch_bounds__(kThreadsT, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kp,
                      const __grid_constant__ CUtensorMap tm_vp,
@@ -152,7 +152,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                      float* __restrict__ ws_o, int n_heads, int hkv, int window,
                      uint32_t* err) {
   using TB = TileBuf<D>;
-  using S = TcDecSmem<D, G, NST>;
+  using S = TcDecSmem<D, G>;
   constexpr int NT_D = D / 8;     // n-tiles of 8 along head_dim
   constexpr int KS_D = D / 16;    // k-steps of 16 along head_dim
   extern __shared__ __align__(1024) char smem_raw[];
@@ -162,9 +162,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   int* s_live = s_rows + n_heads;
   int* s_base = s_live + n_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int* counters = ws_ctrl;
-  int* next_chunk = ws_ctrl + n_heads;
-  int* done_ctas = ws_ctrl + n_heads + 1;
+  int* next_chunk = ws_ctrl + n_heads;  // reset by the merge kernel
 
   // ---- plan (identical in every CTA) ---------------------------------------------
   int my_rows = 0;
@@ -181,14 +179,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   for (int m = 16; m > 0; m >>= 1) my_rows += __shfl_xor_sync(0xffffffffu, my_rows, m);
   if (lane == 0) sm.red[warp] = my_rows;
   if (tid == 0) {
-    for (int s = 0; s < NST; ++s) {
+    for (int s = 0; s < kStagesT; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], kCons);
     }
-    mbar_init(&sm.q_free[0], kConsThreads);
-    mbar_init(&sm.q_free[1], kConsThreads);
-    mbar_init(&sm.chunk_done, kConsThreads);
-    mbar_init(&sm.red_free, 32);
+    mbar_init(&sm.q_free[0], kCons);
+    mbar_init(&sm.q_free[1], kCons);
     fence_mbar_init();
   }
   __syncthreads();
@@ -203,35 +199,38 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   __syncthreads();
   const int chunk_rows = sm.misc[0];
   {
+    // chunks per head, exclusive prefix over heads: thread segments, warp shuffle scan
     const int per = (n_heads + kThreadsT - 1) / kThreadsT;
     const int lo = tid * per, hi = min(n_heads, lo + per);
     int s = 0;
     for (int bh = lo; bh < hi; ++bh) s += (s_rows[bh] + chunk_rows - 1) / chunk_rows;
-    sm.red[tid] = s;
-    __syncthreads();
-    if (tid == 0) {
-      int acc = 0;
-      for (int i = 0; i < kThreadsT; ++i) {
-        const int v = sm.red[i];
-        sm.red[i] = acc;
-        acc += v;
-      }
-      s_base[n_heads] = acc;
+    int inc = s;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += v;
     }
+    if (lane == 31) sm.red[warp] = inc;
     __syncthreads();
-    int acc = sm.red[tid];
+    int before = 0, total = 0;
+#pragma unroll
+    for (int w = 0; w < kThreadsT / 32; ++w) {
+      const int v = sm.red[w];
+      before += w < warp ? v : 0;
+      total += v;
+    }
+    int acc = before + inc - s;
     for (int bh = lo; bh < hi; ++bh) {
       s_base[bh] = acc;
       acc += (s_rows[bh] + chunk_rows - 1) / chunk_rows;
     }
+    if (tid == 0) s_base[n_heads] = total;
   }
   __syncthreads();
   const int total_chunks = s_base[n_heads];
 
-  if (warp == kProducer) {
+  if (warp == kCons) {
     // ------------------------------ producer ------------------------------------
-    // The whole warp fetches a stretch of the chunk's page-table entries at once (one
-    // round trip instead of one per tile); lane 0 then issues the copies.
     int it = 0;
     for (int seq = 0;; ++seq) {
       int c = 0;
@@ -248,45 +247,39 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       const int r1 = min(s_rows[bh], r0 + chunk_rows);
       const int nl = s_live[bh];
       const int nlp = ((nl + kTileR - 1) / kTileR) * kTileR;
-      const int live_pages = (nl + kPageRows - 1) / kPageRows;
       const int b = bh / hkv, kh = bh % hkv;
       const int t = __ldg(t_pos + b);
       const int nw = t + 1 < window ? t + 1 : window;
       const int k0 = r0 / kTileR, k1 = (r1 + kTileR - 1) / kTileR;
+      const int kc1 = min(k1, nlp / kTileR);  // cache tiles are k0 .. kc1-1
       const int qslot = seq & 1;
       if (lane == 0) mbar_wait(&sm.q_free[qslot], ((seq >> 1) & 1) ^ 1, err);
-      for (int ks = k0; ks < k1; ks += kSegTiles) {
-        const int ke = min(k1, ks + kSegTiles);
-        const int pg_lo = 2 * ks, pg_hi = min(2 * ke, live_pages);
+      for (int ks = k0; ks < k1; ks += kChunkPages) {
+        const int ke = min(k1, ks + kChunkPages);
         __syncwarp();
-        for (int i = lane; i < pg_hi - pg_lo; i += 32)
-          sm.pages[i] = __ldg(cache.page_table + (size_t)bh * cache.max_pages + pg_lo + i);
+        for (int i = ks + lane; i < min(ke, kc1); i += 32)
+          sm.pages[i - ks] = __ldg(cache.page_table + (size_t)bh * cache.max_pages + i);
         __syncwarp();
         if (lane == 0) {
           for (int k = ks; k < ke; ++k, ++it) {
-            const int s = it % NST;
-            mbar_wait(&sm.empty[s], ((it / NST) & 1) ^ 1, err);
+            const int s = it % kStagesT;
+            mbar_wait(&sm.empty[s], ((it / kStagesT) & 1) ^ 1, err);
             TB& tb = sm.st[s];
-            const bool from_cache = k * kTileR < nlp;
+            const bool from_cache = k < kc1;
             const int slot = k * kTileR - nlp;
             const int valid = from_cache ? min(kTileR, nl - k * kTileR) : min(kTileR, nw - slot);
             // the tile description must be in place before the phase can complete
-            sm.info[s] = TileRef{c, bh, valid, qslot};
+            sm.info[s] = TileRef{c, bh, valid, k == k1 - 1, qslot};
             const bool first = k == k0;
             mbar_arrive_expect_tx(&sm.full[s], 2 * TB::kBytes + (first ? G * D * 2 : 0));
             if (first)
               bulk_g2s(sm.qbuf[qslot], q + ((size_t)b * hkv + kh) * G * D, G * D * 2, &sm.full[s]);
             if (from_cache) {
-              const int pg0 = 2 * k;
-              const int page0 = sm.pages[pg0 - pg_lo];
-              // a missing second page is replaced by the first (its rows are masked)
-              const int page1 = pg0 + 1 < live_pages ? sm.pages[pg0 + 1 - pg_lo] : page0;
+              const int page = sm.pages[k - ks];
 #pragma unroll
               for (int hf = 0; hf < TB::kHalves; ++hf) {
-                tma2d(tb.k[hf], &tm_kp, hf * 64, page0 * kPageRows, &sm.full[s]);
-                tma2d(tb.k[hf] + 64 * 128, &tm_kp, hf * 64, page1 * kPageRows, &sm.full[s]);
-                tma2d(tb.v[hf], &tm_vp, hf * 64, page0 * kPageRows, &sm.full[s]);
-                tma2d(tb.v[hf] + 64 * 128, &tm_vp, hf * 64, page1 * kPageRows, &sm.full[s]);
+                tma2d(tb.k[hf], &tm_kp, hf * 64, page * kPageRows, &sm.full[s]);
+                tma2d(tb.v[hf], &tm_vp, hf * 64, page * kPageRows, &sm.full[s]);
               }
             } else {
 #pragma unroll
@@ -301,142 +294,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       }
     }
     if (lane == 0) {
-      const int s = it % NST;
-      mbar_wait(&sm.empty[s], ((it / NST) & 1) ^ 1, err);
+      const int s = it % kStagesT;
+      mbar_wait(&sm.empty[s], ((it / kStagesT) & 1) ^ 1, err);
       sm.info[s].chunk = -1;
       mbar_arrive(&sm.full[s]);
-    }
-  } else if (warp == kFinisher) {
-    // ------------------------------ finisher ------------------------------------
-    for (int n = 0;; ++n) {
-      mbar_wait(&sm.chunk_done, n & 1, err);
-      const int c = sm.red_chunk, bh = sm.red_bh;
-      if (c < 0) break;
-      const int b = bh / hkv, kh = bh % hkv;
-      const size_t hrow = (size_t)b * hkv * G + (size_t)kh * G;
-      const int nch = s_base[bh + 1] - s_base[bh];
-      float Mg[G], Lg[G];
-#pragma unroll
-      for (int g = 0; g < G; ++g) {
-        float M = -INFINITY;
-#pragma unroll
-        for (int w = 0; w < kCons; ++w) M = fmaxf(M, sm.red_m[w][g]);
-        float L = 0.f;
-#pragma unroll
-        for (int w = 0; w < kCons; ++w) {
-          const float mw = sm.red_m[w][g];
-          L += (mw == -INFINITY ? 0.f : exp2f(mw - M)) * sm.red_l[w][g];
-        }
-        Mg[g] = M;
-        Lg[g] = L;
-      }
-      for (int e = lane; e < G * D / 4; e += 32) {
-        const int g = (e * 4) / D, d = (e * 4) % D;
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int w = 0; w < kCons; ++w) {
-          const float mw = sm.red_m[w][g];
-          const float ww = mw == -INFINITY ? 0.f : exp2f(mw - Mg[g]);
-          const float4 v = *reinterpret_cast<const float4*>(&sm.red_o[w][g][d]);
-          acc.x += ww * v.x;
-          acc.y += ww * v.y;
-          acc.z += ww * v.z;
-          acc.w += ww * v.w;
-        }
-        if (nch == 1) {
-          const float L = Lg[g], inv = L > 0.f ? 1.f / L : 0.f;
-          uint2 pk;
-          pk.x = pack2(acc.x * inv, acc.y * inv);
-          pk.y = pack2(acc.z * inv, acc.w * inv);
-          *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
-        } else {
-          *reinterpret_cast<float4*>(ws_o + ((size_t)c * G + g) * D + d) = acc;
-        }
-      }
-      if (nch == 1) {
-        if (lane < G && lse_out)
-          lse_out[hrow + lane] = Lg[lane] > 0.f ? (Mg[lane] + log2f(Lg[lane])) * kLn2T : -INFINITY;
-      } else if (lane < G) {
-        ws_ml[((size_t)c * G + lane) * 2 + 0] = Mg[lane];
-        ws_ml[((size_t)c * G + lane) * 2 + 1] = Lg[lane];
-      }
-      mbar_arrive(&sm.red_free);  // the consumers may overwrite red_* now
-      if (nch > 1) {
-        __syncwarp();
-        int last = 0;
-        if (lane == 0) {
-          __threadfence();
-          const int prev = atomicAdd(counters + bh, 1);
-          last = prev == nch - 1;
-          if (last) counters[bh] = 0;
-        }
-        last = __shfl_sync(0xffffffffu, last, 0);
-        if (last) {
-          // ---- merge all partials of the head ----------------------------------------
-          // Lane l works on the (chunk, head) pairs e = c*G + g with e = l (mod 32), so its
-          // head is g = l % G throughout; the outputs (head g, 4 columns) are spread over
-          // the lanes, and the chunk weights are staged in shared memory per batch.
-          __threadfence();
-          const size_t e0 = (size_t)s_base[bh] * G;
-          float Mx = -INFINITY;
-          for (int e = lane; e < nch * G; e += 32) Mx = fmaxf(Mx, __ldcg(ws_ml + (e0 + e) * 2));
-#pragma unroll
-          for (int m = G; m < 32; m <<= 1) Mx = fmaxf(Mx, __shfl_xor_sync(0xffffffffu, Mx, m));
-          constexpr int kPairs = G * D / 4;           // (head, 4 columns) outputs
-          constexpr int kPerLane = (kPairs + 31) / 32;
-          float4 acc[kPerLane];
-#pragma unroll
-          for (int k = 0; k < kPerLane; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-          float Lx = 0.f;
-          for (int cb = 0; cb < nch; cb += kMergeBatch) {
-            const int nb = min(kMergeBatch, nch - cb);
-            for (int e = lane; e < nb * G; e += 32) {
-              const size_t idx = (e0 + (size_t)cb * G + e) * 2;
-              const float mc = __ldcg(ws_ml + idx);
-              const float wc = mc == -INFINITY ? 0.f : exp2f(mc - Mx);
-              sm.fin_w[e] = wc;
-              Lx += wc * __ldcg(ws_ml + idx + 1);
-            }
-            __syncwarp();
-#pragma unroll
-            for (int k = 0; k < kPerLane; ++k) {
-              const int pi = lane + 32 * k;
-              if (pi < kPairs) {
-                const int g = pi / (D / 4), d = (pi % (D / 4)) * 4;
-                const float* src = ws_o + (e0 + (size_t)cb * G + g) * D + d;
-#pragma unroll 4
-                for (int c = 0; c < nb; ++c) {
-                  const float wc = sm.fin_w[c * G + g];
-                  const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)c * G * D));
-                  acc[k].x += wc * v.x;
-                  acc[k].y += wc * v.y;
-                  acc[k].z += wc * v.z;
-                  acc[k].w += wc * v.w;
-                }
-              }
-            }
-            __syncwarp();
-          }
-#pragma unroll
-          for (int m = G; m < 32; m <<= 1) Lx += __shfl_xor_sync(0xffffffffu, Lx, m);
-#pragma unroll
-          for (int k = 0; k < kPerLane; ++k) {
-            const int pi = lane + 32 * k;
-            const int g = (pi < kPairs ? pi : 0) / (D / 4);
-            const float L = __shfl_sync(0xffffffffu, Lx, g);  // lane g holds head g's sum
-            if (pi < kPairs) {
-              const int d = (pi % (D / 4)) * 4;
-              const float inv = L > 0.f ? 1.f / L : 0.f;
-              uint2 pk;
-              pk.x = pack2(acc[k].x * inv, acc[k].y * inv);
-              pk.y = pack2(acc[k].z * inv, acc[k].w * inv);
-              *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
-            }
-          }
-          if (lane < G && lse_out)
-            lse_out[hrow + lane] = Lx > 0.f ? (Mx + log2f(Lx)) * kLn2T : -INFINITY;
-        }
-      }
     }
   } else {
     // ------------------------------ consumers -----------------------------------
@@ -448,39 +309,13 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     uint32_t qa[KS_D][2];
     float o[NT_D][4];
     float m_run = -INFINITY, l_run = 0.f;
-    int cur = -1, cur_bh = 0, n_ev = 0;
-    // hand this warp's state of the finished chunk to the finisher
-    auto dump = [&](int chunk, int bh) {
-      mbar_wait(&sm.red_free, (n_ev & 1) ^ 1, err);
-      float l = l_run;
-      l += __shfl_xor_sync(0xffffffffu, l, 1);
-      l += __shfl_xor_sync(0xffffffffu, l, 2);
-      if (qrow < G) {
-#pragma unroll
-        for (int n = 0; n < NT_D; ++n)
-          *reinterpret_cast<float2*>(&sm.red_o[warp][qrow][8 * n + qcol]) = make_float2(o[n][0], o[n][1]);
-        if (qcol == 0) {
-          sm.red_m[warp][qrow] = m_run;
-          sm.red_l[warp][qrow] = l;
-        }
-      }
-      if (warp == 0 && lane == 0) {
-        sm.red_chunk = chunk;
-        sm.red_bh = bh;
-      }
-      mbar_arrive(&sm.chunk_done);
-      ++n_ev;
-    };
+    int cur = -1, cur_bh = 0;
     for (int it = 0;; ++it) {
-      const int s = it % NST;
-      mbar_wait(&sm.full[s], (it / NST) & 1, err);
+      const int s = it % kStagesT;
+      mbar_wait(&sm.full[s], (it / kStagesT) & 1, err);
       const TileRef ti = sm.info[s];
-      if (ti.chunk < 0) {
-        if (cur >= 0) dump(cur, cur_bh);
-        break;
-      }
-      if (ti.chunk != cur) {
-        if (cur >= 0) dump(cur, cur_bh);
+      if (ti.chunk < 0) break;
+      if (ti.chunk != cur) {  // new chunk: its head's queries (staged), fresh state
         cur = ti.chunk;
         cur_bh = ti.bh;
         const __nv_bfloat16* qh = sm.qbuf[ti.qslot] + qrow * D;
@@ -489,7 +324,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           qa[k][0] = qrow < G ? *reinterpret_cast<const uint32_t*>(qh + 16 * k + qcol) : 0u;
           qa[k][1] = qrow < G ? *reinterpret_cast<const uint32_t*>(qh + 16 * k + 8 + qcol) : 0u;
         }
-        mbar_arrive(&sm.q_free[ti.qslot]);
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.q_free[ti.qslot]);
 #pragma unroll
         for (int n = 0; n < NT_D; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
         m_run = -INFINITY;
@@ -550,18 +386,156 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
+
+      if (ti.last) {
+        // ---- warps -> CTA ----------------------------------------------------------
+        float l = l_run;
+        l += __shfl_xor_sync(0xffffffffu, l, 1);
+        l += __shfl_xor_sync(0xffffffffu, l, 2);
+        if (qrow < G) {
+#pragma unroll
+          for (int n = 0; n < NT_D; ++n) {
+            sm.red_o[warp][qrow][8 * n + qcol] = o[n][0];
+            sm.red_o[warp][qrow][8 * n + qcol + 1] = o[n][1];
+          }
+          if (qcol == 0) {
+            sm.red_m[warp][qrow] = m_run;
+            sm.red_l[warp][qrow] = l;
+          }
+        }
+        named_bar_sync(1, kConsThreads);
+        const int bh = cur_bh;
+        const int b = bh / hkv, kh = bh % hkv;
+        const size_t hrow = (size_t)b * hkv * G + (size_t)kh * G;
+        const int nch = s_base[bh + 1] - s_base[bh];
+        for (int e = tid; e < G * D; e += kConsThreads) {
+          const int g = e / D, d = e % D;
+          float M = -INFINITY;
+#pragma unroll
+          for (int w = 0; w < kCons; ++w) M = fmaxf(M, sm.red_m[w][g]);
+          float O = 0.f, L = 0.f;
+#pragma unroll
+          for (int w = 0; w < kCons; ++w) {
+            const float mw = sm.red_m[w][g];
+            const float ww = mw == -INFINITY ? 0.f : exp2f(mw - M);
+            O += ww * sm.red_o[w][g][d];
+            L += ww * sm.red_l[w][g];
+          }
+          if (nch == 1) {
+            from_f32(L > 0.f ? O / L : 0.f, out + (hrow + g) * D + d);
+            if (d == 0 && lse_out) lse_out[hrow + g] = L > 0.f ? (M + log2f(L)) * kLn2T : -INFINITY;
+          } else {
+            ws_o[((size_t)cur * G + g) * D + d] = O;
+            if (d == 0) {
+              ws_ml[((size_t)cur * G + g) * 2 + 0] = M;
+              ws_ml[((size_t)cur * G + g) * 2 + 1] = L;
+            }
+          }
+        }
+        // red_* may be reused by the next chunk
+        named_bar_sync(1, kConsThreads);
+      }
     }
-    // no more chunks: tell the finisher
-    mbar_wait(&sm.red_free, (n_ev & 1) ^ 1, err);
-    if (warp == 0 && lane == 0) sm.red_chunk = -1;
-    mbar_arrive(&sm.chunk_done);
+  }
+  // the chunk prefix for the merge kernel (identical in every CTA; CTA 0 publishes it)
+  if (blockIdx.x == 0)
+    for (int i = tid; i <= n_heads; i += kThreadsT) ws_ctrl[n_heads + 2 + i] = s_base[i];
+}
+
+// Second kernel of a decode step: merges the chunk partials of every head that was
+// split (o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i), one CTA per (batch row, key
+// head).  Thread t works on the (chunk, head) pairs e = c*G + g with e = t (mod 128),
+// so its head is g = t % G; the outputs (head, 4 columns) are spread over the threads
+// and the chunk weights are staged in shared memory per batch.  It also clears the
+// work counter for the next decode launch.
+template <int D, int G>
+__global__ void __launch_bounds__(kMergeThreads)
+    decode_merge_kernel(int* __restrict__ ws_ctrl, const float* __restrict__ ws_ml,
+                        const float* __restrict__ ws_o, __nv_bfloat16* __restrict__ out,
+                        float* __restrict__ lse_out, int n_heads, int hkv) {
+  __shared__ float mrg_w[kMergeBatch * G];
+  __shared__ float part[kMergeThreads / 32][G];
+  __shared__ float Ms[G], Ls[G];
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int bh = blockIdx.x;
+  if (bh == 0 && tid == 0) ws_ctrl[n_heads] = 0;  // work counter of the next launch
+  const int* plan = ws_ctrl + n_heads + 2;
+  const int c0 = plan[bh], nch = plan[bh + 1] - c0;
+  if (nch <= 1) return;  // a single chunk wrote its output directly
+  const int b = bh / hkv, kh = bh % hkv;
+  const size_t hrow = (size_t)b * hkv * G + (size_t)kh * G;
+  const size_t e0 = (size_t)c0 * G;
+  float mx = -INFINITY;
+  for (int e = tid; e < nch * G; e += kMergeThreads) mx = fmaxf(mx, __ldcg(ws_ml + (e0 + e) * 2));
+#pragma unroll
+  for (int m = G; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
+  if (lane < G) part[warp][lane] = mx;
+  __syncthreads();
+  if (tid < G) {
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) M = fmaxf(M, part[w][tid]);
+    Ms[tid] = M;
   }
   __syncthreads();
-  if (tid == 0) {
-    const int d = atomicAdd(done_ctas, 1);
-    if (d == (int)gridDim.x - 1) {  // every CTA has stopped pulling work
-      *next_chunk = 0;
-      *done_ctas = 0;
+  constexpr int kPairs = G * D / 4;
+  constexpr int kPer = (kPairs + kMergeThreads - 1) / kMergeThreads;
+  float4 acc[kPer];
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
+  float lx = 0.f;
+  const float Mown = Ms[tid % G];
+  for (int cb = 0; cb < nch; cb += kMergeBatch) {
+    const int nb = min(kMergeBatch, nch - cb);
+    for (int e = tid; e < nb * G; e += kMergeThreads) {
+      const size_t idx = (e0 + (size_t)cb * G + e) * 2;
+      const float mc = __ldcg(ws_ml + idx);
+      const float wc = mc == -INFINITY ? 0.f : exp2f(mc - Mown);
+      mrg_w[e] = wc;
+      lx += wc * __ldcg(ws_ml + idx + 1);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int pi = tid + kMergeThreads * k;
+      if (pi < kPairs) {
+        const int g = pi / (D / 4), d = (pi % (D / 4)) * 4;
+        const float* src = ws_o + (e0 + (size_t)cb * G + g) * D + d;
+#pragma unroll 4
+        for (int c = 0; c < nb; ++c) {
+          const float wc = mrg_w[c * G + g];
+          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)c * G * D));
+          acc[k].x += wc * v.x;
+          acc[k].y += wc * v.y;
+          acc[k].z += wc * v.z;
+          acc[k].w += wc * v.w;
+        }
+      }
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int m = G; m < 32; m <<= 1) lx += __shfl_xor_sync(0xffffffffu, lx, m);
+  if (lane < G) part[warp][lane] = lx;
+  __syncthreads();
+  if (tid < G) {
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kMergeThreads / 32; ++w) L += part[w][tid];
+    Ls[tid] = L;
+    if (lse_out) lse_out[hrow + tid] = L > 0.f ? (Ms[tid] + log2f(L)) * kLn2T : -INFINITY;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int k = 0; k < kPer; ++k) {
+    const int pi = tid + kMergeThreads * k;
+    if (pi < kPairs) {
+      const int g = pi / (D / 4), d = (pi % (D / 4)) * 4;
+      const float L = Ls[g], inv = L > 0.f ? 1.f / L : 0.f;
+      uint2 pk;
+      pk.x = pack2(acc[k].x * inv, acc[k].y * inv);
+      pk.y = pack2(acc[k].z * inv, acc[k].w * inv);
+      *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
     }
   }
 }
@@ -589,20 +563,23 @@ bool map_bf16(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Control words at the front of the workspace: [n_heads] unused, work counter,
+// spare, chunk prefix [n_heads + 1] (written by the decode kernel for the merge).
+size_t ctrl_bytes_tc(int n_heads) { return ((size_t)(2 * n_heads + 3) * 4 + 255) / 256 * 256; }
+
 size_t max_chunks_tc(const spkv_params& p, int num_sms) {
   return (size_t)num_sms * kUnitsPerCta + (size_t)p.B * p.Hkv;
 }
 
-template <int D, int G, int NST>
-cudaError_t run_nst(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
+template <int D, int G>
+cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
                    const int32_t* t_pos, void* o, float* lse, void* ws, int num_sms,
                    cudaStream_t stream) {
-  using S = TcDecSmem<D, G, NST>;
-  const int n_heads_ = p.B * p.Hkv;
-  const size_t smem = sizeof(S) + 1024 + ((size_t)3 * n_heads_ + 1) * 4;
+  using S = TcDecSmem<D, G>;
+  const size_t smem = sizeof(S) + 1024 + ((size_t)3 * p.B * p.Hkv + 1) * 4;
   static int configured = 0;
   if ((int)smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, G, NST>,
+    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, G>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured = (int)smem;
@@ -612,7 +589,7 @@ cudaError_t run_nst(const spkv_params& p, const spkv_cache& c, const spkv_ring& 
   {
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.num_pages * kPageRows};
     const cuuint64_t str[1] = {(cuuint64_t)D * es};
-    const cuuint32_t box[2] = {64, kPageRows};  // one cache page per box; a tile takes two
+    const cuuint32_t box[2] = {64, kTileR};
     if (!map_bf16(&tkp, c.K_pool, 2, dims, str, box) || !map_bf16(&tvp, c.V_pool, 2, dims, str, box))
       return cudaErrorInvalidValue;
   }
@@ -626,27 +603,21 @@ cudaError_t run_nst(const spkv_params& p, const spkv_cache& c, const spkv_ring& 
   }
   const int n_heads = p.B * p.Hkv;
   char* w = static_cast<char*>(ws);
-  const size_t ctrl_bytes = ((size_t)(n_heads + 2) * 4 + 255) / 256 * 256;
+  const size_t ctrl_bytes = ctrl_bytes_tc(n_heads);
   const size_t ml_bytes = (max_chunks_tc(p, num_sms) * G * 2 * 4 + 255) / 256 * 256;
   CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
                c.page_table, c.count, c.max_pages_per_head};
-  decode_tc_kernel<D, G, NST><<<num_sms, kThreadsT, smem, stream>>>(
+  int* ctrl = reinterpret_cast<int*>(w);
+  float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
+  float* po = reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes);
+  decode_tc_kernel<D, G><<<num_sms, kThreadsT, smem, stream>>>(
       tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
-      static_cast<__nv_bfloat16*>(o), lse, reinterpret_cast<int*>(w),
-      reinterpret_cast<float*>(w + ctrl_bytes), reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes),
-      n_heads, p.Hkv, p.window, c.err_flag);
+      static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv, p.window, c.err_flag);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  decode_merge_kernel<D, G><<<n_heads, kMergeThreads, 0, stream>>>(
+      ctrl, ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
   return cudaGetLastError();
-}
-
-// Three stages when they fit in shared memory with the plan, else two.
-template <int D, int G>
-cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
-                   const int32_t* t_pos, void* o, float* lse, void* ws, int num_sms,
-                   cudaStream_t stream) {
-  const size_t plan = ((size_t)3 * p.B * p.Hkv + 1) * 4 + 1024;
-  if (sizeof(TcDecSmem<D, G, 3>) + plan <= 227 * 1024)
-    return run_nst<D, G, 3>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
-  return run_nst<D, G, 2>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
 }
 
 template <int D>
@@ -672,7 +643,7 @@ bool decode_tc_supported(const spkv_params& p) {
 size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms) {
   const int n_heads = p.B * p.Hkv;
   const int G = p.Hq / p.Hkv;
-  const size_t ctrl_bytes = ((size_t)(n_heads + 2) * 4 + 255) / 256 * 256;
+  const size_t ctrl_bytes = ctrl_bytes_tc(n_heads);
   const size_t mc = max_chunks_tc(p, num_sms);
   const size_t ml_bytes = (mc * G * 2 * 4 + 255) / 256 * 256;
   return ctrl_bytes + ml_bytes + mc * G * p.head_dim * 4;
