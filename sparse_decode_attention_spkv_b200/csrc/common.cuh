@@ -74,6 +74,37 @@ __device__ __forceinline__ float2 mul2(float2 a, float2 b) {
   return *reinterpret_cast<float2*>(&rd);
 }
 
+// ---- programmatic dependent launch ---------------------------------------------------
+// Kernels launched with launch_pdl may start while the previous kernel on the stream
+// is still running; each of them calls grid_dependency_wait() before it touches memory
+// that the previous kernel writes (the wait returns once that grid has completed and
+// its writes are visible).  grid_dependents_launch() lets the next such kernel start
+// its own launch early.  Both are no-ops for a kernel launched the ordinary way.
+
+__device__ __forceinline__ void grid_dependency_wait() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+__device__ __forceinline__ void grid_dependents_launch() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t stream, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // ---- time and bounded waits ------------------------------------------------------------
 
 __device__ __forceinline__ uint64_t global_ns() {

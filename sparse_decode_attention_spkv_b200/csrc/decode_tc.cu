@@ -50,7 +50,10 @@ constexpr int kStagesT = 4;
 constexpr int kUnitsPerCta = 4;      // target chunks per CTA
 constexpr int kMaxHeadsT = 2048;
 constexpr int kChunkPages = 256;     // page numbers staged per fetch
-constexpr int kMergeBatch = 128;     // partials whose weights are staged at once
+constexpr int kPgRegs = kChunkPages / 32;
+constexpr int kLookClaim = 4;        // tiles before a chunk's end: claim the next chunk
+constexpr int kLookPages = 2;        // ... and fetch its page-table entries
+constexpr int kMergeBatch = 8;       // partials a merge thread loads at once
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kLn2T = 0.6931471805599453f;
 constexpr float kSlackT = 8.f;
@@ -86,7 +89,7 @@ struct TcDecSmem {
   TileRef info[kStagesT];
   int red[kThreadsT];
   int misc[4];
-  // followed (dynamic) by rows[n_heads], live[n_heads], base[n_heads + 1]
+  // followed (dynamic) by rows[n_heads], live[n_heads], nw[n_heads], base[n_heads + 1]
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -140,6 +143,53 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
   return (uint32_t)(r * 128 + ((c ^ (r & 7)) << 4));
 }
 
+// One chunk of one head's key rows, in 64-row tiles: cache tiles k0 .. kc1-1 (page
+// list order), then the window slots.
+struct ChunkDesc {
+  int c;    // chunk id (>= total: no more work)
+  int bh;   // head: b * hkv + kh
+  int k0, k1, kc1;
+  int nl, nlp, nw;  // live cache rows, rounded up to tiles, window rows
+};
+
+__device__ __forceinline__ ChunkDesc describe_chunk(int c, int total, int chunk_rows,
+                                                    const int* s_base, const int* s_rows,
+                                                    const int* s_live, const int* s_nw,
+                                                    int n_heads, int hkv) {
+  ChunkDesc d;
+  d.c = c;
+  if (c >= total) {
+    d.bh = d.k0 = d.k1 = d.kc1 = d.nl = d.nlp = d.nw = 0;
+    return d;
+  }
+  int lo = 0, hi = n_heads - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (s_base[mid] <= c) lo = mid; else hi = mid - 1;
+  }
+  d.bh = lo;
+  const int r0 = (c - s_base[lo]) * chunk_rows;
+  const int r1 = min(s_rows[lo], r0 + chunk_rows);
+  d.nl = s_live[lo];
+  d.nlp = ((d.nl + kTileR - 1) / kTileR) * kTileR;
+  d.nw = s_nw[lo];
+  d.k0 = r0 / kTileR;
+  d.k1 = (r1 + kTileR - 1) / kTileR;
+  d.kc1 = min(d.k1, d.nlp / kTileR);
+  return d;
+}
+
+// Page numbers of a chunk's first kChunkPages cache tiles, lane-strided into registers
+// (the loads stay in flight until the registers are stored to shared memory).
+__device__ __forceinline__ void fetch_pages(int (&pg)[kPgRegs], const ChunkDesc& d,
+                                            const CacheView& cache, int lane) {
+#pragma unroll
+  for (int j = 0; j < kPgRegs; ++j) {
+    const int k = d.k0 + lane + 32 * j;
+    pg[j] = k < d.kc1 ? __ldg(cache.page_table + (size_t)d.bh * cache.max_pages + k) : 0;
+  }
+}
+
 template <int D, int G>
 __global__ void __launch_bounds__(kThreadsT, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kp,
@@ -160,9 +210,15 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   S& sm = *reinterpret_cast<S*>(smem_raw + pad);
   int* s_rows = reinterpret_cast<int*>(smem_raw + pad + sizeof(S));
   int* s_live = s_rows + n_heads;
-  int* s_base = s_live + n_heads;
+  int* s_nw = s_live + n_heads;
+  int* s_base = s_nw + n_heads;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* next_chunk = ws_ctrl + n_heads;  // reset by the merge kernel
+
+  // the merge kernel may be scheduled now (it waits for this grid to complete); the
+  // cache counts and the ring are written by the kernel before this one
+  grid_dependents_launch();
+  grid_dependency_wait();
 
   // ---- plan (identical in every CTA) ---------------------------------------------
   int my_rows = 0;
@@ -172,6 +228,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     const int nw = t + 1 < window ? t + 1 : window;
     const int rows = ((nl + kTileR - 1) / kTileR) * kTileR + nw;
     s_live[bh] = nl;
+    s_nw[bh] = nw;
     s_rows[bh] = rows;
     my_rows += rows;
   }
@@ -231,67 +288,78 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 
   if (warp == kCons) {
     // ------------------------------ producer ------------------------------------
+    // The whole warp walks the tiles; lane 0 issues the copies.  The next chunk is
+    // claimed kLookClaim tiles before the current one ends and its page-table entries
+    // are fetched into registers kLookPages tiles before the end, so neither the
+    // global atomic nor the page-table read stalls the stage ring between chunks.
     int it = 0;
-    for (int seq = 0;; ++seq) {
-      int c = 0;
-      if (lane == 0) c = atomicAdd(next_chunk, 1);
-      c = __shfl_sync(0xffffffffu, c, 0);
-      if (c >= total_chunks) break;
-      int lo = 0, hi = n_heads - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_base[mid] <= c) lo = mid; else hi = mid - 1;
-      }
-      const int bh = lo;
-      const int r0 = (c - s_base[bh]) * chunk_rows;
-      const int r1 = min(s_rows[bh], r0 + chunk_rows);
-      const int nl = s_live[bh];
-      const int nlp = ((nl + kTileR - 1) / kTileR) * kTileR;
-      const int b = bh / hkv, kh = bh % hkv;
-      const int t = __ldg(t_pos + b);
-      const int nw = t + 1 < window ? t + 1 : window;
-      const int k0 = r0 / kTileR, k1 = (r1 + kTileR - 1) / kTileR;
-      const int kc1 = min(k1, nlp / kTileR);  // cache tiles are k0 .. kc1-1
+    int c = 0;
+    if (lane == 0) c = atomicAdd(next_chunk, 1);
+    c = __shfl_sync(0xffffffffu, c, 0);
+    ChunkDesc cd = describe_chunk(c, total_chunks, chunk_rows, s_base, s_rows, s_live, s_nw,
+                                  n_heads, hkv);
+    int pg[kPgRegs];
+    fetch_pages(pg, cd, cache, lane);
+    for (int seq = 0; cd.c < total_chunks; ++seq) {
+      __syncwarp();
+#pragma unroll
+      for (int j = 0; j < kPgRegs; ++j) sm.pages[lane + 32 * j] = pg[j];
+      __syncwarp();
       const int qslot = seq & 1;
       if (lane == 0) mbar_wait(&sm.q_free[qslot], ((seq >> 1) & 1) ^ 1, err);
-      for (int ks = k0; ks < k1; ks += kChunkPages) {
-        const int ke = min(k1, ks + kChunkPages);
-        __syncwarp();
-        for (int i = ks + lane; i < min(ke, kc1); i += 32)
-          sm.pages[i - ks] = __ldg(cache.page_table + (size_t)bh * cache.max_pages + i);
-        __syncwarp();
+      int c_next = 0;
+      ChunkDesc nd;
+      nd.c = total_chunks;
+      const int k_claim = max(cd.k0, cd.k1 - kLookClaim);
+      const int k_pages = max(cd.k0, cd.k1 - kLookPages);
+      for (int k = cd.k0; k < cd.k1; ++k, ++it) {
+        if (k != cd.k0 && (k - cd.k0) % kChunkPages == 0) {
+          // a chunk longer than the staged page list: next segment, read in place
+          __syncwarp();
+          for (int i = lane; i < kChunkPages; i += 32) {
+            const int kk = k + i;
+            sm.pages[i] = kk < cd.kc1 ? __ldg(cache.page_table + (size_t)cd.bh * cache.max_pages + kk) : 0;
+          }
+          __syncwarp();
+        }
+        const int s = it % kStagesT;
+        mbar_wait(&sm.empty[s], ((it / kStagesT) & 1) ^ 1, err);
         if (lane == 0) {
-          for (int k = ks; k < ke; ++k, ++it) {
-            const int s = it % kStagesT;
-            mbar_wait(&sm.empty[s], ((it / kStagesT) & 1) ^ 1, err);
-            TB& tb = sm.st[s];
-            const bool from_cache = k < kc1;
-            const int slot = k * kTileR - nlp;
-            const int valid = from_cache ? min(kTileR, nl - k * kTileR) : min(kTileR, nw - slot);
-            // the tile description must be in place before the phase can complete
-            sm.info[s] = TileRef{c, bh, valid, k == k1 - 1, qslot};
-            const bool first = k == k0;
-            mbar_arrive_expect_tx(&sm.full[s], 2 * TB::kBytes + (first ? G * D * 2 : 0));
-            if (first)
-              bulk_g2s(sm.qbuf[qslot], q + ((size_t)b * hkv + kh) * G * D, G * D * 2, &sm.full[s]);
-            if (from_cache) {
-              const int page = sm.pages[k - ks];
+          TB& tb = sm.st[s];
+          const bool from_cache = k < cd.kc1;
+          const int slot = k * kTileR - cd.nlp;
+          const int valid = from_cache ? min(kTileR, cd.nl - k * kTileR) : min(kTileR, cd.nw - slot);
+          // the tile description must be in place before the phase can complete
+          sm.info[s] = TileRef{cd.c, cd.bh, valid, k == cd.k1 - 1, qslot};
+          const bool first = k == cd.k0;
+          mbar_arrive_expect_tx(&sm.full[s], 2 * TB::kBytes + (first ? G * D * 2 : 0));
+          if (first)
+            bulk_g2s(sm.qbuf[qslot], q + (size_t)cd.bh * G * D, G * D * 2, &sm.full[s]);
+          if (from_cache) {
+            const int page = sm.pages[(k - cd.k0) % kChunkPages];
 #pragma unroll
-              for (int hf = 0; hf < TB::kHalves; ++hf) {
-                tma2d(tb.k[hf], &tm_kp, hf * 64, page * kPageRows, &sm.full[s]);
-                tma2d(tb.v[hf], &tm_vp, hf * 64, page * kPageRows, &sm.full[s]);
-              }
-            } else {
+            for (int hf = 0; hf < TB::kHalves; ++hf) {
+              tma2d(tb.k[hf], &tm_kp, hf * 64, page * kPageRows, &sm.full[s]);
+              tma2d(tb.v[hf], &tm_vp, hf * 64, page * kPageRows, &sm.full[s]);
+            }
+          } else {
+            const int b = cd.bh / hkv, kh = cd.bh % hkv;
 #pragma unroll
-              for (int hf = 0; hf < TB::kHalves; ++hf) {
-                tma4d(tb.k[hf], &tm_kr, hf * 64, slot, kh, b, &sm.full[s]);
-                tma4d(tb.v[hf], &tm_vr, hf * 64, slot, kh, b, &sm.full[s]);
-              }
+            for (int hf = 0; hf < TB::kHalves; ++hf) {
+              tma4d(tb.k[hf], &tm_kr, hf * 64, slot, kh, b, &sm.full[s]);
+              tma4d(tb.v[hf], &tm_vr, hf * 64, slot, kh, b, &sm.full[s]);
             }
           }
+          if (k == k_claim) c_next = atomicAdd(next_chunk, 1);
         }
-        it = __shfl_sync(0xffffffffu, it, 0);
+        if (k == k_pages) {
+          c_next = __shfl_sync(0xffffffffu, c_next, 0);
+          nd = describe_chunk(c_next, total_chunks, chunk_rows, s_base, s_rows, s_live, s_nw,
+                              n_heads, hkv);
+          fetch_pages(pg, nd, cache, lane);
+        }
       }
+      cd = nd;
     }
     if (lane == 0) {
       const int s = it % kStagesT;
@@ -444,99 +512,77 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 
 // Second kernel of a decode step: merges the chunk partials of every head that was
 // split (o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i), one CTA per (batch row, key
-// head).  Thread t works on the (chunk, head) pairs e = c*G + g with e = t (mod 128),
-// so its head is g = t % G; the outputs (head, 4 columns) are spread over the threads
-// and the chunk weights are staged in shared memory per batch.  It also clears the
-// work counter for the next decode launch.
+// head).  Each thread owns 4 output columns of one query head and walks that head's
+// partials kMergeBatch at a time: the batch's loads are issued together, then folded
+// in with a running maximum, so a merge costs a few memory round trips.  Launched as
+// a programmatic dependent of the decode kernel: it waits for the decode grid to
+// complete before reading anything.  It also clears the work counter for the next
+// decode launch.
 template <int D, int G>
 __global__ void __launch_bounds__(kMergeThreads)
     decode_merge_kernel(int* __restrict__ ws_ctrl, const float* __restrict__ ws_ml,
                         const float* __restrict__ ws_o, __nv_bfloat16* __restrict__ out,
                         float* __restrict__ lse_out, int n_heads, int hkv) {
-  __shared__ float mrg_w[kMergeBatch * G];
-  __shared__ float part[kMergeThreads / 32][G];
-  __shared__ float Ms[G], Ls[G];
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dependency_wait();
+  grid_dependents_launch();
+  const int tid = threadIdx.x;
   const int bh = blockIdx.x;
   if (bh == 0 && tid == 0) ws_ctrl[n_heads] = 0;  // work counter of the next launch
   const int* plan = ws_ctrl + n_heads + 2;
-  const int c0 = plan[bh], nch = plan[bh + 1] - c0;
+  const int c0 = __ldcg(plan + bh), nch = __ldcg(plan + bh + 1) - c0;
   if (nch <= 1) return;  // a single chunk wrote its output directly
-  const int b = bh / hkv, kh = bh % hkv;
-  const size_t hrow = (size_t)b * hkv * G + (size_t)kh * G;
-  const size_t e0 = (size_t)c0 * G;
-  float mx = -INFINITY;
-  for (int e = tid; e < nch * G; e += kMergeThreads) mx = fmaxf(mx, __ldcg(ws_ml + (e0 + e) * 2));
+  const size_t hrow = (size_t)bh * G;  // == (b * hkv + kh) * G
+  constexpr int kVec = D / 4;
+  constexpr int kPairs = G * kVec;
 #pragma unroll
-  for (int m = G; m < 32; m <<= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, m));
-  if (lane < G) part[warp][lane] = mx;
-  __syncthreads();
-  if (tid < G) {
-    float M = -INFINITY;
+  for (int pi = tid; pi < kPairs; pi += kMergeThreads) {
+    const int g = pi / kVec, d = (pi % kVec) * 4;
+    float M = -INFINITY, L = 0.f;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int cb = 0; cb < nch; cb += kMergeBatch) {
+      float mv[kMergeBatch], lv[kMergeBatch];
+      float4 ov[kMergeBatch];
 #pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) M = fmaxf(M, part[w][tid]);
-    Ms[tid] = M;
-  }
-  __syncthreads();
-  constexpr int kPairs = G * D / 4;
-  constexpr int kPer = (kPairs + kMergeThreads - 1) / kMergeThreads;
-  float4 acc[kPer];
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) acc[k] = make_float4(0.f, 0.f, 0.f, 0.f);
-  float lx = 0.f;
-  const float Mown = Ms[tid % G];
-  for (int cb = 0; cb < nch; cb += kMergeBatch) {
-    const int nb = min(kMergeBatch, nch - cb);
-    for (int e = tid; e < nb * G; e += kMergeThreads) {
-      const size_t idx = (e0 + (size_t)cb * G + e) * 2;
-      const float mc = __ldcg(ws_ml + idx);
-      const float wc = mc == -INFINITY ? 0.f : exp2f(mc - Mown);
-      mrg_w[e] = wc;
-      lx += wc * __ldcg(ws_ml + idx + 1);
-    }
-    __syncthreads();
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int pi = tid + kMergeThreads * k;
-      if (pi < kPairs) {
-        const int g = pi / (D / 4), d = (pi % (D / 4)) * 4;
-        const float* src = ws_o + (e0 + (size_t)cb * G + g) * D + d;
-#pragma unroll 4
-        for (int c = 0; c < nb; ++c) {
-          const float wc = mrg_w[c * G + g];
-          const float4 v = __ldcg(reinterpret_cast<const float4*>(src + (size_t)c * G * D));
-          acc[k].x += wc * v.x;
-          acc[k].y += wc * v.y;
-          acc[k].z += wc * v.z;
-          acc[k].w += wc * v.w;
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const int c = cb + j;
+        if (c < nch) {
+          const size_t e = ((size_t)(c0 + c) * G + g);
+          mv[j] = __ldcg(ws_ml + e * 2);
+          lv[j] = __ldcg(ws_ml + e * 2 + 1);
+          ov[j] = __ldcg(reinterpret_cast<const float4*>(ws_o + e * D + d));
+        } else {
+          mv[j] = -INFINITY;
+          lv[j] = 0.f;
+          ov[j] = make_float4(0.f, 0.f, 0.f, 0.f);
         }
       }
+      float mb = M;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) mb = fmaxf(mb, mv[j]);
+      if (mb == -INFINITY) continue;
+      const float sc = M == -INFINITY ? 0.f : exp2f(M - mb);
+      acc.x *= sc;
+      acc.y *= sc;
+      acc.z *= sc;
+      acc.w *= sc;
+      L *= sc;
+#pragma unroll
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const float w = mv[j] == -INFINITY ? 0.f : exp2f(mv[j] - mb);
+        acc.x = fmaf(w, ov[j].x, acc.x);
+        acc.y = fmaf(w, ov[j].y, acc.y);
+        acc.z = fmaf(w, ov[j].z, acc.z);
+        acc.w = fmaf(w, ov[j].w, acc.w);
+        L = fmaf(w, lv[j], L);
+      }
+      M = mb;
     }
-    __syncthreads();
-  }
-#pragma unroll
-  for (int m = G; m < 32; m <<= 1) lx += __shfl_xor_sync(0xffffffffu, lx, m);
-  if (lane < G) part[warp][lane] = lx;
-  __syncthreads();
-  if (tid < G) {
-    float L = 0.f;
-#pragma unroll
-    for (int w = 0; w < kMergeThreads / 32; ++w) L += part[w][tid];
-    Ls[tid] = L;
-    if (lse_out) lse_out[hrow + tid] = L > 0.f ? (Ms[tid] + log2f(L)) * kLn2T : -INFINITY;
-  }
-  __syncthreads();
-#pragma unroll
-  for (int k = 0; k < kPer; ++k) {
-    const int pi = tid + kMergeThreads * k;
-    if (pi < kPairs) {
-      const int g = pi / (D / 4), d = (pi % (D / 4)) * 4;
-      const float L = Ls[g], inv = L > 0.f ? 1.f / L : 0.f;
-      uint2 pk;
-      pk.x = pack2(acc[k].x * inv, acc[k].y * inv);
-      pk.y = pack2(acc[k].z * inv, acc[k].w * inv);
-      *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
-    }
+    const float inv = L > 0.f ? 1.f / L : 0.f;
+    uint2 pk;
+    pk.x = pack2(acc.x * inv, acc.y * inv);
+    pk.y = pack2(acc.z * inv, acc.w * inv);
+    *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+    if (d == 0 && lse_out) lse_out[hrow + g] = L > 0.f ? (M + log2f(L)) * kLn2T : -INFINITY;
   }
 }
 
@@ -576,7 +622,7 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
                    const int32_t* t_pos, void* o, float* lse, void* ws, int num_sms,
                    cudaStream_t stream) {
   using S = TcDecSmem<D, G>;
-  const size_t smem = sizeof(S) + 1024 + ((size_t)3 * p.B * p.Hkv + 1) * 4;
+  const size_t smem = sizeof(S) + 1024 + ((size_t)4 * p.B * p.Hkv + 1) * 4;
   static int configured = 0;
   if ((int)smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, G>,
@@ -610,14 +656,13 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
   int* ctrl = reinterpret_cast<int*>(w);
   float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
   float* po = reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes);
-  decode_tc_kernel<D, G><<<num_sms, kThreadsT, smem, stream>>>(
-      tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
-      static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv, p.window, c.err_flag);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = launch_pdl(decode_tc_kernel<D, G>, dim3(num_sms), dim3(kThreadsT), smem, stream,
+                             tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
+                             static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv,
+                             p.window, c.err_flag);
   if (e != cudaSuccess) return e;
-  decode_merge_kernel<D, G><<<n_heads, kMergeThreads, 0, stream>>>(
-      ctrl, ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
-  return cudaGetLastError();
+  return launch_pdl(decode_merge_kernel<D, G>, dim3(n_heads), dim3(kMergeThreads), 0, stream, ctrl,
+                    ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
 }
 
 template <int D>

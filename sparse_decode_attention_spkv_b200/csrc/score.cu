@@ -179,6 +179,17 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
     mbar_init(&hbar, 1);
     fence_mbar_init();
   }
+  // the weights do not depend on the previous kernel: their loads are issued before
+  // waiting for it (programmatic dependent launch)
+  uint4 wv[kSmallMaxVec];
+  if (active) {
+    const uint4* wrow = reinterpret_cast<const uint4*>(W1 + (size_t)j * d_model);
+#pragma unroll
+    for (int i = 0; i < kSmallMaxVec; ++i)
+      if (i < nv) wv[i] = __ldg(wrow + lane + 32 * i);
+  }
+  grid_dependency_wait();
+  grid_dependents_launch();
   __syncthreads();
   if (tid == 0) {  // the tokens' hidden states: one contiguous block
     const uint32_t bytes = (uint32_t)nt * d_model * E::kSize;
@@ -186,13 +197,6 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
     const char* src = reinterpret_cast<const char*>(h + (size_t)tok0 * d_model);
     for (uint32_t off = 0; off < bytes; off += kBulkPiece)
       bulk_g2s(reinterpret_cast<char*>(hs) + off, src + off, min(kBulkPiece, bytes - off), &hbar);
-  }
-  uint4 wv[kSmallMaxVec];
-  if (active) {
-    const uint4* wrow = reinterpret_cast<const uint4*>(W1 + (size_t)j * d_model);
-#pragma unroll
-    for (int i = 0; i < kSmallMaxVec; ++i)
-      if (i < nv) wv[i] = __ldg(wrow + lane + 32 * i);
   }
   mbar_wait(&hbar, 0, nullptr);
 
@@ -280,10 +284,9 @@ cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const v
     configured_smem = (int)smem;
   }
   const int groups = (n_tok + NT - 1) / NT;
-  score_small_kernel<E, NT, APPEND><<<groups * kSmallRanks, kSmallThreads, smem, stream>>>(
-      static_cast<const T*>(h), n_tok, p.d_model, static_cast<const T*>(W1), b1, W2, b2, p.hid,
-      p.Hkv, p.tau, u_out, z_out, ap);
-  return cudaGetLastError();
+  return launch_pdl(score_small_kernel<E, NT, APPEND>, dim3(groups * kSmallRanks),
+                    dim3(kSmallThreads), smem, stream, static_cast<const T*>(h), n_tok, p.d_model,
+                    static_cast<const T*>(W1), b1, W2, b2, p.hid, p.Hkv, p.tau, u_out, z_out, ap);
 }
 
 template <bool APPEND>
