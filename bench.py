@@ -144,9 +144,10 @@ def _kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def _profiled_traffic():
+def _profiled_traffic(launch_bytes: float):
     """DRAM bytes per decode launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None)."""
+    on the current kernel source (else None).  The capture is one layer of the same
+    workload; its traffic is scaled to this launch by the algorithmic bytes."""
     path = os.path.join(ROOT, "profiles", "decode_attn_decode32k.md")
     if not os.path.exists(path):
         return None
@@ -159,7 +160,10 @@ def _profiled_traffic():
                 vals[k.strip()] = v.strip()
     if vals.get("source_hash") != want or "traffic_bytes_per_launch" not in vals:
         return None
-    return float(vals["traffic_bytes_per_launch"])
+    traffic = float(vals["traffic_bytes_per_launch"])
+    if "algorithmic_bytes_per_launch" in vals:
+        traffic *= launch_bytes / float(vals["algorithmic_bytes_per_launch"])
+    return traffic
 
 
 def run_gpu(args, world, rank, local):
@@ -257,7 +261,7 @@ def run_gpu(args, world, rank, local):
 
     peak, peak_kind = _peaks()
     achieved = launch_bytes / (attn_avg_ms / 1e3) / 1e9
-    traffic = _profiled_traffic()
+    traffic = _profiled_traffic(launch_bytes)
     tokens_s = world * p.B * K / (elapsed_max / 1e3)
     ms_step = elapsed_max / K
     live = sum(int(L.cache.count.sum().item()) for L in Ls)

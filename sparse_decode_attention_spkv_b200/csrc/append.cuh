@@ -91,4 +91,108 @@ __device__ __forceinline__ void decode_append_warp(const CacheMut& c, const Ring
   if (lane == 0) *zslot = z_new;
 }
 
+// ---- the same step split in two, for kernels that know the new gate late -------------
+//
+// append_prefetch issues every read of the step that does not depend on the new gate
+// (the old row in slot t % window and its gate, the head's count and current page, the
+// new k/v rows) with the old and new rows copied into `stage` (4 * row_bytes of shared
+// memory, 16-byte aligned) by cp.async; append_commit then writes the step once the gate
+// is known.  Together they do exactly what decode_append_warp does.
+struct AppendPre {
+  int t;     // query position (< 0: no step for this row)
+  int zs;    // stored gate of the retiring slot
+  int cnt;   // head's cache count before the step
+  int page;  // page holding row cnt when cnt is not at a page boundary
+};
+
+__device__ __forceinline__ void cp_async16(void* dst_smem, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst_smem)), "l"(src)
+               : "memory");
+}
+
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
+__device__ __forceinline__ AppendPre append_prefetch(const CacheMut& c, const RingMut& r, int bh,
+                                                     int b, int kh, int t, const char* k_new,
+                                                     const char* v_new, int hkv, int window,
+                                                     int row_bytes, int lane, char* stage) {
+  AppendPre a;
+  a.t = t;
+  a.zs = 0;
+  a.cnt = 0;
+  a.page = -1;
+  if (t < 0) return a;
+  const int slot = t % window;
+  const size_t ring_row = (size_t)bh * window + slot;
+  const int lpr = row_bytes >> 4;
+  for (int e = lane; e < 4 * lpr; e += 32) {
+    const int which = e / lpr, off = (e % lpr) * 16;
+    const char* src = which == 0   ? r.K + ring_row * row_bytes
+                      : which == 1 ? r.V + ring_row * row_bytes
+                      : which == 2 ? k_new + (size_t)bh * row_bytes
+                                   : v_new + (size_t)bh * row_bytes;
+    cp_async16(stage + which * row_bytes + off, src + off);
+  }
+  a.zs = r.z[((size_t)b * window + slot) * hkv + kh];
+  a.cnt = c.count[bh];
+  if (t - window >= 0 && a.zs && (a.cnt & 63) != 0 && (a.cnt >> 6) < c.max_pages)
+    a.page = c.page_table[(size_t)bh * c.max_pages + (a.cnt >> 6)];
+  return a;
+}
+
+__device__ __forceinline__ void append_commit(const CacheMut& c, const RingMut& r, const AppendPre& a,
+                                              int bh, int b, int kh, uint8_t z_new, int hkv,
+                                              int window, int row_bytes, int lane,
+                                              const char* stage) {
+  if (a.t < 0) return;
+  const int t = a.t;
+  const int slot = t % window;
+  const int s = t - window;
+  const int lpr = row_bytes >> 4;
+  const size_t ring_row = (size_t)bh * window + slot;
+  cp_async_wait_all();
+  __syncwarp();
+  if (s >= 0 && a.zs) {
+    const int i = a.cnt;
+    int page = a.page;
+    if ((i & 63) == 0) {
+      page = -1;
+      if (lane == 0) {
+        if ((i >> 6) >= c.max_pages) {
+          atomicOr(c.err, SPKV_FLAG_TABLE_FULL);
+        } else {
+          const int pg = atomicAdd(c.pool_top, 1);
+          if (pg >= c.num_pages) {
+            atomicOr(c.err, SPKV_FLAG_POOL_FULL);
+          } else {
+            page = pg;
+            c.page_table[(size_t)bh * c.max_pages + (i >> 6)] = pg;
+          }
+        }
+      }
+      page = __shfl_sync(0xffffffffu, page, 0);
+    }
+    if (page >= 0) {
+      const size_t drow = (size_t)page * kPageRows + (i & 63);
+      for (int e = lane; e < 2 * lpr; e += 32) {
+        const int which = e / lpr, off = (e % lpr) * 16;
+        const uint4 v = *reinterpret_cast<const uint4*>(stage + which * row_bytes + off);
+        *reinterpret_cast<uint4*>((which == 0 ? c.K : c.V) + drow * row_bytes + off) = v;
+      }
+      if (lane == 0) {
+        c.pos[drow] = s;
+        c.count[bh] = i + 1;
+      }
+    }
+  }
+  for (int e = lane; e < 2 * lpr; e += 32) {
+    const int which = e / lpr, off = (e % lpr) * 16;
+    const uint4 v = *reinterpret_cast<const uint4*>(stage + (2 + which) * row_bytes + off);
+    *reinterpret_cast<uint4*>((which == 0 ? r.K : r.V) + ring_row * row_bytes + off) = v;
+  }
+  if (lane == 0) r.z[((size_t)b * window + slot) * hkv + kh] = z_new;
+}
+
 }  // namespace spkv

@@ -303,6 +303,166 @@ cudaError_t dispatch_small(const spkv_params& p, const void* h, int n_tok, const
              : launch_small<F32, 16, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }
 
+// ---- few tokens, bf16, hid = 128: the first layer on tensor cores ---------------------
+//
+// h W1^T for up to 8 tokens is a skinny GEMM: M = 128 hidden units (W1 rows), N = 8
+// tokens, K = d_model.  A cluster of 8 CTAs takes 8 tokens; CTA rank r owns hidden
+// units 16r .. 16r+15 (one m16n8k16 row tile) and its 16 warps split K.  Inside each
+// pair of k-steps the K index is permuted the same way for W1 and h, so that a lane's
+// A and B fragments of both k-steps are 16 contiguous bytes of a W1 row or an h row
+// (one 16-byte load each, no shared-memory staging).  The K-split partials are summed
+// in shared memory, bias + GELU follow, and the 128 x 8 GELU outputs are all-gathered
+// into every CTA of the cluster with distributed shared-memory stores; rank n then
+// finishes token n (second layer in fp32, sigmoid, threshold).  W1 and W2 loads are
+// issued before the kernel waits for the preceding kernel on the stream.  With APPEND
+// the per-token ring/cache reads of the step are issued while the MLP runs and the
+// step is written once the gate is known.
+constexpr int kMmaRanks = 8;
+constexpr int kMmaWarps = 16;
+constexpr int kMmaThreads = kMmaWarps * 32;
+constexpr int kMmaTok = 8;          // tokens per cluster (the MMA's N)
+constexpr int kMmaHid = 16 * kMmaRanks;
+constexpr int kMmaMaxPairs = 8;     // 32-column k-step pairs per warp (d_model <= 4096)
+constexpr int kMmaMaxHkv = 16;
+constexpr int kMmaMaxRowBytes = 256;
+
+__device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+template <bool APPEND>
+__global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads, 1)
+    score_mma_kernel(const __nv_bfloat16* __restrict__ h, int n_tok, int d_model,
+                     const __nv_bfloat16* __restrict__ W1, const float* __restrict__ b1,
+                     const float* __restrict__ W2, const float* __restrict__ b2, int hkv,
+                     float tau, float* __restrict__ u_out, uint8_t* __restrict__ z_out,
+                     SmallAppend ap) {
+  __shared__ float red[kMmaWarps][16][kMmaTok];
+  __shared__ float xs[kMmaHid][kMmaTok];  // GELU outputs of all hidden units (all-gathered)
+  __shared__ __align__(16) char stage[APPEND ? kMmaMaxHkv : 1][4 * kMmaMaxRowBytes];
+  cg::cluster_group cluster = cg::this_cluster();
+  const int rank = (int)cluster.block_rank();
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int r = lane >> 2, q = lane & 3;
+  const int tok0 = (blockIdx.x / kMmaRanks) * kMmaTok;
+  const int nt = min(kMmaTok, n_tok - tok0);
+  const int pairs = d_model / (32 * kMmaWarps);
+  const int kbeg = warp * pairs * 32;
+
+  // weights first: they do not depend on the preceding kernel
+  uint4 a_lo[kMmaMaxPairs], a_hi[kMmaMaxPairs];
+  {
+    const __nv_bfloat16* w0 = W1 + (size_t)(16 * rank + r) * d_model + kbeg + 8 * q;
+    const __nv_bfloat16* w1 = w0 + (size_t)8 * d_model;
+#pragma unroll
+    for (int i = 0; i < kMmaMaxPairs; ++i) {
+      if (i < pairs) {
+        a_lo[i] = __ldg(reinterpret_cast<const uint4*>(w0 + 32 * i));
+        a_hi[i] = __ldg(reinterpret_cast<const uint4*>(w1 + 32 * i));
+      }
+    }
+  }
+  const int my_n = rank;  // token finished by this rank
+  float w2v[4];
+  float b2v = 0.f;
+  if (warp < hkv) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) w2v[i] = __ldg(W2 + (size_t)warp * kMmaHid + lane + 32 * i);
+    b2v = __ldg(b2 + warp);
+  }
+  const float b1v = tid < 16 * kMmaTok ? __ldg(b1 + 16 * rank + tid / kMmaTok) : 0.f;
+  grid_dependency_wait();
+  grid_dependents_launch();
+
+  AppendPre pre;
+  pre.t = -1;
+  if constexpr (APPEND) {
+    if (warp < hkv && my_n < nt) {
+      const int b = tok0 + my_n, bh = b * hkv + warp;
+      pre = append_prefetch(ap.c, ap.r, bh, b, warp, __ldg(ap.t_pos + b), ap.k_new, ap.v_new, hkv,
+                            ap.window, ap.row_bytes, lane, stage[warp]);
+    }
+  }
+
+  // first layer: this warp's K slice, tokens as the MMA's N
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  {
+    const bool tok_ok = r < nt;
+    const __nv_bfloat16* hp = h + (size_t)(tok0 + (tok_ok ? r : 0)) * d_model + kbeg + 8 * q;
+    uint4 bv[kMmaMaxPairs];
+#pragma unroll
+    for (int i = 0; i < kMmaMaxPairs; ++i)
+      if (i < pairs) bv[i] = tok_ok ? __ldg(reinterpret_cast<const uint4*>(hp + 32 * i)) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+    for (int i = 0; i < kMmaMaxPairs; ++i) {
+      if (i < pairs) {
+        mma_bf16_16816(acc, a_lo[i].x, a_hi[i].x, a_lo[i].y, a_hi[i].y, bv[i].x, bv[i].y);
+        mma_bf16_16816(acc, a_lo[i].z, a_hi[i].z, a_lo[i].w, a_hi[i].w, bv[i].z, bv[i].w);
+      }
+    }
+  }
+  red[warp][r][2 * q] = acc[0];
+  red[warp][r][2 * q + 1] = acc[1];
+  red[warp][r + 8][2 * q] = acc[2];
+  red[warp][r + 8][2 * q + 1] = acc[3];
+  __syncthreads();
+  if (tid < 16 * kMmaTok) {
+    const int j = tid / kMmaTok, n = tid % kMmaTok;
+    float a = b1v;
+#pragma unroll
+    for (int w = 0; w < kMmaWarps; ++w) a += red[w][j][n];
+    const float x = 0.5f * a * (1.f + erff(a * 0.70710678118654752440f));
+#pragma unroll
+    for (int dst = 0; dst < kMmaRanks; ++dst)
+      cluster.map_shared_rank(&xs[0][0], dst)[(16 * rank + j) * kMmaTok + n] = x;
+  }
+  cluster.sync();  // every rank now holds all 128 x 8 GELU outputs; no remote access follows
+
+  // second layer: token my_n, one warp per key head
+  if (warp < hkv && my_n < nt) {
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) sum = fmaf(xs[lane + 32 * i][my_n], w2v[i], sum);
+#pragma unroll
+    for (int m = 16; m > 0; m >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, m);
+    const float logit = sum + b2v;
+    const float uval = 1.f / (1.f + expf(-logit));
+    const uint8_t z = (uval >= tau) ? 1 : 0;
+    const size_t o = (size_t)(tok0 + my_n) * hkv + warp;
+    if (lane == 0) {
+      if (u_out) u_out[o] = uval;
+      z_out[o] = z;
+    }
+    if constexpr (APPEND) {
+      const int b = tok0 + my_n;
+      append_commit(ap.c, ap.r, pre, b * hkv + warp, b, warp, z, hkv, ap.window, ap.row_bytes,
+                    lane, stage[warp]);
+    }
+  }
+}
+
+bool mma_ok(const spkv_params& p, int n_tok) {
+  return p.dtype == SPKV_BF16 && p.hid == kMmaHid && p.d_model % (32 * kMmaWarps) == 0 &&
+         p.d_model / (32 * kMmaWarps) <= kMmaMaxPairs && p.Hkv <= kMmaMaxHkv &&
+         p.head_dim * 2 <= kMmaMaxRowBytes && n_tok >= 1 && n_tok <= 64;
+}
+
+template <bool APPEND>
+cudaError_t launch_mma(const spkv_params& p, const void* h, int n_tok, const void* W1,
+                       const float* b1, const float* W2, const float* b2, float* u_out,
+                       uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
+  const int groups = (n_tok + kMmaTok - 1) / kMmaTok;
+  return launch_pdl(score_mma_kernel<APPEND>, dim3(groups * kMmaRanks), dim3(kMmaThreads), 0,
+                    stream, static_cast<const __nv_bfloat16*>(h), n_tok, p.d_model,
+                    static_cast<const __nv_bfloat16*>(W1), b1, W2, b2, p.Hkv, p.tau, u_out, z_out,
+                    ap);
+}
+
 // The few-token kernel applies when the tokens fit in shared memory, every lane
 // holds whole 16-byte W1 vectors, and one warp per hidden unit covers a rank.
 bool small_ok(const spkv_params& p, int n_tok) {
@@ -319,6 +479,8 @@ bool small_ok(const spkv_params& p, int n_tok) {
 cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const void* W1,
                          const float* b1, const float* W2, const float* b2, float* u_out,
                          uint8_t* z_out, cudaStream_t stream) {
+  if (mma_ok(p, n_tok))
+    return launch_mma<false>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   if (small_ok(p, n_tok))
     return dispatch_small<false>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   dim3 grid((n_tok + kTok - 1) / kTok, kKS);
@@ -339,7 +501,8 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
                                 const float* b1, const float* W2, const float* b2,
                                 const void* k_new, const void* v_new, float* u_out,
                                 uint8_t* z_out, cudaStream_t stream) {
-  if (!small_ok(p, p.B)) {  // many rows: the two steps as separate launches
+  const bool mma = mma_ok(p, p.B);
+  if (!mma && !small_ok(p, p.B)) {  // many rows: the two steps as separate launches
     cudaError_t e = launch_score(p, h, p.B, W1, b1, W2, b2, u_out, z_out, stream);
     if (e != cudaSuccess) return e;
     return launch_decode_append(p, c, ring, t_pos, k_new, v_new, z_out, 1, stream);
@@ -349,6 +512,7 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
                  RingMut{static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win},
                  t_pos, static_cast<const char*>(k_new), static_cast<const char*>(v_new), p.window,
                  p.head_dim * esize};
+  if (mma) return launch_mma<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
   return dispatch_small<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }
 
