@@ -16,6 +16,10 @@ Learning When to Write by Predicting Future Utility" (arXiv 2605.14037):
                        query head h reads key head h // (Hq/Hkv), §1).
 * ``cache_rows``       §2.1 "efficient implementation at deployment": the
                        persistent cache holds exactly the KV pairs with z = 1.
+* ``rethreshold``      §3.3 (end of "Hybrids"): sparsity can be changed after the
+                       fact by changing the threshold; with the stored utility of
+                       every cached row, the cache for tau' keeps the rows with
+                       u >= tau' (rows dropped earlier cannot come back).
 
 Readings where the page is silent (each listed in the design notes):
 * f is one perceptron per layer, d_model -> hid -> Hkv, with a GELU (exact erf
@@ -133,3 +137,12 @@ def cache_rows(z_col: np.ndarray, upto: int) -> np.ndarray:
 def keep_fraction(z: np.ndarray) -> float:
     """Fraction of gated-in keys (the density statistic of §3.2)."""
     return float(np.mean(np.asarray(z, dtype=np.float64)))
+
+
+def rethreshold(cached_pos: np.ndarray, cached_u: np.ndarray, tau_new: float) -> np.ndarray:
+    """Post-hoc threshold change (§3.3) applied to one key head's cache: of the cached
+    positions (increasing) with their stored utilities, keep those with u >= tau_new,
+    in the same order.  Eq. (2) with the new threshold, restricted to what is stored."""
+    cached_pos = np.asarray(cached_pos, dtype=np.int64)
+    keep = np.asarray(cached_u, dtype=np.float64) >= float(tau_new)
+    return cached_pos[keep].astype(np.int32)

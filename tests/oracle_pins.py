@@ -249,9 +249,29 @@ def pin_cache_rows():
             assert set(np.nonzero(O.visible(t, s, z, w))[0].tolist()) == window | cached
 
 
+def pin_rethreshold():
+    """Post-hoc threshold change (§3.3): a hand example with a row exactly at the new
+    threshold (kept: Eq. (2) uses >=), the extremes, and the composition law: gating at
+    tau then re-thresholding at tau' gives the cache gated at max(tau, tau')."""
+    pos = np.array([2, 5, 7, 9], dtype=np.int32)
+    u = np.array([0.55, 0.7, 0.6, 0.9])
+    assert O.rethreshold(pos, u, 0.6).tolist() == [5, 7, 9]
+    assert O.rethreshold(pos, u, 0.95).tolist() == []
+    assert O.rethreshold(pos, u, 0.5).tolist() == [2, 5, 7, 9]
+    assert O.rethreshold(pos[:0], u[:0], 0.5).tolist() == []
+    rng = np.random.default_rng(11)
+    for _ in range(50):
+        T = int(rng.integers(1, 200))
+        uu = rng.random(T)
+        tau, tau2 = rng.random(2)
+        cached = O.cache_rows(O.gate(uu, tau), T)
+        again = O.rethreshold(cached, uu[cached], tau2)
+        assert again.tolist() == O.cache_rows(O.gate(uu, max(tau, tau2)), T).tolist()
+
+
 ALL_PINS = [
     pin_gelu_textbook, pin_gelu_library, pin_utility_zero_weights, pin_utility_hand_example,
     pin_utility_library, pin_gate_threshold, pin_gate_extremes, pin_keysets_golden,
     pin_two_key_softmax, pin_tau0_is_causal, pin_tau_gt1_is_sliding_window,
-    pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows,
+    pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows, pin_rethreshold,
 ]

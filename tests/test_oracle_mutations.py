@@ -63,6 +63,16 @@ def _gelu_wrong_scale(a):
     return 0.5 * a * (1 + erf(a))
 
 
+def _rethreshold_strict(cached_pos, cached_u, tau_new):
+    keep = np.asarray(cached_u, dtype=np.float64) > tau_new
+    return np.asarray(cached_pos)[keep].astype(np.int32)
+
+
+def _rethreshold_inverted(cached_pos, cached_u, tau_new):
+    keep = np.asarray(cached_u, dtype=np.float64) < tau_new
+    return np.asarray(cached_pos)[keep].astype(np.int32)
+
+
 _ORIG_ATTEND = O.attend
 _ORIG_LOGITS = O.utility_logits
 
@@ -77,6 +87,8 @@ MUTANTS = {
     "dropped_b1": ("utility_logits", _utility_no_b1),
     "sigmoid_sign": ("sigmoid", _sigmoid_flipped),
     "gqa_modulo_mapping": ("gated_attention", _gqa_modulo),
+    "rethreshold_strict_inequality": ("rethreshold", _rethreshold_strict),
+    "rethreshold_inverted": ("rethreshold", _rethreshold_inverted),
 }
 
 
