@@ -43,7 +43,7 @@ namespace {
 
 constexpr int kTileR = 64;           // rows per tile (one cache page)
 constexpr int kCons = 4;             // consumer warps, 16 rows each
-constexpr int kThreadsT = (kCons + 1) * 32;   // + producer
+constexpr int kThreadsT = (kCons + 2) * 32;   // + producer + finisher
 constexpr int kMergeThreads = 128;
 constexpr int kConsThreads = kCons * 32;
 constexpr int kStagesT = 4;
@@ -79,9 +79,13 @@ template <int D, int G>
 struct TcDecSmem {
   TileBuf<D> st[kStagesT];
   alignas(16) __nv_bfloat16 qbuf[2][G * D];
-  float red_o[kCons][G][D];
-  float red_m[kCons][G];
-  float red_l[kCons][G];
+  float red_o[2][kCons][G][D];  // per-warp chunk partials, two chunks in flight
+  float red_m[2][kCons][G];
+  float red_l[2][kCons][G];
+  int fin_chunk[2];
+  int fin_bh[2];
+  uint64_t cdone[2];   // consumers -> finisher: a chunk's partials are in red_*[parity]
+  uint64_t cfree[2];   // finisher -> consumers: red_*[parity] may be rewritten
   int pages[kChunkPages];
   uint64_t full[kStagesT];
   uint64_t empty[kStagesT];
@@ -242,6 +246,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     }
     mbar_init(&sm.q_free[0], kCons);
     mbar_init(&sm.q_free[1], kCons);
+    mbar_init(&sm.cdone[0], kConsThreads);
+    mbar_init(&sm.cdone[1], kConsThreads);
+    mbar_init(&sm.cfree[0], 1);
+    mbar_init(&sm.cfree[1], 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -293,9 +301,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     // are fetched into registers kLookPages tiles before the end, so neither the
     // global atomic nor the page-table read stalls the stage ring between chunks.
     int it = 0;
-    int c = 0;
-    if (lane == 0) c = atomicAdd(next_chunk, 1);
-    c = __shfl_sync(0xffffffffu, c, 0);
+    const int c = blockIdx.x;  // first chunk: static; later ones from the counter
     ChunkDesc cd = describe_chunk(c, total_chunks, chunk_rows, s_base, s_rows, s_live, s_nw,
                                   n_heads, hkv);
     int pg[kPgRegs];
@@ -350,7 +356,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
               tma4d(tb.v[hf], &tm_vr, hf * 64, slot, kh, b, &sm.full[s]);
             }
           }
-          if (k == k_claim) c_next = atomicAdd(next_chunk, 1);
+          if (k == k_claim) c_next = atomicAdd(next_chunk, 1) + (int)gridDim.x;
         }
         if (k == k_pages) {
           c_next = __shfl_sync(0xffffffffu, c_next, 0);
@@ -367,6 +373,64 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       sm.info[s].chunk = -1;
       mbar_arrive(&sm.full[s]);
     }
+  } else if (warp == kCons + 1) {
+    // ------------------------------ finisher ------------------------------------
+    // Combines the 4 consumer warps' partials of each finished chunk (max-weighted
+    // sums) and writes the head's output (single-chunk head) or the chunk partial for
+    // the merge kernel, while the consumers already work on the next chunk.
+    for (int nf = 0;; ++nf) {
+      const int par = nf & 1;
+      mbar_wait(&sm.cdone[par], (nf >> 1) & 1, err);
+      const int c = sm.fin_chunk[par];
+      if (c < 0) break;
+      const int bh = sm.fin_bh[par];
+      const size_t hrow = (size_t)bh * G;
+      const int nch = s_base[bh + 1] - s_base[bh];
+#pragma unroll
+      for (int g = 0; g < G; ++g) {
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kCons; ++w) M = fmaxf(M, sm.red_m[par][w][g]);
+        float wt[kCons], L = 0.f;
+#pragma unroll
+        for (int w = 0; w < kCons; ++w) {
+          const float mw = sm.red_m[par][w][g];
+          wt[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
+          L += wt[w] * sm.red_l[par][w][g];
+        }
+#pragma unroll
+        for (int d = 4 * lane; d < D; d += 128) {
+          float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+          for (int w = 0; w < kCons; ++w) {
+            const float4 v = *reinterpret_cast<const float4*>(&sm.red_o[par][w][g][d]);
+            O.x = fmaf(wt[w], v.x, O.x);
+            O.y = fmaf(wt[w], v.y, O.y);
+            O.z = fmaf(wt[w], v.z, O.z);
+            O.w = fmaf(wt[w], v.w, O.w);
+          }
+          if (nch == 1) {
+            const float inv = L > 0.f ? 1.f / L : 0.f;
+            uint2 pk;
+            pk.x = pack2(O.x * inv, O.y * inv);
+            pk.y = pack2(O.z * inv, O.w * inv);
+            *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+          } else {
+            *reinterpret_cast<float4*>(ws_o + ((size_t)c * G + g) * D + d) = O;
+          }
+        }
+        if (lane == 0) {
+          if (nch == 1) {
+            if (lse_out) lse_out[hrow + g] = L > 0.f ? (M + log2f(L)) * kLn2T : -INFINITY;
+          } else {
+            ws_ml[((size_t)c * G + g) * 2 + 0] = M;
+            ws_ml[((size_t)c * G + g) * 2 + 1] = L;
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.cfree[par]);
+    }
   } else {
     // ------------------------------ consumers -----------------------------------
     const float sc = kLog2eT * rsqrtf((float)D);
@@ -378,6 +442,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     float o[NT_D][4];
     float m_run = -INFINITY, l_run = 0.f;
     int cur = -1, cur_bh = 0;
+    int nfin = 0;  // chunks handed to the finisher
     for (int it = 0;; ++it) {
       const int s = it % kStagesT;
       mbar_wait(&sm.full[s], (it / kStagesT) & 1, err);
@@ -456,54 +521,35 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       if (lane == 0) mbar_arrive(&sm.empty[s]);
 
       if (ti.last) {
-        // ---- warps -> CTA ----------------------------------------------------------
+        // ---- this warp's chunk partial -> finisher ---------------------------------
         float l = l_run;
         l += __shfl_xor_sync(0xffffffffu, l, 1);
         l += __shfl_xor_sync(0xffffffffu, l, 2);
+        const int par = nfin & 1;
+        mbar_wait(&sm.cfree[par], ((nfin >> 1) & 1) ^ 1, err);
         if (qrow < G) {
 #pragma unroll
-          for (int n = 0; n < NT_D; ++n) {
-            sm.red_o[warp][qrow][8 * n + qcol] = o[n][0];
-            sm.red_o[warp][qrow][8 * n + qcol + 1] = o[n][1];
-          }
+          for (int n = 0; n < NT_D; ++n)
+            *reinterpret_cast<float2*>(&sm.red_o[par][warp][qrow][8 * n + qcol]) =
+                make_float2(o[n][0], o[n][1]);
           if (qcol == 0) {
-            sm.red_m[warp][qrow] = m_run;
-            sm.red_l[warp][qrow] = l;
+            sm.red_m[par][warp][qrow] = m_run;
+            sm.red_l[par][warp][qrow] = l;
           }
         }
-        named_bar_sync(1, kConsThreads);
-        const int bh = cur_bh;
-        const int b = bh / hkv, kh = bh % hkv;
-        const size_t hrow = (size_t)b * hkv * G + (size_t)kh * G;
-        const int nch = s_base[bh + 1] - s_base[bh];
-        for (int e = tid; e < G * D; e += kConsThreads) {
-          const int g = e / D, d = e % D;
-          float M = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < kCons; ++w) M = fmaxf(M, sm.red_m[w][g]);
-          float O = 0.f, L = 0.f;
-#pragma unroll
-          for (int w = 0; w < kCons; ++w) {
-            const float mw = sm.red_m[w][g];
-            const float ww = mw == -INFINITY ? 0.f : exp2f(mw - M);
-            O += ww * sm.red_o[w][g][d];
-            L += ww * sm.red_l[w][g];
-          }
-          if (nch == 1) {
-            from_f32(L > 0.f ? O / L : 0.f, out + (hrow + g) * D + d);
-            if (d == 0 && lse_out) lse_out[hrow + g] = L > 0.f ? (M + log2f(L)) * kLn2T : -INFINITY;
-          } else {
-            ws_o[((size_t)cur * G + g) * D + d] = O;
-            if (d == 0) {
-              ws_ml[((size_t)cur * G + g) * 2 + 0] = M;
-              ws_ml[((size_t)cur * G + g) * 2 + 1] = L;
-            }
-          }
+        if (warp == 0 && lane == 0) {
+          sm.fin_chunk[par] = cur;
+          sm.fin_bh[par] = cur_bh;
         }
-        // red_* may be reused by the next chunk
-        named_bar_sync(1, kConsThreads);
+        mbar_arrive(&sm.cdone[par]);
+        ++nfin;
       }
     }
+    // no more chunks: tell the finisher
+    const int par = nfin & 1;
+    mbar_wait(&sm.cfree[par], ((nfin >> 1) & 1) ^ 1, err);
+    if (warp == 0 && lane == 0) sm.fin_chunk[par] = -1;
+    mbar_arrive(&sm.cdone[par]);
   }
   // the chunk prefix for the merge kernel (identical in every CTA; CTA 0 publishes it)
   if (blockIdx.x == 0)

@@ -131,18 +131,21 @@ class DecodeStep:
         self.z = torch.empty((n, p.B, p.Hkv), dtype=torch.uint8, device=device)
 
     def launch(self, h, q, k, v, t, ev=None):
-        """h [L][B][D], q [L][B][Hq][d], k, v [L][B][Hkv][d], t [B]; ev: per-layer
-        (start, end) timing events around the decode-attention launch."""
+        """h [L][B][D], q [L][B][Hq][d], k, v [L][B][Hkv][d], t [B]; ev: {layer: (start,
+        end)} timing events around the decode-attention call of the listed layers (an
+        event between two launches keeps the second from starting early, so only a
+        sample of layers carries them)."""
         S, p = self.S, self.p
         for l, L in enumerate(self.layers):
             # score the new token, retire t - w, store the new token: one launch
             S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2, k[l],
                                        v[l], self.u[l], self.z[l])
-            if ev is not None:
-                ev[l][0].record()
+            e = ev.get(l) if ev else None
+            if e is not None:
+                e[0].record()
             S.spkv_decode_attn(p, L.cache, L.ring, q[l], t, self.o[l], self.lse[l], L.ws)
-            if ev is not None:
-                ev[l][1].record()
+            if e is not None:
+                e[1].record()
 
     LAUNCHES_PER_LAYER = 2
 
@@ -151,8 +154,11 @@ def kv_bytes(p, layers, t_min):
     """Algorithmic K/V bytes of one decode step: every head reads its live cache rows and
     its window rows once (K and V, bf16).  (The cache holds only rows <= t - w in the
     per-token schedule, so count is the live row count.)"""
-    total = 0
+    return sum(kv_bytes_layers(p, layers, t_min))
+
+
+def kv_bytes_layers(p, layers, t_min):
+    """kv_bytes per layer (a list)."""
     n_win = min(p.window, t_min + 1)
-    for L in layers:
-        total += int((L.cache.count.to(torch.int64) + n_win).sum().item())
-    return total * 2 * p.head_dim * 2
+    return [int((L.cache.count.to(torch.int64) + n_win).sum().item()) * 2 * p.head_dim * 2
+            for L in layers]
