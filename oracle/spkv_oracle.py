@@ -20,6 +20,11 @@ Learning When to Write by Predicting Future Utility" (arXiv 2605.14037):
                        fact by changing the threshold; with the stored utility of
                        every cached row, the cache for tau' keeps the rows with
                        u >= tau' (rows dropped earlier cannot come back).
+* ``soft_gate``        §2.1 "soft relaxation at training time", Eq. (5):
+                       alpha_s = sigmoid((u_s - tau) / beta).
+* ``soft_mask``        Eq. (6): additive score 0 inside the causal window,
+                       c (alpha_s - 1) outside it (and -inf for s > t: causal).
+* ``soft_gated_attention``  Eq. (3) with the mask of Eq. (6), every key s <= t.
 
 Readings where the page is silent (each listed in the design notes):
 * f is one perceptron per layer, d_model -> hid -> Hkv, with a GELU (exact erf
@@ -146,3 +151,47 @@ def rethreshold(cached_pos: np.ndarray, cached_u: np.ndarray, tau_new: float) ->
     cached_pos = np.asarray(cached_pos, dtype=np.int64)
     keep = np.asarray(cached_u, dtype=np.float64) >= float(tau_new)
     return cached_pos[keep].astype(np.int32)
+
+
+def soft_gate(u, tau: float, beta: float) -> np.ndarray:
+    """Eq. (5): the differentiable stand-in for z, alpha = sigmoid((u - tau) / beta)."""
+    return sigmoid((np.asarray(u, dtype=np.float64) - float(tau)) / float(beta))
+
+
+def soft_mask(t: int, s: np.ndarray, alpha: np.ndarray, w: int, c: float) -> np.ndarray:
+    """Eq. (6) for query t over keys s: 0 when 0 <= t - s < w (the causal window),
+    c (alpha_s - 1) for the older keys, -inf for keys after t (causal language model)."""
+    s = np.asarray(s, dtype=np.int64)
+    alpha = np.asarray(alpha, dtype=np.float64)
+    m = np.where(t - s < w, 0.0, float(c) * (alpha - 1.0))
+    return np.where(s <= t, m, -np.inf)
+
+
+def soft_gated_attention(Q, K, V, u, tau: float, beta: float, c: float, w: int, q_pos):
+    """Eqs. (3), (5), (6) for one batch row: softmax(q k^T / sqrt(d_k) + M_soft) V.
+
+    Q [n_q][Hq][d] at positions q_pos; K, V [T][Hkv][d]; u [T][Hkv] utilities.
+    Returns o [n_q][Hq][d] and lse [n_q][Hq] (natural log)."""
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    n_q, Hq, d = Q.shape
+    T, Hkv, _ = K.shape
+    G = Hq // Hkv
+    s = np.arange(T)
+    alpha = soft_gate(u, tau, beta)
+    o = np.zeros((n_q, Hq, d))
+    lse = np.zeros((n_q, Hq))
+    for i, t in enumerate(q_pos):
+        for hk in range(Hkv):
+            M = soft_mask(int(t), s, alpha[:, hk], w, c)
+            logits_k = K[:, hk] / np.sqrt(d)
+            for g in range(G):
+                h = hk * G + g
+                x = logits_k @ Q[i, h] + M
+                m = np.max(x)
+                p = np.exp(x - m)
+                l = np.sum(p)
+                o[i, h] = (p @ V[:, hk]) / l
+                lse[i, h] = m + np.log(l)
+    return o, lse

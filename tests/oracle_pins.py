@@ -269,9 +269,57 @@ def pin_rethreshold():
         assert again.tolist() == O.cache_rows(O.gate(uu, max(tau, tau2)), T).tolist()
 
 
+def pin_soft_gate_values():
+    """Eq. (5) at hand-picked points: u = tau gives 1/2; u - tau = +-beta gives the
+    logistic function at +-1; large |u - tau| / beta saturates to 0 or 1."""
+    g = O.soft_gate(np.array([0.5, 0.51, 0.49, 0.9, 0.1]), 0.5, 0.01)
+    _close(g[0], 0.5, 1e-15, "alpha at u = tau")
+    _close(g[1], 1.0 / (1.0 + math.exp(-1.0)), 1e-12, "alpha at u = tau + beta")
+    _close(g[2], 1.0 / (1.0 + math.exp(1.0)), 1e-12, "alpha at u = tau - beta")
+    _close(g[3:], [1.0, 0.0], 1e-15, "saturation")
+
+
+def pin_soft_two_key_closed_form():
+    """Eq. (6) by hand: one query at t = 1, w = 1, two keys with equal scores (q = 0);
+    key 0 lies outside the window and gets c (alpha - 1) with alpha = 1/2 (u = tau),
+    key 1 is the window.  With c = 2 the weights are e^{-1} : 1."""
+    Q = np.zeros((1, 1, 4))
+    K = np.zeros((2, 1, 4))
+    V = np.array([[[1.0, 0.0, 0.0, 0.0]], [[0.0, 1.0, 0.0, 0.0]]])
+    u = np.array([[0.5], [0.9]])
+    o, lse = O.soft_gated_attention(Q, K, V, u, 0.5, 0.01, 2.0, 1, [1])
+    e = math.exp(-1.0)
+    _close(o[0, 0], [e / (1 + e), 1 / (1 + e), 0.0, 0.0], 1e-12, "two-key soft mask")
+    _close(lse[0, 0], math.log(1 + e), 1e-12, "two-key lse")
+    # the key after the query never counts, whatever its utility
+    o2, _ = O.soft_gated_attention(Q, K, V, u, 0.5, 0.01, 2.0, 1, [0])
+    _close(o2[0, 0], [1.0, 0.0, 0.0, 0.0], 1e-15, "causal")
+
+
+def pin_soft_special_cases():
+    """c = 0 and w >= T reduce Eq. (6) to causal attention (torch SDPA, fp64); with a
+    vanishing temperature and utilities away from tau, the soft mask equals the hard
+    gate of Eq. (4) (the pinned ``gated_attention``)."""
+    rng = np.random.default_rng(21)
+    T, Hq, Hkv, d, w = 40, 4, 2, 16, 6
+    Q, K, V = _rand_qkv(rng, T, Hq, Hkv, d)
+    u = rng.random((T, Hkv))
+    u = np.where(np.abs(u - 0.5) < 0.02, u + 0.05, u)
+    causal = np.tril(np.ones((T, T), dtype=bool))
+    ref = _sdpa(Q, K, V, causal)
+    o, _ = O.soft_gated_attention(Q, K, V, u, 0.5, 0.01, 0.0, w, np.arange(T))
+    _close(o, ref, 1e-12, "c = 0 is causal attention")
+    o, _ = O.soft_gated_attention(Q, K, V, u, 0.5, 0.01, 1e6, T, np.arange(T))
+    _close(o, ref, 1e-12, "w >= T is causal attention")
+    o_soft, _ = O.soft_gated_attention(Q, K, V, u, 0.5, 1e-12, 1e6, w, np.arange(T))
+    o_hard, _ = O.gated_attention(Q, K, V, O.gate(u, 0.5), w, np.arange(T))
+    _close(o_soft, o_hard, 1e-12, "beta -> 0 is the hard gate")
+
+
 ALL_PINS = [
     pin_gelu_textbook, pin_gelu_library, pin_utility_zero_weights, pin_utility_hand_example,
     pin_utility_library, pin_gate_threshold, pin_gate_extremes, pin_keysets_golden,
     pin_two_key_softmax, pin_tau0_is_causal, pin_tau_gt1_is_sliding_window,
     pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows, pin_rethreshold,
+    pin_soft_gate_values, pin_soft_two_key_closed_form, pin_soft_special_cases,
 ]

@@ -41,7 +41,8 @@ def _utility_no_b1(h, W1, b1, W2, b2):
 
 
 def _sigmoid_flipped(x):
-    return 1.0 / (1.0 + np.exp(np.asarray(x, dtype=np.float64)))
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(np.asarray(x, dtype=np.float64)))
 
 
 def _gqa_modulo(Q, K, V, z, w, q_pos):
@@ -73,6 +74,27 @@ def _rethreshold_inverted(cached_pos, cached_u, tau_new):
     return np.asarray(cached_pos)[keep].astype(np.int32)
 
 
+def _soft_gate_flipped(u, tau, beta):
+    return O.sigmoid((float(tau) - np.asarray(u, dtype=np.float64)) / float(beta))
+
+
+def _soft_mask_window_off_by_one(t, s, alpha, w, c):
+    s = np.asarray(s, dtype=np.int64)
+    m = np.where(t - s <= w, 0.0, float(c) * (np.asarray(alpha) - 1.0))
+    return np.where(s <= t, m, -np.inf)
+
+
+def _soft_mask_sign(t, s, alpha, w, c):
+    s = np.asarray(s, dtype=np.int64)
+    m = np.where(t - s < w, 0.0, float(c) * (1.0 - np.asarray(alpha)))
+    return np.where(s <= t, m, -np.inf)
+
+
+def _soft_mask_acausal(t, s, alpha, w, c):
+    s = np.asarray(s, dtype=np.int64)
+    return np.where((t - s < w) & (t - s >= 0), 0.0, float(c) * (np.asarray(alpha) - 1.0))
+
+
 _ORIG_ATTEND = O.attend
 _ORIG_LOGITS = O.utility_logits
 
@@ -89,6 +111,10 @@ MUTANTS = {
     "gqa_modulo_mapping": ("gated_attention", _gqa_modulo),
     "rethreshold_strict_inequality": ("rethreshold", _rethreshold_strict),
     "rethreshold_inverted": ("rethreshold", _rethreshold_inverted),
+    "soft_gate_flipped": ("soft_gate", _soft_gate_flipped),
+    "soft_window_off_by_one": ("soft_mask", _soft_mask_window_off_by_one),
+    "soft_bias_sign": ("soft_mask", _soft_mask_sign),
+    "soft_not_causal": ("soft_mask", _soft_mask_acausal),
 }
 
 
