@@ -301,7 +301,10 @@ def run_gpu(args, world, rank, local):
     del Ls, inp, step
     torch.cuda.empty_cache()
     if not args.no_aux:
-        out["aux"] = {"prefill16k": measure_prefill(device, reps=3)}
+        out["aux"] = {"prefill16k": measure_prefill(device, reps=3),
+                      "rethreshold_decode32k": measure_rethreshold(device),
+                      "soft_attn_16k": measure_soft(device),
+                      "hybrid_3to1_decode32k": measure_hybrid(device)}
     return out
 
 
@@ -346,13 +349,14 @@ def measure_prefill(device, reps=3):
     def run(evs=None):
         for i in range(n_ch):
             S.spkv_score(p, hs[i], chunk, L.W1, L.b1, L.W2, L.b2, u, z)
-            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, ks[i], vs[i], z, src[i], chunk, chunk)
+            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, ks[i], vs[i], z, u, src[i], chunk,
+                                 chunk)
             if evs:
                 evs[i][0].record()
             S.spkv_prefill_attn(p, L.cache, L.ring, qs[i], ks[i], vs[i], i * chunk, chunk, o, lse)
             if evs:
                 evs[i][1].record()
-            S.spkv_ring_write(p, L.ring, ks[i], vs[i], z, chunk, src[i], chunk, chunk)
+            S.spkv_ring_write(p, L.ring, ks[i], vs[i], z, u, chunk, src[i], chunk, chunk)
 
     totals, attn = [], []
     for r in range(reps + 1):
@@ -395,6 +399,182 @@ def measure_prefill(device, reps=3):
                          "peak_kind": "measured (burst)" if txt else "fallback"},
             "density_nonlocal": float(sum(len(pp) for pp in pos)) / (wl.Hkv * T),
             "l2": "512 MB buffer written before each repetition"}
+
+
+def measure_rethreshold(device, reps=3):
+    """Secondary measurement: post-hoc re-threshold (in-place stable compaction of every
+    key head's cache by the stored utilities) of one decode32k layer at 32768-token
+    context from tau = 0.5 to the median stored utility (about half the rows stay).
+    The cache is restored from a device copy before each repetition (which also evicts
+    it from L2).  Algorithmic bytes: every stored row read once (K, V, position,
+    utility) and every kept row written once."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.states import build_decode_state
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+
+    wl = W.small_case("decode32k", layers=1)
+    p, Ls, _ = build_decode_state(wl, 1, 1, device, store_u=True)
+    L = Ls[0]
+    c = L.cache
+    saved = {k: getattr(c, k).clone() for k in ("K_pool", "V_pool", "pos_pool", "u_pool",
+                                                  "count", "count_prev", "page_table")}
+    z_saved = L.ring.z_win.clone()
+    # median utility of the stored rows (setup on the host side of the measurement)
+    n_rows = c.count.tolist()
+    vals = []
+    table = c.page_table.cpu()
+    for bh, n in enumerate(n_rows):
+        idx = torch.arange(n)
+        vals.append(c.u_pool[table[bh, idx // S.PAGE_ROWS].to(device).long(), (idx % S.PAGE_ROWS).to(device)])
+    tau_new = float(torch.cat(vals).median().item())
+    ws = S.alloc_rethreshold_workspace(p, c)
+    times = []
+    rows_before = int(saved["count"].sum().item())
+    rows_after = 0
+    for r in range(reps + 1):
+        for k, v in saved.items():
+            getattr(c, k).copy_(v)
+        L.ring.z_win.copy_(z_saved)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        S.spkv_cache_rethreshold(p, c, L.ring, tau_new, ws)
+        b.record()
+        torch.cuda.synchronize()
+        if r:
+            times.append(a.elapsed_time(b))
+        rows_after = int(c.count.sum().item())
+    status, flags = S.spkv_cache_check(c)
+    if status != S.OK:
+        raise RuntimeError(f"rethreshold measurement: {S.status_str(status)} flags={flags}")
+    row = 2 * p.head_dim * 2 + 8
+    nbytes = rows_before * row + rows_after * row
+    t = statistics.median(times) / 1e3
+    peak, peak_kind = _peaks()
+    return {"unit": "GB/s", "tau": [p.tau, tau_new], "rows_before": rows_before,
+            "rows_after": rows_after, "ms": t * 1e3, "algorithmic_bytes": nbytes,
+            "roofline": {"bound": "hbm", "kernel": "cache_rethreshold", "achieved": nbytes / t / 1e9,
+                         "peak": peak, "unit": "GB/s", "frac": nbytes / t / 1e9 / peak,
+                         "peak_kind": peak_kind}}
+
+
+def measure_soft(device, reps=3, beta=0.01, c=1e6):
+    """Secondary measurement: soft-gated training-time attention (Eqs. (5)-(6)) over one
+    16384-token sequence with the prefill16k shapes (32 query / 8 key heads, head_dim
+    128, RoPE'd q/k), the utilities from the utility perceptron of that workload.
+    FLOPs: every (query, key <= query) pair of every query head, QK^T and PV:
+    4 * head_dim * Hq * T (T + 1) / 2."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.inputs import device as D
+    from sparse_decode_attention_spkv_b200.inputs import gen
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+
+    wl = W.WORKLOADS["prefill16k"]
+    T = wl.ctx[0]
+    bf = torch.bfloat16
+    p = S.make_params(1, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau, S.BF16)
+    h = torch.empty((T, wl.d_model), dtype=bf, device=device)
+    q = torch.empty((1, T, wl.Hq, wl.head_dim), dtype=bf, device=device)
+    k = torch.empty((1, T, wl.Hkv, wl.head_dim), dtype=bf, device=device)
+    v = torch.empty_like(k)
+    D.fill_normal(h, wl.key(0, gen.T_H), 1.0)
+    D.fill_rope(q, wl.key(0, gen.T_Q), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_rope(k, wl.key(0, gen.T_K), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale)
+    W1 = torch.from_numpy(wl.w1(0)).to(bf).to(device)
+    u = torch.empty((T, wl.Hkv), dtype=torch.float32, device=device)
+    z = torch.empty((T, wl.Hkv), dtype=torch.uint8, device=device)
+    S.spkv_score(p, h, T, W1, torch.from_numpy(wl.b1(0)).to(device),
+                 torch.from_numpy(wl.w2(0)).to(device), torch.from_numpy(wl.b2(0)).to(device), u, z)
+    o = torch.empty_like(q)
+    lse = torch.empty((1, T, wl.Hq), dtype=torch.float32, device=device)
+    ws = torch.empty(S.spkv_soft_attn_workspace_bytes(p, T), dtype=torch.uint8, device=device)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=device)
+    times = []
+    for r in range(reps + 1):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        S.spkv_soft_attn(p, q, k, v, u, T, beta, c, o, lse, ws)
+        b.record()
+        torch.cuda.synchronize()
+        if r:
+            times.append(a.elapsed_time(b))
+    if not torch.isfinite(o.float()).all():
+        raise RuntimeError("soft attention: non-finite output")
+    flops = 4.0 * wl.head_dim * wl.Hq * T * (T + 1) / 2
+    t = statistics.median(times) / 1e3
+    peak_tf = _bf16_peak()
+    return {"unit": "TFLOP/s", "seq_len": T, "beta": beta, "c": c, "flops": flops,
+            "ms": t * 1e3, "roofline": {"bound": "tensor", "kernel": "soft_attn",
+                                        "achieved": flops / t / 1e12, "peak": peak_tf[0],
+                                        "unit": "TFLOP/s", "frac": flops / t / 1e12 / peak_tf[0],
+                                        "peak_kind": peak_tf[1]},
+            "l2": "512 MB buffer written before each repetition"}
+
+
+def _bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured (burst)"
+    return 1590.0, "fallback"
+
+
+def measure_hybrid(device, steps=10, warmup=3, period=4):
+    """Secondary measurement: per-token decode over a 32-layer hybrid local/global stack
+    (SP-KV page §3.3 "Hybrids"): every 4th layer global with the decode32k gated cache
+    (32768-token context; the 8 global layers are decode32k layers 0-7), the other 24
+    local (window of 128, no cache).  Same batch, heads and step as the headline
+    workload; graph-replayed steps timed with CUDA events."""
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200.inputs import device as D
+    from sparse_decode_attention_spkv_b200.inputs import gen
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    from sparse_decode_attention_spkv_b200.states import HybridStep, build_decode_state
+
+    wl = W.WORKLOADS[WORKLOAD]
+    n_layers = wl.layers
+    n_glob = n_layers // period
+    p, G, inp = build_decode_state(wl, n_glob, warmup + steps, device)
+    loc = []
+    for l in range(n_layers - n_glob):
+        L = R.Layer.create_local(p, device)
+        D.fill_normal(L.ring.K_win, wl.key(l, gen.T_K), wl.qkv_scale)
+        D.fill_normal(L.ring.V_win, wl.key(l, gen.T_V), wl.qkv_scale)
+        loc.append(L)
+    step = HybridStep(p, G, loc, period, device)
+    graphs = []
+    for i in range(warmup + steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
+        graphs.append(g)
+    torch.cuda.synchronize()
+    for i in range(warmup):
+        graphs[i].replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(warmup, warmup + steps):
+        graphs[i].replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    for L in G:
+        status, flags = S_check(L)
+        if status:
+            raise RuntimeError(f"hybrid measurement: cache error {flags}")
+    del graphs
+    return {"unit": "tokens/s", "value": p.B / (ms / 1e3), "ms_per_step": ms,
+            "layers": {"global": n_glob, "local": n_layers - n_glob, "period": period},
+            "launches_per_step": 2 * n_layers}
+
+
+def S_check(L):
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    status, flags = S.spkv_cache_check(L.cache)
+    return (0 if status == S.OK else status), flags
 
 
 # -------------------------------------------------------------- CPU oracle arm -----

@@ -94,6 +94,8 @@ typedef struct spkv_cache {
   int32_t* count_prev; /* [B*Hkv] value of count before the last chunk append */
   int32_t* pool_top;   /* [1] next free page */
   uint32_t* err_flag;  /* [1] SPKV_FLAG_* bits, sticky until spkv_cache_reset */
+  float* u_pool;       /* [num_pages][page_rows] utility u (Eq. (1)) of every stored row, or
+                          NULL: utilities are not kept (spkv_cache_rethreshold needs them) */
   int num_pages;
   int page_rows; /* must be 64 */
   int max_pages_per_head;
@@ -101,11 +103,14 @@ typedef struct spkv_cache {
 
 /* Local window (Eq. (4), 1_win): the last `window` keys/values of every
  * (batch row, key head), position p in slot p % window; z_win holds the gate of
- * the token in each slot (for retirement into the cache). */
+ * the token in each slot (for retirement into the cache).  u_win (optional) holds
+ * the utility of a slot's token while its retirement is pending, and NaN (all bits
+ * set) when the token is not pending (already cached, or not yet scored). */
 typedef struct spkv_ring {
   void* K_win;    /* [B][Hkv][window][head_dim] dtype */
   void* V_win;    /* [B][Hkv][window][head_dim] dtype */
   uint8_t* z_win; /* [B][window][Hkv] */
+  float* u_win;   /* [B][window][Hkv] f32, or NULL */
 } spkv_ring;
 
 /* Static text for a status code. */
@@ -115,7 +120,7 @@ const char* spkv_status_str(int status);
 int spkv_version(void);
 
 /* Zero the cache (count, count_prev, pool_top, err_flag), set page_table to -1
- * and, if ring is not NULL, zero its z_win. */
+ * and, if ring is not NULL, zero its z_win and set its u_win (if any) to NaN. */
 int spkv_cache_reset(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                      spkv_stream_t stream);
 
@@ -136,33 +141,39 @@ int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, c
 
 /* a2 -- stream compaction (§2.1 deployment): for every (b, key head), append the
  * rows i in [0, n_rows) with z = 1, in increasing i, to the cache, recording
- * position src_pos[b] + i.
+ * position src_pos[b] + i (and utility u[b][i][kh] when cache->u_pool is set).
  *   src_kind SPKV_SRC_CHUNK: K_src/V_src [B][src_batch_rows][Hkv][head_dim];
  *   src_kind SPKV_SRC_RING: rows are read from ring->K_win/V_win (K_src/V_src
  *     ignored), row i of batch b from slot (src_pos[b] + i) % window; requires
  *     n_rows <= window.
- * z [B][src_batch_rows][Hkv] uint8 (device); src_pos [B] int32 (device).
+ * z [B][src_batch_rows][Hkv] uint8, u [B][src_batch_rows][Hkv] f32 (required when
+ * cache->u_pool is not NULL, else ignored); src_pos [B] int32; all device.
  * Positions must exceed those already stored for that head.  Rows that do not fit
  * are dropped and flagged in err_flag.  Two kernels: plan (page allocation), then
  * scatter. */
 int spkv_write_compact(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                        int src_kind, const void* K_src, const void* V_src, const uint8_t* z,
-                       const int32_t* src_pos, int n_rows, int src_batch_rows,
+                       const float* u, const int32_t* src_pos, int n_rows, int src_batch_rows,
                        spkv_stream_t stream);
 
 /* a2 + a3 for one decode step per batch row (per-token retirement): with
  * t = t_pos[b], if retire != 0 and t - window >= 0, the token s = t - window
  * leaves the window; it is appended to the cache if its gate (ring->z_win of its
- * slot) is 1.  Then k_new, v_new (and z_new, if not NULL; else 0) are stored in
- * slot t % window.  k_new, v_new [B][Hkv][head_dim] dtype; z_new [B][Hkv] uint8;
- * t_pos [B] int32, all device. */
+ * slot) is 1 (with its utility from ring->u_win when cache->u_pool is set).  Then
+ * k_new, v_new (and z_new, if not NULL; else 0) are stored in slot t % window, and
+ * u_new in ring->u_win if that is set (NaN when z_new is NULL).  k_new, v_new
+ * [B][Hkv][head_dim] dtype; z_new [B][Hkv] uint8; u_new [B][Hkv] f32 (required when
+ * ring->u_win and z_new are set); t_pos [B] int32, all device.  cache may be NULL for
+ * a window-only layer (a local layer of a hybrid local/global stack, §3.3
+ * "Hybrids": it keeps no long-range cache); retire must then be 0. */
 int spkv_decode_append(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                        const int32_t* t_pos, const void* k_new, const void* v_new,
-                       const uint8_t* z_new, int retire, spkv_stream_t stream);
+                       const uint8_t* z_new, const float* u_new, int retire,
+                       spkv_stream_t stream);
 
 /* a1 + a2 + a3 fused for one per-token decode step: the same result as spkv_score on
  * the B new tokens (h [B][d_model], one per batch row, at positions t_pos) followed by
- * spkv_decode_append(..., z_new = z_out, retire = 1).  The warp that finishes the gate
+ * spkv_decode_append(..., z_new = z_out, u_new = u_out, retire = 1).  The warp that finishes the gate
  * of (batch row b, key head kh) also retires token t-window of (b, kh) and stores the
  * new token, so the step costs one launch.  u_out [B][Hkv] (may be NULL), z_out
  * [B][Hkv] as in spkv_score; k_new, v_new [B][Hkv][head_dim]. */
@@ -176,10 +187,12 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* cache, cons
  * batch b (position src_pos[b] + i) goes to slot (src_pos[b] + i) % window.  The
  * slot's gate is 0 for rows i < gated_from (already in the cache, so retiring them
  * appends nothing) and z_src[b][i][kh] for the others (z_src may be NULL when
- * gated_from >= n_rows).  K_src/V_src [B][src_batch_rows][Hkv][head_dim],
- * z_src [B][src_batch_rows][Hkv]. */
+ * gated_from >= n_rows); ring->u_win, if set, gets NaN for the former and
+ * u_src[b][i][kh] for the latter (u_src is then required when gated_from < n_rows).
+ * K_src/V_src [B][src_batch_rows][Hkv][head_dim], z_src [B][src_batch_rows][Hkv],
+ * u_src [B][src_batch_rows][Hkv] f32. */
 int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
-                    const void* V_src, const uint8_t* z_src, int gated_from,
+                    const void* V_src, const uint8_t* z_src, const float* u_src, int gated_from,
                     const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream);
 
 /* Bytes of decode workspace spkv_decode_attn needs for this cache geometry.  The
@@ -194,7 +207,9 @@ size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* cache
  * Split-K over balanced chunks of rows (a5: the chunk partials of a head are
  * combined by their log-sum-exp weights in a second kernel on the same stream).
  * q [B][Hq][head_dim] dtype; o [B][Hq][head_dim] dtype; lse [B][Hq] f32 natural
- * log (may be NULL).  The token t itself must already be in the ring. */
+ * log (may be NULL).  The token t itself must already be in the ring.  cache may be
+ * NULL: a window-only layer (the local layers of a hybrid stack, §3.3 "Hybrids"),
+ * whose keys are the window slots alone. */
 int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                      const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
                      size_t ws_bytes, spkv_stream_t stream);
@@ -234,10 +249,53 @@ int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* cache,
  * cache rows with position <= t - window (the cache may already hold rows of
  * this chunk; those are used only by queries they have left the window of).
  * q [B][chunk_len][Hq][head_dim]; K_chunk, V_chunk [B][chunk_len][Hkv][head_dim];
- * o [B][chunk_len][Hq][head_dim]; lse [B][chunk_len][Hq] f32 (may be NULL). */
+ * o [B][chunk_len][Hq][head_dim]; lse [B][chunk_len][Hq] f32 (may be NULL).  cache
+ * may be NULL for a window-only layer. */
 int spkv_prefill_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                       const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
                       int chunk_len, void* o, float* lse, spkv_stream_t stream);
+
+/* Bytes of workspace spkv_cache_rethreshold needs for this cache geometry.  The
+ * workspace must be zero-filled once before its first use; the library leaves its
+ * work counter at zero after every call.  Calls sharing a workspace must not overlap. */
+size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* cache);
+
+/* Post-hoc re-threshold ("Self-Pruned Key-Value Attention", §3.3: at inference the
+ * sparsity can be changed after the fact by changing the threshold): every key head
+ * keeps exactly its cache rows whose stored utility satisfies u >= tau_new, in their
+ * order (an in-place stable compaction inside the head's pages), and count and
+ * count_prev become the kept count.  Rows removed earlier are not recovered, so a
+ * tau_new below the threshold the rows were gated with removes nothing.  Pages a head
+ * no longer fills stay in its page list and are reused by its later appends (they
+ * are not returned to the pool).  If ring and ring->u_win are set, every slot's gate
+ * becomes z = 1[u_win >= tau_new] (NaN slots: 0), so the tokens still in the window
+ * retire under the new threshold; later scoring should be given tau_new in p.
+ * Requires cache->u_pool.  Three kernels (plan, move, finish); a bounded wait inside
+ * the move kernel that gives up latches SPKV_FLAG_TIMEOUT and skips its writes. */
+int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
+                           float tau_new, void* workspace, size_t ws_bytes,
+                           spkv_stream_t stream);
+
+/* Bytes of workspace spkv_soft_attn needs (a per-key bias buffer). */
+size_t spkv_soft_attn_workspace_bytes(const spkv_params* p, int seq_len);
+
+/* Soft-gated attention of SP-KV training ("Self-Pruned Key-Value Attention", §2.1,
+ * soft relaxation at training time), forward pass over whole sequences:
+ *   alpha_s = sigmoid((u_s - tau) / beta)                                  (Eq. (5))
+ *   M(t,s)  = 0 if 0 <= t-s < window, c (alpha_s - 1) if s <= t-window,
+ *             -inf if s > t                                                 (Eq. (6))
+ *   o_t     = softmax_s(q_t . k_s / sqrt(head_dim) + M(t,s)) v_s             (Eq. (3))
+ * for every batch row, query head and position t < seq_len (GQA grouping as
+ * elsewhere; tau and window from p).  No key is skipped: this is the dense training
+ * form; the backward pass is not provided.
+ * q [B][seq_len][Hq][head_dim], K, V [B][seq_len][Hkv][head_dim] dtype, u
+ * [B][seq_len][Hkv] f32 (e.g. from spkv_score), o like q, lse [B][seq_len][Hq] f32
+ * natural log (may be NULL).  workspace: spkv_soft_attn_workspace_bytes, no
+ * initialisation needed.  beta > 0, c >= 0.  err_flag (may be NULL) latches
+ * SPKV_FLAG_TIMEOUT if a bounded wait inside the kernel gives up. */
+int spkv_soft_attn(const spkv_params* p, const void* q, const void* K, const void* V,
+                   const float* u, int seq_len, float beta, float c, void* o, float* lse,
+                   void* workspace, size_t ws_bytes, uint32_t* err_flag, spkv_stream_t stream);
 
 #ifdef __cplusplus
 }

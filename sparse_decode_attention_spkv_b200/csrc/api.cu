@@ -1,6 +1,7 @@
 // api.cu -- the C ABI (include/spkv.h): host-side validation, then launches.
 // Validation touches no CUDA API, so argument errors are reported without a GPU.
 #include <cuda_runtime.h>
+#include <math.h>
 #include <stdint.h>
 
 #include <mutex>
@@ -42,6 +43,13 @@ bool cache_ok(const spkv_params* p, const spkv_cache* c) {
 
 bool ring_ok(const spkv_ring* r) {
   return r && r->K_win && r->V_win && r->z_win && aligned16(r->K_win) && aligned16(r->V_win);
+}
+
+// A layer without a persistent cache (window-only, e.g. the local layers of a hybrid
+// local/global stack) passes cache == NULL; the kernels see an all-zero cache.
+const spkv_cache& cache_or_none(const spkv_cache* c) {
+  static const spkv_cache none = {};
+  return c ? *c : none;
 }
 
 int sm_count() {
@@ -89,6 +97,8 @@ int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring*
   if (e == cudaSuccess) e = cudaMemsetAsync(c->pool_top, 0, 4, s);
   if (e == cudaSuccess) e = cudaMemsetAsync(c->err_flag, 0, 4, s);
   if (e == cudaSuccess && ring) e = cudaMemsetAsync(ring->z_win, 0, (size_t)p->B * p->window * p->Hkv, s);
+  if (e == cudaSuccess && ring && ring->u_win)  // NaN: no pending utility
+    e = cudaMemsetAsync(ring->u_win, 0xff, (size_t)p->B * p->window * p->Hkv * 4, s);
   return status_of(e);
 }
 
@@ -119,11 +129,12 @@ int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, c
 
 int spkv_write_compact(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                        int src_kind, const void* K_src, const void* V_src, const uint8_t* z,
-                       const int32_t* src_pos, int n_rows, int src_batch_rows,
+                       const float* u, const int32_t* src_pos, int n_rows, int src_batch_rows,
                        spkv_stream_t stream) {
   if (!params_ok(p) || !cache_ok(p, c) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
   if (n_rows == 0) return SPKV_OK;
   if (!z || !src_pos) return SPKV_ERR_ARG;
+  if (c->u_pool && !u) return SPKV_ERR_ARG;
   if (src_kind == SPKV_SRC_CHUNK) {
     if (!K_src || !V_src || !aligned16(K_src) || !aligned16(V_src)) return SPKV_ERR_ARG;
   } else if (src_kind == SPKV_SRC_RING) {
@@ -131,17 +142,20 @@ int spkv_write_compact(const spkv_params* p, const spkv_cache* c, const spkv_rin
   } else {
     return SPKV_ERR_ARG;
   }
-  return status_of(spkv::launch_write_compact(*p, *c, ring, src_kind, K_src, V_src, z, src_pos,
+  return status_of(spkv::launch_write_compact(*p, *c, ring, src_kind, K_src, V_src, z, u, src_pos,
                                               n_rows, src_batch_rows,
                                               static_cast<cudaStream_t>(stream)));
 }
 
 int spkv_decode_append(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                        const int32_t* t_pos, const void* k_new, const void* v_new,
-                       const uint8_t* z_new, int retire, spkv_stream_t stream) {
-  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+                       const uint8_t* z_new, const float* u_new, int retire,
+                       spkv_stream_t stream) {
+  if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!c && retire) return SPKV_ERR_ARG;  // nowhere to retire into
   if (!t_pos || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
-  return status_of(spkv::launch_decode_append(*p, *c, *ring, t_pos, k_new, v_new, z_new, retire,
+  if (ring->u_win && z_new && !u_new) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_decode_append(*p, cache_or_none(c), *ring, t_pos, k_new, v_new, z_new, u_new, retire,
                                               static_cast<cudaStream_t>(stream)));
 }
 
@@ -154,20 +168,22 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const sp
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (!t_pos || !h || !W1 || !b1 || !W2 || !b2 || !k_new || !v_new || !z_out) return SPKV_ERR_ARG;
   if (!aligned16(h) || !aligned16(W1) || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
+  if (ring->u_win && !u_out) return SPKV_ERR_ARG;
   if (!spkv::score_supported(*p)) return SPKV_ERR_UNSUPPORTED;
   return status_of(spkv::launch_score_append(*p, *c, *ring, t_pos, h, W1, b1, W2, b2, k_new, v_new,
                                              u_out, z_out, static_cast<cudaStream_t>(stream)));
 }
 
 int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
-                    const void* V_src, const uint8_t* z_src, int gated_from,
+                    const void* V_src, const uint8_t* z_src, const float* u_src, int gated_from,
                     const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream) {
   if (!params_ok(p) || !ring_ok(ring) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
   if (n_rows == 0) return SPKV_OK;
   if (!K_src || !V_src || !src_pos || !aligned16(K_src) || !aligned16(V_src)) return SPKV_ERR_ARG;
   if (gated_from < 0) return SPKV_ERR_ARG;
   if (!z_src && gated_from < n_rows) return SPKV_ERR_ARG;
-  return status_of(spkv::launch_ring_write(*p, *ring, K_src, V_src, z_src, gated_from, src_pos,
+  if (ring->u_win && !u_src && gated_from < n_rows) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_ring_write(*p, *ring, K_src, V_src, z_src, u_src, gated_from, src_pos,
                                            n_rows, src_batch_rows,
                                            static_cast<cudaStream_t>(stream)));
 }
@@ -183,25 +199,63 @@ size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* c) {
 int spkv_decode_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                      const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
                      size_t ws_bytes, spkv_stream_t stream) {
-  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
   if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
   const int sms = sm_count();
   if (sms <= 0) return SPKV_ERR_CUDA;
   if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
-  return status_of(spkv::launch_decode(*p, *c, *ring, q, t_pos, o, lse, workspace, ws_bytes, sms,
+  return status_of(spkv::launch_decode(*p, cache_or_none(c), *ring, q, t_pos, o, lse, workspace, ws_bytes, sms,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* c) {
+  if (!params_ok(p) || !cache_ok(p, c)) return 0;
+  return spkv::rethreshold_workspace_bytes(*p, *c);
+}
+
+int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                           float tau_new, void* workspace, size_t ws_bytes,
+                           spkv_stream_t stream) {
+  if (!params_ok(p) || !cache_ok(p, c) || !c->u_pool) return SPKV_ERR_ARG;
+  if (ring && !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!(tau_new == tau_new) || !workspace) return SPKV_ERR_ARG;
+  if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
+  if (ws_bytes < spkv::rethreshold_workspace_bytes(*p, *c)) return SPKV_ERR_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  return status_of(spkv::launch_rethreshold(*p, *c, ring, tau_new, workspace, sms,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+size_t spkv_soft_attn_workspace_bytes(const spkv_params* p, int seq_len) {
+  if (!params_ok(p) || seq_len < 0) return 0;
+  return spkv::soft_workspace_bytes(*p, seq_len);
+}
+
+int spkv_soft_attn(const spkv_params* p, const void* q, const void* K, const void* V,
+                   const float* u, int seq_len, float beta, float c, void* o, float* lse,
+                   void* workspace, size_t ws_bytes, uint32_t* err_flag, spkv_stream_t stream) {
+  if (!params_ok(p) || seq_len < 0) return SPKV_ERR_ARG;
+  if (!(beta > 0.f) || !(c >= 0.f) || !(c < INFINITY)) return SPKV_ERR_ARG;
+  if (seq_len == 0) return SPKV_OK;
+  if (!q || !K || !V || !u || !o || !workspace) return SPKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(K) || !aligned16(V) || !aligned16(o) || !aligned16(workspace))
+    return SPKV_ERR_ARG;
+  if (ws_bytes < spkv::soft_workspace_bytes(*p, seq_len)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_soft(*p, q, K, V, u, seq_len, beta, c, o, lse, workspace, err_flag,
+                                     static_cast<cudaStream_t>(stream)));
 }
 
 int spkv_prefill_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                       const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
                       int chunk_len, void* o, float* lse, spkv_stream_t stream) {
-  if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (chunk_start < 0 || chunk_len < 0) return SPKV_ERR_ARG;
   if (chunk_len == 0) return SPKV_OK;
   if (!q || !K_chunk || !V_chunk || !o) return SPKV_ERR_ARG;
   if (!aligned16(q) || !aligned16(K_chunk) || !aligned16(V_chunk) || !aligned16(o)) return SPKV_ERR_ARG;
-  return status_of(spkv::launch_prefill(*p, *c, *ring, q, K_chunk, V_chunk, chunk_start,
+  return status_of(spkv::launch_prefill(*p, cache_or_none(c), *ring, q, K_chunk, V_chunk, chunk_start,
                                         chunk_len, o, lse, static_cast<cudaStream_t>(stream)));
 }
 

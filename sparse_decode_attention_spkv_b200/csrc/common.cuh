@@ -198,8 +198,8 @@ struct CacheView {
 
 // Position of cache row i of head bh.
 __device__ __forceinline__ int cache_pos(const CacheView& c, int bh, int i) {
-  const int page = __ldg(c.page_table + (size_t)bh * c.max_pages + (i >> 6));
-  return __ldg(c.pos + (size_t)page * kPageRows + (i & 63));
+  const int page = __ldcg(c.page_table + (size_t)bh * c.max_pages + (i >> 6));
+  return __ldcg(c.pos + (size_t)page * kPageRows + (i & 63));
 }
 
 // Number of cache rows of head bh whose position is <= limit (positions are
@@ -207,7 +207,8 @@ __device__ __forceinline__ int cache_pos(const CacheView& c, int bh, int i) {
 // exceed the limit: in decode the cache holds no position beyond the query t, so
 // at most `window` rows lie in (t - window, t]; prefill passes the row count.
 __device__ __forceinline__ int cache_live_rows(const CacheView& c, int bh, int limit, int tail) {
-  const int n = __ldg(c.count + bh);
+  if (!c.count) return 0;  // no cache: a local (window-only) layer
+  const int n = __ldcg(c.count + bh);
   if (n == 0) return 0;
   if (cache_pos(c, bh, n - 1) <= limit) return n;
   int lo = n - tail > 0 ? n - tail : 0;  // rows before lo are <= limit

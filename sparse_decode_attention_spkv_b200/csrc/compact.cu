@@ -32,47 +32,59 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 }
 
 // One CTA per (batch row, key head): count this call's gated rows, extend the
-// head's page list from the bump allocator, and publish count_prev / count.
+// head's page list (pages it still owns past its count, left by a re-threshold, first;
+// then new ones from the bump allocator), and publish count_prev / count.
 __global__ void __launch_bounds__(256)
     compact_plan(CacheMut c, const uint8_t* __restrict__ z, int n_rows, int src_batch_rows,
                  int hkv) {
   __shared__ int red[8];
-  __shared__ int s_first, s_have, s_grant;
+  __shared__ int s_have, s_need, s_free, s_first, s_grant;
   const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
   const uint8_t* zb = z + (size_t)b * src_batch_rows * hkv + kh;
+  int32_t* table = c.page_table + (size_t)bh * c.max_pages;
   int kept = 0;
   for (int i = threadIdx.x; i < n_rows; i += blockDim.x) kept += zb[(size_t)i * hkv];
   const int total = block_sum(kept, red);
+  int old = 0, want = 0;
   if (threadIdx.x == 0) {
-    const int old = c.count[bh];
+    old = c.count[bh];
     const int cap = c.max_pages * kPageRows;
-    int want = old + total;
+    want = old + total;
     if (want > cap) {
       atomicOr(c.err, SPKV_FLAG_TABLE_FULL);
       want = cap;
     }
-    const int have = (old + kPageRows - 1) / kPageRows;
-    int need = (want + kPageRows - 1) / kPageRows;
+    s_have = (old + kPageRows - 1) / kPageRows;
+    s_need = (want + kPageRows - 1) / kPageRows;
+    s_free = s_need;
+  }
+  __syncthreads();
+  // owned pages form a prefix of the table: find the first unowned entry we need
+  for (int j = s_have + threadIdx.x; j < s_need; j += blockDim.x)
+    if (table[j] < 0) atomicMin(&s_free, j);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int need = s_need;
+    const int own_end = s_free;
     int first = 0, grant = 0;
-    if (need > have) {
-      first = atomicAdd(c.pool_top, need - have);
-      grant = need - have;
+    if (need > own_end) {
+      first = atomicAdd(c.pool_top, need - own_end);
+      grant = need - own_end;
       if (first + grant > c.num_pages) {
         grant = c.num_pages - first > 0 ? c.num_pages - first : 0;
         atomicOr(c.err, SPKV_FLAG_POOL_FULL);
-        need = have + grant;
+        need = own_end + grant;
         if (want > need * kPageRows) want = need * kPageRows;
       }
     }
     c.count_prev[bh] = old;
     c.count[bh] = want;
     s_first = first;
-    s_have = have;
+    s_free = own_end;
     s_grant = grant;
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < s_grant; j += blockDim.x)
-    c.page_table[(size_t)bh * c.max_pages + s_have + j] = s_first + j;
+  for (int j = threadIdx.x; j < s_grant; j += blockDim.x) table[s_free + j] = s_first + j;
 }
 
 constexpr int kScatterTile = 1024;
@@ -83,7 +95,8 @@ constexpr int kScatterThreads = 256;
 // rounds are ranked with a warp-ballot prefix sum and copied by lane groups.
 __global__ void __launch_bounds__(kScatterThreads)
     compact_scatter(CacheMut c, const char* __restrict__ Ksrc, const char* __restrict__ Vsrc,
-                    const uint8_t* __restrict__ z, const int32_t* __restrict__ src_pos,
+                    const uint8_t* __restrict__ z, const float* __restrict__ u,
+                    const int32_t* __restrict__ src_pos,
                     int n_rows, int src_batch_rows, int hkv, int row_bytes, int from_ring,
                     int window) {
   __shared__ int red[8];
@@ -142,7 +155,10 @@ __global__ void __launch_bounds__(kScatterThreads)
       const uint4 vv = *reinterpret_cast<const uint4*>(Vsrc + srow * row_bytes + col * 16);
       *reinterpret_cast<uint4*>(c.K + drow * row_bytes + col * 16) = kv;
       *reinterpret_cast<uint4*>(c.V + drow * row_bytes + col * 16) = vv;
-      if (col == 0) c.pos[drow] = p0 + src_i;
+      if (col == 0) {
+        c.pos[drow] = p0 + src_i;
+        if (c.u) c.u[drow] = u[((size_t)b * src_batch_rows + src_i) * hkv + kh];
+      }
     }
     running += round_total;
     __syncthreads();
@@ -151,26 +167,27 @@ __global__ void __launch_bounds__(kScatterThreads)
 
 // One warp per (batch row, key head).
 __global__ void __launch_bounds__(128)
-    decode_append_kernel(CacheMut c, char* __restrict__ Kwin, char* __restrict__ Vwin,
-                         uint8_t* __restrict__ zwin, const int32_t* __restrict__ t_pos,
+    decode_append_kernel(CacheMut c, RingMut r, const int32_t* __restrict__ t_pos,
                          const char* __restrict__ k_new, const char* __restrict__ v_new,
-                         const uint8_t* __restrict__ z_new, int retire, int n_heads, int hkv,
-                         int window, int row_bytes) {
+                         const uint8_t* __restrict__ z_new, const float* __restrict__ u_new,
+                         int retire, int n_heads, int hkv, int window, int row_bytes) {
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (bh >= n_heads) return;
   const int b = bh / hkv, kh = bh % hkv;
   const int t = t_pos[b];
   if (t < 0) return;  // positions are non-negative by contract
-  decode_append_warp(c, RingMut{Kwin, Vwin, zwin}, bh, b, kh, t, k_new, v_new,
-                     z_new ? z_new[bh] : (uint8_t)0, retire, hkv, window, row_bytes, lane);
+  decode_append_warp(c, r, bh, b, kh, t, k_new, v_new, z_new ? z_new[bh] : (uint8_t)0,
+                     (z_new && u_new) ? u_new[bh] : no_utility(), retire, hkv, window, row_bytes,
+                     lane);
 }
 
 // grid (B*Hkv); the last min(n_rows, window) rows of a chunk go to their slots.
 __global__ void __launch_bounds__(256)
     ring_write_kernel(char* __restrict__ Kwin, char* __restrict__ Vwin, uint8_t* __restrict__ zwin,
-                      const char* __restrict__ Ksrc, const char* __restrict__ Vsrc,
-                      const uint8_t* __restrict__ z_src, int gated_from,
+                      float* __restrict__ uwin, const char* __restrict__ Ksrc,
+                      const char* __restrict__ Vsrc, const uint8_t* __restrict__ z_src,
+                      const float* __restrict__ u_src, int gated_from,
                       const int32_t* __restrict__ src_pos, int n_rows, int src_batch_rows, int hkv,
                       int window, int row_bytes) {
   const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
@@ -188,7 +205,11 @@ __global__ void __launch_bounds__(256)
     const uint4 vv = *reinterpret_cast<const uint4*>(Vsrc + srow * row_bytes + col * 16);
     *reinterpret_cast<uint4*>(Kwin + drow * row_bytes + col * 16) = kv;
     *reinterpret_cast<uint4*>(Vwin + drow * row_bytes + col * 16) = vv;
-    if (col == 0) zwin[((size_t)b * window + slot) * hkv + kh] = (i >= gated_from) ? z_src[srow] : 0;
+    if (col == 0) {
+      const size_t zi = ((size_t)b * window + slot) * hkv + kh;
+      zwin[zi] = (i >= gated_from) ? z_src[srow] : 0;
+      if (uwin) uwin[zi] = (i >= gated_from) ? u_src[srow] : no_utility();
+    }
   }
 }
 
@@ -196,8 +217,8 @@ __global__ void __launch_bounds__(256)
 
 cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
                                  int src_kind, const void* K_src, const void* V_src,
-                                 const uint8_t* z, const int32_t* src_pos, int n_rows,
-                                 int src_batch_rows, cudaStream_t stream) {
+                                 const uint8_t* z, const float* u, const int32_t* src_pos,
+                                 int n_rows, int src_batch_rows, cudaStream_t stream) {
   const int n_heads = p.B * p.Hkv;
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
   const int row_bytes = p.head_dim * esize;
@@ -206,7 +227,7 @@ cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, cons
   const char* Ks = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->K_win : K_src);
   const char* Vs = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->V_win : V_src);
   dim3 grid(n_heads, (n_rows + kScatterTile - 1) / kScatterTile);
-  compact_scatter<<<grid, kScatterThreads, 0, stream>>>(m, Ks, Vs, z, src_pos, n_rows,
+  compact_scatter<<<grid, kScatterThreads, 0, stream>>>(m, Ks, Vs, z, u, src_pos, n_rows,
                                                         src_batch_rows, p.Hkv, row_bytes,
                                                         src_kind == SPKV_SRC_RING, p.window);
   return cudaGetLastError();
@@ -214,26 +235,27 @@ cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, cons
 
 cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                                  const int32_t* t_pos, const void* k_new, const void* v_new,
-                                 const uint8_t* z_new, int retire, cudaStream_t stream) {
+                                 const uint8_t* z_new, const float* u_new, int retire,
+                                 cudaStream_t stream) {
   const int n_heads = p.B * p.Hkv;
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
   decode_append_kernel<<<(n_heads + 3) / 4, 128, 0, stream>>>(
-      mut(c), static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win, t_pos,
-      static_cast<const char*>(k_new), static_cast<const char*>(v_new), z_new, retire, n_heads,
-      p.Hkv, p.window, p.head_dim * esize);
+      mut(c), ring_mut(ring), t_pos, static_cast<const char*>(k_new),
+      static_cast<const char*>(v_new), z_new, u_new, retire, n_heads, p.Hkv, p.window,
+      p.head_dim * esize);
   return cudaGetLastError();
 }
 
 cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const void* K_src,
-                              const void* V_src, const uint8_t* z_src, int gated_from,
-                              const int32_t* src_pos, int n_rows, int src_batch_rows,
-                              cudaStream_t stream) {
+                              const void* V_src, const uint8_t* z_src, const float* u_src,
+                              int gated_from, const int32_t* src_pos, int n_rows,
+                              int src_batch_rows, cudaStream_t stream) {
   const int n_heads = p.B * p.Hkv;
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
   ring_write_kernel<<<n_heads, 256, 0, stream>>>(
-      static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win,
-      static_cast<const char*>(K_src), static_cast<const char*>(V_src), z_src, gated_from, src_pos,
-      n_rows, src_batch_rows, p.Hkv, p.window, p.head_dim * esize);
+      static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win, ring.u_win,
+      static_cast<const char*>(K_src), static_cast<const char*>(V_src), z_src, u_src, gated_from,
+      src_pos, n_rows, src_batch_rows, p.Hkv, p.window, p.head_dim * esize);
   return cudaGetLastError();
 }
 

@@ -190,7 +190,7 @@ __device__ __forceinline__ void fetch_pages(int (&pg)[kPgRegs], const ChunkDesc&
 #pragma unroll
   for (int j = 0; j < kPgRegs; ++j) {
     const int k = d.k0 + lane + 32 * j;
-    pg[j] = k < d.kc1 ? __ldg(cache.page_table + (size_t)d.bh * cache.max_pages + k) : 0;
+    pg[j] = k < d.kc1 ? __ldcg(cache.page_table + (size_t)d.bh * cache.max_pages + k) : 0;
   }
 }
 
@@ -219,6 +219,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* next_chunk = ws_ctrl + n_heads;  // reset by the merge kernel
 
+  if (tid == 0) {  // descriptor fetches overlap the wait below
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_kp)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vp)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_kr)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vr)) : "memory");
+  }
   // the merge kernel may be scheduled now (it waits for this grid to complete); the
   // cache counts and the ring are written by the kernel before this one
   grid_dependents_launch();
@@ -227,7 +233,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   // ---- plan (identical in every CTA) ---------------------------------------------
   int my_rows = 0;
   for (int bh = tid; bh < n_heads; bh += kThreadsT) {
-    const int t = __ldg(t_pos + bh / hkv);
+    const int t = __ldcg(t_pos + bh / hkv);
     const int nl = cache_live_rows(cache, bh, t - window, window);
     const int nw = t + 1 < window ? t + 1 : window;
     const int rows = ((nl + kTileR - 1) / kTileR) * kTileR + nw;
@@ -324,7 +330,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           __syncwarp();
           for (int i = lane; i < kChunkPages; i += 32) {
             const int kk = k + i;
-            sm.pages[i] = kk < cd.kc1 ? __ldg(cache.page_table + (size_t)cd.bh * cache.max_pages + kk) : 0;
+            sm.pages[i] = kk < cd.kc1 ? __ldcg(cache.page_table + (size_t)cd.bh * cache.max_pages + kk) : 0;
           }
           __syncwarp();
         }
@@ -678,7 +684,7 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
   }
   const cuuint64_t es = 2;
   CUtensorMap tkp, tvp, tkr, tvr;
-  {
+  if (c.K_pool) {  // else a window-only layer: the cache maps are never used
     const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)c.num_pages * kPageRows};
     const cuuint64_t str[1] = {(cuuint64_t)D * es};
     const cuuint32_t box[2] = {64, kTileR};
@@ -692,6 +698,10 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
     const cuuint32_t box[4] = {64, kTileR, 1, 1};
     if (!map_bf16(&tkr, ring.K_win, 4, dims, str, box) || !map_bf16(&tvr, ring.V_win, 4, dims, str, box))
       return cudaErrorInvalidValue;
+  }
+  if (!c.K_pool) {
+    tkp = tkr;
+    tvp = tvr;
   }
   const int n_heads = p.B * p.Hkv;
   char* w = static_cast<char*>(ws);

@@ -21,17 +21,18 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
 
 cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
                                  int src_kind, const void* K_src, const void* V_src,
-                                 const uint8_t* z, const int32_t* src_pos, int n_rows,
-                                 int src_batch_rows, cudaStream_t stream);
+                                 const uint8_t* z, const float* u, const int32_t* src_pos,
+                                 int n_rows, int src_batch_rows, cudaStream_t stream);
 
 cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                                  const int32_t* t_pos, const void* k_new, const void* v_new,
-                                 const uint8_t* z_new, int retire, cudaStream_t stream);
+                                 const uint8_t* z_new, const float* u_new, int retire,
+                                 cudaStream_t stream);
 
 cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const void* K_src,
-                              const void* V_src, const uint8_t* z_src, int gated_from,
-                              const int32_t* src_pos, int n_rows, int src_batch_rows,
-                              cudaStream_t stream);
+                              const void* V_src, const uint8_t* z_src, const float* u_src,
+                              int gated_from, const int32_t* src_pos, int n_rows,
+                              int src_batch_rows, cudaStream_t stream);
 
 size_t decode_workspace_bytes(const spkv_params& p, int num_sms);
 bool decode_tc_supported(const spkv_params& p);
@@ -48,9 +49,22 @@ cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const s
                               const void* q, const void* K_chunk, const void* V_chunk,
                               int chunk_start, int chunk_len, void* o, float* lse,
                               cudaStream_t stream);
+size_t rethreshold_workspace_bytes(const spkv_params& p, const spkv_cache& c);
+cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
+                               float tau_new, void* workspace, int num_sms, cudaStream_t stream);
+
 cudaError_t launch_prefill(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                            const void* q, const void* K_chunk, const void* V_chunk,
                            int chunk_start, int chunk_len, void* o, float* lse,
                            cudaStream_t stream);
+
+bool soft_tc_supported(const spkv_params& p, int seq_len);
+cudaError_t launch_soft_tc(const spkv_params& p, const void* q, const void* K, const void* V,
+                           const float* bias, int seq_len, void* o, float* lse, uint32_t* err,
+                           cudaStream_t stream);
+size_t soft_workspace_bytes(const spkv_params& p, int seq_len);
+cudaError_t launch_soft(const spkv_params& p, const void* q, const void* K, const void* V,
+                        const float* u, int seq_len, float beta, float c, void* o, float* lse,
+                        void* workspace, uint32_t* err, cudaStream_t stream);
 
 }  // namespace spkv

@@ -23,6 +23,12 @@
 // Softmax runs in the log2 domain; the running max is raised only when a score
 // exceeds it by more than 8, and only then is the O row in TMEM rescaled.
 // Every mbarrier wait is bounded (a stuck wait raises SPKV_FLAG_TIMEOUT).
+//
+// The same kernel (SOFT = true) computes the soft-gated attention used at training
+// time (§2.1, "soft relaxation", Eqs. (5)-(6)): every key s <= t of the sequence,
+// read in 64-key blocks from the sequence K/V, with the additive score 0 inside the
+// causal window and c (alpha_s - 1) outside it; the per-key bias (already scaled to
+// the log2 domain) rides with each block.  No key block is skipped.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -157,6 +163,7 @@ struct Blocks {
   int nw;      // window blocks
 };
 
+template <bool SOFT>
 __global__ void __launch_bounds__(kThr, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tm_q,
                       const __grid_constant__ CUtensorMap tm_kc,
@@ -166,7 +173,8 @@ __global__ void __launch_bounds__(kThr, 1)
                       const __grid_constant__ CUtensorMap tm_kr,
                       const __grid_constant__ CUtensorMap tm_vr, CacheView cache,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
-                      int chunk_start, int chunk_len, int hkv, int G, uint32_t* err) {
+                      int chunk_start, int chunk_len, int hkv, int G, uint32_t* err,
+                      const float* __restrict__ soft_bias) {
   extern __shared__ __align__(1024) char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;  // 128B-swizzle atoms
   TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw + pad);
@@ -200,43 +208,52 @@ __global__ void __launch_bounds__(kThr, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  const int n = __ldg(cache.count + bh);
-  const int npages = (n + kPageRows - 1) / kPageRows;
-  const int lim_full = t0 - kWin, lim_any = t0 + kQT - 1 - kWin;
-  for (int pg = tid; pg < npages; pg += kThr) sm.first_pos[pg] = cache_pos(cache, bh, pg * kPageRows);
-  __syncthreads();
-  {
-    int pf = 0, pa = 0;
-    for (int pg = tid; pg < npages; pg += kThr) {
-      pf += sm.first_pos[pg] <= lim_full;
-      pa += sm.first_pos[pg] <= lim_any;
-    }
-    if (pf) atomicAdd(&sm.cnt[0], pf);
-    if (pa) atomicAdd(&sm.cnt[1], pa);
-  }
-  __syncthreads();
-  {
-    const int Pf = sm.cnt[0], Pa = sm.cnt[1];
-    if (tid < 64 && Pf > 0) {
-      const int row = (Pf - 1) * kPageRows + tid;
-      if (row < n && cache_pos(cache, bh, row) <= lim_full) atomicAdd(&sm.cnt[2], 1);
-    } else if (tid >= 64 && tid < 128 && Pa > 0) {
-      const int row = (Pa - 1) * kPageRows + (tid - 64);
-      if (row < n && cache_pos(cache, bh, row) <= lim_any) atomicAdd(&sm.cnt[3], 1);
-    }
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   Blocks bl;
-  {
-    const int Pf = sm.cnt[0], Pa = sm.cnt[1];
-    bl.nfull = Pf > 0 ? (Pf - 1) * kPageRows + sm.cnt[2] : 0;
-    const int n_any = Pa > 0 ? (Pa - 1) * kPageRows + sm.cnt[3] : 0;
-    bl.nc = (n_any + kKB - 1) / kKB;
-    bl.nrows = n;
-    bl.wfirst = t0 >= kWin ? t0 - kWin : t0;
-    bl.nw = (t0 + kQT - bl.wfirst) / kKB;
+  if constexpr (SOFT) {
+    bl.nc = bl.nfull = bl.nrows = 0;
+    bl.wfirst = 0;                    // every key block from the start of the sequence
+    bl.nw = (t0 + kQT) / kKB;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  } else {
+    const int n = cache.count ? __ldg(cache.count + bh) : 0;  // no cache: window only
+    const int npages = (n + kPageRows - 1) / kPageRows;
+    const int lim_full = t0 - kWin, lim_any = t0 + kQT - 1 - kWin;
+    for (int pg = tid; pg < npages; pg += kThr) sm.first_pos[pg] = cache_pos(cache, bh, pg * kPageRows);
+    __syncthreads();
+    {
+      int pf = 0, pa = 0;
+      for (int pg = tid; pg < npages; pg += kThr) {
+        pf += sm.first_pos[pg] <= lim_full;
+        pa += sm.first_pos[pg] <= lim_any;
+      }
+      if (pf) atomicAdd(&sm.cnt[0], pf);
+      if (pa) atomicAdd(&sm.cnt[1], pa);
+    }
+    __syncthreads();
+    {
+      const int Pf = sm.cnt[0], Pa = sm.cnt[1];
+      if (tid < 64 && Pf > 0) {
+        const int row = (Pf - 1) * kPageRows + tid;
+        if (row < n && cache_pos(cache, bh, row) <= lim_full) atomicAdd(&sm.cnt[2], 1);
+      } else if (tid >= 64 && tid < 128 && Pa > 0) {
+        const int row = (Pa - 1) * kPageRows + (tid - 64);
+        if (row < n && cache_pos(cache, bh, row) <= lim_any) atomicAdd(&sm.cnt[3], 1);
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    {
+      const int Pf = sm.cnt[0], Pa = sm.cnt[1];
+      bl.nfull = Pf > 0 ? (Pf - 1) * kPageRows + sm.cnt[2] : 0;
+      const int n_any = Pa > 0 ? (Pa - 1) * kPageRows + sm.cnt[3] : 0;
+      bl.nc = (n_any + kKB - 1) / kKB;
+      bl.nrows = n;
+      bl.wfirst = t0 >= kWin ? t0 - kWin : t0;
+      bl.nw = (t0 + kQT - bl.wfirst) / kKB;
+    }
   }
   const int J = bl.nc + bl.nw;
   const uint32_t tmem = sm.tmem_base;
@@ -261,7 +278,9 @@ __global__ void __launch_bounds__(kThr, 1)
           bulk_g2s(sm.pos[s], cache.pos + (size_t)page * kPageRows, kKB * 4, &sm.kv_full[s]);
         } else {
           const int pb = bl.wfirst + (j - bl.nc) * kKB;
-          mbar_arrive_expect_tx(&sm.kv_full[s], 4 * kKB * 128);
+          mbar_arrive_expect_tx(&sm.kv_full[s], 4 * kKB * 128 + (SOFT ? kKB * 4 : 0));
+          if constexpr (SOFT)  // the block's per-key bias, [B][Hkv][T] layout
+            bulk_g2s(sm.pos[s], soft_bias + (size_t)bh * chunk_len + pb, kKB * 4, &sm.kv_full[s]);
           for (int half = 0; half < 2; ++half) {
             if (pb >= chunk_start) {
               tma_4d(sm.k[s][half], &tm_kc, half * 64, kh, pb - chunk_start, b, &sm.kv_full[s]);
@@ -346,12 +365,23 @@ __global__ void __launch_bounds__(kThr, 1)
         }
       } else {
         const int pb = bl.wfirst + (j - bl.nc) * kKB;
+        if constexpr (SOFT) {
+          const float* bias = reinterpret_cast<const float*>(sm.pos[s]);
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const int dlt = t - (pb + i);
-          const bool vis = dlt >= 0 && dlt < kWin;
-          x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
-          rmax = fmaxf(rmax, x[i]);
+          for (int i = 0; i < 64; ++i) {
+            const int dlt = t - (pb + i);
+            x[i] = dlt < 0 ? -INFINITY
+                           : __uint_as_float(raw[i]) * c + (dlt >= kWin ? bias[i] : 0.f);
+            rmax = fmaxf(rmax, x[i]);
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 64; ++i) {
+            const int dlt = t - (pb + i);
+            const bool vis = dlt >= 0 && dlt < kWin;
+            x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
+            rmax = fmaxf(rmax, x[i]);
+          }
         }
       }
       const bool need = rmax > m + kSlack;
@@ -445,6 +475,20 @@ bool make_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+constexpr size_t kSmem = sizeof(TcSmem) + 1024;  // + alignment slack
+
+template <bool SOFT>
+cudaError_t configure() {
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel<SOFT>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
+    if (err != cudaSuccess) return err;
+    configured = true;
+  }
+  return cudaSuccess;
+}
+
 }  // namespace
 
 bool prefill_tc_supported(const spkv_params& p, const spkv_cache& c, int chunk_start, int chunk_len) {
@@ -474,12 +518,15 @@ cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const s
     if (!make_map(&tkc, K_chunk, 4, dims, str, box) || !make_map(&tvc, V_chunk, 4, dims, str, box))
       return cudaErrorInvalidValue;
   }
-  {
+  if (c.K_pool) {
     const cuuint64_t dims[2] = {(cuuint64_t)kHD, (cuuint64_t)c.num_pages * kPageRows};
     const cuuint64_t str[1] = {kHD * e};
     const cuuint32_t box[2] = {64, kKB};
     if (!make_map(&tkp, c.K_pool, 2, dims, str, box) || !make_map(&tvp, c.V_pool, 2, dims, str, box))
       return cudaErrorInvalidValue;
+  } else {  // window-only layer: no cache block is ever loaded
+    tkp = tkc;
+    tvp = tvc;
   }
   {
     const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)kWin, (cuuint64_t)p.Hkv, (cuuint64_t)p.B};
@@ -488,19 +535,50 @@ cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const s
     if (!make_map(&tkr, ring.K_win, 4, dims, str, box) || !make_map(&tvr, ring.V_win, 4, dims, str, box))
       return cudaErrorInvalidValue;
   }
-  const size_t smem = sizeof(TcSmem) + 1024;  // + alignment slack
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (err != cudaSuccess) return err;
-    configured = true;
-  }
+  cudaError_t e2 = configure<false>();
+  if (e2 != cudaSuccess) return e2;
   CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
                c.page_table, c.count, c.max_pages_per_head};
   dim3 grid(chunk_len / kQT, G / 2, p.B * p.Hkv);
-  prefill_tc_kernel<<<grid, kThr, smem, stream>>>(tq, tkc, tvc, tkp, tvp, tkr, tvr, cv,
-                                                  static_cast<__nv_bfloat16*>(o), lse, chunk_start,
-                                                  chunk_len, p.Hkv, G, c.err_flag);
+  prefill_tc_kernel<false><<<grid, kThr, kSmem, stream>>>(
+      tq, tkc, tvc, tkp, tvp, tkr, tvr, cv, static_cast<__nv_bfloat16*>(o), lse, chunk_start,
+      chunk_len, p.Hkv, G, c.err_flag, nullptr);
+  return cudaGetLastError();
+}
+
+bool soft_tc_supported(const spkv_params& p, int seq_len) {
+  const int G = p.Hq / p.Hkv;
+  return p.dtype == SPKV_BF16 && p.head_dim == kHD && p.window == kWin && G % 2 == 0 &&
+         seq_len % kQT == 0 && seq_len > 0 && encode_fn() != nullptr;
+}
+
+cudaError_t launch_soft_tc(const spkv_params& p, const void* q, const void* K, const void* V,
+                           const float* bias, int seq_len, void* o, float* lse, uint32_t* err,
+                           cudaStream_t stream) {
+  const int G = p.Hq / p.Hkv;
+  const cuuint64_t e = 2;
+  CUtensorMap tq, tk, tv;
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)p.Hq, (cuuint64_t)seq_len, (cuuint64_t)p.B};
+    const cuuint64_t str[3] = {kHD * e, (cuuint64_t)p.Hq * kHD * e, (cuuint64_t)seq_len * p.Hq * kHD * e};
+    const cuuint32_t box[4] = {64, 1, kQT, 1};
+    if (!make_map(&tq, q, 4, dims, str, box)) return cudaErrorInvalidValue;
+  }
+  {
+    const cuuint64_t dims[4] = {(cuuint64_t)kHD, (cuuint64_t)p.Hkv, (cuuint64_t)seq_len, (cuuint64_t)p.B};
+    const cuuint64_t str[3] = {kHD * e, (cuuint64_t)p.Hkv * kHD * e, (cuuint64_t)seq_len * p.Hkv * kHD * e};
+    const cuuint32_t box[4] = {64, 1, kKB, 1};
+    if (!make_map(&tk, K, 4, dims, str, box) || !make_map(&tv, V, 4, dims, str, box))
+      return cudaErrorInvalidValue;
+  }
+  cudaError_t e2 = configure<true>();
+  if (e2 != cudaSuccess) return e2;
+  CacheView cv{nullptr, nullptr, nullptr, nullptr, nullptr, 0};
+  dim3 grid(seq_len / kQT, G / 2, p.B * p.Hkv);
+  // the cache and ring maps are not read in this mode: the sequence maps stand in
+  prefill_tc_kernel<true><<<grid, kThr, kSmem, stream>>>(
+      tq, tk, tv, tk, tv, tk, tv, cv, static_cast<__nv_bfloat16*>(o), lse, 0, seq_len, p.Hkv, G,
+      err, bias);
   return cudaGetLastError();
 }
 

@@ -262,7 +262,7 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
       const int b = tok0 + n;  // one new token per batch row
       const int t = ap.t_pos[b];
       if (t >= 0)
-        decode_append_warp(ap.c, ap.r, b * hkv + kh, b, kh, t, ap.k_new, ap.v_new, z, 1, hkv,
+        decode_append_warp(ap.c, ap.r, b * hkv + kh, b, kh, t, ap.k_new, ap.v_new, z, uval, 1, hkv,
                            ap.window, ap.row_bytes, lane);
     }
   }
@@ -440,7 +440,7 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
     }
     if constexpr (APPEND) {
       const int b = tok0 + my_n;
-      append_commit(ap.c, ap.r, pre, b * hkv + warp, b, warp, z, hkv, ap.window, ap.row_bytes,
+      append_commit(ap.c, ap.r, pre, b * hkv + warp, b, warp, z, uval, hkv, ap.window, ap.row_bytes,
                     lane, stage[warp]);
     }
   }
@@ -505,11 +505,11 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
   if (!mma && !small_ok(p, p.B)) {  // many rows: the two steps as separate launches
     cudaError_t e = launch_score(p, h, p.B, W1, b1, W2, b2, u_out, z_out, stream);
     if (e != cudaSuccess) return e;
-    return launch_decode_append(p, c, ring, t_pos, k_new, v_new, z_out, 1, stream);
+    return launch_decode_append(p, c, ring, t_pos, k_new, v_new, z_out, u_out, 1, stream);
   }
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
   SmallAppend ap{cache_mut(c),
-                 RingMut{static_cast<char*>(ring.K_win), static_cast<char*>(ring.V_win), ring.z_win},
+                 ring_mut(ring),
                  t_pos, static_cast<const char*>(k_new), static_cast<const char*>(v_new), p.window,
                  p.head_dim * esize};
   if (mma) return launch_mma<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);

@@ -50,6 +50,7 @@ T_QDEC = 11    # per-step decode queries
 T_KDEC = 12    # per-step decode keys
 T_VDEC = 13    # per-step decode values
 T_HDEC = 14    # per-step decode hidden states
+T_U = 15       # utilities drawn directly (inputs of the soft-gated attention tests)
 
 
 def _mix64_int(z: int) -> int:

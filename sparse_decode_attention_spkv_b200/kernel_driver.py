@@ -64,10 +64,10 @@ def run_compact(args):
     D.fill_normal(k, wl.key(0, gen.T_K), wl.qkv_scale)
     D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale)
     D.fill_normal(h, wl.key(0, gen.T_H), 1.0)
-    _, z = R.score(L, h, n)
+    u, z = R.score(L, h, n)
     for i in range(args.steps):
         src = torch.full((1,), i * n, dtype=torch.int32, device="cuda")
-        S.spkv_write_compact(L.p, L.cache, L.ring, S.SRC_CHUNK, k, v, z, src, n, n)
+        S.spkv_write_compact(L.p, L.cache, L.ring, S.SRC_CHUNK, k, v, z, u, src, n, n)
     torch.cuda.synchronize()
 
 

@@ -1,7 +1,9 @@
 """Schedules of the SP-KV hot path, driven through the C ABI.
 
 A ``Layer`` holds one attention layer's utility-perceptron weights, gated cache,
-window ring and decode workspace on the device.  The functions below sequence the
+window ring and decode workspace on the device.  A local layer of a hybrid
+local/global stack (``Layer.create_local``) has only the ring: it keeps no
+long-range cache and attends to its window alone.  The functions below sequence the
 library calls for the three schedules the workloads use:
 
 * chunked prefill, compacting each chunk right after scoring it (the chunk's
@@ -29,19 +31,33 @@ from . import spkv as S
 @dataclass
 class Layer:
     p: S.spkv_params
-    W1: torch.Tensor
-    b1: torch.Tensor
-    W2: torch.Tensor
-    b2: torch.Tensor
-    cache: S.Cache
+    W1: Optional[torch.Tensor]
+    b1: Optional[torch.Tensor]
+    W2: Optional[torch.Tensor]
+    b2: Optional[torch.Tensor]
+    cache: Optional[S.Cache]
     ring: S.Ring
     ws: torch.Tensor
 
+    @property
+    def local(self) -> bool:
+        return self.cache is None
+
+    @staticmethod
+    def create_local(p: S.spkv_params, device="cuda") -> "Layer":
+        """A window-only layer (the local layers of a hybrid stack, §3.3 "Hybrids"):
+        no utility perceptron, no cache."""
+        ring = S.Ring.allocate(p, device)
+        ws = S.alloc_decode_workspace(p, None, device)
+        return Layer(p, None, None, None, None, None, ring, ws)
+
     @staticmethod
     def create(p: S.spkv_params, W1, b1, W2, b2, num_pages: int, max_pages_per_head: int,
-               device="cuda") -> "Layer":
-        cache = S.Cache.allocate(p, num_pages, max_pages_per_head, device)
-        ring = S.Ring.allocate(p, device)
+               device="cuda", store_u: bool = False) -> "Layer":
+        """store_u: keep the utility of every cached row and pending window slot, so
+        that the cache can be re-thresholded later (spkv_cache_rethreshold)."""
+        cache = S.Cache.allocate(p, num_pages, max_pages_per_head, device, store_u=store_u)
+        ring = S.Ring.allocate(p, device, store_u=store_u)
         ws = S.alloc_decode_workspace(p, cache, device)
         layer = Layer(p, W1, b1, W2, b2, cache, ring, ws)
         S.spkv_cache_reset(p, cache, ring)
@@ -76,19 +92,26 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
     stay only in the ring with their gates, to be retired by per-token decode.
     Returns (o [B][Tc][Hq][d], lse [B][Tc][Hq], u, z [B][Tc][Hkv])."""
     p = layer.p
-    B, Tc = h.shape[0], h.shape[1]
-    dev = h.device
+    B, Tc = q.shape[0], q.shape[1]
+    dev = q.device
     if n_compact is None:
         n_compact = Tc
     if src_pos is None:
         src_pos = torch.full((B,), chunk_start, dtype=torch.int32, device=dev)
+    if layer.local:  # window only: attend, then keep the chunk's last rows in the ring
+        o = torch.empty_like(q)
+        lse = torch.empty((B, Tc, p.Hq), dtype=torch.float32, device=dev)
+        S.spkv_prefill_attn(p, None, layer.ring, q, k, v, chunk_start, Tc, o, lse)
+        S.spkv_ring_write(p, layer.ring, k, v, None, None, Tc, src_pos, Tc, Tc)
+        return o, lse, None, None
     u, z = score(layer, h, B * Tc)
     if n_compact > 0:
-        S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, k, v, z, src_pos, n_compact, Tc)
+        S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, k, v, z, u, src_pos, n_compact,
+                             Tc)
     o = torch.empty_like(q)
     lse = torch.empty((B, Tc, p.Hq), dtype=torch.float32, device=dev)
     S.spkv_prefill_attn(p, layer.cache, layer.ring, q, k, v, chunk_start, Tc, o, lse)
-    S.spkv_ring_write(p, layer.ring, k, v, z, n_compact, src_pos, Tc, Tc)
+    S.spkv_ring_write(p, layer.ring, k, v, z, u, n_compact, src_pos, Tc, Tc)
     return o, lse, u.view(B, Tc, p.Hkv), z.view(B, Tc, p.Hkv)
 
 
@@ -102,15 +125,24 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
     launch (spkv_decode_score_append), else spkv_score then spkv_decode_append.
     Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
     p = layer.p
-    z_t = None
+    z_t = u_t = None
+    if layer.local:  # store the new token in the ring; nothing ever retires
+        S.spkv_decode_append(p, None, layer.ring, t_pos, k_t, v_t, None, None, 0)
+        if o is None:
+            o = torch.empty_like(q_t)
+        if lse is None:
+            lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
+        S.spkv_decode_attn(p, None, layer.ring, q_t, t_pos, o, lse, layer.ws)
+        return o, lse, None
     if retire and fused:
         z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
+        u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)
         S.spkv_decode_score_append(p, layer.cache, layer.ring, t_pos, h_t, layer.W1, layer.b1,
-                                   layer.W2, layer.b2, k_t, v_t, None, z_t)
+                                   layer.W2, layer.b2, k_t, v_t, u_t, z_t)
     else:
         if retire:
-            _, z_t = score(layer, h_t, p.B)
-        S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, z_t, retire)
+            u_t, z_t = score(layer, h_t, p.B)
+        S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, z_t, u_t, retire)
     if o is None:
         o = torch.empty_like(q_t)
     if lse is None:
@@ -125,7 +157,7 @@ def bulk_compact(layer: Layer, h_buf: torch.Tensor, start_pos: torch.Tensor):
     p = layer.p
     B, n = h_buf.shape[0], h_buf.shape[1]
     u, z = score(layer, h_buf, B * n)
-    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_RING, None, None, z, start_pos, n, n)
+    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_RING, None, None, z, u, start_pos, n, n)
     return u.view(B, n, p.Hkv), z.view(B, n, p.Hkv)
 
 

@@ -39,11 +39,12 @@ class spkv_params(ctypes.Structure):
 class spkv_cache(ctypes.Structure):
     _fields_ = [("K_pool", _vp), ("V_pool", _vp), ("pos_pool", _vp), ("page_table", _vp),
                 ("count", _vp), ("count_prev", _vp), ("pool_top", _vp), ("err_flag", _vp),
-                ("num_pages", _i32), ("page_rows", _i32), ("max_pages_per_head", _i32)]
+                ("u_pool", _vp), ("num_pages", _i32), ("page_rows", _i32),
+                ("max_pages_per_head", _i32)]
 
 
 class spkv_ring(ctypes.Structure):
-    _fields_ = [("K_win", _vp), ("V_win", _vp), ("z_win", _vp)]
+    _fields_ = [("K_win", _vp), ("V_win", _vp), ("z_win", _vp), ("u_win", _vp)]
 
 
 _P = ctypes.POINTER
@@ -54,11 +55,17 @@ _sigs = {
     "spkv_cache_check": (_i32, [_P(spkv_cache), _vp, _P(ctypes.c_uint32)]),
     "spkv_score": (_i32, [_P(spkv_params), _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "spkv_write_compact": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _i32, _vp, _vp,
-                                  _vp, _vp, _i32, _i32, _vp]),
+                                  _vp, _vp, _vp, _i32, _i32, _vp]),
     "spkv_decode_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp,
-                                  _vp, _i32, _vp]),
-    "spkv_ring_write": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _i32, _vp, _i32, _i32,
-                                _vp]),
+                                  _vp, _vp, _i32, _vp]),
+    "spkv_ring_write": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _vp, _i32, _vp, _i32,
+                                _i32, _vp]),
+    "spkv_rethreshold_workspace_bytes": (ctypes.c_size_t, [_P(spkv_params), _P(spkv_cache)]),
+    "spkv_cache_rethreshold": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring),
+                                      ctypes.c_float, _vp, ctypes.c_size_t, _vp]),
+    "spkv_soft_attn_workspace_bytes": (ctypes.c_size_t, [_P(spkv_params), _i32]),
+    "spkv_soft_attn": (_i32, [_P(spkv_params), _vp, _vp, _vp, _vp, _i32, ctypes.c_float,
+                              ctypes.c_float, _vp, _vp, _vp, ctypes.c_size_t, _vp, _vp]),
     "spkv_decode_workspace_bytes": (ctypes.c_size_t, [_P(spkv_params), _P(spkv_cache)]),
     "spkv_decode_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _vp,
                                 _vp, ctypes.c_size_t, _vp]),
@@ -121,10 +128,14 @@ class Cache:
     count_prev: torch.Tensor
     pool_top: torch.Tensor
     err_flag: torch.Tensor
+    u_pool: Optional[torch.Tensor]
     c: spkv_cache
 
     @staticmethod
-    def allocate(p: spkv_params, num_pages: int, max_pages_per_head: int, device="cuda") -> "Cache":
+    def allocate(p: spkv_params, num_pages: int, max_pages_per_head: int, device="cuda",
+                 store_u: bool = False) -> "Cache":
+        """store_u: keep the utility of every stored row (needed by
+        spkv_cache_rethreshold)."""
         dt = torch_dtype(p.dtype)
         heads = p.B * p.Hkv
         K = torch.zeros((num_pages, PAGE_ROWS, p.head_dim), dtype=dt, device=device)
@@ -135,10 +146,12 @@ class Cache:
         count_prev = torch.zeros(heads, dtype=torch.int32, device=device)
         top = torch.zeros(1, dtype=torch.int32, device=device)
         err = torch.zeros(1, dtype=torch.int32, device=device)
+        u = torch.zeros((num_pages, PAGE_ROWS), dtype=torch.float32, device=device) if store_u else None
         c = spkv_cache(K.data_ptr(), V.data_ptr(), pos.data_ptr(), table.data_ptr(),
                        count.data_ptr(), count_prev.data_ptr(), top.data_ptr(), err.data_ptr(),
-                       num_pages, PAGE_ROWS, max_pages_per_head)
-        return Cache(K, V, pos, table, count, count_prev, top, err, c)
+                       u.data_ptr() if u is not None else None, num_pages, PAGE_ROWS,
+                       max_pages_per_head)
+        return Cache(K, V, pos, table, count, count_prev, top, err, u, c)
 
 
 @dataclass
@@ -146,15 +159,20 @@ class Ring:
     K_win: torch.Tensor
     V_win: torch.Tensor
     z_win: torch.Tensor
+    u_win: Optional[torch.Tensor]
     r: spkv_ring
 
     @staticmethod
-    def allocate(p: spkv_params, device="cuda") -> "Ring":
+    def allocate(p: spkv_params, device="cuda", store_u: bool = False) -> "Ring":
+        """store_u: keep the pending utility of every slot (NaN: none pending)."""
         dt = torch_dtype(p.dtype)
         K = torch.zeros((p.B, p.Hkv, p.window, p.head_dim), dtype=dt, device=device)
         V = torch.zeros_like(K)
         z = torch.zeros((p.B, p.window, p.Hkv), dtype=torch.uint8, device=device)
-        return Ring(K, V, z, spkv_ring(K.data_ptr(), V.data_ptr(), z.data_ptr()))
+        u = torch.full((p.B, p.window, p.Hkv), float("nan"), dtype=torch.float32,
+                       device=device) if store_u else None
+        return Ring(K, V, z, u, spkv_ring(K.data_ptr(), V.data_ptr(), z.data_ptr(),
+                                          u.data_ptr() if u is not None else None))
 
 
 # ---- entry points (same names as the C ABI) -------------------------------------------
@@ -177,29 +195,53 @@ def spkv_score(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream=None):
         _ptr(z_out), _stream(stream)))
 
 
-def spkv_write_compact(p, cache: Cache, ring: Optional[Ring], src_kind, K_src, V_src, z, src_pos,
-                       n_rows, src_batch_rows, stream=None):
+def spkv_write_compact(p, cache: Cache, ring: Optional[Ring], src_kind, K_src, V_src, z, u,
+                       src_pos, n_rows, src_batch_rows, stream=None):
     return _check("spkv_write_compact", lib.spkv_write_compact(
         ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r) if ring else None, src_kind,
-        _ptr(K_src), _ptr(V_src), _ptr(z), _ptr(src_pos), n_rows, src_batch_rows, _stream(stream)))
+        _ptr(K_src), _ptr(V_src), _ptr(z), _ptr(u), _ptr(src_pos), n_rows, src_batch_rows,
+        _stream(stream)))
 
 
-def spkv_decode_append(p, cache: Cache, ring: Ring, t_pos, k_new, v_new, z_new, retire,
-                       stream=None):
+def _cache_ref(cache: Optional[Cache]):
+    return ctypes.byref(cache.c) if cache is not None else None
+
+
+def spkv_decode_append(p, cache: Optional[Cache], ring: Ring, t_pos, k_new, v_new, z_new, u_new,
+                       retire, stream=None):
+    """cache None: a window-only layer (retire must be 0)."""
     return _check("spkv_decode_append", lib.spkv_decode_append(
-        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(t_pos), _ptr(k_new),
-        _ptr(v_new), _ptr(z_new), int(retire), _stream(stream)))
+        ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(t_pos), _ptr(k_new),
+        _ptr(v_new), _ptr(z_new), _ptr(u_new), int(retire), _stream(stream)))
 
 
-def spkv_ring_write(p, ring: Ring, K_src, V_src, z_src, gated_from, src_pos, n_rows,
+def spkv_ring_write(p, ring: Ring, K_src, V_src, z_src, u_src, gated_from, src_pos, n_rows,
                     src_batch_rows, stream=None):
     return _check("spkv_ring_write", lib.spkv_ring_write(
-        ctypes.byref(p), ctypes.byref(ring.r), _ptr(K_src), _ptr(V_src), _ptr(z_src),
+        ctypes.byref(p), ctypes.byref(ring.r), _ptr(K_src), _ptr(V_src), _ptr(z_src), _ptr(u_src),
         int(gated_from), _ptr(src_pos), n_rows, src_batch_rows, _stream(stream)))
 
 
-def spkv_decode_workspace_bytes(p, cache: Cache) -> int:
-    return int(lib.spkv_decode_workspace_bytes(ctypes.byref(p), ctypes.byref(cache.c)))
+def spkv_rethreshold_workspace_bytes(p, cache: Cache) -> int:
+    return int(lib.spkv_rethreshold_workspace_bytes(ctypes.byref(p), ctypes.byref(cache.c)))
+
+
+def alloc_rethreshold_workspace(p, cache: Cache, device="cuda") -> torch.Tensor:
+    n = spkv_rethreshold_workspace_bytes(p, cache)
+    if n == 0:
+        raise SpkvError("spkv_rethreshold_workspace_bytes", ERR_ARG)
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def spkv_cache_rethreshold(p, cache: Cache, ring: Optional[Ring], tau_new, workspace,
+                           stream=None):
+    return _check("spkv_cache_rethreshold", lib.spkv_cache_rethreshold(
+        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r) if ring else None,
+        float(tau_new), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def spkv_decode_workspace_bytes(p, cache: Optional[Cache]) -> int:
+    return int(lib.spkv_decode_workspace_bytes(ctypes.byref(p), _cache_ref(cache)))
 
 
 def alloc_decode_workspace(p, cache: Cache, device="cuda") -> torch.Tensor:
@@ -209,16 +251,19 @@ def alloc_decode_workspace(p, cache: Cache, device="cuda") -> torch.Tensor:
     return torch.zeros(n, dtype=torch.uint8, device=device)
 
 
-def spkv_decode_attn(p, cache: Cache, ring: Ring, q, t_pos, o, lse, workspace, stream=None):
+def spkv_decode_attn(p, cache: Optional[Cache], ring: Ring, q, t_pos, o, lse, workspace,
+                     stream=None):
+    """cache None: a window-only layer (attends to the ring only)."""
     return _check("spkv_decode_attn", lib.spkv_decode_attn(
-        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
+        ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
         _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
-def spkv_prefill_attn(p, cache: Cache, ring: Ring, q, K_chunk, V_chunk, chunk_start, chunk_len,
-                      o, lse, stream=None):
+def spkv_prefill_attn(p, cache: Optional[Cache], ring: Ring, q, K_chunk, V_chunk, chunk_start,
+                      chunk_len, o, lse, stream=None):
+    """cache None: a window-only layer."""
     return _check("spkv_prefill_attn", lib.spkv_prefill_attn(
-        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(K_chunk),
+        ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(K_chunk),
         _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _stream(stream)))
 
 
@@ -236,3 +281,15 @@ def spkv_decode_score_append(p, cache: Cache, ring: Ring, t_pos, h, W1, b1, W2, 
         ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(t_pos), _ptr(h), _ptr(W1),
         _ptr(b1), _ptr(W2), _ptr(b2), _ptr(k_new), _ptr(v_new), _ptr(u_out), _ptr(z_out),
         _stream(stream)))
+
+
+def spkv_soft_attn_workspace_bytes(p, seq_len: int) -> int:
+    return int(lib.spkv_soft_attn_workspace_bytes(ctypes.byref(p), int(seq_len)))
+
+
+def spkv_soft_attn(p, q, K, V, u, seq_len, beta, c, o, lse, workspace, err_flag=None,
+                   stream=None):
+    """Soft-gated training-time attention (Eqs. (5)-(6)); see include/spkv.h."""
+    return _check("spkv_soft_attn", lib.spkv_soft_attn(
+        ctypes.byref(p), _ptr(q), _ptr(K), _ptr(V), _ptr(u), int(seq_len), float(beta), float(c),
+        _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(err_flag), _stream(stream)))

@@ -20,9 +20,10 @@ import torch
 
 
 def build_decode_state(wl, layers, steps_total, device, compact_window: bool = False,
-                       chunk: int = 0):
+                       chunk: int = 0, store_u: bool = False):
     """Returns (params, [Layer], inputs) where inputs["h"|"q"|"k"|"v"][i][l] are step i's
-    tensors of layer l and inputs["t"][i] the positions [B] of step i."""
+    tensors of layer l and inputs["t"][i] the positions [B] of step i.  store_u keeps the
+    utilities of cached rows and pending window slots (for re-thresholding)."""
     from sparse_decode_attention_spkv_b200 import runner as R
     from sparse_decode_attention_spkv_b200 import spkv as S
     from sparse_decode_attention_spkv_b200.inputs import device as D
@@ -55,7 +56,7 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
                          int(keep_table[l][kh] * 1.15 * Tmax) + steps_total + 512) for kh in range(Hkv)]
         max_pages = R.pages_for(max(rows_head))
         num_pages = B * sum(R.pages_for(r) for r in rows_head)
-        L = R.Layer.create(p, W1, b1, W2, b2, num_pages, max_pages, device)
+        L = R.Layer.create(p, W1, b1, W2, b2, num_pages, max_pages, device, store_u=store_u)
         kh_, kk_, kv_ = wl.key(l, gen.T_H), wl.key(l, gen.T_K), wl.key(l, gen.T_V)
         n_lim = max(limit.tolist())
         for c0 in range(0, n_lim, chunk):
@@ -67,12 +68,12 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
             hc = h_c[:, :n].contiguous() if n < chunk else h_c
             kc = k_c[:, :n].contiguous() if n < chunk else k_c
             vc = v_c[:, :n].contiguous() if n < chunk else v_c
-            _, z = R.score(L, hc, B * n)
+            u, z = R.score(L, hc, B * n)
             z = z.view(B, n, Hkv)
             pos = torch.arange(c0, c0 + n, dtype=torch.int32, device=device)
             z.mul_((pos[None, :] < limit[:, None]).to(torch.uint8)[:, :, None])  # beyond a row's prefix
             src = torch.full((B,), c0, dtype=torch.int32, device=device)
-            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, src, n, n)
+            S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, u, src, n, n)
         # the ring: each row's last w tokens, gated (per-token) or marked as cached
         kr = torch.empty((B, w, Hkv, d), dtype=bf, device=device)
         vr = torch.empty_like(kr)
@@ -82,9 +83,9 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
             D.fill_normal(hr[b], kh_, 1.0, offset=(b * Tt + s0) * Dm)
             D.fill_normal(kr[b], kk_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
             D.fill_normal(vr[b], kv_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
-        _, zr = R.score(L, hr, B * w)
+        ur, zr = R.score(L, hr, B * w)
         src = torch.tensor([c - w for c in ctx], dtype=torch.int32, device=device)
-        S.spkv_ring_write(p, L.ring, kr, vr, zr, w if compact_window else 0, src, w, w)
+        S.spkv_ring_write(p, L.ring, kr, vr, zr, ur, w if compact_window else 0, src, w, w)
         Ls.append(L)
     del h_c, k_c, v_c
     # per-step inputs [steps][layers][B][...]; row b's step i is position ctx[b] + i
@@ -162,3 +163,42 @@ def kv_bytes_layers(p, layers, t_min):
     n_win = min(p.window, t_min + 1)
     return [int((L.cache.count.to(torch.int64) + n_win).sum().item()) * 2 * p.head_dim * 2
             for L in layers]
+
+
+class HybridStep:
+    """Launch sequence of one decode step over a hybrid local/global stack: layer l is
+    global (SP-KV: score, retire, attend over cache + window) when l % period ==
+    period - 1, else local (window only, no cache)."""
+
+    def __init__(self, p, global_layers, local_layers, period, device):
+        from sparse_decode_attention_spkv_b200 import spkv as S
+        self.S, self.p, self.period = S, p, period
+        self.glob, self.loc = global_layers, local_layers
+        n = len(global_layers) + len(local_layers)
+        self.n = n
+        self.o = torch.empty((n, p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
+        self.lse = torch.empty((n, p.B, p.Hq), dtype=torch.float32, device=device)
+        self.u = torch.empty((len(global_layers), p.B, p.Hkv), dtype=torch.float32, device=device)
+        self.z = torch.empty((len(global_layers), p.B, p.Hkv), dtype=torch.uint8, device=device)
+
+    def launch(self, h, q, k, v, t):
+        """h, q, k, v indexed by global-layer number (local layers reuse q, k, v of
+        global layer l // period: their values do not change the work)."""
+        S, p = self.S, self.p
+        gi = li = 0
+        for l in range(self.n):
+            g = l // self.period
+            if l % self.period == self.period - 1:
+                L = self.glob[gi]
+                S.spkv_decode_score_append(p, L.cache, L.ring, t, h[g], L.W1, L.b1, L.W2, L.b2,
+                                           k[g], v[g], self.u[gi], self.z[gi])
+                S.spkv_decode_attn(p, L.cache, L.ring, q[g], t, self.o[l], self.lse[l], L.ws)
+                gi += 1
+            else:
+                L = self.loc[li]
+                S.spkv_decode_append(p, None, L.ring, t, k[g], v[g], None, None, 0)
+                S.spkv_decode_attn(p, None, L.ring, q[g], t, self.o[l], self.lse[l], L.ws)
+                li += 1
+
+    LAUNCHES_GLOBAL = 2
+    LAUNCHES_LOCAL = 2

@@ -60,17 +60,32 @@ def test_argument_validation_without_gpu():
     assert S.lib.spkv_prefill_attn(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
                                    None, None, None, 0, 16, None, None, None) == S.ERR_ARG
     # misaligned pool pointer
-    cache = S.spkv_cache(8, 16, 16, 16, 16, 16, 16, 16, 4, 64, 4)
+    cache = S.spkv_cache(8, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
     assert S.lib.spkv_cache_reset(ctypes.byref(good), ctypes.byref(cache), None, None) == S.ERR_ARG
     # page_rows other than 64
-    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, 4, 32, 4)
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 32, 4)
     assert S.lib.spkv_cache_reset(ctypes.byref(good), ctypes.byref(cache), None, None) == S.ERR_ARG
     # ring compaction longer than the window, negative gated_from
-    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, 4, 64, 4)
-    ring = S.spkv_ring(16, 16, 16)
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
+    ring = S.spkv_ring(16, 16, 16, None)
     assert S.lib.spkv_write_compact(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
-                                    S.SRC_RING, None, None, 16, 16, 129, 129, None) == S.ERR_ARG
-    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, 16, -1, 16, 4, 4,
-                                 None) == S.ERR_ARG
-    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, None, 0, 16, 4, 4,
-                                 None) == S.ERR_ARG
+                                    S.SRC_RING, None, None, 16, None, 16, 129, 129, None) == S.ERR_ARG
+    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, 16, None, -1, 16, 4,
+                                 4, None) == S.ERR_ARG
+    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring), 16, 16, None, None, 0, 16, 4,
+                                 4, None) == S.ERR_ARG
+    # utilities kept in the cache: the compaction needs them; the ring's pending
+    # utilities need u_src / u_new; re-threshold needs the cache's utilities
+    cache_u = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, 16, 4, 64, 4)
+    assert S.lib.spkv_write_compact(ctypes.byref(good), ctypes.byref(cache_u), None, S.SRC_CHUNK,
+                                    16, 16, 16, None, 16, 4, 4, None) == S.ERR_ARG
+    ring_u = S.spkv_ring(16, 16, 16, 16)
+    assert S.lib.spkv_ring_write(ctypes.byref(good), ctypes.byref(ring_u), 16, 16, 16, None, 0, 16,
+                                 4, 4, None) == S.ERR_ARG
+    assert S.lib.spkv_decode_append(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring_u),
+                                    16, 16, 16, 16, None, 1, None) == S.ERR_ARG
+    assert S.lib.spkv_cache_rethreshold(ctypes.byref(good), ctypes.byref(cache), None,
+                                        ctypes.c_float(0.6), 16, 1 << 20, None) == S.ERR_ARG
+    assert S.lib.spkv_cache_rethreshold(ctypes.byref(good), ctypes.byref(cache_u), None,
+                                        ctypes.c_float(float("nan")), 16, 1 << 20, None) == S.ERR_ARG
+    assert S.lib.spkv_rethreshold_workspace_bytes(ctypes.byref(good), ctypes.byref(cache_u)) > 0

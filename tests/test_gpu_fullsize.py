@@ -138,3 +138,82 @@ def test_prefill16k_full_size():
     for i, t in enumerate(ts):
         o_ref, _ = O.gated_attention(Q[i:i + 1], K[:t + 1], V[:t + 1], z[:t + 1], wl.window, [t])
         C.check_attn(o_gpu[t], o_ref[0], "bf16", f"prefill16k query {t}")
+
+
+def test_decode32k_rethreshold_full_size():
+    """One decode32k layer (32768-token context, utilities kept) re-thresholded from
+    0.5 to 0.6 in place, then one per-token decode step at 0.6: sampled heads' index
+    lists and stored rows, and sampled batch rows' outputs, against the oracle."""
+    wl = _one_layer("decode32k")
+    tau2 = 0.6
+    p, Ls, inp = build_decode_state(wl, 1, 2, torch.device("cuda"), store_u=True)
+    L = Ls[0]
+    before = R.cache_lists(L)
+    ws = S.alloc_rethreshold_workspace(p, L.cache)
+    S.spkv_cache_rethreshold(p, L.cache, L.ring, tau2, ws)
+    status, flags = S.spkv_cache_check(L.cache)
+    assert status == S.OK, flags
+    after = R.cache_lists(L)
+    L.p = S.make_params(p.B, p.Hq, p.Hkv, p.head_dim, p.d_model, p.hid, p.window, tau2, p.dtype)
+    step = DecodeStep(L.p, Ls, "cuda")
+    step.launch(inp["h"][0], inp["q"][0], inp["k"][0], inp["v"][0], inp["t"][0])
+    torch.cuda.synchronize()
+    assert S.spkv_cache_check(L.cache)[0] == S.OK
+    o = step.o[0].float().cpu().numpy()
+    t = inp["t"][0].cpu().numpy()
+    W1, b1, W2, b2 = C.weights(wl)
+    for b in (1, 6):
+        tb = int(t[b])
+        u, _ = C.oracle_gates_rows(wl, 0, b, tb + 1, W1, b1, W2, b2)
+        z2 = O.gate(u, tau2)
+        K, V = C.kv_rows(wl, 0, b, tb + 1)
+        for kh in (0, 5):
+            bh = b * wl.Hkv + kh
+            want = O.rethreshold(before[bh], u[before[bh], kh], tau2)
+            near = set(np.nonzero((np.abs(u[:, kh] - tau2) < C.EXCLUDE) |
+                                  (np.abs(u[:, kh] - wl.tau) < C.EXCLUDE))[0].tolist())
+            got = [int(x) for x in after[bh] if int(x) not in near]
+            assert got == [int(x) for x in want if int(x) not in near]
+            Kc, Vc = R.cache_rows_kv(L, bh)
+            assert np.array_equal(Kc.float().numpy(), K[after[bh], kh])
+            assert np.array_equal(Vc.float().numpy(), V[after[bh], kh])
+        q = wl.q_rows(0, b, [tb])
+        o_ref, _ = O.gated_attention(q, K, V, z2, wl.window, [tb])
+        C.check_attn(o[b], o_ref[0], "bf16", f"rethreshold decode row {b}")
+
+
+def test_soft_attention_16k_full_size():
+    """Soft-gated training-time attention (Eqs. (5)-(6)) over a 16384-token sequence
+    with the prefill16k shapes, utilities from the utility perceptron (each side
+    computes its own: GPU spkv_score, oracle in fp64; Eq. (5) is smooth, so their
+    rounding differences do not flip anything), sampled query positions."""
+    from sparse_decode_attention_spkv_b200.inputs import gen as G_
+    wl = W.WORKLOADS["prefill16k"]
+    T = wl.ctx[0]
+    beta, c = 0.01, 1e6
+    W1, b1, W2, b2 = C.weights(wl)
+    p = S.make_params(1, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau, S.BF16)
+    h = torch.empty((T, wl.d_model), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((1, T, wl.Hq, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    k = torch.empty((1, T, wl.Hkv, wl.head_dim), dtype=torch.bfloat16, device="cuda")
+    v = torch.empty_like(k)
+    D.fill_normal(h, wl.key(0, G_.T_H), 1.0)
+    D.fill_rope(q, wl.key(0, G_.T_Q), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_rope(k, wl.key(0, G_.T_K), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_normal(v, wl.key(0, G_.T_V), wl.qkv_scale)
+    u = torch.empty((T, wl.Hkv), dtype=torch.float32, device="cuda")
+    z = torch.empty((T, wl.Hkv), dtype=torch.uint8, device="cuda")
+    S.spkv_score(p, h, T, C.dev(W1, "bf16"), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2), u, z)
+    o = torch.empty_like(q)
+    ws = torch.empty(S.spkv_soft_attn_workspace_bytes(p, T), dtype=torch.uint8, device="cuda")
+    S.spkv_soft_attn(p, q, k, v, u, T, beta, c, o, None, ws)
+    o_gpu = o[0].float().cpu().numpy()
+    u_ref, _ = C.oracle_gates_rows(wl, 0, 0, T, W1, b1, W2, b2)
+    K, V = C.kv_rows(wl, 0, 0, T)
+    rng = np.random.default_rng(1)
+    ts = sorted(set([0, 127, 128, 4096, 16383] + rng.integers(0, T, 10).tolist()))
+    Q = wl.q_rows(0, 0, ts)
+    for i, t in enumerate(ts):
+        o_ref, _ = O.soft_gated_attention(Q[i:i + 1], K[:t + 1], V[:t + 1], u_ref[:t + 1], wl.tau,
+                                          beta, c, wl.window, [t])
+        C.check_attn(o_gpu[t], o_ref[0], "bf16", f"soft attention query {t}")

@@ -92,14 +92,14 @@ def test_compact_chunks_and_ring(dtype):
         src_pos = torch.full((wl.B,), c0, dtype=torch.int32, device="cuda")
         S.spkv_write_compact(layer.p, layer.cache, layer.ring, S.SRC_CHUNK,
                              kd[:, c0:].contiguous(), vd[:, c0:].contiguous(),
-                             zd[:, c0:].contiguous(), src_pos, c1 - c0, T - c0)
+                             zd[:, c0:].contiguous(), None, src_pos, c1 - c0, T - c0)
     # the last 128 rows through the ring
     w = wl.window
     src_pos = torch.full((wl.B,), 2372, dtype=torch.int32, device="cuda")
     S.spkv_ring_write(layer.p, layer.ring, kd[:, 2372:].contiguous(), vd[:, 2372:].contiguous(),
-                      zd[:, 2372:].contiguous(), 0, src_pos, T - 2372, T - 2372)
+                      zd[:, 2372:].contiguous(), None, 0, src_pos, T - 2372, T - 2372)
     S.spkv_write_compact(layer.p, layer.cache, layer.ring, S.SRC_RING, None, None,
-                         zd[:, 2372:].contiguous(), src_pos, T - 2372, T - 2372)
+                         zd[:, 2372:].contiguous(), None, src_pos, T - 2372, T - 2372)
     assert T - 2372 == w
     status, flags = S.spkv_cache_check(layer.cache)
     assert status == S.OK and flags == 0
@@ -121,7 +121,7 @@ def test_compact_capacity_is_flagged():
                            num_pages=2, max_pages_per_head=8)
     z = torch.ones((1, 1000, 1), dtype=torch.uint8, device="cuda")
     kv = torch.randn((1, 1000, 1, 128), device="cuda").to(torch.bfloat16)
-    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, kv, kv, z,
+    S.spkv_write_compact(p, layer.cache, layer.ring, S.SRC_CHUNK, kv, kv, z, None,
                          torch.zeros(1, dtype=torch.int32, device="cuda"), 1000, 1000)
     status, flags = S.spkv_cache_check(layer.cache)
     assert status == S.ERR_CAPACITY and flags & S.FLAG_POOL_FULL

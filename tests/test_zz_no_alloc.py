@@ -42,9 +42,9 @@ def _state(wl, T0):
                     C.dev(k[:, :T0], wl.dtype), C.dev(v[:, :T0], wl.dtype), 0,
                     n_compact=max(0, T0 - w))
     t_pos = torch.full((wl.B,), T0, dtype=torch.int32, device="cuda")
-    _, z_t = R.score(layer, C.dev(h[:, T0], wl.dtype), wl.B)
+    u_t, z_t = R.score(layer, C.dev(h[:, T0], wl.dtype), wl.B)
     S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, C.dev(k[:, T0], wl.dtype),
-                         C.dev(v[:, T0], wl.dtype), z_t, 1)
+                         C.dev(v[:, T0], wl.dtype), z_t, u_t, 1)
     return p, layer, C.dev(q[:, T0], wl.dtype), t_pos
 
 
@@ -81,8 +81,10 @@ def test_noalloc_rejects_shapes_beyond_the_scratch():
     assert need > S.NOALLOC_SCRATCH_BYTES
     buf = torch.zeros(1024, dtype=torch.uint8, device="cuda")
     a = buf.data_ptr()
-    cache = S.spkv_cache(a, a, a, a, a, a, a, a, 1, S.PAGE_ROWS, 1)
-    ring = S.spkv_ring(a, a, a)
+    cache = S.spkv_cache(K_pool=a, V_pool=a, pos_pool=a, page_table=a, count=a, count_prev=a,
+                         pool_top=a, err_flag=a, u_pool=None, num_pages=1,
+                         page_rows=S.PAGE_ROWS, max_pages_per_head=1)
+    ring = S.spkv_ring(K_win=a, V_win=a, z_win=a, u_win=None)
     st = S.lib.spkv_decode_attn_noalloc(ctypes.byref(p), ctypes.byref(cache), ctypes.byref(ring),
                                         a, a, a, None, None)
     assert st == S.ERR_UNSUPPORTED
