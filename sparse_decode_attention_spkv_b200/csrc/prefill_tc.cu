@@ -13,7 +13,10 @@
 // Both contractions are dense tensor-core tiles: S = Q K^T (M=128 queries, N=64
 // keys, K=128) and O += P V (M=128, N=128, K=64 keys), bf16 operands, fp32
 // accumulators in TMEM.  P is written back into TMEM over S and fed to the second
-// MMA as its A operand.
+// MMA as its A operand.  S is double-buffered per head (TMEM: O0, O1, then two S
+// buffers per head, 512 columns), and the MMA thread issues S(j+1) before PV(j):
+// the softmax of block j+1 runs while the tensor cores do PV(j) and the other
+// head's work, so the tensor pipe is not left waiting on one softmax at a time.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q once, then K/V (+ positions) per block, 3 stages;
@@ -21,7 +24,8 @@
 //   warps 4-7   softmax of head 0 (one query row per thread, TMEM lanes 0..127);
 //   warps 8-11  softmax of head 1.
 // Softmax runs in the log2 domain; the running max is raised only when a score
-// exceeds it by more than 8, and only then is the O row in TMEM rescaled.
+// exceeds it by more than 8, and only then is the O row in TMEM rescaled (after the
+// previous block's PV has completed: pv_done).
 // Every mbarrier wait is bounded (a stuck wait raises SPKV_FLAG_TIMEOUT).
 //
 // The same kernel (SOFT = true) computes the soft-gated attention used at training
@@ -51,7 +55,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kSlack = 8.f;
 
-constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS0 = 256, kColS1 = 320;
+constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS = 256;  // S[h][buf] at kColS + 128 h + 64 buf
 
 struct __align__(1024) TcSmem {
   char q[2][2][kQT * 128];        // [head][d half] 128 rows x 128 B, 128B-swizzled
@@ -62,8 +66,9 @@ struct __align__(1024) TcSmem {
   uint64_t q_full;
   uint64_t kv_full[kStg];
   uint64_t kv_empty[kStg];
-  uint64_t s_ready[2];
+  uint64_t s_ready[2][2];  // [head][buffer]
   uint64_t p_ready[2];
+  uint64_t pv_done[2];
   uint64_t o_ready[2];
   uint32_t tmem_base;
   int cnt[4];
@@ -150,6 +155,14 @@ __device__ __forceinline__ void tma_4d(void* dst, const CUtensorMap* map, int c0
       : "memory");
 }
 
+// 2^x on the MUFU unit (ex2.approx, flush-to-zero): the scores are <= 8 above the
+// running max, so x < 8 and the result is a normal number or 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
   return *reinterpret_cast<const uint32_t*>(&v);
@@ -195,8 +208,10 @@ __global__ void __launch_bounds__(kThr, 1)
       mbar_init(&sm.kv_empty[s], 1);
     }
     for (int h = 0; h < 2; ++h) {
-      mbar_init(&sm.s_ready[h], 1);
+      mbar_init(&sm.s_ready[h][0], 1);
+      mbar_init(&sm.s_ready[h][1], 1);
       mbar_init(&sm.p_ready[h], 128);
+      mbar_init(&sm.pv_done[h], 1);
       mbar_init(&sm.o_ready[h], 1);
     }
     sm.cnt[0] = sm.cnt[1] = sm.cnt[2] = sm.cnt[3] = 0;
@@ -300,38 +315,45 @@ __global__ void __launch_bounds__(kThr, 1)
                                    ((uint32_t)(kQT >> 4) << 24);
       constexpr uint32_t idesc_pv = (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) |
                                     ((uint32_t)(kHD >> 3) << 17) | ((uint32_t)(kQT >> 4) << 24);
-      const uint32_t colS[2] = {kColS0, kColS1}, colO[2] = {kColO0, kColO1};
+      const uint32_t colO[2] = {kColO0, kColO1};
       mbar_wait(&sm.q_full, 0, err);
       tc_fence_after();
-      for (int j = 0; j <= J; ++j) {
-        const int s = j % kStg, sp = (j + kStg - 1) % kStg;
-        if (j < J) {
-          mbar_wait(&sm.kv_full[s], (j / kStg) & 1, err);
-          tc_fence_after();
-        }
+      // S_h(j) = Q_h K(j)^T into buffer j % 2 of head h
+      auto issue_s = [&](int j) {
+        const int s = j % kStg;
+        mbar_wait(&sm.kv_full[s], (j / kStg) & 1, err);
+        tc_fence_after();
         for (int hh = 0; hh < 2; ++hh) {
-          if (j > 0) {  // O_h += P_h(j-1) V(j-1)
-            mbar_wait(&sm.p_ready[hh], (j - 1) & 1, err);
-            tc_fence_after();
+          const uint32_t col = kColS + 128 * hh + 64 * (j & 1);
 #pragma unroll
-            for (int kk = 0; kk < kKB / 16; ++kk) {
-              const uint64_t bd = smem_desc(sm.v[sp][0] + kk * 16 * 128, 8192, 1024);
-              mma_ts(tmem + colO[hh], tmem + colS[hh] + kk * 8, bd, idesc_pv, (j > 1 || kk > 0) ? 1u : 0u);
-            }
-            if (j == J) mma_commit(&sm.o_ready[hh]);
+          for (int kk = 0; kk < kHD / 16; ++kk) {
+            const uint64_t ad = smem_desc(sm.q[hh][kk >> 2] + (kk & 3) * 32, 16, 1024);
+            const uint64_t bd = smem_desc(sm.k[s][kk >> 2] + (kk & 3) * 32, 16, 1024);
+            mma_ss(tmem + col, ad, bd, idesc_s, kk > 0 ? 1u : 0u);
           }
-          if (j < J) {  // S_h = Q_h K(j)^T
-#pragma unroll
-            for (int kk = 0; kk < kHD / 16; ++kk) {
-              const uint64_t ad = smem_desc(sm.q[hh][kk >> 2] + (kk & 3) * 32, 16, 1024);
-              const uint64_t bd = smem_desc(sm.k[s][kk >> 2] + (kk & 3) * 32, 16, 1024);
-              mma_ss(tmem + colS[hh], ad, bd, idesc_s, kk > 0 ? 1u : 0u);
-            }
-            mma_commit(&sm.s_ready[hh]);
-          }
+          mma_commit(&sm.s_ready[hh][j & 1]);
         }
-        if (j > 0) mma_commit(&sm.kv_empty[sp]);
+      };
+      if (J > 0) issue_s(0);
+      for (int j = 0; j < J; ++j) {
+        // the next block's scores go ahead of this block's PV (double-buffered S; the
+        // buffer they overwrite held P(j-1), whose PV was issued before)
+        if (j + 1 < J) issue_s(j + 1);
+        const int s = j % kStg;
+        for (int hh = 0; hh < 2; ++hh) {  // O_h += P_h(j) V(j)
+          mbar_wait(&sm.p_ready[hh], j & 1, err);
+          tc_fence_after();
+          const uint32_t col = kColS + 128 * hh + 64 * (j & 1);
+#pragma unroll
+          for (int kk = 0; kk < kKB / 16; ++kk) {
+            const uint64_t bd = smem_desc(sm.v[s][0] + kk * 16 * 128, 8192, 1024);
+            mma_ts(tmem + colO[hh], tmem + col + kk * 8, bd, idesc_pv, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sm.pv_done[hh]);
+        }
+        mma_commit(&sm.kv_empty[s]);
       }
+      for (int hh = 0; hh < 2; ++hh) mma_commit(&sm.o_ready[hh]);
     }
   } else if (warp >= 4) {
     // ------------------------------ softmax --------------------------------------
@@ -340,12 +362,13 @@ __global__ void __launch_bounds__(kThr, 1)
     const int r = quad * 32 + lane;
     const int t = t0 + r;
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
-    const uint32_t colS = hh ? kColS1 : kColS0, colO = hh ? kColO1 : kColO0;
+    const uint32_t colO = hh ? kColO1 : kColO0;
     const float c = kLog2e * rsqrtf((float)kHD);
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < J; ++j) {
       const int s = j % kStg;
-      mbar_wait(&sm.s_ready[hh], j & 1, err);
+      const uint32_t colS = kColS + 128 * hh + 64 * (j & 1);
+      mbar_wait(&sm.s_ready[hh][j & 1], (j >> 1) & 1, err);
       mbar_wait(&sm.kv_full[s], (j / kStg) & 1, err);
       tc_fence_after();
       uint32_t raw[64];
@@ -385,9 +408,24 @@ __global__ void __launch_bounds__(kThr, 1)
         }
       }
       const bool need = rmax > m + kSlack;
-      if (__any_sync(0xffffffffu, need)) {
-        const float mnew = need ? fmaxf(m, rmax) : m;
-        const float alpha = (m == -INFINITY) ? 0.f : exp2f(m - mnew);
+      const bool any_need = __any_sync(0xffffffffu, need);
+      const float mnew = need ? fmaxf(m, rmax) : m;
+      uint32_t pk[32];
+      float ps = 0.f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) {
+        const float p0 = x[2 * i] == -INFINITY ? 0.f : fast_exp2(x[2 * i] - mnew);
+        const float p1 = x[2 * i + 1] == -INFINITY ? 0.f : fast_exp2(x[2 * i + 1] - mnew);
+        ps += p0 + p1;
+        pk[i] = pack_bf16(p0, p1);
+      }
+      // O may be touched only once the previous block's PV has landed in it
+      if (j > 0) {
+        mbar_wait(&sm.pv_done[hh], (j - 1) & 1, err);
+        tc_fence_after();
+      }
+      if (any_need) {
+        const float alpha = (m == -INFINITY) ? 0.f : fast_exp2(m - mnew);
         if (j > 0) {  // O holds P V of earlier blocks: rescale it in TMEM
 #pragma unroll
           for (int cc = 0; cc < kHD; cc += 32) {
@@ -398,19 +436,9 @@ __global__ void __launch_bounds__(kThr, 1)
             for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
             tmem_st32(lane_addr + colO + cc, o);
           }
-          tmem_wait_st();
         }
         l *= alpha;
         m = mnew;
-      }
-      uint32_t pk[32];
-      float ps = 0.f;
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = x[2 * i] == -INFINITY ? 0.f : exp2f(x[2 * i] - m);
-        const float p1 = x[2 * i + 1] == -INFINITY ? 0.f : exp2f(x[2 * i + 1] - m);
-        ps += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
       }
       l += ps;
       tmem_st32(lane_addr + colS, pk);
