@@ -364,6 +364,7 @@ __global__ void __launch_bounds__(kThr, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t colO = hh ? kColO1 : kColO0;
     const float c = kLog2e * rsqrtf((float)kHD);
+    const float inv_c = 1.f / c;  // soft bias (log2 units) back to raw-score units
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < J; ++j) {
       const int s = j % kStg;
@@ -375,16 +376,16 @@ __global__ void __launch_bounds__(kThr, 1)
       tmem_ld32(lane_addr + colS, raw);
       tmem_ld32(lane_addr + colS + 32, raw + 32);
       tmem_wait_ld();
+      // scores in the raw (unscaled) domain, masked keys at -inf; for the soft mask the
+      // per-key bias is pre-divided by the scale so that one fma gives the exponent
       float x[64];
-      float rmax = -INFINITY;
       if (j < bl.nc) {
         const bool dense = (j + 1) * kKB <= bl.nfull;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
           const int row = j * kKB + i;
           const bool vis = dense || (row < bl.nrows && sm.pos[s][i] <= t - kWin);
-          x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
-          rmax = fmaxf(rmax, x[i]);
+          x[i] = vis ? __uint_as_float(raw[i]) : -INFINITY;
         }
       } else {
         const int pb = bl.wfirst + (j - bl.nc) * kKB;
@@ -394,31 +395,43 @@ __global__ void __launch_bounds__(kThr, 1)
           for (int i = 0; i < 64; ++i) {
             const int dlt = t - (pb + i);
             x[i] = dlt < 0 ? -INFINITY
-                           : __uint_as_float(raw[i]) * c + (dlt >= kWin ? bias[i] : 0.f);
-            rmax = fmaxf(rmax, x[i]);
+                           : __uint_as_float(raw[i]) + (dlt >= kWin ? bias[i] * inv_c : 0.f);
           }
         } else {
 #pragma unroll
           for (int i = 0; i < 64; ++i) {
             const int dlt = t - (pb + i);
             const bool vis = dlt >= 0 && dlt < kWin;
-            x[i] = vis ? __uint_as_float(raw[i]) * c : -INFINITY;
-            rmax = fmaxf(rmax, x[i]);
+            x[i] = vis ? __uint_as_float(raw[i]) : -INFINITY;
           }
         }
       }
+      // row maximum: 8 independent partial maxima, then a short tree
+      float mx[8];
+#pragma unroll
+      for (int a = 0; a < 8; ++a) mx[a] = x[a];
+#pragma unroll
+      for (int i = 8; i < 64; ++i) mx[i & 7] = fmaxf(mx[i & 7], x[i]);
+      const float rmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7]))) * c;
       const bool need = rmax > m + kSlack;
       const bool any_need = __any_sync(0xffffffffu, need);
       const float mnew = need ? fmaxf(m, rmax) : m;
+      // p = 2^(x c - m): one packed fma per pair, then MUFU; masked keys give 2^-inf = 0
+      const float msafe = mnew == -INFINITY ? 0.f : mnew;
       uint32_t pk[32];
-      float ps = 0.f;
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-msafe, -msafe);
 #pragma unroll
       for (int i = 0; i < 32; ++i) {
-        const float p0 = x[2 * i] == -INFINITY ? 0.f : fast_exp2(x[2 * i] - mnew);
-        const float p1 = x[2 * i + 1] == -INFINITY ? 0.f : fast_exp2(x[2 * i + 1] - mnew);
-        ps += p0 + p1;
-        pk[i] = pack_bf16(p0, p1);
+        const float2 e = fma2(make_float2(x[2 * i], x[2 * i + 1]), c2, nm2);
+        const float2 pp = make_float2(fast_exp2(e.x), fast_exp2(e.y));
+        acc[i & 3] = add2(acc[i & 3], pp);
+        pk[i] = pack_bf16(pp.x, pp.y);
       }
+      const float ps = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
+                       (acc[3].x + acc[3].y);
       // O may be touched only once the previous block's PV has landed in it
       if (j > 0) {
         mbar_wait(&sm.pv_done[hh], (j - 1) & 1, err);
