@@ -102,10 +102,10 @@ __global__ void __launch_bounds__(kMoveThreads)
   extern __shared__ __align__(16) char smem[];
   char* kbuf = smem;                                    // [64][row_bytes]
   char* vbuf = kbuf + (size_t)kPageRows * row_bytes;    // [64][row_bytes]
+  int* s_base = reinterpret_cast<int*>(vbuf + (size_t)kPageRows * row_bytes);  // [n_heads + 1]
   __shared__ int s_pos[kPageRows];
   __shared__ float s_u[kPageRows];
   __shared__ int s_dst[kPageRows];                      // new row index, or -1
-  __shared__ int s_base[kMaxHeadsR + 1];
   __shared__ int s_item, s_ok, s_wc[2];
   __shared__ __align__(8) uint64_t bar;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -256,7 +256,7 @@ cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const 
   CacheMut m = cache_mut(c);
   RethrWs ws = carve(workspace, n_heads, c.max_pages_per_head);
   rethr_plan<<<n_heads, kPlanThreads, 0, stream>>>(m, ws, tau_new);
-  const size_t smem = (size_t)2 * kPageRows * row_bytes;
+  const size_t smem = (size_t)2 * kPageRows * row_bytes + (size_t)(n_heads + 1) * 4;
   static int configured = 0;
   if ((int)smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(rethr_move, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -265,8 +265,8 @@ cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const 
     configured = (int)smem;
   }
   // as many CTAs per SM as shared memory allows (each streams one page at a time)
-  int per_sm = (int)((200u << 10) / (smem + (10u << 10)));
-  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
+  int per_sm = (int)((216u << 10) / (smem + (2u << 10)));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
   rethr_move<<<num_sms * per_sm, kMoveThreads, smem, stream>>>(m, ws, tau_new, n_heads, row_bytes);
   RingMut r = ring ? ring_mut(*ring) : RingMut{nullptr, nullptr, nullptr, nullptr};
   const int ring_entries = ring ? p.B * p.window * p.Hkv : 0;

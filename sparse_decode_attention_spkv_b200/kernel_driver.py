@@ -4,6 +4,8 @@
     python -m sparse_decode_attention_spkv_b200.kernel_driver score   [--tokens 8]
     python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096]
     python -m sparse_decode_attention_spkv_b200.kernel_driver prefill [--chunk 4096]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver rethreshold [--steps 2]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver soft [--seq 8192]
 
 ``decode`` builds the decode32k state (batch 8, 32K context, ~300 MB of live K/V per
 layer, more than L2) for a few layers and runs eager decode steps; the others run
@@ -90,17 +92,58 @@ def run_prefill(args):
     torch.cuda.synchronize()
 
 
+def run_rethreshold(args):
+    """One decode32k layer with utilities kept, re-thresholded at the median stored
+    utility; the cache is restored from a copy before each repetition."""
+    from .states import build_decode_state
+    wl = W.small_case("decode32k", layers=1)
+    p, Ls, _ = build_decode_state(wl, 1, 1, torch.device("cuda"), store_u=True)
+    c = Ls[0].cache
+    saved = {k: getattr(c, k).clone() for k in ("K_pool", "V_pool", "pos_pool", "u_pool", "count",
+                                                  "count_prev", "page_table")}
+    ws = S.alloc_rethreshold_workspace(p, c)
+    n = int(c.count.sum().item())
+    tau = float(c.u_pool.flatten()[: max(1, n)].median().item())
+    for _ in range(args.steps):
+        for k, v in saved.items():
+            getattr(c, k).copy_(v)
+        S.spkv_cache_rethreshold(p, c, Ls[0].ring, tau, ws)
+    torch.cuda.synchronize()
+
+
+def run_soft(args):
+    """Soft-gated attention over one sequence with the prefill16k shapes."""
+    wl = W.WORKLOADS["prefill16k"]
+    T = args.seq
+    bf = torch.bfloat16
+    p = S.make_params(1, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, wl.tau, S.BF16)
+    q = torch.empty((1, T, wl.Hq, wl.head_dim), dtype=bf, device="cuda")
+    k = torch.empty((1, T, wl.Hkv, wl.head_dim), dtype=bf, device="cuda")
+    v = torch.empty_like(k)
+    D.fill_rope(q, wl.key(0, gen.T_Q), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_rope(k, wl.key(0, gen.T_K), 0, wl.T_total, wl.qkv_scale, wl.rope_base)
+    D.fill_normal(v, wl.key(0, gen.T_V), wl.qkv_scale)
+    u = torch.rand((1, T, wl.Hkv), device="cuda") * 0.6 + 0.2
+    o = torch.empty_like(q)
+    ws = torch.empty(S.spkv_soft_attn_workspace_bytes(p, T), dtype=torch.uint8, device="cuda")
+    for _ in range(args.steps):
+        S.spkv_soft_attn(p, q, k, v, u, T, 0.01, 1e6, o, None, ws)
+    torch.cuda.synchronize()
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("kernel", choices=["decode", "score", "compact", "prefill"])
+    ap.add_argument("kernel", choices=["decode", "score", "compact", "prefill", "rethreshold", "soft"])
     ap.add_argument("--layers", type=int, default=1)
     ap.add_argument("--steps", type=int, default=3)
     ap.add_argument("--tokens", type=int, default=8)
     ap.add_argument("--rows", type=int, default=4096)
     ap.add_argument("--chunk", type=int, default=4096)
+    ap.add_argument("--seq", type=int, default=8192)
     args = ap.parse_args()
     torch.cuda.set_device(0)
-    {"decode": run_decode, "score": run_score, "compact": run_compact, "prefill": run_prefill}[args.kernel](args)
+    {"decode": run_decode, "score": run_score, "compact": run_compact, "prefill": run_prefill,
+     "rethreshold": run_rethreshold, "soft": run_soft}[args.kernel](args)
     st, flags = (S.OK, 0)
     print(f"kernel_driver {args.kernel} done")
 
