@@ -31,8 +31,9 @@
 // The same kernel (SOFT = true) computes the soft-gated attention used at training
 // time (§2.1, "soft relaxation", Eqs. (5)-(6)): every key s <= t of the sequence,
 // read in 64-key blocks from the sequence K/V, with the additive score 0 inside the
-// causal window and c (alpha_s - 1) outside it; the per-key bias (already scaled to
-// the log2 domain) rides with each block.  No key block is skipped.
+// causal window and c (alpha_s - 1) outside it; the per-key bias (already divided by
+// the score scale, i.e. in raw q.k units) rides with each block.  No key block is
+// skipped.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
@@ -364,7 +365,6 @@ __global__ void __launch_bounds__(kThr, 1)
     const uint32_t lane_addr = tmem + ((uint32_t)(quad * 32) << 16);
     const uint32_t colO = hh ? kColO1 : kColO0;
     const float c = kLog2e * rsqrtf((float)kHD);
-    const float inv_c = 1.f / c;  // soft bias (log2 units) back to raw-score units
     float m = -INFINITY, l = 0.f;
     for (int j = 0; j < J; ++j) {
       const int s = j % kStg;
@@ -390,12 +390,16 @@ __global__ void __launch_bounds__(kThr, 1)
       } else {
         const int pb = bl.wfirst + (j - bl.nc) * kKB;
         if constexpr (SOFT) {
-          const float* bias = reinterpret_cast<const float*>(sm.pos[s]);
+          const float* bias = reinterpret_cast<const float*>(sm.pos[s]);  // raw-score units
+          if (pb + kKB - 1 <= t0 - kWin) {  // every key of the block is outside every window
 #pragma unroll
-          for (int i = 0; i < 64; ++i) {
-            const int dlt = t - (pb + i);
-            x[i] = dlt < 0 ? -INFINITY
-                           : __uint_as_float(raw[i]) + (dlt >= kWin ? bias[i] * inv_c : 0.f);
+            for (int i = 0; i < 64; ++i) x[i] = __uint_as_float(raw[i]) + bias[i];
+          } else {
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              const int dlt = t - (pb + i);
+              x[i] = dlt < 0 ? -INFINITY : __uint_as_float(raw[i]) + (dlt >= kWin ? bias[i] : 0.f);
+            }
           }
         } else {
 #pragma unroll

@@ -8,8 +8,8 @@
 // bias instead of being removed.  The forward pass here is
 //   o_t = softmax_s(q_t k_s / sqrt(d_k) + M_soft(t, s)) v_s   over all s <= t.
 // soft_bias computes the per-key bias c (alpha_s - 1) = -c / (1 + exp((u_s - tau) /
-// beta)) (the second form has no cancellation for alpha near 1), scaled to the log2
-// domain, into a [B][Hkv][T] buffer; the attention itself runs on the tensor cores
+// beta)) (the second form has no cancellation for alpha near 1) into a [B][Hkv][T]
+// buffer, in the units the attention kernel adds it in; the attention itself runs on the tensor cores
 // (prefill_tc.cu, SOFT mode) or, for other shapes, in soft_simple_kernel below.
 #include <math.h>
 
@@ -23,10 +23,11 @@ constexpr int kWarps = 4;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// u [B][T][Hkv] -> bias [B][Hkv][T], log2 units.
+// u [B][T][Hkv] -> bias [B][Hkv][T] in units of out_scale (1/(score scale) for the
+// tensor-core path, which adds it to raw q.k; log2 e for the CUDA-core path).
 __global__ void __launch_bounds__(256)
     soft_bias_kernel(const float* __restrict__ u, float* __restrict__ bias, int B, int T, int hkv,
-                     float tau, float inv_beta, float c) {
+                     float tau, float inv_beta, float c, float out_scale) {
   const size_t n = (size_t)B * T * hkv;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
        i += (size_t)gridDim.x * blockDim.x) {
@@ -35,7 +36,7 @@ __global__ void __launch_bounds__(256)
     const int t = (int)(bt % T), b = (int)(bt / T);
     const float x = (u[i] - tau) * inv_beta;
     const float m = -c / (1.f + expf(x));  // c (alpha - 1)
-    bias[((size_t)b * hkv + kh) * T + t] = m * kLog2e;
+    bias[((size_t)b * hkv + kh) * T + t] = m * out_scale;
   }
 }
 
@@ -188,11 +189,15 @@ cudaError_t launch_soft(const spkv_params& p, const void* q, const void* K, cons
   float* bias = static_cast<float*>(workspace);
   const size_t n = (size_t)p.B * seq_len * p.Hkv;
   const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
-  soft_bias_kernel<<<blocks, 256, 0, stream>>>(u, bias, p.B, seq_len, p.Hkv, p.tau, 1.f / beta, c);
+  const bool tc = soft_tc_supported(p, seq_len);
+  // the tensor-core path adds the bias to raw q.k (scaled by log2 e / sqrt(d) later);
+  // the CUDA-core path adds it to scores already in the log2 domain
+  const float out_scale = tc ? sqrtf((float)p.head_dim) : kLog2e;
+  soft_bias_kernel<<<blocks, 256, 0, stream>>>(u, bias, p.B, seq_len, p.Hkv, p.tau, 1.f / beta, c,
+                                               out_scale);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  if (soft_tc_supported(p, seq_len))
-    return launch_soft_tc(p, q, K, V, bias, seq_len, o, lse, err, stream);
+  if (tc) return launch_soft_tc(p, q, K, V, bias, seq_len, o, lse, err, stream);
   if (p.dtype == SPKV_BF16)
     return p.head_dim == 128 ? dispatch_g<BF16, 128>(p, q, K, V, bias, seq_len, o, lse, stream)
                              : dispatch_g<BF16, 64>(p, q, K, V, bias, seq_len, o, lse, stream);
