@@ -181,7 +181,7 @@ def run_gpu(args, world, rank, local):
                                                           kv_bytes_layers)
     p, Ls, inp = build_decode_state(wl, layers, steps_total, device)
     T0 = wl.ctx[0]
-    step = DecodeStep(p, Ls, device)
+    step = DecodeStep(p, Ls, device, split=args.decode_step == "split")
 
     # one eager decode-attention call per layer sets kernel attributes before capture
     for l, L in enumerate(Ls):
@@ -280,6 +280,7 @@ def run_gpu(args, world, rank, local):
         "config": {"workload": "decode32k: batch 8 x 32 layers, 32q/8kv heads, head_dim 128, "
                                "d_model 4096, utility MLP 4096->128->8, w=128, tau=0.5, 32768-token "
                                "context, per-head keep U[5%,50%], per-token retirement",
+                   "decode_step": args.decode_step,
                    "global_batch": world * p.B, "seq_len": T0, "layers": layers,
                    "parallelism": f"replicas x{world} (no data-path collective)",
                    "l2": "inputs larger than L2 (every step reads all live K/V, ~GBs)"},
@@ -294,7 +295,7 @@ def run_gpu(args, world, rank, local):
                                        f"{timed_layers[1] if len(timed_layers) > 1 else ''}.."
                                        f"{timed_layers[-1]} in every timed step (CUDA events on "
                                        f"the launching stream)"},
-        "gpu_launches": DecodeStep.LAUNCHES_PER_LAYER * layers * K,
+        "gpu_launches": (DecodeStep.LAUNCHES_PER_LAYER + (1 if step.split else 0) + 1) * layers * K,
         "clocks": clocks.summary(),
         "e2e": e2e,
     }
@@ -660,7 +661,10 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=20)
     ap.add_argument("--cpu-units", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-aux", action="store_true", help="skip the secondary prefill measurement")
+    ap.add_argument("--no-aux", action="store_true", help="skip the secondary measurements")
+    ap.add_argument("--decode-step", default="split", choices=["split", "fused"],
+                    help="split: the new tokens are scored on a second stream beside the "
+                         "attention; fused: score, retirement and ring write in one launch")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -183,6 +183,20 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* cache, cons
                              const void* v_new, float* u_out, uint8_t* z_out,
                              spkv_stream_t stream);
 
+/* a1 for one per-token decode step, kept off the attention's critical path: the
+ * utility and gate of the B new tokens (h [B][d_model], the token of batch row b at
+ * position t_pos[b]) exactly as spkv_score computes them, each gate (and utility, if
+ * ring->u_win is set) stored in its token's window slot t_pos[b] % window.  Use it after
+ * spkv_decode_append(..., z_new = NULL, u_new = NULL, retire = 1) of the same step
+ * (which retires token t - window and stores the new token with gate 0).  The gate of a
+ * token is read only when it leaves the window, so this call may run on another stream
+ * while spkv_decode_attn of the step (and later layers) proceed; it must finish before
+ * the step that retires the token.  u_out [B][Hkv] f32 (required when ring->u_win is
+ * set, else may be NULL), z_out [B][Hkv] uint8. */
+int spkv_decode_score(const spkv_params* p, const spkv_ring* ring, const int32_t* t_pos,
+                      const void* h, const void* W1, const float* b1, const float* W2,
+                      const float* b2, float* u_out, uint8_t* z_out, spkv_stream_t stream);
+
 /* a3 -- store the last min(n_rows, window) rows of a chunk in the ring: row i of
  * batch b (position src_pos[b] + i) goes to slot (src_pos[b] + i) % window.  The
  * slot's gate is 0 for rows i < gated_from (already in the cache, so retiring them

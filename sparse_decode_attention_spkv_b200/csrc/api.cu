@@ -174,6 +174,19 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const sp
                                              u_out, z_out, static_cast<cudaStream_t>(stream)));
 }
 
+int spkv_decode_score(const spkv_params* p, const spkv_ring* ring, const int32_t* t_pos,
+                      const void* h, const void* W1, const float* b1, const float* W2,
+                      const float* b2, float* u_out, uint8_t* z_out, spkv_stream_t stream) {
+  if (!params_ok(p) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
+  if (!t_pos || !h || !W1 || !b1 || !W2 || !b2 || !z_out) return SPKV_ERR_ARG;
+  if (!aligned16(h) || !aligned16(W1)) return SPKV_ERR_ARG;
+  if (ring->u_win && !u_out) return SPKV_ERR_ARG;
+  if (!spkv::score_supported(*p)) return SPKV_ERR_UNSUPPORTED;
+  return status_of(spkv::launch_score_gates(*p, *ring, t_pos, h, W1, b1, W2, b2, u_out, z_out,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
 int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
                     const void* V_src, const uint8_t* z_src, const float* u_src, int gated_from,
                     const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream) {

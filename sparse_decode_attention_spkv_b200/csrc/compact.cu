@@ -171,6 +171,8 @@ __global__ void __launch_bounds__(128)
                          const char* __restrict__ k_new, const char* __restrict__ v_new,
                          const uint8_t* __restrict__ z_new, const float* __restrict__ u_new,
                          int retire, int n_heads, int hkv, int window, int row_bytes) {
+  grid_dependency_wait();    // programmatic dependent launch: inputs may come from the
+  grid_dependents_launch();  // kernel before; the attention after may start its launch
   const int lane = threadIdx.x & 31;
   const int bh = blockIdx.x * 4 + (threadIdx.x >> 5);
   if (bh >= n_heads) return;
@@ -239,11 +241,10 @@ cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, cons
                                  cudaStream_t stream) {
   const int n_heads = p.B * p.Hkv;
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
-  decode_append_kernel<<<(n_heads + 3) / 4, 128, 0, stream>>>(
-      mut(c), ring_mut(ring), t_pos, static_cast<const char*>(k_new),
-      static_cast<const char*>(v_new), z_new, u_new, retire, n_heads, p.Hkv, p.window,
-      p.head_dim * esize);
-  return cudaGetLastError();
+  return launch_pdl(decode_append_kernel, dim3((n_heads + 3) / 4), dim3(128), 0, stream, mut(c),
+                    ring_mut(ring), t_pos, static_cast<const char*>(k_new),
+                    static_cast<const char*>(v_new), z_new, u_new, retire, n_heads, p.Hkv, p.window,
+                    p.head_dim * esize);
 }
 
 cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const void* K_src,

@@ -134,12 +134,18 @@ __global__ void __cluster_dims__(1, kKS, 1) __launch_bounds__(kThreads)
 // unit: the warp's W1 row is loaded into registers all at once while one bulk copy
 // brings the tokens' h into shared memory, the dot products use packed fp32 FMAs,
 // and the GELU outputs are exchanged through distributed shared memory for the
-// second layer.  With APPEND the warp that finishes (token b, key head kh) of a
-// per-token decode step also does that step's ring/cache update for (b, kh).
+// second layer.  In kScoreAppend mode the warp that finishes (token b, key head kh) of
+// a per-token decode step also does that step's ring/cache update for (b, kh); in
+// kScoreGates mode it stores the gate in the token's window slot.
 constexpr int kSmallRanks = 8;
 constexpr int kSmallThreads = 512;   // one warp per hidden unit of the rank (<= 16 units)
 constexpr int kSmallMaxVec = 16;     // 16-byte W1 vectors per lane
 constexpr uint32_t kBulkPiece = 32768;
+
+// What the few-token kernels do after the gates: nothing, the per-token decode step's
+// ring/cache update (retire t - window, store the new token), or store each new token's
+// gate and utility in its window slot (the step's update having been done before).
+constexpr int kScoreOnly = 0, kScoreAppend = 1, kScoreGates = 2;
 
 struct SmallAppend {
   CacheMut c;
@@ -151,7 +157,27 @@ struct SmallAppend {
   int row_bytes;
 };
 
-template <typename E, int NT, bool APPEND>
+// The gate (and, if the ring keeps them, the utility) of the token of batch row b at
+// its window slot t_pos[b] % window.
+__device__ __forceinline__ void store_gate(const SmallAppend& ap, int b, int kh, int hkv,
+                                           uint8_t z, float u) {
+  const int t = ap.t_pos[b];
+  if (t < 0) return;
+  const size_t zi = ((size_t)b * ap.window + t % ap.window) * hkv + kh;
+  ap.r.z[zi] = z;
+  if (ap.r.u) ap.r.u[zi] = u;
+}
+
+// Gates of a scored batch into their window slots (after the separate score kernel).
+__global__ void __launch_bounds__(256)
+    store_gates_kernel(SmallAppend ap, const uint8_t* __restrict__ z, const float* __restrict__ u,
+                       int B, int hkv) {
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < B * hkv) store_gate(ap, i / hkv, i % hkv, hkv, z[i], u ? u[i] : no_utility());
+}
+
+
+template <typename E, int NT, int MODE>
 __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThreads, 1)
     score_small_kernel(const typename E::T* __restrict__ h, int n_tok, int d_model,
                        const typename E::T* __restrict__ W1, const float* __restrict__ b1,
@@ -258,18 +284,21 @@ __global__ void __cluster_dims__(kSmallRanks, 1, 1) __launch_bounds__(kSmallThre
       if (u_out) u_out[o] = uval;
       z_out[o] = z;
     }
-    if constexpr (APPEND) {
+    if constexpr (MODE == kScoreAppend) {
       const int b = tok0 + n;  // one new token per batch row
       const int t = ap.t_pos[b];
       if (t >= 0)
         decode_append_warp(ap.c, ap.r, b * hkv + kh, b, kh, t, ap.k_new, ap.v_new, z, uval, 1, hkv,
                            ap.window, ap.row_bytes, lane);
+    } else if constexpr (MODE == kScoreGates) {
+      const int b = tok0 + n;
+      if (lane == 0) store_gate(ap, b, kh, hkv, z, uval);
     }
   }
   cluster.sync();
 }
 
-template <typename E, int NT, bool APPEND>
+template <typename E, int NT, int MODE>
 cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const void* W1,
                          const float* b1, const float* W2, const float* b2, float* u_out,
                          uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
@@ -278,29 +307,29 @@ cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const v
   const size_t smem = (size_t)NT * p.d_model * E::kSize + (size_t)units * NT * 4;
   static int configured_smem = 0;
   if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT, APPEND>,
+    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT, MODE>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     configured_smem = (int)smem;
   }
   const int groups = (n_tok + NT - 1) / NT;
-  return launch_pdl(score_small_kernel<E, NT, APPEND>, dim3(groups * kSmallRanks),
+  return launch_pdl(score_small_kernel<E, NT, MODE>, dim3(groups * kSmallRanks),
                     dim3(kSmallThreads), smem, stream, static_cast<const T*>(h), n_tok, p.d_model,
                     static_cast<const T*>(W1), b1, W2, b2, p.hid, p.Hkv, p.tau, u_out, z_out, ap);
 }
 
-template <bool APPEND>
+template <int MODE>
 cudaError_t dispatch_small(const spkv_params& p, const void* h, int n_tok, const void* W1,
                            const float* b1, const float* W2, const float* b2, float* u_out,
                            uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
   if (p.dtype == SPKV_BF16) {
     return n_tok <= 8
-               ? launch_small<BF16, 8, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
-               : launch_small<BF16, 16, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
+               ? launch_small<BF16, 8, MODE>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
+               : launch_small<BF16, 16, MODE>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
   }
   return n_tok <= 8
-             ? launch_small<F32, 8, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
-             : launch_small<F32, 16, APPEND>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
+             ? launch_small<F32, 8, MODE>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream)
+             : launch_small<F32, 16, MODE>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }
 
 // ---- few tokens, bf16, hid = 128: the first layer on tensor cores ---------------------
@@ -314,9 +343,10 @@ cudaError_t dispatch_small(const spkv_params& p, const void* h, int n_tok, const
 // in shared memory, bias + GELU follow, and the 128 x 8 GELU outputs are all-gathered
 // into every CTA of the cluster with distributed shared-memory stores; rank n then
 // finishes token n (second layer in fp32, sigmoid, threshold).  W1 and W2 loads are
-// issued before the kernel waits for the preceding kernel on the stream.  With APPEND
-// the per-token ring/cache reads of the step are issued while the MLP runs and the
-// step is written once the gate is known.
+// issued before the kernel waits for the preceding kernel on the stream.  In
+// kScoreAppend mode the per-token ring/cache reads of the step are issued while the MLP
+// runs and the step is written once the gate is known; in kScoreGates mode the gates
+// go to the tokens' window slots.
 constexpr int kMmaRanks = 8;
 constexpr int kMmaWarps = 16;
 constexpr int kMmaThreads = kMmaWarps * 32;
@@ -335,7 +365,7 @@ __device__ __forceinline__ void mma_bf16_16816(float* d, uint32_t a0, uint32_t a
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
-template <bool APPEND>
+template <int MODE>
 __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads, 1)
     score_mma_kernel(const __nv_bfloat16* __restrict__ h, int n_tok, int d_model,
                      const __nv_bfloat16* __restrict__ W1, const float* __restrict__ b1,
@@ -344,7 +374,7 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
                      SmallAppend ap) {
   __shared__ float red[kMmaWarps][16][kMmaTok];
   __shared__ float xs[kMmaHid][kMmaTok];  // GELU outputs of all hidden units (all-gathered)
-  __shared__ __align__(16) char stage[APPEND ? kMmaMaxHkv : 1][4 * kMmaMaxRowBytes];
+  __shared__ __align__(16) char stage[MODE == kScoreAppend ? kMmaMaxHkv : 1][4 * kMmaMaxRowBytes];
   cg::cluster_group cluster = cg::this_cluster();
   const int rank = (int)cluster.block_rank();
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -381,7 +411,7 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
 
   AppendPre pre;
   pre.t = -1;
-  if constexpr (APPEND) {
+  if constexpr (MODE == kScoreAppend) {
     if (warp < hkv && my_n < nt) {
       const int b = tok0 + my_n, bh = b * hkv + warp;
       pre = append_prefetch(ap.c, ap.r, bh, b, warp, __ldg(ap.t_pos + b), ap.k_new, ap.v_new, hkv,
@@ -438,7 +468,10 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
       if (u_out) u_out[o] = uval;
       z_out[o] = z;
     }
-    if constexpr (APPEND) {
+    if constexpr (MODE == kScoreGates) {
+      if (lane == 0) store_gate(ap, tok0 + my_n, warp, hkv, z, uval);
+    }
+    if constexpr (MODE == kScoreAppend) {
       const int b = tok0 + my_n;
       append_commit(ap.c, ap.r, pre, b * hkv + warp, b, warp, z, uval, hkv, ap.window, ap.row_bytes,
                     lane, stage[warp]);
@@ -452,12 +485,12 @@ bool mma_ok(const spkv_params& p, int n_tok) {
          p.head_dim * 2 <= kMmaMaxRowBytes && n_tok >= 1 && n_tok <= 64;
 }
 
-template <bool APPEND>
+template <int MODE>
 cudaError_t launch_mma(const spkv_params& p, const void* h, int n_tok, const void* W1,
                        const float* b1, const float* W2, const float* b2, float* u_out,
                        uint8_t* z_out, const SmallAppend& ap, cudaStream_t stream) {
   const int groups = (n_tok + kMmaTok - 1) / kMmaTok;
-  return launch_pdl(score_mma_kernel<APPEND>, dim3(groups * kMmaRanks), dim3(kMmaThreads), 0,
+  return launch_pdl(score_mma_kernel<MODE>, dim3(groups * kMmaRanks), dim3(kMmaThreads), 0,
                     stream, static_cast<const __nv_bfloat16*>(h), n_tok, p.d_model,
                     static_cast<const __nv_bfloat16*>(W1), b1, W2, b2, p.Hkv, p.tau, u_out, z_out,
                     ap);
@@ -480,9 +513,9 @@ cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const v
                          const float* b1, const float* W2, const float* b2, float* u_out,
                          uint8_t* z_out, cudaStream_t stream) {
   if (mma_ok(p, n_tok))
-    return launch_mma<false>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
+    return launch_mma<kScoreOnly>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   if (small_ok(p, n_tok))
-    return dispatch_small<false>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
+    return dispatch_small<kScoreOnly>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   dim3 grid((n_tok + kTok - 1) / kTok, kKS);
   if (p.dtype == SPKV_BF16) {
     score_kernel<BF16><<<grid, kThreads, 0, stream>>>(
@@ -512,8 +545,25 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
                  ring_mut(ring),
                  t_pos, static_cast<const char*>(k_new), static_cast<const char*>(v_new), p.window,
                  p.head_dim * esize};
-  if (mma) return launch_mma<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
-  return dispatch_small<true>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
+  if (mma) return launch_mma<kScoreAppend>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
+  return dispatch_small<kScoreAppend>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
+}
+
+cudaError_t launch_score_gates(const spkv_params& p, const spkv_ring& ring, const int32_t* t_pos,
+                               const void* h, const void* W1, const float* b1, const float* W2,
+                               const float* b2, float* u_out, uint8_t* z_out, cudaStream_t stream) {
+  SmallAppend ap{};
+  ap.r = ring_mut(ring);
+  ap.t_pos = t_pos;
+  ap.window = p.window;
+  if (mma_ok(p, p.B))
+    return launch_mma<kScoreGates>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
+  if (small_ok(p, p.B))
+    return dispatch_small<kScoreGates>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
+  cudaError_t e = launch_score(p, h, p.B, W1, b1, W2, b2, u_out, z_out, stream);
+  if (e != cudaSuccess) return e;
+  store_gates_kernel<<<(p.B * p.Hkv + 255) / 256, 256, 0, stream>>>(ap, z_out, u_out, p.B, p.Hkv);
+  return cudaGetLastError();
 }
 
 bool score_supported(const spkv_params& p) {

@@ -117,12 +117,15 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
 
 def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: bool = True,
                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                fused: bool = True):
+                fused: bool = True, score_stream=None):
     """One decode step for every batch row at positions t_pos [B] (device int32).
 
     h_t [B][d_model] (ignored when retire is False: buffered scoring), q_t [B][Hq][d],
     k_t, v_t [B][Hkv][d].  With ``fused`` the score and the ring/cache update are one
-    launch (spkv_decode_score_append), else spkv_score then spkv_decode_append.
+    launch (spkv_decode_score_append), else spkv_score then spkv_decode_append.  With a
+    ``score_stream`` the update comes first (new gate 0), then the attention, and the new
+    tokens are scored on that stream with their gates stored in the window
+    (spkv_decode_score); the caller joins that stream before the gates are needed.
     Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
     p = layer.p
     z_t = u_t = None
@@ -134,6 +137,21 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
             lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
         S.spkv_decode_attn(p, None, layer.ring, q_t, t_pos, o, lse, layer.ws)
         return o, lse, None
+    if retire and score_stream is not None:
+        z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
+        u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)
+        S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, None, None, 1)
+        if o is None:
+            o = torch.empty_like(q_t)
+        if lse is None:
+            lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
+        S.spkv_decode_attn(p, layer.cache, layer.ring, q_t, t_pos, o, lse, layer.ws)
+        score_stream.wait_stream(torch.cuda.current_stream())
+        S.spkv_decode_score(p, layer.ring, t_pos, h_t, layer.W1, layer.b1, layer.W2, layer.b2, u_t,
+                            z_t, stream=score_stream)
+        for x in (h_t, t_pos, z_t, u_t):
+            x.record_stream(score_stream)
+        return o, lse, z_t
     if retire and fused:
         z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
         u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)

@@ -75,6 +75,8 @@ _sigs = {
                                         _vp, _vp, _vp]),
     "spkv_decode_score_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "spkv_decode_score": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _vp, _vp]),
 }
 NOALLOC_SCRATCH_BYTES = 8 << 20
 for _name, (_res, _args) in _sigs.items():
@@ -293,3 +295,11 @@ def spkv_soft_attn(p, q, K, V, u, seq_len, beta, c, o, lse, workspace, err_flag=
     return _check("spkv_soft_attn", lib.spkv_soft_attn(
         ctypes.byref(p), _ptr(q), _ptr(K), _ptr(V), _ptr(u), int(seq_len), float(beta), float(c),
         _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(), _ptr(err_flag), _stream(stream)))
+
+
+def spkv_decode_score(p, ring: Ring, t_pos, h, W1, b1, W2, b2, u_out, z_out, stream=None):
+    """Score one decode step's new tokens and store their gates in their window slots
+    (to run beside the attention; see include/spkv.h)."""
+    return _check("spkv_decode_score", lib.spkv_decode_score(
+        ctypes.byref(p), ctypes.byref(ring.r), _ptr(t_pos), _ptr(h), _ptr(W1), _ptr(b1), _ptr(W2),
+        _ptr(b2), _ptr(u_out), _ptr(z_out), _stream(stream)))

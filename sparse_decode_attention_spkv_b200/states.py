@@ -120,9 +120,15 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
 
 
 class DecodeStep:
-    """Launch sequence of one decode step (all layers) on fixed buffers."""
+    """Launch sequence of one decode step (all layers) on fixed buffers.
 
-    def __init__(self, p, layers, device):
+    Default: per layer, the fused score + retire + ring write, then the attention.  With
+    ``split``, the scoring leaves the attention's path: per layer the retirement and ring
+    write (gate of the new token left at 0), then the attention, and on a second stream
+    the scoring of the layer's new tokens, which stores their gates in their window slots
+    while the next layers run (a gate is read only when its token leaves the window)."""
+
+    def __init__(self, p, layers, device, split: bool = False):
         from sparse_decode_attention_spkv_b200 import spkv as S
         self.S, self.p, self.layers = S, p, layers
         n = len(layers)
@@ -130,6 +136,10 @@ class DecodeStep:
         self.lse = torch.empty((n, p.B, p.Hq), dtype=torch.float32, device=device)
         self.u = torch.empty((n, p.B, p.Hkv), dtype=torch.float32, device=device)
         self.z = torch.empty((n, p.B, p.Hkv), dtype=torch.uint8, device=device)
+        self.split = split
+        if split:
+            self.side = torch.cuda.Stream(device=device)
+            self.fork = [torch.cuda.Event() for _ in layers]
 
     def launch(self, h, q, k, v, t, ev=None):
         """h [L][B][D], q [L][B][Hq][d], k, v [L][B][Hkv][d], t [B]; ev: {layer: (start,
@@ -137,18 +147,28 @@ class DecodeStep:
         event between two launches keeps the second from starting early, so only a
         sample of layers carries them)."""
         S, p = self.S, self.p
+        main = torch.cuda.current_stream()
         for l, L in enumerate(self.layers):
-            # score the new token, retire t - w, store the new token: one launch
-            S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2, k[l],
-                                       v[l], self.u[l], self.z[l])
+            if self.split:  # retire t - w, store the new token (gate 0 for now)
+                S.spkv_decode_append(p, L.cache, L.ring, t, k[l], v[l], None, None, 1)
+            else:  # score the new token, retire t - w, store the new token: one launch
+                S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2,
+                                           k[l], v[l], self.u[l], self.z[l])
             e = ev.get(l) if ev else None
             if e is not None:
                 e[0].record()
             S.spkv_decode_attn(p, L.cache, L.ring, q[l], t, self.o[l], self.lse[l], L.ws)
             if e is not None:
                 e[1].record()
+            if self.split:  # the new tokens' gates, beside the following layers
+                self.fork[l].record(main)
+                self.side.wait_event(self.fork[l])
+                S.spkv_decode_score(p, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2, self.u[l],
+                                    self.z[l], stream=self.side)
+        if self.split:
+            main.wait_stream(self.side)
 
-    LAUNCHES_PER_LAYER = 2
+    LAUNCHES_PER_LAYER = 2  # plus one on the second stream when split
 
 
 def kv_bytes(p, layers, t_min):

@@ -280,3 +280,69 @@ def test_fused_and_separate_decode_steps_agree():
         assert np.array_equal(a[i], b[i]), f"step {i}"
     for x, y in zip(R.cache_lists(la), R.cache_lists(lb)):
         assert np.array_equal(x, y)
+
+
+SPLIT_CASES = {
+    # d_model 4096, hid 128: tensor-core score, gates stored by the score kernel
+    "mma": W.small_case("decode32k", cid=55, B=4, ctx=[1100], decode_steps=140, layers=1,
+                        keep="fixed25"),
+    # few-token CUDA-core score
+    "small": W.small_case("decode32k", cid=56, B=3, Hq=8, Hkv=2, d_model=256, hid=64, ctx=[900],
+                          decode_steps=135, layers=1, keep="u05_50"),
+    # batch above the few-token kernels: spkv_score, then the gates stored by a second kernel
+    "batch20": W.small_case("decode32k", cid=57, B=20, Hq=4, Hkv=2, d_model=128, hid=32,
+                            ctx=[700], decode_steps=130, layers=1, keep="fixed25"),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SPLIT_CASES))
+def test_split_decode_step_matches_fused(name):
+    """The decode step with the scoring on a second stream (the retirement and ring
+    write with the new gate at 0, the attention, then spkv_decode_score storing the new
+    gates in the window) gives the fused step's outputs, gates, utilities and cache bit
+    for bit, and the oracle's outputs; retirements after w steps use the stored gates."""
+    wl = SPLIT_CASES[name]
+    T0, steps, w = wl.ctx[0], wl.decode_steps, wl.window
+    T = T0 + steps
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    mp = R.pages_for(T)
+    layers = [R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                             num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp, store_u=True)
+              for _ in range(2)]
+    h, q, k, v = _rows(wl, T)
+    for L in layers:
+        for c0 in range(0, T0, 512):
+            c1 = min(T0, c0 + 512)
+            R.prefill_chunk(L, C.dev(h[:, c0:c1], wl.dtype), C.dev(q[:, c0:c1], wl.dtype),
+                            C.dev(k[:, c0:c1], wl.dtype), C.dev(v[:, c0:c1], wl.dtype), c0,
+                            n_compact=max(0, min(c1, T0 - w) - c0))
+    side = torch.cuda.Stream()
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        args = (C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype), C.dev(k[:, t], wl.dtype),
+                C.dev(v[:, t], wl.dtype))
+        o_a, _, z_a = R.decode_step(layers[0], t_pos, *args)
+        o_b, _, z_b = R.decode_step(layers[1], t_pos, *args, score_stream=side)
+        torch.cuda.current_stream().wait_stream(side)
+        assert torch.equal(o_a, o_b), f"step {i}: outputs differ"
+        assert torch.equal(z_a, z_b), f"step {i}: gates differ"
+        if i % 29 == 0 or i == steps - 1:
+            og = C.to_np(o_b)
+            for b in range(wl.B):
+                o_ref, _ = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
+                                             z_ref[b, :t + 1], w, [t])
+                C.check_attn(og[b], o_ref[0], wl.dtype, f"split {name} step {i} b={b}")
+    torch.cuda.synchronize()
+    for x, y in ((layers[0].ring.z_win, layers[1].ring.z_win),
+                 (layers[0].ring.u_win, layers[1].ring.u_win),
+                 (layers[0].cache.count, layers[1].cache.count)):
+        assert torch.equal(x, y)
+    la, lb = R.cache_lists(layers[0]), R.cache_lists(layers[1])
+    for bh in range(wl.B * wl.Hkv):
+        assert np.array_equal(la[bh], lb[bh])
+    for L in layers:
+        assert S.spkv_cache_check(L.cache)[0] == S.OK
