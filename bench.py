@@ -301,7 +301,7 @@ def run_gpu(args, world, rank, local):
     }
     del Ls, inp, step
     torch.cuda.empty_cache()
-    if not args.no_aux:
+    if not args.no_aux and world == 1:  # per-GPU kernel measurements: once, at N = 1
         out["aux"] = {"prefill16k": measure_prefill(device, reps=3),
                       "rethreshold_decode32k": measure_rethreshold(device),
                       "soft_attn_16k": measure_soft(device),
