@@ -384,6 +384,20 @@ def measure_prefill(device, reps=3):
     pairs_win = sum(min(w, t + 1) for t in range(T))
     pairs_cache = sum(int(np.maximum(0, T - (pp + w)).sum()) for pp in pos)
     flops = 4.0 * wl.head_dim * wl.G * (pairs_win * wl.Hkv + pairs_cache)
+    # tile FLOPs: every 128-query x 64-key block the kernel computes (masked entries
+    # included): per chunk, query tile and key head, the window band (from 128 keys
+    # before the tile to its last query) and the cache pages holding a row with
+    # pos <= last query - w at the time of that chunk (its own rows included)
+    qt, kb = 128, 64
+    blocks = 0
+    for c0 in range(0, T, chunk):
+        for t0 in range(c0, c0 + chunk, qt):
+            wfirst = t0 - w if t0 >= w else t0
+            nwin = (t0 + qt - wfirst) // kb
+            for pp in pos:
+                n_any = int(np.sum(pp[pp < c0 + chunk] <= t0 + qt - 1 - w))
+                blocks += nwin + (n_any + kb - 1) // kb
+    tile_flops = 4.0 * wl.head_dim * wl.G * blocks * qt * kb
     t_total = statistics.median(totals) / 1e3
     t_attn = statistics.median(attn) / 1e3
     import json as _json
@@ -393,7 +407,8 @@ def measure_prefill(device, reps=3):
     peak_tf = float(_json.loads(txt)["bf16_tflops"]) if txt else 1590.0
     return {"unit": "TFLOP/s", "live_pair_flops": flops, "ms_total": t_total * 1e3,
             "ms_prefill_attn": t_attn * 1e3, "tflops_total": flops / t_total / 1e12,
-            "tflops_prefill_attn": flops / t_attn / 1e12,
+            "tflops_prefill_attn": flops / t_attn / 1e12, "tile_flops": tile_flops,
+            "tile_tflops_prefill_attn": tile_flops / t_attn / 1e12,
             "roofline": {"bound": "tensor", "kernel": "prefill_attn",
                          "achieved": flops / t_attn / 1e12, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": flops / t_attn / 1e12 / peak_tf,

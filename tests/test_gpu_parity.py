@@ -346,3 +346,38 @@ def test_split_decode_step_matches_fused(name):
         assert np.array_equal(la[bh], lb[bh])
     for L in layers:
         assert S.spkv_cache_check(L.cache)[0] == S.OK
+
+
+def test_tau_zero_decode_is_causal_attention():
+    """tau = 0 gates every token in (u >= 0 always): the cache holds every position that
+    left the window and per-token decode equals plain causal attention over the whole
+    context (torch SDPA in fp64 as the reference of that special case)."""
+    wl = W.small_case("decode32k", cid=58, B=2, Hq=8, Hkv=2, d_model=128, hid=32, ctx=[700],
+                      decode_steps=4, layers=1, keep="fixed25")
+    T0, steps = wl.ctx[0], wl.decode_steps
+    T = T0 + steps
+    W1, b1, W2, b2 = C.weights(wl)
+    p = S.make_params(wl.B, wl.Hq, wl.Hkv, wl.head_dim, wl.d_model, wl.hid, wl.window, 0.0, S.BF16)
+    mp = R.pages_for(T)
+    layer = R.Layer.create(p, C.dev(W1, "bf16"), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                           num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp)
+    h, q, k, v = _rows(wl, T)
+    R.prefill_chunk(layer, C.dev(h[:, :T0], "bf16"), C.dev(q[:, :T0], "bf16"),
+                    C.dev(k[:, :T0], "bf16"), C.dev(v[:, :T0], "bf16"), 0,
+                    n_compact=T0 - wl.window)
+    G = wl.Hq // wl.Hkv
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        o, _, z = R.decode_step(layer, t_pos, C.dev(h[:, t], "bf16"), C.dev(q[:, t], "bf16"),
+                                C.dev(k[:, t], "bf16"), C.dev(v[:, t], "bf16"))
+        assert int(z.min()) == 1
+        og = C.to_np(o)
+        for b in range(wl.B):
+            Kx = torch.from_numpy(k[b, :t + 1]).double().permute(1, 0, 2)   # [Hkv][t+1][d]
+            Vx = torch.from_numpy(v[b, :t + 1]).double().permute(1, 0, 2)
+            Qx = torch.from_numpy(q[b, t]).double().view(wl.Hkv, G, 1, wl.head_dim)
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                Qx, Kx[:, None], Vx[:, None]).view(wl.Hq, wl.head_dim).numpy()
+            C.check_attn(og[b], ref, "bf16", f"tau=0 step {i} b={b}")
+    assert int(layer.cache.count.min().item()) == T - wl.window
