@@ -32,6 +32,12 @@
  *   page_rows 64.  Pointers to tensors must be 16-byte aligned.
  * - Positions are absolute token indices (int32).  Query head h reads key head
  *   h / (Hq/Hkv) (grouped-query attention).
+ * - The decode-step kernels (few-token scoring, retirement, decode attention and its
+ *   merge) are launched as programmatic dependents: each may start while the kernel
+ *   before it on the stream is finishing, and waits for that kernel to complete before
+ *   touching memory it may write.  The perceptron weights (W1, b1, W2, b2) are read
+ *   before that wait, so they must not be written by the kernel launched immediately
+ *   before a scoring call (weights written earlier on the stream are fine).
  */
 #ifndef SPKV_H
 #define SPKV_H

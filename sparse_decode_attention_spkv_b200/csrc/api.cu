@@ -83,7 +83,7 @@ const char* spkv_status_str(int status) {
   return "unknown status";
 }
 
-int spkv_version(void) { return 100; }
+int spkv_version(void) { return 200; }
 
 int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                      spkv_stream_t stream) {
