@@ -305,7 +305,9 @@ def run_gpu(args, world, rank, local):
         out["aux"] = {"prefill16k": measure_prefill(device, reps=3),
                       "rethreshold_decode32k": measure_rethreshold(device),
                       "soft_attn_16k": measure_soft(device),
-                      "hybrid_3to1_decode32k": measure_hybrid(device)}
+                      "hybrid_3to1_decode32k": measure_hybrid(device),
+                      "ragged128k": measure_ragged(device),
+                      "serving_e2e": measure_serving(device)}
     return out
 
 
@@ -585,6 +587,92 @@ def measure_hybrid(device, steps=10, warmup=3, period=4):
     return {"unit": "tokens/s", "value": p.B / (ms / 1e3), "ms_per_step": ms,
             "layers": {"global": n_glob, "local": n_layers - n_glob, "period": period},
             "launches_per_step": 2 * n_layers}
+
+
+def measure_ragged(device, warmup=3):
+    """Secondary measurement: ragged128k (batch 4, contexts 128K / 96K / 64K / 32K, one
+    layer, per-head keep 60% / 2% / 5-15%) per-token decode, the workload's 64 steps:
+    every step scores the new tokens, retires t - 128 and attends (split step, graph
+    replay, CUDA events).  Effective GB/s = live K/V bytes read per step / step time."""
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    from sparse_decode_attention_spkv_b200.states import DecodeStep, build_decode_state, kv_bytes
+
+    wl = W.WORKLOADS["ragged128k"]
+    steps = wl.decode_steps - warmup
+    p, Ls, inp = build_decode_state(wl, 1, wl.decode_steps, device)
+    step = DecodeStep(p, Ls, device, split=True)
+    graphs = []
+    for i in range(wl.decode_steps):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
+        graphs.append(g)
+    for i in range(warmup):
+        graphs[i].replay()
+    torch.cuda.synchronize()
+    b0 = kv_bytes(p, Ls, min(wl.ctx))
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for i in range(warmup, wl.decode_steps):
+        graphs[i].replay()
+    b.record()
+    torch.cuda.synchronize()
+    b1 = kv_bytes(p, Ls, min(wl.ctx))
+    ms = a.elapsed_time(b) / steps
+    status, flags = S_check(Ls[0])
+    if status:
+        raise RuntimeError(f"ragged measurement: cache error {flags}")
+    nbytes = 0.5 * (b0 + b1)
+    peak, peak_kind = _peaks()
+    del graphs
+    return {"unit": "tokens/s", "value": p.B / (ms / 1e3), "ms_per_step": ms, "steps": steps,
+            "kv_bytes_per_step": nbytes, "kv_gbs": nbytes / (ms / 1e3) / 1e9,
+            "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind}
+
+
+def measure_serving(device):
+    """Secondary measurement: serving (batch 32, contexts U[8K, 64K], one layer, keep
+    U[5%, 25%]) end to end over its 256 decode steps: tokens enter the window ungated,
+    and every 128 steps the 128 buffered tokens of every row are scored and their gated
+    rows compacted from the window into the cache, then decoding goes on.  tokens/s =
+    32 x 256 / the whole run's device time (CUDA events around all of it)."""
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    from sparse_decode_attention_spkv_b200.states import build_decode_state
+
+    wl = W.WORKLOADS["serving"]
+    steps, bulk = wl.decode_steps, wl.bulk
+    p, Ls, inp = build_decode_state(wl, 1, steps, device, compact_window=True)
+    L = Ls[0]
+    o = torch.empty((p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=device)
+    h_rows = inp["h_layer_row"][0]                      # [B][steps][d_model]
+    starts = [inp["t"][i0].clone() for i0 in range(0, steps, bulk)]
+    h_bufs = [h_rows[:, i0:i0 + bulk].contiguous() for i0 in range(0, steps, bulk)]
+
+    def run():
+        for i in range(steps):
+            R.decode_step(L, inp["t"][i], None, inp["q"][i][0], inp["k"][i][0], inp["v"][i][0],
+                          retire=False, o=o, lse=lse)
+            if (i + 1) % bulk == 0:
+                R.bulk_compact(L, h_bufs[i // bulk], starts[i // bulk])
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        run()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    g.replay()
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    status, flags = S_check(L)
+    if status:
+        raise RuntimeError(f"serving measurement: cache error {flags}")
+    del g
+    return {"unit": "tokens/s", "value": p.B * steps / (ms / 1e3), "ms_total": ms,
+            "steps": steps, "bulk": bulk,
+            "note": "one pass of the 256 steps (decode state advances; not repeated)"}
 
 
 def S_check(L):
