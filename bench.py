@@ -6,8 +6,9 @@ d_model 4096, utility perceptron 4096 -> 128 -> 8, window 128, tau 0.5, 32 layer
 32768 tokens already processed per row (per-head keep rates drawn in [5%, 50%]).
 One step = one decode token for every batch row through all 32 layers: per layer
 score the new token (a1), retire token t-128 into the gated cache if its gate is 1
-and store the new token in the ring (a2, a3), then gated decode attention with the
-split merge (a4, a5).  Steps are real consecutive decode steps (positions 32768,
+and store the new token in the ring (a2, a3), and gated decode attention with the
+split merge (a4, a5); by default the attention runs first, on the state before the
+step's update (the new rows passed in), and a1-a3 follow on a second stream.  Steps are real consecutive decode steps (positions 32768,
 32769, ...), each captured once in a CUDA graph; every step reads ~9.5 GB of K/V,
 far more than the 126 MB L2, so no flush is needed between steps.
 
@@ -181,7 +182,8 @@ def run_gpu(args, world, rank, local):
                                                           kv_bytes_layers)
     p, Ls, inp = build_decode_state(wl, layers, steps_total, device)
     T0 = wl.ctx[0]
-    step = DecodeStep(p, Ls, device, split=args.decode_step == "split")
+    step = DecodeStep(p, Ls, device, split=args.decode_step != "fused",
+                      attn_first=args.decode_step == "attn-first")
 
     # one eager decode-attention call per layer sets kernel attributes before capture
     for l, L in enumerate(Ls):
@@ -630,12 +632,16 @@ def measure_ragged(device, warmup=3):
             "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind}
 
 
-def measure_serving(device):
+def measure_serving(device, reps=3):
     """Secondary measurement: serving (batch 32, contexts U[8K, 64K], one layer, keep
     U[5%, 25%]) end to end over its 256 decode steps: tokens enter the window ungated,
     and every 128 steps the 128 buffered tokens of every row are scored and their gated
-    rows compacted from the window into the cache, then decoding goes on.  tokens/s =
-    32 x 256 / the whole run's device time (CUDA events around all of it)."""
+    rows compacted from the window into the cache, then decoding goes on.  The whole run
+    is one CUDA graph; the cache and ring are snapshotted before it and restored after
+    every replay, so each timed replay starts from the same state (one untimed replay
+    first).  tokens/s = 32 x 256 / the run's device time (median over `reps`); the K/V
+    bytes per step count every head's live cache rows (pos <= t - w) and window rows,
+    averaged over the first and last step."""
     from sparse_decode_attention_spkv_b200 import runner as R
     from sparse_decode_attention_spkv_b200.inputs import workloads as W
     from sparse_decode_attention_spkv_b200.states import build_decode_state
@@ -649,6 +655,11 @@ def measure_serving(device):
     h_rows = inp["h_layer_row"][0]                      # [B][steps][d_model]
     starts = [inp["t"][i0].clone() for i0 in range(0, steps, bulk)]
     h_bufs = [h_rows[:, i0:i0 + bulk].contiguous() for i0 in range(0, steps, bulk)]
+    state = [x for x in (L.cache.K_pool, L.cache.V_pool, L.cache.pos_pool, L.cache.page_table,
+                         L.cache.count, L.cache.count_prev, L.cache.pool_top, L.cache.err_flag,
+                         L.cache.u_pool, L.ring.K_win, L.ring.V_win, L.ring.z_win, L.ring.u_win)
+             if x is not None]
+    snap = [x.clone() for x in state]
 
     def run():
         for i in range(steps):
@@ -656,23 +667,61 @@ def measure_serving(device):
                           retire=False, o=o, lse=lse)
             if (i + 1) % bulk == 0:
                 R.bulk_compact(L, h_bufs[i // bulk], starts[i // bulk])
+
+    def restore():
+        for x, y in zip(state, snap):
+            x.copy_(y)
+
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         run()
     torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    g.replay()
-    b.record()
+    bytes_first = _live_kv_bytes(p, L, inp["t"][0])
+    g.replay()  # untimed
     torch.cuda.synchronize()
-    ms = a.elapsed_time(b)
     status, flags = S_check(L)
     if status:
         raise RuntimeError(f"serving measurement: cache error {flags}")
+    bytes_last = _live_kv_bytes(p, L, inp["t"][steps - 1])
+    restore()
+    times = []
+    for _ in range(reps):
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        times.append(a.elapsed_time(b))
+        status, flags = S_check(L)
+        if status:
+            raise RuntimeError(f"serving measurement: cache error {flags}")
+        restore()
     del g
+    ms = statistics.median(times)
+    step_bytes = 0.5 * (bytes_first + bytes_last)
+    peak, peak_kind = _peaks()
+    gbs = step_bytes / (ms / steps / 1e3) / 1e9
     return {"unit": "tokens/s", "value": p.B * steps / (ms / 1e3), "ms_total": ms,
-            "steps": steps, "bulk": bulk,
-            "note": "one pass of the 256 steps (decode state advances; not repeated)"}
+            "ms_runs": times, "steps": steps, "bulk": bulk,
+            "kv_bytes_per_step": step_bytes, "kv_gbs": gbs, "frac_of_hbm_peak": gbs / peak,
+            "peak_kind": peak_kind,
+            "l2": "the state restore between replays writes GBs (larger than L2)"}
+
+
+def _live_kv_bytes(p, L, t):
+    """K/V bytes one decode step reads at query positions t [B]: per head, the cache
+    rows with pos <= t - w plus min(w, t + 1) window rows (K and V, bf16)."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    count = L.cache.count.long()
+    table = L.cache.page_table.long()
+    idx = torch.arange(table.shape[1] * S.PAGE_ROWS, device=table.device)
+    pages = table[:, idx // S.PAGE_ROWS].clamp(min=0)
+    pos = L.cache.pos_pool[pages, idx % S.PAGE_ROWS]
+    th = t.long().repeat_interleave(p.Hkv)
+    live = ((pos <= (th - p.window)[:, None]) & (idx[None, :] < count[:, None])).sum(1)
+    nw = torch.clamp(th + 1, max=p.window)
+    return float((live + nw).sum().item()) * 2 * p.head_dim * 2
 
 
 def S_check(L):
@@ -765,9 +814,12 @@ def main():
     ap.add_argument("--cpu-units", type=int, default=48)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-aux", action="store_true", help="skip the secondary measurements")
-    ap.add_argument("--decode-step", default="split", choices=["split", "fused"],
-                    help="split: the new tokens are scored on a second stream beside the "
-                         "attention; fused: score, retirement and ring write in one launch")
+    ap.add_argument("--decode-step", default="attn-first", choices=["attn-first", "split", "fused"],
+                    help="attn-first: per layer the attention on the state before the step's "
+                         "update (new rows passed in), then retirement, ring write and scoring "
+                         "on a second stream; split: retirement and ring write, attention, "
+                         "scoring on a second stream; fused: score, retirement and ring write "
+                         "in one launch, then the attention")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")

@@ -234,6 +234,30 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_r
                      const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
                      size_t ws_bytes, spkv_stream_t stream);
 
+/* a4 + a5 before the step's retirement and ring write -- the same attention as
+ * spkv_decode_attn (Eqs. (3)-(4) at query t = t_pos[b]), taken from the state the
+ * cache and ring are in BEFORE spkv_decode_append of this step:
+ *   - the ring holds positions max(0, t-window) .. t-1; the slot t % window (position
+ *     t - window, which leaves the window at query t and belongs to the cache from
+ *     now on, Eq. (4)) counts iff its stored gate ring->z_win is 1;
+ *   - cache rows count up to position t - window - 1;
+ *   - the new token t is k_new / v_new [B][Hkv][head_dim] dtype (the rows the step's
+ *     spkv_decode_append will store).
+ * The step's spkv_decode_append (and spkv_decode_score) may then run after this call,
+ * off the attention's path: they must start after it has finished (they overwrite
+ * slot t % window) and finish before the next step's call on the same layer.  Same
+ * workspace, q, o and lse as spkv_decode_attn; ring->z_win is required; cache may be
+ * NULL (window-only layer).  Returns SPKV_ERR_UNSUPPORTED where
+ * spkv_decode_attn_before_append_supported says 0. */
+int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* cache,
+                                   const spkv_ring* ring, const void* q, const int32_t* t_pos,
+                                   const void* k_new, const void* v_new, void* o, float* lse,
+                                   void* workspace, size_t ws_bytes, spkv_stream_t stream);
+
+/* 1 if spkv_decode_attn_before_append runs for these parameters (bf16, head_dim 64 or
+ * 128, window a multiple of 64), else 0.  Host only; enqueues nothing. */
+int spkv_decode_attn_before_append_supported(const spkv_params* p);
+
 /* Size of the fixed device scratch used by spkv_decode_attn_noalloc (8 MiB).  Every
  * GPU on which the library is loaded keeps this much memory until the process exits. */
 #define SPKV_NOALLOC_SCRATCH_BYTES (8u << 20)

@@ -83,7 +83,7 @@ const char* spkv_status_str(int status) {
   return "unknown status";
 }
 
-int spkv_version(void) { return 200; }
+int spkv_version(void) { return 300; }
 
 int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                      spkv_stream_t stream) {
@@ -220,6 +220,26 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring*
   if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
   return status_of(spkv::launch_decode(*p, cache_or_none(c), *ring, q, t_pos, o, lse, workspace, ws_bytes, sms,
                                        static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_decode_attn_before_append_supported(const spkv_params* p) {
+  return params_ok(p) && spkv::decode_tc_supported(*p) ? 1 : 0;
+}
+
+int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* c,
+                                   const spkv_ring* ring, const void* q, const int32_t* t_pos,
+                                   const void* k_new, const void* v_new, void* o, float* lse,
+                                   void* workspace, size_t ws_bytes, spkv_stream_t stream) {
+  if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
+  if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
+  if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
+  if (!spkv::decode_tc_supported(*p)) return SPKV_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_decode_tc(*p, cache_or_none(c), *ring, q, t_pos, o, lse, workspace,
+                                          sms, static_cast<cudaStream_t>(stream), k_new, v_new));
 }
 
 size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* c) {

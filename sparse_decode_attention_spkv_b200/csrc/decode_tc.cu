@@ -29,6 +29,12 @@
 //    same stream) combines the partials: o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i,
 //    and resets the work counter for the next call.  A second launch costs less than
 //    the decode CTAs waiting on an arrival count at the end of every head.
+//  * Before-append mode (k_new given): the step's retirement and ring write have not
+//    run yet.  The ring then holds rows t-w .. t-1; slot t mod w (row t - w, which
+//    leaves the window at query t) counts only if its stored gate is 1, cache rows
+//    count up to pos t - w - 1, and the new row t is folded into the head's last
+//    chunk by the finisher as one more (m, l, o) term.  The retirement and ring write
+//    can then run after the attention, off its path.
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <math.h>
@@ -73,6 +79,7 @@ struct TileRef {
   int valid;  // valid rows
   int last;   // last tile of its chunk
   int qslot;  // query staging slot of the chunk
+  int hide;   // row of the tile that does not count (-1: none)
 };
 
 template <int D, int G>
@@ -93,7 +100,8 @@ struct TcDecSmem {
   TileRef info[kStagesT];
   int red[kThreadsT];
   int misc[4];
-  // followed (dynamic) by rows[n_heads], live[n_heads], nw[n_heads], base[n_heads + 1]
+  // followed (dynamic) by rows[n_heads], live[n_heads], nw[n_heads], hide[n_heads],
+  // base[n_heads + 1]
 };
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
@@ -118,6 +126,11 @@ __device__ __forceinline__ void mma16816(float* d, uint32_t a0, uint32_t a1, uin
       "{%8,%9}, {%0,%1,%2,%3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two bf16 (low half first) widened to fp32 (exact: a bf16 is the top half of an fp32).
+__device__ __forceinline__ float2 bf2_to_f2(uint32_t x) {
+  return make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xffff0000u));
 }
 
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
@@ -154,16 +167,18 @@ struct ChunkDesc {
   int bh;   // head: b * hkv + kh
   int k0, k1, kc1;
   int nl, nlp, nw;  // live cache rows, rounded up to tiles, window rows
+  int hide;         // window slot that does not count (-1: none)
 };
 
 __device__ __forceinline__ ChunkDesc describe_chunk(int c, int total, int chunk_rows,
                                                     const int* s_base, const int* s_rows,
                                                     const int* s_live, const int* s_nw,
-                                                    int n_heads, int hkv) {
+                                                    const int* s_hide, int n_heads, int hkv) {
   ChunkDesc d;
   d.c = c;
   if (c >= total) {
     d.bh = d.k0 = d.k1 = d.kc1 = d.nl = d.nlp = d.nw = 0;
+    d.hide = -1;
     return d;
   }
   int lo = 0, hi = n_heads - 1;
@@ -177,6 +192,7 @@ __device__ __forceinline__ ChunkDesc describe_chunk(int c, int total, int chunk_
   d.nl = s_live[lo];
   d.nlp = ((d.nl + kTileR - 1) / kTileR) * kTileR;
   d.nw = s_nw[lo];
+  d.hide = s_hide[lo];
   d.k0 = r0 / kTileR;
   d.k1 = (r1 + kTileR - 1) / kTileR;
   d.kc1 = min(d.k1, d.nlp / kTileR);
@@ -204,7 +220,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                      __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
                      int* __restrict__ ws_ctrl, float* __restrict__ ws_ml,
                      float* __restrict__ ws_o, int n_heads, int hkv, int window,
-                     uint32_t* err) {
+                     uint32_t* err, const __nv_bfloat16* __restrict__ k_new,
+                     const __nv_bfloat16* __restrict__ v_new, const uint8_t* __restrict__ z_win) {
   using TB = TileBuf<D>;
   using S = TcDecSmem<D, G>;
   constexpr int NT_D = D / 8;     // n-tiles of 8 along head_dim
@@ -215,7 +232,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   int* s_rows = reinterpret_cast<int*>(smem_raw + pad + sizeof(S));
   int* s_live = s_rows + n_heads;
   int* s_nw = s_live + n_heads;
-  int* s_base = s_nw + n_heads;
+  int* s_hide = s_nw + n_heads;
+  int* s_base = s_hide + n_heads;
+  const bool pre = k_new != nullptr;  // before the step's retirement and ring write
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   int* next_chunk = ws_ctrl + n_heads;  // reset by the merge kernel
 
@@ -233,12 +252,23 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   // ---- plan (identical in every CTA) ---------------------------------------------
   int my_rows = 0;
   for (int bh = tid; bh < n_heads; bh += kThreadsT) {
-    const int t = __ldcg(t_pos + bh / hkv);
-    const int nl = cache_live_rows(cache, bh, t - window, window);
-    const int nw = t + 1 < window ? t + 1 : window;
-    const int rows = ((nl + kTileR - 1) / kTileR) * kTileR + nw;
+    const int b = bh / hkv;
+    const int t = __ldcg(t_pos + b);
+    int nl, nw, hide = -1;
+    if (!pre) {
+      nl = cache_live_rows(cache, bh, t - window, window);
+      nw = t + 1 < window ? t + 1 : window;
+    } else {  // ring rows t-w .. t-1; row t - w (slot t mod w) counts if its gate is 1
+      nl = cache_live_rows(cache, bh, t - window - 1, window + 1);
+      nw = t < window ? t : window;
+      if (t >= window && __ldcg(z_win + ((size_t)b * window + t % window) * hkv + bh % hkv) == 0)
+        hide = t % window;
+    }
+    int rows = ((nl + kTileR - 1) / kTileR) * kTileR + nw;
+    if (pre && rows == 0) rows = 1;  // one empty tile: its chunk carries the new row
     s_live[bh] = nl;
     s_nw[bh] = nw;
+    s_hide[bh] = hide;
     s_rows[bh] = rows;
     my_rows += rows;
   }
@@ -309,7 +339,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     int it = 0;
     const int c = blockIdx.x;  // first chunk: static; later ones from the counter
     ChunkDesc cd = describe_chunk(c, total_chunks, chunk_rows, s_base, s_rows, s_live, s_nw,
-                                  n_heads, hkv);
+                                  s_hide, n_heads, hkv);
     int pg[kPgRegs];
     fetch_pages(pg, cd, cache, lane);
     for (int seq = 0; cd.c < total_chunks; ++seq) {
@@ -340,9 +370,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           TB& tb = sm.st[s];
           const bool from_cache = k < cd.kc1;
           const int slot = k * kTileR - cd.nlp;
-          const int valid = from_cache ? min(kTileR, cd.nl - k * kTileR) : min(kTileR, cd.nw - slot);
+          const int valid = from_cache ? min(kTileR, cd.nl - k * kTileR) : max(0, min(kTileR, cd.nw - slot));
+          const int hide = !from_cache && cd.hide >= slot && cd.hide < slot + kTileR ? cd.hide - slot : -1;
           // the tile description must be in place before the phase can complete
-          sm.info[s] = TileRef{cd.c, cd.bh, valid, k == cd.k1 - 1, qslot};
+          sm.info[s] = TileRef{cd.c, cd.bh, valid, k == cd.k1 - 1, qslot, hide};
           const bool first = k == cd.k0;
           mbar_arrive_expect_tx(&sm.full[s], 2 * TB::kBytes + (first ? G * D * 2 : 0));
           if (first)
@@ -367,7 +398,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         if (k == k_pages) {
           c_next = __shfl_sync(0xffffffffu, c_next, 0);
           nd = describe_chunk(c_next, total_chunks, chunk_rows, s_base, s_rows, s_live, s_nw,
-                              n_heads, hkv);
+                              s_hide, n_heads, hkv);
           fetch_pages(pg, nd, cache, lane);
         }
       }
@@ -392,9 +423,27 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       const int bh = sm.fin_bh[par];
       const size_t hrow = (size_t)bh * G;
       const int nch = s_base[bh + 1] - s_base[bh];
+      // before-append mode: the head's last chunk also takes the new row t
+      const bool fold = pre && c == s_base[bh + 1] - 1;
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
+        float s_new = -INFINITY;  // q . k_new in the log2 domain
+        if (fold) {
+          float part = 0.f;
+#pragma unroll
+          for (int d = 4 * lane; d < D; d += 128) {
+            const uint2 qa = __ldg(reinterpret_cast<const uint2*>(q + (hrow + g) * D + d));
+            const uint2 ka = __ldg(reinterpret_cast<const uint2*>(k_new + (size_t)bh * D + d));
+            const float2 q0 = bf2_to_f2(qa.x), q1 = bf2_to_f2(qa.y);
+            const float2 k0 = bf2_to_f2(ka.x), k1 = bf2_to_f2(ka.y);
+            part = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q1.x, k1.x, fmaf(q1.y, k1.y, part))));
+          }
+#pragma unroll
+          for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
+          s_new = part * (kLog2eT * rsqrtf((float)D));
+          M = s_new;
+        }
 #pragma unroll
         for (int w = 0; w < kCons; ++w) M = fmaxf(M, sm.red_m[par][w][g]);
         float wt[kCons], L = 0.f;
@@ -404,9 +453,16 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           wt[w] = mw == -INFINITY ? 0.f : exp2f(mw - M);
           L += wt[w] * sm.red_l[par][w][g];
         }
+        const float w_new = fold ? exp2f(s_new - M) : 0.f;
+        L += w_new;
 #pragma unroll
         for (int d = 4 * lane; d < D; d += 128) {
           float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (fold) {
+            const uint2 va = __ldg(reinterpret_cast<const uint2*>(v_new + (size_t)bh * D + d));
+            const float2 v0 = bf2_to_f2(va.x), v1 = bf2_to_f2(va.y);
+            O = make_float4(w_new * v0.x, w_new * v0.y, w_new * v1.x, w_new * v1.y);
+          }
 #pragma unroll
           for (int w = 0; w < kCons; ++w) {
             const float4 v = *reinterpret_cast<const float4*>(&sm.red_o[par][w][g][d]);
@@ -486,10 +542,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         mma16816(sb, qa[k][0], 0u, qa[k][1], 0u, b2, b3);
       }
       float x[4];
-      x[0] = row0 + qcol < ti.valid ? sa[0] * sc : -INFINITY;
-      x[1] = row0 + qcol + 1 < ti.valid ? sa[1] * sc : -INFINITY;
-      x[2] = row0 + 8 + qcol < ti.valid ? sb[0] * sc : -INFINITY;
-      x[3] = row0 + 9 + qcol < ti.valid ? sb[1] * sc : -INFINITY;
+      const int r0 = row0 + qcol;
+      x[0] = r0 < ti.valid && r0 != ti.hide ? sa[0] * sc : -INFINITY;
+      x[1] = r0 + 1 < ti.valid && r0 + 1 != ti.hide ? sa[1] * sc : -INFINITY;
+      x[2] = r0 + 8 < ti.valid && r0 + 8 != ti.hide ? sb[0] * sc : -INFINITY;
+      x[3] = r0 + 9 < ti.valid && r0 + 9 != ti.hide ? sb[1] * sc : -INFINITY;
       float rmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
       rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
       rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
@@ -671,10 +728,10 @@ size_t max_chunks_tc(const spkv_params& p, int num_sms) {
 
 template <int D, int G>
 cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
-                   const int32_t* t_pos, void* o, float* lse, void* ws, int num_sms,
-                   cudaStream_t stream) {
+                   const int32_t* t_pos, const void* k_new, const void* v_new, void* o, float* lse,
+                   void* ws, int num_sms, cudaStream_t stream) {
   using S = TcDecSmem<D, G>;
-  const size_t smem = sizeof(S) + 1024 + ((size_t)4 * p.B * p.Hkv + 1) * 4;
+  const size_t smem = sizeof(S) + 1024 + ((size_t)5 * p.B * p.Hkv + 1) * 4;
   static int configured = 0;
   if ((int)smem > configured) {
     cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, G>,
@@ -715,7 +772,8 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
   cudaError_t e = launch_pdl(decode_tc_kernel<D, G>, dim3(num_sms), dim3(kThreadsT), smem, stream,
                              tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
                              static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv,
-                             p.window, c.err_flag);
+                             p.window, c.err_flag, static_cast<const __nv_bfloat16*>(k_new),
+                             static_cast<const __nv_bfloat16*>(v_new), ring.z_win);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_merge_kernel<D, G>, dim3(n_heads), dim3(kMergeThreads), 0, stream, ctrl,
                     ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
@@ -723,13 +781,13 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
 
 template <int D>
 cudaError_t dispatch_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
-                        const void* q, const int32_t* t_pos, void* o, float* lse, void* ws,
-                        int num_sms, cudaStream_t stream) {
+                        const void* q, const int32_t* t_pos, const void* k_new, const void* v_new,
+                        void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
   switch (p.Hq / p.Hkv) {
-    case 1: return run_tc<D, 1>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
-    case 2: return run_tc<D, 2>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
-    case 4: return run_tc<D, 4>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
-    case 8: return run_tc<D, 8>(p, c, ring, q, t_pos, o, lse, ws, num_sms, stream);
+    case 1: return run_tc<D, 1>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
+    case 2: return run_tc<D, 2>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
+    case 4: return run_tc<D, 4>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
+    case 8: return run_tc<D, 8>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -752,9 +810,11 @@ size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms) {
 
 cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                              const void* q, const int32_t* t_pos, void* o, float* lse,
-                             void* workspace, int num_sms, cudaStream_t stream) {
-  if (p.head_dim == 128) return dispatch_tc<128>(p, c, ring, q, t_pos, o, lse, workspace, num_sms, stream);
-  return dispatch_tc<64>(p, c, ring, q, t_pos, o, lse, workspace, num_sms, stream);
+                             void* workspace, int num_sms, cudaStream_t stream,
+                             const void* k_new, const void* v_new) {
+  if (p.head_dim == 128)
+    return dispatch_tc<128>(p, c, ring, q, t_pos, k_new, v_new, o, lse, workspace, num_sms, stream);
+  return dispatch_tc<64>(p, c, ring, q, t_pos, k_new, v_new, o, lse, workspace, num_sms, stream);
 }
 
 }  // namespace spkv

@@ -41,9 +41,12 @@ cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const
 size_t decode_workspace_bytes(const spkv_params& p, int num_sms);
 bool decode_tc_supported(const spkv_params& p);
 size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms);
+// k_new / v_new given: before-append mode (the ring holds rows t-w .. t-1, the new row
+// comes from k_new / v_new, row t - w counts if its gate in the ring is 1).
 cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                              const void* q, const int32_t* t_pos, void* o, float* lse,
-                             void* workspace, int num_sms, cudaStream_t stream);
+                             void* workspace, int num_sms, cudaStream_t stream,
+                             const void* k_new = nullptr, const void* v_new = nullptr);
 cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                           const void* q, const int32_t* t_pos, void* o, float* lse,
                           void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream);

@@ -1,6 +1,7 @@
 """Run one kernel of the SP-KV path on a small, fixed configuration (for profilers).
 
     python -m sparse_decode_attention_spkv_b200.kernel_driver decode  [--layers 1] [--steps 3]
+                                      [--decode-step attn-first|split|fused]
     python -m sparse_decode_attention_spkv_b200.kernel_driver score   [--tokens 8]
     python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096]
     python -m sparse_decode_attention_spkv_b200.kernel_driver prefill [--chunk 4096]
@@ -40,7 +41,8 @@ def run_decode(args):
     from .states import DecodeStep, build_decode_state
     wl = W.WORKLOADS["decode32k"]
     p, Ls, inp = build_decode_state(wl, args.layers, args.steps, torch.device("cuda"))
-    step = DecodeStep(p, Ls, "cuda")
+    step = DecodeStep(p, Ls, "cuda", split=args.decode_step != "fused",
+                      attn_first=args.decode_step == "attn-first")
     for i in range(args.steps):
         step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
     torch.cuda.synchronize()
@@ -140,6 +142,7 @@ def main():
     ap.add_argument("--rows", type=int, default=4096)
     ap.add_argument("--chunk", type=int, default=4096)
     ap.add_argument("--seq", type=int, default=8192)
+    ap.add_argument("--decode-step", default="attn-first", choices=["attn-first", "split", "fused"])
     args = ap.parse_args()
     torch.cuda.set_device(0)
     {"decode": run_decode, "score": run_score, "compact": run_compact, "prefill": run_prefill,

@@ -117,7 +117,7 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
 
 def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: bool = True,
                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                fused: bool = True, score_stream=None):
+                fused: bool = True, score_stream=None, attn_first: bool = False):
     """One decode step for every batch row at positions t_pos [B] (device int32).
 
     h_t [B][d_model] (ignored when retire is False: buffered scoring), q_t [B][Hq][d],
@@ -125,7 +125,10 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
     launch (spkv_decode_score_append), else spkv_score then spkv_decode_append.  With a
     ``score_stream`` the update comes first (new gate 0), then the attention, and the new
     tokens are scored on that stream with their gates stored in the window
-    (spkv_decode_score); the caller joins that stream before the gates are needed.
+    (spkv_decode_score); the caller joins that stream before the gates are needed.  With
+    a ``score_stream`` and ``attn_first`` the attention runs first, on the state before
+    the step's update (spkv_decode_attn_before_append, the new rows passed in), and the
+    update and the scoring both go to that stream.
     Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
     p = layer.p
     z_t = u_t = None
@@ -137,6 +140,23 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
             lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
         S.spkv_decode_attn(p, None, layer.ring, q_t, t_pos, o, lse, layer.ws)
         return o, lse, None
+    if retire and score_stream is not None and attn_first:
+        z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
+        u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)
+        if o is None:
+            o = torch.empty_like(q_t)
+        if lse is None:
+            lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
+        S.spkv_decode_attn_before_append(p, layer.cache, layer.ring, q_t, t_pos, k_t, v_t, o, lse,
+                                         layer.ws)
+        score_stream.wait_stream(torch.cuda.current_stream())
+        S.spkv_decode_append(p, layer.cache, layer.ring, t_pos, k_t, v_t, None, None, 1,
+                             stream=score_stream)
+        S.spkv_decode_score(p, layer.ring, t_pos, h_t, layer.W1, layer.b1, layer.W2, layer.b2, u_t,
+                            z_t, stream=score_stream)
+        for x in (h_t, k_t, v_t, t_pos, z_t, u_t):
+            x.record_stream(score_stream)
+        return o, lse, z_t
     if retire and score_stream is not None:
         z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
         u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)

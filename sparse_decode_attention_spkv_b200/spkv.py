@@ -69,6 +69,9 @@ _sigs = {
     "spkv_decode_workspace_bytes": (ctypes.c_size_t, [_P(spkv_params), _P(spkv_cache)]),
     "spkv_decode_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _vp,
                                 _vp, ctypes.c_size_t, _vp]),
+    "spkv_decode_attn_before_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp,
+                                              _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "spkv_decode_attn_before_append_supported": (_i32, [_P(spkv_params)]),
     "spkv_prefill_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _i32,
                                  _i32, _vp, _vp, _vp]),
     "spkv_decode_attn_noalloc": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
@@ -259,6 +262,20 @@ def spkv_decode_attn(p, cache: Optional[Cache], ring: Ring, q, t_pos, o, lse, wo
     return _check("spkv_decode_attn", lib.spkv_decode_attn(
         ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
         _ptr(lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def spkv_decode_attn_before_append(p, cache: Optional[Cache], ring: Ring, q, t_pos, k_new, v_new,
+                                   o, lse, workspace, stream=None):
+    """The decode attention of a step taken before the step's spkv_decode_append (the
+    new rows k_new / v_new passed in); see include/spkv.h."""
+    return _check("spkv_decode_attn_before_append", lib.spkv_decode_attn_before_append(
+        ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos),
+        _ptr(k_new), _ptr(v_new), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
+        _stream(stream)))
+
+
+def spkv_decode_attn_before_append_supported(p) -> bool:
+    return bool(lib.spkv_decode_attn_before_append_supported(ctypes.byref(p)))
 
 
 def spkv_prefill_attn(p, cache: Optional[Cache], ring: Ring, q, K_chunk, V_chunk, chunk_start,

@@ -126,11 +126,20 @@ class DecodeStep:
     ``split``, the scoring leaves the attention's path: per layer the retirement and ring
     write (gate of the new token left at 0), then the attention, and on a second stream
     the scoring of the layer's new tokens, which stores their gates in their window slots
-    while the next layers run (a gate is read only when its token leaves the window)."""
+    while the next layers run (a gate is read only when its token leaves the window).
+    With ``split`` and ``attn_first`` (the default where the kernels support it) the
+    attention runs first, on the state before the step's update, and the retirement, ring
+    write and scoring all run on the second stream: the attention of the next layer
+    follows the previous one directly."""
 
-    def __init__(self, p, layers, device, split: bool = False):
+    def __init__(self, p, layers, device, split: bool = False, attn_first=None):
         from sparse_decode_attention_spkv_b200 import spkv as S
         self.S, self.p, self.layers = S, p, layers
+        if attn_first is None:
+            attn_first = split and S.spkv_decode_attn_before_append_supported(p)
+        if attn_first and not split:
+            raise ValueError("attn_first needs split")
+        self.attn_first = bool(attn_first)
         n = len(layers)
         self.o = torch.empty((n, p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((n, p.B, p.Hq), dtype=torch.float32, device=device)
@@ -149,6 +158,23 @@ class DecodeStep:
         S, p = self.S, self.p
         main = torch.cuda.current_stream()
         for l, L in enumerate(self.layers):
+            if self.attn_first:
+                e = ev.get(l) if ev else None
+                if e is not None:
+                    e[0].record()
+                S.spkv_decode_attn_before_append(p, L.cache, L.ring, q[l], t, k[l], v[l],
+                                                 self.o[l], self.lse[l], L.ws)
+                if e is not None:
+                    e[1].record()
+                # retire t - w, store the new token (gate 0), then its gate: beside the
+                # following layers' attention
+                self.fork[l].record(main)
+                self.side.wait_event(self.fork[l])
+                S.spkv_decode_append(p, L.cache, L.ring, t, k[l], v[l], None, None, 1,
+                                     stream=self.side)
+                S.spkv_decode_score(p, L.ring, t, h[l], L.W1, L.b1, L.W2, L.b2, self.u[l],
+                                    self.z[l], stream=self.side)
+                continue
             if self.split:  # retire t - w, store the new token (gate 0 for now)
                 S.spkv_decode_append(p, L.cache, L.ring, t, k[l], v[l], None, None, 1)
             else:  # score the new token, retire t - w, store the new token: one launch

@@ -89,3 +89,15 @@ def test_argument_validation_without_gpu():
     assert S.lib.spkv_cache_rethreshold(ctypes.byref(good), ctypes.byref(cache_u), None,
                                         ctypes.c_float(float("nan")), 16, 1 << 20, None) == S.ERR_ARG
     assert S.lib.spkv_rethreshold_workspace_bytes(ctypes.byref(good), ctypes.byref(cache_u)) > 0
+    # attention before the step's update: needs the new rows; fp32 is not supported
+    assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
+                                                ctypes.byref(ring), 16, 16, None, 16, 16, None,
+                                                16, 1 << 20, None) == S.ERR_ARG
+    assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
+                                                ctypes.byref(ring), 16, 16, 16, 8, 16, None,
+                                                16, 1 << 20, None) == S.ERR_ARG
+    assert S.lib.spkv_decode_attn_before_append_supported(ctypes.byref(good)) == 0
+    assert S.lib.spkv_decode_attn_before_append_supported(None) == 0
+    assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
+                                                ctypes.byref(ring), 16, 16, 16, 16, 16, None,
+                                                16, 1 << 20, None) == S.ERR_UNSUPPORTED

@@ -348,6 +348,106 @@ def test_split_decode_step_matches_fused(name):
         assert S.spkv_cache_check(L.cache)[0] == S.OK
 
 
+ATTN_FIRST_CASES = dict(SPLIT_CASES)
+# from an empty state: t = 0 (no key but the new token), t < w, the first retirement at t = w
+ATTN_FIRST_CASES["from_empty"] = W.small_case("decode32k", cid=59, B=2, Hq=8, Hkv=2, d_model=128,
+                                              hid=32, ctx=[0], decode_steps=150, layers=1,
+                                              keep="u05_50")
+# head_dim 64, 8 query heads per key head
+ATTN_FIRST_CASES["d64_g8"] = W.small_case("decode32k", cid=63, B=2, Hq=8, Hkv=1, head_dim=64,
+                                          d_model=128, hid=32, ctx=[300], decode_steps=140,
+                                          layers=1, keep="fixed25")
+
+
+@pytest.mark.parametrize("name", sorted(ATTN_FIRST_CASES))
+def test_attention_first_decode_step(name):
+    """The decode step with the attention first (spkv_decode_attn_before_append on the
+    state before the step's retirement and ring write, the new rows passed in; the
+    update and the scoring after it on a second stream): outputs against the oracle at
+    every step, and gates, utilities, ring and cache bit for bit equal to the fused
+    step's (the update kernels are the same, only their order changes)."""
+    wl = ATTN_FIRST_CASES[name]
+    T0, steps, w = wl.ctx[0], wl.decode_steps, wl.window
+    T = T0 + steps
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    assert S.spkv_decode_attn_before_append_supported(p)
+    mp = R.pages_for(T)
+    layers = [R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                             num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp, store_u=True)
+              for _ in range(2)]
+    h, q, k, v = _rows(wl, T)
+    for L in layers:
+        for c0 in range(0, T0, 512):
+            c1 = min(T0, c0 + 512)
+            R.prefill_chunk(L, C.dev(h[:, c0:c1], wl.dtype), C.dev(q[:, c0:c1], wl.dtype),
+                            C.dev(k[:, c0:c1], wl.dtype), C.dev(v[:, c0:c1], wl.dtype), c0,
+                            n_compact=max(0, min(c1, T0 - w) - c0))
+    side = torch.cuda.Stream()
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        args = (C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype), C.dev(k[:, t], wl.dtype),
+                C.dev(v[:, t], wl.dtype))
+        o_a, _, z_a = R.decode_step(layers[0], t_pos, *args)
+        o_b, lse_b, z_b = R.decode_step(layers[1], t_pos, *args, score_stream=side,
+                                        attn_first=True)
+        torch.cuda.current_stream().wait_stream(side)
+        assert torch.equal(z_a, z_b), f"step {i}: gates differ"
+        og = C.to_np(o_b)
+        assert np.all(np.isfinite(og)) and np.all(np.isfinite(lse_b.cpu().numpy()))
+        for b in range(wl.B):
+            o_ref, _ = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
+                                         z_ref[b, :t + 1], w, [t])
+            C.check_attn(og[b], o_ref[0], wl.dtype, f"attn-first {name} step {i} b={b}")
+    torch.cuda.synchronize()
+    for x, y in ((layers[0].ring.z_win, layers[1].ring.z_win),
+                 (layers[0].ring.u_win, layers[1].ring.u_win),
+                 (layers[0].ring.K_win, layers[1].ring.K_win),
+                 (layers[0].ring.V_win, layers[1].ring.V_win),
+                 (layers[0].cache.count, layers[1].cache.count)):
+        assert torch.equal(x.nan_to_num() if x.is_floating_point() else x,
+                           y.nan_to_num() if y.is_floating_point() else y)
+    la, lb = R.cache_lists(layers[0]), R.cache_lists(layers[1])
+    for bh in range(wl.B * wl.Hkv):
+        assert np.array_equal(la[bh], lb[bh])
+    for L in layers:
+        assert S.spkv_cache_check(L.cache)[0] == S.OK
+
+
+def test_attention_first_lse():
+    """lse of the attention-first step against the oracle's log-sum-exp (natural log of
+    the softmax denominator over the key set, scores scaled by 1/sqrt(d))."""
+    wl = ATTN_FIRST_CASES["small"]
+    T0, steps, w = wl.ctx[0], 3, wl.window
+    T = T0 + steps
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    mp = R.pages_for(T)
+    L = R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                       num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp)
+    h, q, k, v = _rows(wl, T)
+    R.prefill_chunk(L, C.dev(h[:, :T0], wl.dtype), C.dev(q[:, :T0], wl.dtype),
+                    C.dev(k[:, :T0], wl.dtype), C.dev(v[:, :T0], wl.dtype), 0, n_compact=T0 - w)
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    side = torch.cuda.Stream()
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        _, lse, _ = R.decode_step(L, t_pos, C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype),
+                                  C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype),
+                                  score_stream=side, attn_first=True)
+        torch.cuda.current_stream().wait_stream(side)
+        got = lse.cpu().numpy()
+        for b in range(wl.B):
+            _, lse_ref = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
+                                           z_ref[b, :t + 1], w, [t])
+            assert np.max(np.abs(got[b] - lse_ref[0])) <= 2e-2, (i, b)
+
+
 def test_tau_zero_decode_is_causal_attention():
     """tau = 0 gates every token in (u >= 0 always): the cache holds every position that
     left the window and per-token decode equals plain causal attention over the whole
