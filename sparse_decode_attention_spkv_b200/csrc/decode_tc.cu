@@ -423,22 +423,30 @@ __global__ void __launch_bounds__(kThreadsT, 1)
       const int bh = sm.fin_bh[par];
       const size_t hrow = (size_t)bh * G;
       const int nch = s_base[bh + 1] - s_base[bh];
-      // before-append mode: the head's last chunk also takes the new row t
+      // before-append mode: the head's last chunk also takes the new row t.  Each lane
+      // owns columns 4 lane .. 4 lane + 3 (D <= 128); the new key, value and the group's
+      // queries are loaded together, one memory round trip.
+      static_assert(D <= 128, "one 4-column slice per finisher lane");
       const bool fold = pre && c == s_base[bh + 1] - 1;
+      const bool has_cols = 4 * lane < D;
+      uint2 kn = make_uint2(0u, 0u), vn = make_uint2(0u, 0u), qn[G];
+#pragma unroll
+      for (int g = 0; g < G; ++g) qn[g] = make_uint2(0u, 0u);
+      if (fold && has_cols) {
+        kn = __ldg(reinterpret_cast<const uint2*>(k_new + (size_t)bh * D + 4 * lane));
+        vn = __ldg(reinterpret_cast<const uint2*>(v_new + (size_t)bh * D + 4 * lane));
+#pragma unroll
+        for (int g = 0; g < G; ++g)
+          qn[g] = __ldg(reinterpret_cast<const uint2*>(q + (hrow + g) * D + 4 * lane));
+      }
 #pragma unroll
       for (int g = 0; g < G; ++g) {
         float M = -INFINITY;
         float s_new = -INFINITY;  // q . k_new in the log2 domain
         if (fold) {
-          float part = 0.f;
-#pragma unroll
-          for (int d = 4 * lane; d < D; d += 128) {
-            const uint2 qa = __ldg(reinterpret_cast<const uint2*>(q + (hrow + g) * D + d));
-            const uint2 ka = __ldg(reinterpret_cast<const uint2*>(k_new + (size_t)bh * D + d));
-            const float2 q0 = bf2_to_f2(qa.x), q1 = bf2_to_f2(qa.y);
-            const float2 k0 = bf2_to_f2(ka.x), k1 = bf2_to_f2(ka.y);
-            part = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q1.x, k1.x, fmaf(q1.y, k1.y, part))));
-          }
+          const float2 q0 = bf2_to_f2(qn[g].x), q1 = bf2_to_f2(qn[g].y);
+          const float2 k0 = bf2_to_f2(kn.x), k1 = bf2_to_f2(kn.y);
+          float part = fmaf(q0.x, k0.x, fmaf(q0.y, k0.y, fmaf(q1.x, k1.x, q1.y * k1.y)));
 #pragma unroll
           for (int o = 16; o > 0; o >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o);
           s_new = part * (kLog2eT * rsqrtf((float)D));
@@ -459,8 +467,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         for (int d = 4 * lane; d < D; d += 128) {
           float4 O = make_float4(0.f, 0.f, 0.f, 0.f);
           if (fold) {
-            const uint2 va = __ldg(reinterpret_cast<const uint2*>(v_new + (size_t)bh * D + d));
-            const float2 v0 = bf2_to_f2(va.x), v1 = bf2_to_f2(va.y);
+            const float2 v0 = bf2_to_f2(vn.x), v1 = bf2_to_f2(vn.y);
             O = make_float4(w_new * v0.x, w_new * v0.y, w_new * v1.x, w_new * v1.y);
           }
 #pragma unroll
