@@ -248,11 +248,21 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_r
  * slot t % window) and finish before the next step's call on the same layer.  Same
  * workspace, q, o and lse as spkv_decode_attn; ring->z_win is required; cache may be
  * NULL (window-only layer).  Returns SPKV_ERR_UNSUPPORTED where
- * spkv_decode_attn_before_append_supported says 0. */
+ * spkv_decode_attn_before_append_supported says 0.
+ * flags: 0, or SPKV_DECODE_STATE_SETTLED -- the caller vouches that t_pos and every
+ * part of this cache and ring (counts, page table, positions, rows, gates) were last
+ * written by work that completes before this call's place on the stream without a
+ * programmatic launch in between: written on another stream joined to this one by an
+ * event, or followed on this stream by an event wait, a copy or a kernel of the
+ * caller's own.  The kernel then plans its chunks from them while the kernel before it
+ * on the stream is still finishing; q, k_new, v_new and the workspace are still read
+ * only after that kernel has completed.  Any other flag bit is an argument error. */
+#define SPKV_DECODE_STATE_SETTLED 1u
 int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* cache,
                                    const spkv_ring* ring, const void* q, const int32_t* t_pos,
                                    const void* k_new, const void* v_new, void* o, float* lse,
-                                   void* workspace, size_t ws_bytes, spkv_stream_t stream);
+                                   void* workspace, size_t ws_bytes, unsigned flags,
+                                   spkv_stream_t stream);
 
 /* 1 if spkv_decode_attn_before_append runs for these parameters (bf16, head_dim 64 or
  * 128, window a multiple of 64), else 0.  Host only; enqueues nothing. */

@@ -229,8 +229,10 @@ int spkv_decode_attn_before_append_supported(const spkv_params* p) {
 int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* c,
                                    const spkv_ring* ring, const void* q, const int32_t* t_pos,
                                    const void* k_new, const void* v_new, void* o, float* lse,
-                                   void* workspace, size_t ws_bytes, spkv_stream_t stream) {
+                                   void* workspace, size_t ws_bytes, unsigned flags,
+                                   spkv_stream_t stream) {
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
+  if (flags & ~SPKV_DECODE_STATE_SETTLED) return SPKV_ERR_ARG;
   if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
   if (!k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
   if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
@@ -239,7 +241,8 @@ int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* c,
   if (sms <= 0) return SPKV_ERR_CUDA;
   if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
   return status_of(spkv::launch_decode_tc(*p, cache_or_none(c), *ring, q, t_pos, o, lse, workspace,
-                                          sms, static_cast<cudaStream_t>(stream), k_new, v_new));
+                                          sms, static_cast<cudaStream_t>(stream), k_new, v_new,
+                                          (flags & SPKV_DECODE_STATE_SETTLED) != 0));
 }
 
 size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* c) {

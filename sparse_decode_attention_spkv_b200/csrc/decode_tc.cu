@@ -221,7 +221,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                      int* __restrict__ ws_ctrl, float* __restrict__ ws_ml,
                      float* __restrict__ ws_o, int n_heads, int hkv, int window,
                      uint32_t* err, const __nv_bfloat16* __restrict__ k_new,
-                     const __nv_bfloat16* __restrict__ v_new, const uint8_t* __restrict__ z_win) {
+                     const __nv_bfloat16* __restrict__ v_new, const uint8_t* __restrict__ z_win,
+                     int early_plan) {
   using TB = TileBuf<D>;
   using S = TcDecSmem<D, G>;
   constexpr int NT_D = D / 8;     // n-tiles of 8 along head_dim
@@ -244,10 +245,12 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_kr)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_vr)) : "memory");
   }
-  // the merge kernel may be scheduled now (it waits for this grid to complete); the
-  // cache counts and the ring are written by the kernel before this one
+  // the merge kernel may be scheduled now (it waits for this grid to complete).  The
+  // cache counts and the ring may be written by the kernel before this one, unless the
+  // caller vouched that they are settled: then the plan, which reads only them and the
+  // positions, runs before the wait, while the previous kernel finishes
   grid_dependents_launch();
-  grid_dependency_wait();
+  if (!early_plan) grid_dependency_wait();
 
   // ---- plan (identical in every CTA) ---------------------------------------------
   int my_rows = 0;
@@ -299,6 +302,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   }
   __syncthreads();
   const int chunk_rows = sm.misc[0];
+  if (early_plan) grid_dependency_wait();  // queries, new rows, workspace: after the wait
   {
     // chunks per head, exclusive prefix over heads: thread segments, warp shuffle scan
     const int per = (n_heads + kThreadsT - 1) / kThreadsT;
@@ -639,8 +643,10 @@ __global__ void __launch_bounds__(kMergeThreads)
     decode_merge_kernel(int* __restrict__ ws_ctrl, const float* __restrict__ ws_ml,
                         const float* __restrict__ ws_o, __nv_bfloat16* __restrict__ out,
                         float* __restrict__ lse_out, int n_heads, int hkv) {
-  grid_dependency_wait();
+  // the next kernel may start launching now (its CTAs take SMs as the decode CTAs exit);
+  // it waits for this grid before touching anything written here
   grid_dependents_launch();
+  grid_dependency_wait();
   const int tid = threadIdx.x;
   const int bh = blockIdx.x;
   if (bh == 0 && tid == 0) ws_ctrl[n_heads] = 0;  // work counter of the next launch
@@ -735,8 +741,8 @@ size_t max_chunks_tc(const spkv_params& p, int num_sms) {
 
 template <int D, int G>
 cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
-                   const int32_t* t_pos, const void* k_new, const void* v_new, void* o, float* lse,
-                   void* ws, int num_sms, cudaStream_t stream) {
+                   const int32_t* t_pos, const void* k_new, const void* v_new, bool early_plan,
+                   void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
   using S = TcDecSmem<D, G>;
   const size_t smem = sizeof(S) + 1024 + ((size_t)5 * p.B * p.Hkv + 1) * 4;
   static int configured = 0;
@@ -780,7 +786,7 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
                              tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
                              static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv,
                              p.window, c.err_flag, static_cast<const __nv_bfloat16*>(k_new),
-                             static_cast<const __nv_bfloat16*>(v_new), ring.z_win);
+                             static_cast<const __nv_bfloat16*>(v_new), ring.z_win, early_plan ? 1 : 0);
   if (e != cudaSuccess) return e;
   return launch_pdl(decode_merge_kernel<D, G>, dim3(n_heads), dim3(kMergeThreads), 0, stream, ctrl,
                     ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
@@ -789,12 +795,13 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
 template <int D>
 cudaError_t dispatch_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                         const void* q, const int32_t* t_pos, const void* k_new, const void* v_new,
-                        void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
+                        bool early_plan, void* o, float* lse, void* ws, int num_sms,
+                        cudaStream_t stream) {
   switch (p.Hq / p.Hkv) {
-    case 1: return run_tc<D, 1>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
-    case 2: return run_tc<D, 2>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
-    case 4: return run_tc<D, 4>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
-    case 8: return run_tc<D, 8>(p, c, ring, q, t_pos, k_new, v_new, o, lse, ws, num_sms, stream);
+    case 1: return run_tc<D, 1>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
+    case 2: return run_tc<D, 2>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
+    case 4: return run_tc<D, 4>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
+    case 8: return run_tc<D, 8>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -818,10 +825,12 @@ size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms) {
 cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                              const void* q, const int32_t* t_pos, void* o, float* lse,
                              void* workspace, int num_sms, cudaStream_t stream,
-                             const void* k_new, const void* v_new) {
+                             const void* k_new, const void* v_new, bool early_plan) {
   if (p.head_dim == 128)
-    return dispatch_tc<128>(p, c, ring, q, t_pos, k_new, v_new, o, lse, workspace, num_sms, stream);
-  return dispatch_tc<64>(p, c, ring, q, t_pos, k_new, v_new, o, lse, workspace, num_sms, stream);
+    return dispatch_tc<128>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, workspace,
+                            num_sms, stream);
+  return dispatch_tc<64>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, workspace,
+                         num_sms, stream);
 }
 
 }  // namespace spkv

@@ -46,7 +46,8 @@ size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms);
 cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                              const void* q, const int32_t* t_pos, void* o, float* lse,
                              void* workspace, int num_sms, cudaStream_t stream,
-                             const void* k_new = nullptr, const void* v_new = nullptr);
+                             const void* k_new = nullptr, const void* v_new = nullptr,
+                             bool early_plan = false);
 cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                           const void* q, const int32_t* t_pos, void* o, float* lse,
                           void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream);

@@ -26,6 +26,7 @@ F32, BF16 = 0, 1
 SRC_CHUNK, SRC_RING = 0, 1
 FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT = 1, 2, 4
 PAGE_ROWS = 64
+DECODE_STATE_SETTLED = 1
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int
@@ -70,7 +71,8 @@ _sigs = {
     "spkv_decode_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _vp,
                                 _vp, ctypes.c_size_t, _vp]),
     "spkv_decode_attn_before_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp,
-                                              _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+                                              _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                              ctypes.c_uint, _vp]),
     "spkv_decode_attn_before_append_supported": (_i32, [_P(spkv_params)]),
     "spkv_prefill_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _i32,
                                  _i32, _vp, _vp, _vp]),
@@ -265,13 +267,14 @@ def spkv_decode_attn(p, cache: Optional[Cache], ring: Ring, q, t_pos, o, lse, wo
 
 
 def spkv_decode_attn_before_append(p, cache: Optional[Cache], ring: Ring, q, t_pos, k_new, v_new,
-                                   o, lse, workspace, stream=None):
+                                   o, lse, workspace, flags=0, stream=None):
     """The decode attention of a step taken before the step's spkv_decode_append (the
-    new rows k_new / v_new passed in); see include/spkv.h."""
+    new rows k_new / v_new passed in); flags: 0 or DECODE_STATE_SETTLED.  See
+    include/spkv.h."""
     return _check("spkv_decode_attn_before_append", lib.spkv_decode_attn_before_append(
         ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos),
         _ptr(k_new), _ptr(v_new), _ptr(o), _ptr(lse), _ptr(workspace), workspace.numel(),
-        _stream(stream)))
+        int(flags), _stream(stream)))
 
 
 def spkv_decode_attn_before_append_supported(p) -> bool:

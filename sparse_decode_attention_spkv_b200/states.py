@@ -162,8 +162,11 @@ class DecodeStep:
                 e = ev.get(l) if ev else None
                 if e is not None:
                     e[0].record()
+                # layer l's cache and ring were last written on the second stream, joined
+                # at the end of the previous step: settled
                 S.spkv_decode_attn_before_append(p, L.cache, L.ring, q[l], t, k[l], v[l],
-                                                 self.o[l], self.lse[l], L.ws)
+                                                 self.o[l], self.lse[l], L.ws,
+                                                 flags=S.DECODE_STATE_SETTLED)
                 if e is not None:
                     e[1].record()
                 # retire t - w, store the new token (gate 0), then its gate: beside the

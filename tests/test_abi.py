@@ -92,12 +92,16 @@ def test_argument_validation_without_gpu():
     # attention before the step's update: needs the new rows; fp32 is not supported
     assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
                                                 ctypes.byref(ring), 16, 16, None, 16, 16, None,
-                                                16, 1 << 20, None) == S.ERR_ARG
+                                                16, 1 << 20, 0, None) == S.ERR_ARG
     assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
                                                 ctypes.byref(ring), 16, 16, 16, 8, 16, None,
-                                                16, 1 << 20, None) == S.ERR_ARG
+                                                16, 1 << 20, 0, None) == S.ERR_ARG
+    assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
+                                                ctypes.byref(ring), 16, 16, 16, 16, 16, None,
+                                                16, 1 << 20, 2, None) == S.ERR_ARG
     assert S.lib.spkv_decode_attn_before_append_supported(ctypes.byref(good)) == 0
     assert S.lib.spkv_decode_attn_before_append_supported(None) == 0
     assert S.lib.spkv_decode_attn_before_append(ctypes.byref(good), ctypes.byref(cache),
                                                 ctypes.byref(ring), 16, 16, 16, 16, 16, None,
-                                                16, 1 << 20, None) == S.ERR_UNSUPPORTED
+                                                16, 1 << 20, S.DECODE_STATE_SETTLED,
+                                                None) == S.ERR_UNSUPPORTED

@@ -47,10 +47,24 @@ def _check_row(wl, L, b, t, o_gpu_b, z_new_b, nrows_retired):
     C.check_attn(o_gpu_b, o_ref[0], "bf16", f"{wl.name} row {b}")
 
 
-def _decode_one_step(wl, rows):
+def _decode_one_step(wl, rows, order="fused"):
+    """One decode step of a full-size state.  order "attn-first" is the bench's launch
+    configuration: attention on the state before the step's update (settled-state
+    flag), update and scoring on the second stream, the whole step captured in a CUDA
+    graph and replayed."""
     p, Ls, inp = build_decode_state(wl, 1, 2, torch.device("cuda"))
-    step = DecodeStep(p, Ls, "cuda")
-    step.launch(inp["h"][0], inp["q"][0], inp["k"][0], inp["v"][0], inp["t"][0])
+    step = DecodeStep(p, Ls, "cuda", split=order != "fused", attn_first=order == "attn-first")
+    if order == "attn-first":
+        L = Ls[0]  # one eager attention (read-only) sets the kernel attributes before capture
+        S.spkv_decode_attn_before_append(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0],
+                                         inp["k"][0][0], inp["v"][0][0], step.o[0], step.lse[0],
+                                         L.ws)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step.launch(inp["h"][0], inp["q"][0], inp["k"][0], inp["v"][0], inp["t"][0])
+        g.replay()
+    else:
+        step.launch(inp["h"][0], inp["q"][0], inp["k"][0], inp["v"][0], inp["t"][0])
     torch.cuda.synchronize()
     status, flags = S.spkv_cache_check(Ls[0].cache)
     assert status == S.OK, flags
@@ -67,6 +81,14 @@ def test_decode32k_one_layer_full_size():
 
 def test_ragged128k_full_size():
     _decode_one_step(_one_layer("ragged128k"), rows=[3, 0])
+
+
+def test_decode32k_attention_first_graph_full_size():
+    _decode_one_step(_one_layer("decode32k"), rows=[2, 7], order="attn-first")
+
+
+def test_ragged128k_attention_first_graph_full_size():
+    _decode_one_step(_one_layer("ragged128k"), rows=[0, 2], order="attn-first")
 
 
 def test_serving_buffered_full_size():
