@@ -59,7 +59,7 @@ constexpr int kChunkPages = 256;     // page numbers staged per fetch
 constexpr int kPgRegs = kChunkPages / 32;
 constexpr int kLookClaim = 4;        // tiles before a chunk's end: claim the next chunk
 constexpr int kLookPages = 2;        // ... and fetch its page-table entries
-constexpr int kMergeBatch = 8;       // partials a merge thread loads at once
+constexpr int kMergeBatch = 16;      // partials a merge thread loads at once
 constexpr float kLog2eT = 1.4426950408889634f;
 constexpr float kLn2T = 0.6931471805599453f;
 constexpr float kSlackT = 8.f;
