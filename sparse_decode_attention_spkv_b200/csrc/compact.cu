@@ -87,10 +87,10 @@ __global__ void __launch_bounds__(256)
   for (int j = threadIdx.x; j < s_grant; j += blockDim.x) table[s_free + j] = s_first + j;
 }
 
-constexpr int kScatterTile = 1024;
+constexpr int kScatterTile = 256;
 constexpr int kScatterThreads = 256;
 
-// grid (B*Hkv, tiles of 1024 rows).  Each CTA counts the gated rows before its
+// grid (B*Hkv, tiles of 256 rows).  Each CTA counts the gated rows before its
 // tile (z is tiny), so tiles need no inter-CTA ordering; inside a tile, 256-row
 // rounds are ranked with a warp-ballot prefix sum and copied by lane groups.
 __global__ void __launch_bounds__(kScatterThreads)

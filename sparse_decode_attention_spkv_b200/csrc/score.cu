@@ -516,6 +516,8 @@ cudaError_t launch_score(const spkv_params& p, const void* h, int n_tok, const v
     return launch_mma<kScoreOnly>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
   if (small_ok(p, n_tok))
     return dispatch_small<kScoreOnly>(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, SmallAppend{}, stream);
+  if (score_tc_supported(p, n_tok))
+    return launch_score_tc(p, h, n_tok, W1, b1, W2, b2, u_out, z_out, stream);
   dim3 grid((n_tok + kTok - 1) / kTok, kKS);
   if (p.dtype == SPKV_BF16) {
     score_kernel<BF16><<<grid, kThreads, 0, stream>>>(
