@@ -239,33 +239,65 @@ def run_gpu(args, world, rank, local):
         raise RuntimeError("non-finite decode output")
 
     # ---- end to end: host inputs in, host outputs back, every step -------------------
+    # Two input/output buffer sets, each with its own captured step: step j's inputs are
+    # copied in (pinned host memory, a copy stream) while step j-1 computes, and step j's
+    # output is read back (another copy stream) while step j+1 computes.  A buffer set is
+    # rewritten only after the step that used it has finished and its output is back.
     e2e = None
     if E > 0:
-        st = {k: torch.empty_like(inp[k][0]) for k in ("h", "q", "k", "v", "t")}
-        host = {k: inp[k][Wm + K:].cpu().pin_memory() for k in ("h", "q", "k", "v", "t")}
+        keys = ("h", "q", "k", "v", "t")
+        host = {k: inp[k][Wm + K:].cpu().pin_memory() for k in keys}
         o_host = torch.empty((E,) + tuple(step.o.shape), dtype=step.o.dtype).pin_memory()
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g):
-            step.launch(st["h"], st["q"], st["k"], st["v"], st["t"])
+        steps2 = [step, DecodeStep(p, Ls, device, split=step.split, attn_first=step.attn_first)]
+        bufs = [{k: torch.empty_like(inp[k][0]) for k in keys} for _ in range(2)]
+        g2 = []
+        for b in range(2):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g):
+                steps2[b].launch(*(bufs[b][k] for k in keys))
+            g2.append(g)
         torch.cuda.synchronize()
+        comp = torch.cuda.current_stream()
+        copy_in, copy_out = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        ev_in = [torch.cuda.Event() for _ in range(E)]
+        ev_done = [torch.cuda.Event() for _ in range(E)]
+        ev_out = [torch.cuda.Event() for _ in range(E)]
         s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         _barrier(world)
         torch.cuda.synchronize()
-        s0.record()
+        s0.record(comp)
+        copy_in.wait_stream(comp)
         for j in range(E):
-            for k_ in st:
-                st[k_].copy_(host[k_][j], non_blocking=True)
-            g.replay()
-            o_host[j].copy_(step.o, non_blocking=True)
-        s1.record()
+            b = j % 2
+            with torch.cuda.stream(copy_in):
+                if j >= 2:
+                    copy_in.wait_event(ev_done[j - 2])  # the step that read bufs[b] is done
+                for k_ in keys:
+                    bufs[b][k_].copy_(host[k_][j], non_blocking=True)
+                ev_in[j].record(copy_in)
+            comp.wait_event(ev_in[j])
+            if j >= 2:
+                comp.wait_event(ev_out[j - 2])  # steps2[b].o of step j-2 is back on the host
+            g2[b].replay()
+            ev_done[j].record(comp)
+            with torch.cuda.stream(copy_out):
+                copy_out.wait_event(ev_done[j])
+                o_host[j].copy_(steps2[b].o, non_blocking=True)
+                ev_out[j].record(copy_out)
+        comp.wait_event(ev_out[E - 1])
+        s1.record(comp)
         torch.cuda.synchronize()
         _barrier(world)
         e2e_ms = _max_over_ranks(s0.elapsed_time(s1), world)
         h2d = sum(host[k_][0].numel() * host[k_][0].element_size() for k_ in host)
         d2h = step.o.numel() * step.o.element_size()
+        if not torch.isfinite(o_host.float()).all():
+            raise RuntimeError("non-finite decode output read back")
         e2e = {"value": world * p.B * E / (e2e_ms / 1e3), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E}
-        del g
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h), "steps": E,
+               "overlap": "inputs of step j copied in during step j-1, output of step j read "
+                          "back during step j+1 (two buffer sets, pinned host memory)"}
+        del g2
     del graphs
 
     peak, peak_kind = _peaks()
