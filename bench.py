@@ -644,9 +644,13 @@ def measure_hybrid(device, steps=10, warmup=3, period=4):
         if status:
             raise RuntimeError(f"hybrid measurement: cache error {flags}")
     del graphs
+    # kernels per layer: decode + merge, the update, and (global layers) the scoring or
+    # the fused score + update
+    per_glob, per_loc = (4, 3) if step.attn_first else (3, 3)
     return {"unit": "tokens/s", "value": p.B / (ms / 1e3), "ms_per_step": ms,
             "layers": {"global": n_glob, "local": n_layers - n_glob, "period": period},
-            "launches_per_step": 2 * n_layers}
+            "order": "attn-first" if step.attn_first else "update first",
+            "launches_per_step": per_glob * n_glob + per_loc * (n_layers - n_glob)}
 
 
 def measure_ragged(device, warmup=3):

@@ -133,11 +133,20 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
     p = layer.p
     z_t = u_t = None
     if layer.local:  # store the new token in the ring; nothing ever retires
-        S.spkv_decode_append(p, None, layer.ring, t_pos, k_t, v_t, None, None, 0)
         if o is None:
             o = torch.empty_like(q_t)
         if lse is None:
             lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=q_t.device)
+        if score_stream is not None and attn_first:
+            S.spkv_decode_attn_before_append(p, None, layer.ring, q_t, t_pos, k_t, v_t, o, lse,
+                                             layer.ws)
+            score_stream.wait_stream(torch.cuda.current_stream())
+            S.spkv_decode_append(p, None, layer.ring, t_pos, k_t, v_t, None, None, 0,
+                                 stream=score_stream)
+            for x in (k_t, v_t, t_pos):
+                x.record_stream(score_stream)
+            return o, lse, None
+        S.spkv_decode_append(p, None, layer.ring, t_pos, k_t, v_t, None, None, 0)
         S.spkv_decode_attn(p, None, layer.ring, q_t, t_pos, o, lse, layer.ws)
         return o, lse, None
     if retire and score_stream is not None and attn_first:

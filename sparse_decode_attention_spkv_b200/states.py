@@ -217,14 +217,23 @@ def kv_bytes_layers(p, layers, t_min):
 class HybridStep:
     """Launch sequence of one decode step over a hybrid local/global stack: layer l is
     global (SP-KV: score, retire, attend over cache + window) when l % period ==
-    period - 1, else local (window only, no cache)."""
+    period - 1, else local (window only, no cache).  With ``attn_first`` (the default
+    where the kernels support it) every layer's attention runs on the state before the
+    step's update, and the updates (and the global layers' scoring) go to a second
+    stream, as in DecodeStep."""
 
-    def __init__(self, p, global_layers, local_layers, period, device):
+    def __init__(self, p, global_layers, local_layers, period, device, attn_first=None):
         from sparse_decode_attention_spkv_b200 import spkv as S
         self.S, self.p, self.period = S, p, period
         self.glob, self.loc = global_layers, local_layers
         n = len(global_layers) + len(local_layers)
         self.n = n
+        if attn_first is None:
+            attn_first = S.spkv_decode_attn_before_append_supported(p)
+        self.attn_first = bool(attn_first)
+        if self.attn_first:
+            self.side = torch.cuda.Stream(device=device)
+            self.fork = [torch.cuda.Event() for _ in range(n)]
         self.o = torch.empty((n, p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
         self.lse = torch.empty((n, p.B, p.Hq), dtype=torch.float32, device=device)
         self.u = torch.empty((len(global_layers), p.B, p.Hkv), dtype=torch.float32, device=device)
@@ -234,6 +243,9 @@ class HybridStep:
         """h, q, k, v indexed by global-layer number (local layers reuse q, k, v of
         global layer l // period: their values do not change the work)."""
         S, p = self.S, self.p
+        if self.attn_first:
+            self._launch_attn_first(h, q, k, v, t)
+            return
         gi = li = 0
         for l in range(self.n):
             g = l // self.period
@@ -248,6 +260,33 @@ class HybridStep:
                 S.spkv_decode_append(p, None, L.ring, t, k[g], v[g], None, None, 0)
                 S.spkv_decode_attn(p, None, L.ring, q[g], t, self.o[l], self.lse[l], L.ws)
                 li += 1
+
+    def _launch_attn_first(self, h, q, k, v, t):
+        S, p = self.S, self.p
+        main = torch.cuda.current_stream()
+        gi = li = 0
+        for l in range(self.n):
+            g = l // self.period
+            glob = l % self.period == self.period - 1
+            L = self.glob[gi] if glob else self.loc[li]
+            cache = L.cache if glob else None
+            # every layer's cache and ring were last written on the second stream, joined
+            # at the end of the previous step: settled
+            S.spkv_decode_attn_before_append(p, cache, L.ring, q[g], t, k[g], v[g], self.o[l],
+                                             self.lse[l], L.ws, flags=S.DECODE_STATE_SETTLED)
+            self.fork[l].record(main)
+            self.side.wait_event(self.fork[l])
+            if glob:
+                S.spkv_decode_append(p, L.cache, L.ring, t, k[g], v[g], None, None, 1,
+                                     stream=self.side)
+                S.spkv_decode_score(p, L.ring, t, h[g], L.W1, L.b1, L.W2, L.b2, self.u[gi],
+                                    self.z[gi], stream=self.side)
+                gi += 1
+            else:
+                S.spkv_decode_append(p, None, L.ring, t, k[g], v[g], None, None, 0,
+                                     stream=self.side)
+                li += 1
+        main.wait_stream(self.side)
 
     LAUNCHES_GLOBAL = 2
     LAUNCHES_LOCAL = 2

@@ -33,9 +33,13 @@ def _params(wl):
                          S.BF16 if wl.dtype == "bf16" else S.F32)
 
 
-@pytest.mark.parametrize("name", sorted(CASES))
-def test_hybrid_stack_matches_oracle(name):
+@pytest.mark.parametrize("name,attn_first", [(n, False) for n in sorted(CASES)] +
+                         [("bf16_3to1", True)])
+def test_hybrid_stack_matches_oracle(name, attn_first):
+    """attn_first: every layer's decode attention on the state before the step's update
+    (spkv_decode_attn_before_append), the update and scoring on a second stream."""
     wl, period = CASES[name]
+    side = torch.cuda.Stream() if attn_first else None
     T0, steps, w = wl.ctx[0], wl.decode_steps, wl.window
     T = T0 + steps
     p = _params(wl)
@@ -75,7 +79,10 @@ def test_hybrid_stack_matches_oracle(name):
         for l, L in enumerate(layers):
             h, q, k, v = host[l]
             o, _, _ = R.decode_step(L, t_pos, C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype),
-                                    C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype))
+                                    C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype),
+                                    score_stream=side, attn_first=attn_first)
+            if side is not None:
+                torch.cuda.current_stream().wait_stream(side)
             og = C.to_np(o)
             for b in range(wl.B):
                 o_ref, _ = O.gated_attention(q[b, t:t + 1], k[b, :t + 1], v[b, :t + 1],
