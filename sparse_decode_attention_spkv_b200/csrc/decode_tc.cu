@@ -9,11 +9,11 @@
 // G query heads of a group are the rows of a 16-row MMA tile, so the same bytes cost
 // a few instructions and the kernel is left bound by HBM.
 //
-// Structure (one CTA per SM, 5 warps):
+// Structure (one CTA per SM, 6 warps: 4 consumers, a producer, a finisher):
 //  * Plan (every CTA, same result): live cache rows per head, rows rounded to 64-row
-//    tiles (cache pages), chunk size so that all heads give a few chunks per CTA,
-//    chunk prefix.  The producer pulls chunks from a global atomic counter, so ragged
-//    heads balance.
+//    tiles (cache pages), chunk size so that all heads give about 4 chunks per CTA,
+//    chunk prefix.  Each CTA's first chunk is its own index; the producer pulls later
+//    chunks from a global atomic counter, so ragged heads balance.
 //  * Producer warp: per chunk, its lanes fetch all the chunk's page-table entries at
 //    once into shared memory; then one lane streams 64-row tiles (TMA boxes of
 //    64 rows x 64 bf16, 128B-swizzled) of K and V from the cache pages or the ring
@@ -23,12 +23,15 @@
 //    = the G heads, zero-padded to 16), fp32 softmax in the log2 domain (running max
 //    raised only when exceeded by > 8), P re-packed in registers as the A operand of
 //    O += P V (V via ldmatrix.trans).
-//  * Chunk end: the warps combine through shared memory; a head with one chunk writes
-//    o and lse, otherwise the chunk's (o, m, l) partial goes to the workspace.
-//  * decode_merge_kernel (one CTA per head with several chunks, launched next on the
-//    same stream) combines the partials: o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i,
-//    and resets the work counter for the next call.  A second launch costs less than
-//    the decode CTAs waiting on an arrival count at the end of every head.
+//  * Chunk end: the consumer warps hand their partials to the finisher warp through
+//    double-buffered shared slots and go on with the next chunk; the finisher combines
+//    them: a head with one chunk gets its o and lse written, otherwise the chunk's
+//    (o, m, l) partial goes to the workspace.
+//  * decode_merge_kernel (one CTA per head, launched next on the same stream as a
+//    programmatic dependent; heads with one chunk return at once) combines the
+//    partials: o = sum_i 2^{m_i-m} o_i / sum_i 2^{m_i-m} l_i, and resets the work counter
+//    for the next call.  A second launch costs less than the decode CTAs waiting on an
+//    arrival count at the end of every head.
 //  * Before-append mode (k_new given): the step's retirement and ring write have not
 //    run yet.  The ring then holds rows t-w .. t-1; slot t mod w (row t - w, which
 //    leaves the window at query t) counts only if its stored gate is 1, cache rows
