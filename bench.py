@@ -179,11 +179,12 @@ def run_gpu(args, world, rank, local):
     device = torch.device("cuda", local)
     wl = W.WORKLOADS[WORKLOAD]
     layers = wl.layers
-    K, Wm, E = args.steps, args.warmup, args.e2e_steps
+    K, Wm = args.steps, args.warmup
     R = 4  # steps with per-layer events, after the timed and end-to-end steps
+    if Wm + K + R > wl.decode_steps:
+        raise SystemExit(f"warmup+steps must be <= {wl.decode_steps - R}")
+    E = max(0, min(args.e2e_steps, wl.decode_steps - R - Wm - K))  # what is left of the steps
     steps_total = Wm + K + E + R
-    if steps_total > wl.decode_steps:
-        raise SystemExit(f"warmup+steps+e2e-steps must be <= {wl.decode_steps - R}")
     from sparse_decode_attention_spkv_b200.states import (DecodeStep, build_decode_state, kv_bytes,
                                                           kv_bytes_layers)
     p, Ls, inp = build_decode_state(wl, layers, steps_total, device)
@@ -893,8 +894,7 @@ def main():
                          "scoring on a second stream; fused: score, retirement and ring write "
                          "in one launch, then the attention")
     args = ap.parse_args()
-    if args.warmup < 3:
-        raise SystemExit("--warmup must be >= 3")
+    args.warmup = max(3, args.warmup)  # at least 3 untimed steps; the line reports the count run
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
