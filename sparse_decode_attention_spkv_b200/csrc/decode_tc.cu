@@ -250,8 +250,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   }
   // the merge kernel may be scheduled now (it waits for this grid to complete).  The
   // cache counts and the ring may be written by the kernel before this one, unless the
-  // caller vouched that they are settled: then the plan, which reads only them and the
-  // positions, runs before the wait, while the previous kernel finishes
+  // caller vouched that they are settled: then the plan and the producer's first
+  // page-table reads, which touch only them and the positions, run before the wait,
+  // while the previous kernel finishes.  The consumer warps read shared memory only.
   grid_dependents_launch();
   if (!early_plan) grid_dependency_wait();
 
@@ -305,7 +306,6 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   }
   __syncthreads();
   const int chunk_rows = sm.misc[0];
-  if (early_plan) grid_dependency_wait();  // queries, new rows, workspace: after the wait
   {
     // chunks per head, exclusive prefix over heads: thread segments, warp shuffle scan
     const int per = (n_heads + kThreadsT - 1) / kThreadsT;
@@ -349,6 +349,9 @@ __global__ void __launch_bounds__(kThreadsT, 1)
                                   s_hide, n_heads, hkv);
     int pg[kPgRegs];
     fetch_pages(pg, cd, cache, lane);
+    // with a settled state the plan and the first page-table reads above ran while the
+    // previous kernel finished; the queries and the work counter come after the wait
+    if (early_plan) grid_dependency_wait();
     for (int seq = 0; cd.c < total_chunks; ++seq) {
       __syncwarp();
 #pragma unroll
@@ -422,6 +425,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     // Combines the 4 consumer warps' partials of each finished chunk (max-weighted
     // sums) and writes the head's output (single-chunk head) or the chunk partial for
     // the merge kernel, while the consumers already work on the next chunk.
+    if (early_plan) grid_dependency_wait();  // new rows, queries, outputs: after the wait
     for (int nf = 0;; ++nf) {
       const int par = nf & 1;
       mbar_wait(&sm.cdone[par], (nf >> 1) & 1, err);
@@ -629,8 +633,10 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     mbar_arrive(&sm.cdone[par]);
   }
   // the chunk prefix for the merge kernel (identical in every CTA; CTA 0 publishes it)
-  if (blockIdx.x == 0)
+  if (blockIdx.x == 0) {
+    grid_dependency_wait();  // returns at once where it was already passed
     for (int i = tid; i <= n_heads; i += kThreadsT) ws_ctrl[n_heads + 2 + i] = s_base[i];
+  }
 }
 
 // Second kernel of a decode step: merges the chunk partials of every head that was
