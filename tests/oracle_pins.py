@@ -316,10 +316,30 @@ def pin_soft_special_cases():
     _close(o_soft, o_hard, 1e-12, "beta -> 0 is the hard gate")
 
 
+def pin_permutation_invariance():
+    """Eq. (3) is a sum over the key set: listing the visible keys in another order (as
+    a cache whose rows were written in another order would) changes nothing but
+    rounding."""
+    rng = np.random.default_rng(21)
+    for _ in range(50):
+        T, d = int(rng.integers(2, 40)), 8
+        q = rng.standard_normal(d)
+        K = rng.standard_normal((T, d))
+        V = rng.standard_normal((T, d))
+        mask = rng.random(T) < 0.6
+        mask[int(rng.integers(T))] = True  # at least one key
+        perm = rng.permutation(T)
+        o1, l1 = O.attend(q, K, V, mask)
+        o2, l2 = O.attend(q, K[perm], V[perm], mask[perm])
+        _close(o1, o2, 1e-12, "permuted keys: output")
+        _close(np.array([l1]), np.array([l2]), 1e-12, "permuted keys: lse")
+
+
 ALL_PINS = [
     pin_gelu_textbook, pin_gelu_library, pin_utility_zero_weights, pin_utility_hand_example,
     pin_utility_library, pin_gate_threshold, pin_gate_extremes, pin_keysets_golden,
     pin_two_key_softmax, pin_tau0_is_causal, pin_tau_gt1_is_sliding_window,
     pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows, pin_rethreshold,
     pin_soft_gate_values, pin_soft_two_key_closed_form, pin_soft_special_cases,
+    pin_permutation_invariance,
 ]

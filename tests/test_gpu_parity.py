@@ -424,6 +424,61 @@ def test_attention_first_decode_step(name):
         assert S.spkv_cache_check(L.cache)[0] == S.OK
 
 
+def test_cache_row_order_does_not_change_decode():
+    """Permutation invariance (the split-K chunking and the merge): every head's cache
+    rows shuffled in place (K, V and positions moved together, pages unchanged) give
+    the same decode output up to rounding, and both orders match the oracle.  The
+    attention runs before the step's update (it leaves the state untouched), so it can
+    be called on the same state twice."""
+    wl = W.small_case("decode32k", cid=65, B=2, Hq=8, Hkv=2, d_model=256, hid=64, ctx=[3000],
+                      decode_steps=1, layers=1, keep="u05_50")
+    T0, w = wl.ctx[0], wl.window
+    T = T0 + 1
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    mp = R.pages_for(T)
+    L = R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                       num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp)
+    h, q, k, v = _rows(wl, T)
+    for c0 in range(0, T0, 512):
+        c1 = min(T0, c0 + 512)
+        R.prefill_chunk(L, C.dev(h[:, c0:c1], wl.dtype), C.dev(q[:, c0:c1], wl.dtype),
+                        C.dev(k[:, c0:c1], wl.dtype), C.dev(v[:, c0:c1], wl.dtype), c0,
+                        n_compact=max(0, min(c1, T0 - w) - c0))
+    t_pos = torch.full((wl.B,), T0, dtype=torch.int32, device="cuda")
+    args = (C.dev(q[:, T0], wl.dtype), t_pos, C.dev(k[:, T0], wl.dtype), C.dev(v[:, T0], wl.dtype))
+
+    def attend():
+        o = torch.empty_like(args[0])
+        lse = torch.empty((wl.B, wl.Hq), dtype=torch.float32, device="cuda")
+        S.spkv_decode_attn_before_append(p, L.cache, L.ring, args[0], args[1], args[2], args[3], o,
+                                         lse, L.ws)
+        return C.to_np(o)
+
+    o1 = attend()
+    gen = torch.Generator().manual_seed(65)
+    count = L.cache.count.cpu()
+    moved = 0
+    for bh in range(wl.B * wl.Hkv):
+        n = int(count[bh])
+        idx = torch.arange(n)
+        pages = L.cache.page_table[bh].cpu()[idx // S.PAGE_ROWS].long().cuda()
+        rows = (idx % S.PAGE_ROWS).cuda()
+        perm = torch.randperm(n, generator=gen).cuda()
+        for pool in (L.cache.K_pool, L.cache.V_pool, L.cache.pos_pool):
+            pool[pages, rows] = pool[pages, rows][perm]
+        moved += n
+    assert moved > 1000
+    o2 = attend()
+    assert np.max(np.abs(o1 - o2)) <= 2e-2
+    _, z_ref = C.oracle_gates(h.reshape(-1, wl.d_model), W1, b1, W2, b2, wl.tau)
+    z_ref = z_ref.reshape(wl.B, T, wl.Hkv)
+    for b in range(wl.B):
+        o_ref, _ = O.gated_attention(q[b, T0:T], k[b, :T], v[b, :T], z_ref[b], w, [T0])
+        C.check_attn(o1[b], o_ref[0], wl.dtype, f"cache in order, b={b}")
+        C.check_attn(o2[b], o_ref[0], wl.dtype, f"cache rows shuffled, b={b}")
+
+
 def test_attention_first_lse():
     """lse of the attention-first step against the oracle's log-sum-exp (natural log of
     the softmax denominator over the key set, scores scaled by 1/sqrt(d))."""
