@@ -254,9 +254,10 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_r
  * written by work that completes before this call's place on the stream without a
  * programmatic launch in between: written on another stream joined to this one by an
  * event, or followed on this stream by an event wait, a copy or a kernel of the
- * caller's own.  The kernel then plans its chunks from them while the kernel before it
- * on the stream is still finishing; q, k_new, v_new and the workspace are still read
- * only after that kernel has completed.  Any other flag bit is an argument error. */
+ * caller's own.  The kernel then plans its chunks from them, and reads its first
+ * page-table entries, while the kernel before it on the stream is still finishing;
+ * q, k_new, v_new and the workspace are still accessed only after that kernel has
+ * completed.  Any other flag bit is an argument error. */
 #define SPKV_DECODE_STATE_SETTLED 1u
 int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* cache,
                                    const spkv_ring* ring, const void* q, const int32_t* t_pos,
