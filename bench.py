@@ -137,17 +137,23 @@ class ClockSampler:
 
 # ------------------------------------------------------------------- GPU arm -------
 
-def _kernel_source_hash() -> str:
-    """Hash of the decode kernels' code (comments and blank lines left out, so that a
-    comment edit does not orphan the profile taken on the same code)."""
+def _code_hash(paths) -> str:
+    """Hash of source files' code, line comments and blank lines left out (so that a
+    comment edit does not orphan a profile taken on the same code)."""
     h = hashlib.sha256()
-    for name in ("decode.cu", "decode_tc.cu", "common.cuh"):
-        with open(os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "csrc", name)) as f:
+    for path in paths:
+        with open(path) as f:
             for line in f:
                 code = line.split("//", 1)[0].rstrip()
                 if code:
                     h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
+
+
+def _kernel_source_hash() -> str:
+    """_code_hash of the decode kernels' sources."""
+    return _code_hash(os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "csrc", name)
+                      for name in ("decode.cu", "decode_tc.cu", "common.cuh"))
 
 
 def _profiled_traffic(launch_bytes: float):

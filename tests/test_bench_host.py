@@ -1,0 +1,40 @@
+"""Host-side logic of bench.py (no GPU): the profile key that ties a committed ncu
+capture to the kernel code it was taken on, and the scaling of its traffic."""
+import os
+
+import bench
+
+
+def test_code_hash_ignores_comments_and_blank_lines(tmp_path):
+    a = tmp_path / "a.cu"
+    b = tmp_path / "b.cu"
+    a.write_text("int x = 1;  // one\n\nint y = 2;\n")
+    b.write_text("// a header comment\nint x = 1;\n   \nint y = 2;   // two\n")
+    assert bench._code_hash([a]) == bench._code_hash([b])
+    b.write_text("int x = 1;\nint y = 3;\n")
+    assert bench._code_hash([a]) != bench._code_hash([b])
+
+
+def test_profiled_traffic_scales_with_the_launch(monkeypatch, tmp_path):
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "decode_attn_decode32k.md").write_text(
+        "text\nbench-key source_hash=abc\nbench-key traffic_bytes_per_launch=1020\n"
+        "bench-key algorithmic_bytes_per_launch=1000\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    monkeypatch.setattr(bench, "_kernel_source_hash", lambda: "abc")
+    assert abs(bench._profiled_traffic(2000.0) - 2040.0) < 1e-9
+    monkeypatch.setattr(bench, "_kernel_source_hash", lambda: "other")
+    assert bench._profiled_traffic(2000.0) is None  # the kernel changed since the capture
+
+
+def test_committed_profile_key_is_well_formed():
+    path = os.path.join(bench.ROOT, "profiles", "decode_attn_decode32k.md")
+    keys = {}
+    with open(path) as f:
+        for line in f:
+            if line.startswith("bench-key "):
+                k, _, v = line[len("bench-key "):].strip().partition("=")
+                keys[k] = v
+    assert set(keys) == {"source_hash", "traffic_bytes_per_launch", "algorithmic_bytes_per_launch"}
+    assert float(keys["traffic_bytes_per_launch"]) >= float(keys["algorithmic_bytes_per_launch"])
