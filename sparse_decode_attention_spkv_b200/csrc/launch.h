@@ -38,7 +38,7 @@ cudaError_t launch_ring_write(const spkv_params& p, const spkv_ring& ring, const
                               int gated_from, const int32_t* src_pos, int n_rows,
                               int src_batch_rows, cudaStream_t stream);
 
-// a1 on tcgen05 tensor cores for more than 64 tokens (bf16, hid 128).
+// a1 on tcgen05 tensor cores for 128 tokens or more (bf16, hid 128).
 bool score_tc_supported(const spkv_params& p, int n_tok);
 cudaError_t launch_score_tc(const spkv_params& p, const void* h, int n_tok, const void* W1,
                             const float* b1, const float* W2, const float* b2, float* u_out,

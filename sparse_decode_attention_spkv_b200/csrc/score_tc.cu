@@ -189,9 +189,12 @@ constexpr size_t kScoreTcSmem = sizeof(ScoreTcSmem) + 1024;  // + alignment slac
 
 }  // namespace
 
+// At least one whole 128-token tile (shorter calls go to the other score kernels, so the
+// tensor map's box never exceeds the token dimension).
 bool score_tc_supported(const spkv_params& p, int n_tok) {
   return p.dtype == SPKV_BF16 && p.hid == kSHid && p.d_model % kSKB == 0 &&
-         p.d_model >= kSKB * kSRanks && p.Hkv <= kSMaxHkv && n_tok > 64 && encode_fn() != nullptr;
+         p.d_model >= kSKB * kSRanks && p.Hkv <= kSMaxHkv && n_tok >= kSTok &&
+         encode_fn() != nullptr;
 }
 
 cudaError_t launch_score_tc(const spkv_params& p, const void* h, int n_tok, const void* W1,

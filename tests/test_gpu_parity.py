@@ -42,7 +42,9 @@ SCORE_CASES = {
     "llama_bf16_300": (W.small_case("decode32k", B=1, ctx=[300], decode_steps=0, layers=1), 300),
     "llama_bf16_1": (W.small_case("decode32k", B=1, ctx=[1], decode_steps=0, layers=1), 1),
     "llama_bf16_33": (W.small_case("decode32k", B=1, ctx=[33], decode_steps=0, layers=1), 33),
-    # more than 64 tokens, bf16, hid 128: the tcgen05 score (128-token tiles, d_model split
+    # 65..127 tokens: the CUDA-core tile kernel (less than one 128-token tile)
+    "llama_bf16_100": (W.small_case("decode32k", B=1, ctx=[100], decode_steps=0, layers=1), 100),
+    # 128 tokens or more, bf16, hid 128: the tcgen05 score (128-token tiles, d_model split
     # over a cluster of 4); a whole 4096-token chunk, a ragged count, and d_model 256 (one
     # K block per rank) with 16 key heads
     "llama_bf16_4096": (W.small_case("decode32k", B=1, ctx=[4096], decode_steps=0, layers=1), 4096),
