@@ -5,7 +5,6 @@ import glob
 import os
 import re
 
-import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 LIB = os.path.join(ROOT, "sparse_decode_attention_spkv_b200", "libspkv.so")

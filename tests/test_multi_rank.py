@@ -4,7 +4,6 @@ import os
 import socket
 
 import pytest
-import torch
 import torch.multiprocessing as mp
 
 from sparse_decode_attention_spkv_b200 import dist as D
