@@ -243,10 +243,11 @@ int spkv_decode_attn(const spkv_params* p, const spkv_cache* cache, const spkv_r
  *   - cache rows count up to position t - window - 1;
  *   - the new token t is k_new / v_new [B][Hkv][head_dim] dtype (the rows the step's
  *     spkv_decode_append will store).
- * This is the state of the per-token schedule, where every window slot holds its
- * token's gate (spkv_decode_score or spkv_decode_score_append wrote it).  A buffered
- * schedule that scores the window in bulk and compacts from the ring without storing
- * the gates back into the ring must use spkv_decode_attn instead.
+ * This is the state of the per-token schedule: no row still in the window has been
+ * compacted into the cache (the cache holds positions <= t - window - 1 only) and every
+ * window slot holds its token's gate.  A schedule that compacts window rows early (bulk
+ * scoring from the ring, or a prefill that compacts every row of its last chunk) must
+ * use spkv_decode_attn instead.
  * The step's spkv_decode_append (and spkv_decode_score) may then run after this call,
  * off the attention's path: they must start after it has finished (they overwrite
  * slot t % window) and finish before the next step's call on the same layer.  Same
