@@ -95,6 +95,13 @@ def _soft_mask_acausal(t, s, alpha, w, c):
     return np.where((t - s < w) & (t - s >= 0), 0.0, float(c) * (np.asarray(alpha) - 1.0))
 
 
+def _attend_lse_without_max(q, K, V, mask):
+    o, lse = _ORIG_ATTEND(q, K, V, mask)
+    logits = np.where(mask, (np.asarray(K, dtype=np.float64) @ np.asarray(q, dtype=np.float64))
+                      / np.sqrt(len(q)), -np.inf)
+    return o, lse - np.max(logits)  # the max subtracted for stability never added back
+
+
 _ORIG_ATTEND = O.attend
 _ORIG_LOGITS = O.utility_logits
 
@@ -106,6 +113,7 @@ MUTANTS = {
     "gated_keys_not_causal": ("visible", _visible_acausal),
     "gate_strict_inequality": ("gate", _gate_strict),
     "missing_inv_sqrt_dk": ("attend", _attend_no_scale),
+    "lse_without_max": ("attend", _attend_lse_without_max),
     "dropped_b1": ("utility_logits", _utility_no_b1),
     "sigmoid_sign": ("sigmoid", _sigmoid_flipped),
     "gqa_modulo_mapping": ("gated_attention", _gqa_modulo),
