@@ -102,6 +102,20 @@ def _attend_lse_without_max(q, K, V, mask):
     return o, lse - np.max(logits)  # the max subtracted for stability never added back
 
 
+def _cache_rows_inclusive(z_col, upto):
+    z_col = np.asarray(z_col, dtype=np.uint8)[:upto + 1]  # one row past the boundary
+    return np.nonzero(z_col == 1)[0].astype(np.int32)
+
+
+def _utility_no_gelu(h, W1, b1, W2, b2):
+    a = np.asarray(h, dtype=np.float64) @ np.asarray(W1, dtype=np.float64).T + np.asarray(b1)
+    return a @ np.asarray(W2, dtype=np.float64).T + np.asarray(b2)
+
+
+def _soft_gate_no_beta(u, tau, beta):
+    return O.sigmoid(np.asarray(u, dtype=np.float64) - float(tau))
+
+
 _ORIG_ATTEND = O.attend
 _ORIG_LOGITS = O.utility_logits
 
@@ -120,6 +134,9 @@ MUTANTS = {
     "rethreshold_strict_inequality": ("rethreshold", _rethreshold_strict),
     "rethreshold_inverted": ("rethreshold", _rethreshold_inverted),
     "soft_gate_flipped": ("soft_gate", _soft_gate_flipped),
+    "soft_gate_missing_beta": ("soft_gate", _soft_gate_no_beta),
+    "cache_rows_past_boundary": ("cache_rows", _cache_rows_inclusive),
+    "perceptron_without_gelu": ("utility_logits", _utility_no_gelu),
     "soft_window_off_by_one": ("soft_mask", _soft_mask_window_off_by_one),
     "soft_bias_sign": ("soft_mask", _soft_mask_sign),
     "soft_not_causal": ("soft_mask", _soft_mask_acausal),
