@@ -122,6 +122,7 @@ int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, c
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (n_tok == 0) return SPKV_OK;
   if (!h || !W1 || !b1 || !W2 || !b2 || !z_out) return SPKV_ERR_ARG;
+  if (!aligned16(h) || !aligned16(W1)) return SPKV_ERR_ARG;  // 16-byte vector and TMA loads
   if (!spkv::score_supported(*p)) return SPKV_ERR_UNSUPPORTED;
   return status_of(spkv::launch_score(*p, h, n_tok, W1, b1, W2, b2, u_out, z_out,
                                       static_cast<cudaStream_t>(stream)));

@@ -48,6 +48,9 @@ def test_argument_validation_without_gpu():
         assert S.lib.spkv_score(ctypes.byref(p), None, 4, None, None, None, None, None, None,
                                 None) == S.ERR_ARG
     good = S.make_params(1, 4, 2, 64, 256, 64, 128, 0.5, S.F32)
+    # h and W1 must be 16-byte aligned (vector and tensor-map loads)
+    assert S.lib.spkv_score(ctypes.byref(good), 8, 4, 16, 16, 16, 16, None, 16, None) == S.ERR_ARG
+    assert S.lib.spkv_score(ctypes.byref(good), 16, 4, 24, 16, 16, 16, None, 16, None) == S.ERR_ARG
     # zero tokens is a no-op that needs no pointers
     assert S.lib.spkv_score(ctypes.byref(good), None, 0, None, None, None, None, None, None,
                             None) == S.OK
