@@ -30,8 +30,9 @@
  * - Layouts are dense row-major with the shapes given below.  head_dim must be
  *   64 or 128, Hq a multiple of Hkv with Hq/Hkv in {1,2,4,8}, window in [1, 1024],
  *   page_rows 64.  Pointers to tensors must be 16-byte aligned.
- * - Positions are absolute token indices (int32).  Query head h reads key head
- *   h / (Hq/Hkv) (grouped-query attention).
+ * - Positions are absolute token indices (int32, >= 0; positions given in device
+ *   memory, such as t_pos, are not range-checked on the device).  Query head h reads
+ *   key head h / (Hq/Hkv) (grouped-query attention).
  * - The decode-step kernels (few-token scoring, retirement, decode attention and its
  *   merge) are launched as programmatic dependents: each may start while the kernel
  *   before it on the stream is finishing, and waits for that kernel to complete before
