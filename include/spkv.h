@@ -24,6 +24,9 @@
  *   only the device can see (cache pool exhausted, page table full, a bounded wait
  *   that gave up) set bits of cache->err_flag, read by spkv_cache_check.
  *   No entry point aborts, throws or traps.
+ * - Every entry point that enqueues work marks an NVTX range named after itself for
+ *   the duration of the host call (visible in Nsight Systems; a no-op call when no
+ *   tool is attached).
  * - Element types: `dtype` SPKV_F32 or SPKV_BF16 applies to h, W1, q, k, v, the
  *   cache pool, the ring and the attention output.  b1, W2, b2, u and lse are fp32
  *   in both cases.  Arithmetic is fp32 (bf16 inputs are widened exactly).

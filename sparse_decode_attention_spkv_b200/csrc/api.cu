@@ -9,6 +9,7 @@
 #include "../../include/spkv.h"
 #include "common.cuh"
 #include "launch.h"
+#include "trace.h"
 
 namespace {
 
@@ -87,6 +88,7 @@ int spkv_version(void) { return 300; }
 
 int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                      spkv_stream_t stream) {
+  SPKV_TRACE("spkv_cache_reset");
   if (!params_ok(p) || !cache_ok(p, c)) return SPKV_ERR_ARG;
   if (ring && !ring_ok(ring)) return SPKV_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -103,6 +105,7 @@ int spkv_cache_reset(const spkv_params* p, const spkv_cache* c, const spkv_ring*
 }
 
 int spkv_cache_check(const spkv_cache* c, spkv_stream_t stream, uint32_t* flags_out) {
+  SPKV_TRACE("spkv_cache_check");
   if (!c || !c->err_flag) return SPKV_ERR_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t flags = 0;
@@ -118,6 +121,7 @@ int spkv_cache_check(const spkv_cache* c, spkv_stream_t stream, uint32_t* flags_
 int spkv_score(const spkv_params* p, const void* h, int n_tok, const void* W1, const float* b1,
                const float* W2, const float* b2, float* u_out, uint8_t* z_out,
                spkv_stream_t stream) {
+  SPKV_TRACE("spkv_score");
   if (!params_ok(p) || n_tok < 0) return SPKV_ERR_ARG;
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (n_tok == 0) return SPKV_OK;
@@ -132,6 +136,7 @@ int spkv_write_compact(const spkv_params* p, const spkv_cache* c, const spkv_rin
                        int src_kind, const void* K_src, const void* V_src, const uint8_t* z,
                        const float* u, const int32_t* src_pos, int n_rows, int src_batch_rows,
                        spkv_stream_t stream) {
+  SPKV_TRACE("spkv_write_compact");
   if (!params_ok(p) || !cache_ok(p, c) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
   if (n_rows == 0) return SPKV_OK;
   if (!z || !src_pos) return SPKV_ERR_ARG;
@@ -152,6 +157,7 @@ int spkv_decode_append(const spkv_params* p, const spkv_cache* c, const spkv_rin
                        const int32_t* t_pos, const void* k_new, const void* v_new,
                        const uint8_t* z_new, const float* u_new, int retire,
                        spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_append");
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (!c && retire) return SPKV_ERR_ARG;  // nowhere to retire into
   if (!t_pos || !k_new || !v_new || !aligned16(k_new) || !aligned16(v_new)) return SPKV_ERR_ARG;
@@ -165,6 +171,7 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const sp
                              const float* W2, const float* b2, const void* k_new,
                              const void* v_new, float* u_out, uint8_t* z_out,
                              spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_score_append");
   if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (!t_pos || !h || !W1 || !b1 || !W2 || !b2 || !k_new || !v_new || !z_out) return SPKV_ERR_ARG;
@@ -178,6 +185,7 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const sp
 int spkv_decode_score(const spkv_params* p, const spkv_ring* ring, const int32_t* t_pos,
                       const void* h, const void* W1, const float* b1, const float* W2,
                       const float* b2, float* u_out, uint8_t* z_out, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_score");
   if (!params_ok(p) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (!t_pos || !h || !W1 || !b1 || !W2 || !b2 || !z_out) return SPKV_ERR_ARG;
@@ -191,6 +199,7 @@ int spkv_decode_score(const spkv_params* p, const spkv_ring* ring, const int32_t
 int spkv_ring_write(const spkv_params* p, const spkv_ring* ring, const void* K_src,
                     const void* V_src, const uint8_t* z_src, const float* u_src, int gated_from,
                     const int32_t* src_pos, int n_rows, int src_batch_rows, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_ring_write");
   if (!params_ok(p) || !ring_ok(ring) || n_rows < 0 || src_batch_rows < n_rows) return SPKV_ERR_ARG;
   if (n_rows == 0) return SPKV_OK;
   if (!K_src || !V_src || !src_pos || !aligned16(K_src) || !aligned16(V_src)) return SPKV_ERR_ARG;
@@ -213,6 +222,7 @@ size_t spkv_decode_workspace_bytes(const spkv_params* p, const spkv_cache* c) {
 int spkv_decode_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                      const void* q, const int32_t* t_pos, void* o, float* lse, void* workspace,
                      size_t ws_bytes, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_attn");
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
   if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
@@ -232,6 +242,7 @@ int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* c,
                                    const void* k_new, const void* v_new, void* o, float* lse,
                                    void* workspace, size_t ws_bytes, unsigned flags,
                                    spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_attn_before_append");
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (flags & ~SPKV_DECODE_STATE_SETTLED) return SPKV_ERR_ARG;
   if (!q || !t_pos || !o || !workspace || !aligned16(q) || !aligned16(o)) return SPKV_ERR_ARG;
@@ -254,6 +265,7 @@ size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* 
 int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                            float tau_new, void* workspace, size_t ws_bytes,
                            spkv_stream_t stream) {
+  SPKV_TRACE("spkv_cache_rethreshold");
   if (!params_ok(p) || !cache_ok(p, c) || !c->u_pool) return SPKV_ERR_ARG;
   if (ring && !ring_ok(ring)) return SPKV_ERR_ARG;
   if (!(tau_new == tau_new) || !workspace) return SPKV_ERR_ARG;
@@ -273,6 +285,7 @@ size_t spkv_soft_attn_workspace_bytes(const spkv_params* p, int seq_len) {
 int spkv_soft_attn(const spkv_params* p, const void* q, const void* K, const void* V,
                    const float* u, int seq_len, float beta, float c, void* o, float* lse,
                    void* workspace, size_t ws_bytes, uint32_t* err_flag, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_soft_attn");
   if (!params_ok(p) || seq_len < 0) return SPKV_ERR_ARG;
   if (!(beta > 0.f) || !(c >= 0.f) || !(c < INFINITY)) return SPKV_ERR_ARG;
   if (seq_len == 0) return SPKV_OK;
@@ -287,6 +300,7 @@ int spkv_soft_attn(const spkv_params* p, const void* q, const void* K, const voi
 int spkv_prefill_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                       const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
                       int chunk_len, void* o, float* lse, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_prefill_attn");
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (chunk_start < 0 || chunk_len < 0) return SPKV_ERR_ARG;
   if (chunk_len == 0) return SPKV_OK;

@@ -15,6 +15,7 @@
 #include "../../include/spkv.h"
 #include "common.cuh"
 #include "launch.h"
+#include "trace.h"
 
 namespace {
 
@@ -59,6 +60,7 @@ extern "C" int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* 
                                         const spkv_ring* ring, const void* q,
                                         const int32_t* t_pos, void* o, float* lse,
                                         spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_attn_noalloc");
   if (!p || !c || !ring || !q || !t_pos || !o) return SPKV_ERR_ARG;
   if (!c->K_pool || !c->V_pool || !c->pos_pool || !c->page_table || !c->count || !c->err_flag ||
       c->page_rows != spkv::kPageRows || !ring->K_win || !ring->V_win || !ring->z_win)
