@@ -38,3 +38,16 @@ def test_committed_profile_key_is_well_formed():
                 keys[k] = v
     assert set(keys) == {"source_hash", "traffic_bytes_per_launch", "algorithmic_bytes_per_launch"}
     assert float(keys["traffic_bytes_per_launch"]) >= float(keys["algorithmic_bytes_per_launch"])
+
+
+def test_reference_arm_line(monkeypatch):
+    """--impl reference: rank 0 prints the oracle's line with the contract's keys; its
+    per-step sample is bounded (about 600 oracle units over all timed steps)."""
+    import argparse
+    args = argparse.Namespace(steps=1, warmup=3, cpu_units=1)
+    out = bench.run_reference(args, world=1, rank=0)
+    assert out["impl"] == "reference" and out["unit"] == "tokens/s" and out["value"] > 0
+    assert out["e2e"]["value"] == out["value"]
+    assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
+    assert out["cpu_baseline"]["kind"] == "oracle" and out["cpu_baseline"]["value"] == out["value"]
+    assert bench.run_reference(args, world=2, rank=1) is None  # other ranks: no work, no line
