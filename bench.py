@@ -157,24 +157,20 @@ def _kernel_source_hash() -> str:
 
 
 def _profiled_traffic(launch_bytes: float):
-    """DRAM bytes per decode launch from the committed ncu summary, if it was taken
-    on the current kernel source (else None).  The capture is one layer of the same
-    workload; its traffic is scaled to this launch by the algorithmic bytes."""
-    path = os.path.join(ROOT, "profiles", "decode_attn_decode32k.md")
+    """DRAM bytes per decode launch from the committed ncu capture's key file
+    (profiles/decode_attn_decode32k.json), if the capture was taken on the current
+    kernel source (else None).  The capture is one layer of the same workload; its
+    traffic is scaled to this launch by the algorithmic bytes."""
+    path = os.path.join(ROOT, "profiles", "decode_attn_decode32k.json")
     if not os.path.exists(path):
         return None
-    want = _kernel_source_hash()
-    vals = {}
     with open(path) as f:
-        for line in f:
-            if line.startswith("bench-key "):
-                k, _, v = line[len("bench-key "):].strip().partition("=")
-                vals[k.strip()] = v.strip()
-    if vals.get("source_hash") != want or "traffic_bytes_per_launch" not in vals:
+        key = json.load(f)
+    if key.get("source_hash") != _kernel_source_hash() or "traffic_bytes_per_launch" not in key:
         return None
-    traffic = float(vals["traffic_bytes_per_launch"])
-    if "algorithmic_bytes_per_launch" in vals:
-        traffic *= launch_bytes / float(vals["algorithmic_bytes_per_launch"])
+    traffic = float(key["traffic_bytes_per_launch"])
+    if key.get("algorithmic_bytes_per_launch"):
+        traffic *= launch_bytes / float(key["algorithmic_bytes_per_launch"])
     return traffic
 
 

@@ -290,18 +290,20 @@ int spkv_decode_attn_before_append_supported(const spkv_params* p);
  * owns all device memory through its own pool, a serving path that must not call
  * cudaMalloc after start-up, or a runtime with no allocator to borrow from.  This
  * entry point computes exactly what spkv_decode_attn computes (same arguments minus
- * the workspace, same kernels) but takes its scratch from a fixed array of
+ * the workspace, the same argument checks, same kernels; cache may be NULL for a
+ * window-only layer) but takes its scratch from a fixed array of
  * SPKV_NOALLOC_SCRATCH_BYTES inside the library.  It allocates and frees nothing.
  *
  * - Shapes whose scratch need (spkv_decode_workspace_bytes) exceeds the fixed size
  *   are rejected with SPKV_ERR_UNSUPPORTED before anything is enqueued.
- * - The first call on a device looks up the array's device address (set-up, once
- *   per device, with that device current); make that first call before any stream
- *   capture.
- * - Every call shares the one array: the counters it needs at zero are cleared on
- *   `stream` at the start of each call, but calls whose work overlaps on the device
- *   (other streams, concurrent graph branches) race on the scratch and must not be
- *   issued. */
+ * - The first call in a CUDA context (per device; again after a device reset, which
+ *   makes a new context) looks up the array's device address with that context
+ *   current; make that first call before any stream capture.
+ * - Every call shares the one array, whatever its shape: each call clears the counters
+ *   of its own shape at the start, on `stream` (one memset before the kernels, which
+ *   also keeps the first kernel from overlapping the previous kernel on the stream).
+ *   Calls whose work overlaps on the device (other streams, concurrent graph
+ *   branches) race on the scratch and must not be issued. */
 int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* cache,
                              const spkv_ring* ring, const void* q, const int32_t* t_pos,
                              void* o, float* lse, spkv_stream_t stream);

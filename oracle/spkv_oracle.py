@@ -139,11 +139,6 @@ def cache_rows(z_col: np.ndarray, upto: int) -> np.ndarray:
     return np.nonzero(z_col == 1)[0].astype(np.int32)
 
 
-def keep_fraction(z: np.ndarray) -> float:
-    """Fraction of gated-in keys (the density statistic of §3.2)."""
-    return float(np.mean(np.asarray(z, dtype=np.float64)))
-
-
 def rethreshold(cached_pos: np.ndarray, cached_u: np.ndarray, tau_new: float) -> np.ndarray:
     """Post-hoc threshold change (§3.3) applied to one key head's cache: of the cached
     positions (increasing) with their stored utilities, keep those with u >= tau_new,

@@ -4,68 +4,25 @@
 #include <math.h>
 #include <stdint.h>
 
-#include <mutex>
-
 #include "../../include/spkv.h"
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 #include "trace.h"
 
 namespace {
 
-using spkv::kPageRows;
+using spkv::aligned16;
+using spkv::cache_or_none;
+using spkv::params_ok;
+using spkv::ring_ok;
+using spkv::sm_count;
 
 int status_of(cudaError_t e) { return e == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA; }
 
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
-bool params_ok(const spkv_params* p) {
-  if (!p) return false;
-  if (p->B < 1 || p->Hkv < 1 || p->Hq < p->Hkv || p->Hq % p->Hkv) return false;
-  const int G = p->Hq / p->Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return false;
-  if (p->head_dim != 64 && p->head_dim != 128) return false;
-  if (p->window < 1 || p->window > 1024) return false;
-  if (p->dtype != SPKV_F32 && p->dtype != SPKV_BF16) return false;
-  if (!(p->tau == p->tau)) return false;  // NaN threshold
-  return true;
-}
-
 bool cache_ok(const spkv_params* p, const spkv_cache* c) {
-  if (!c) return false;
-  if (!c->K_pool || !c->V_pool || !c->pos_pool || !c->page_table || !c->count ||
-      !c->count_prev || !c->pool_top || !c->err_flag)
-    return false;
-  if (c->page_rows != kPageRows || c->num_pages < 1 || c->max_pages_per_head < 1) return false;
-  if (!aligned16(c->K_pool) || !aligned16(c->V_pool)) return false;
   (void)p;
-  return true;
-}
-
-bool ring_ok(const spkv_ring* r) {
-  return r && r->K_win && r->V_win && r->z_win && aligned16(r->K_win) && aligned16(r->V_win);
-}
-
-// A layer without a persistent cache (window-only, e.g. the local layers of a hybrid
-// local/global stack) passes cache == NULL; the kernels see an all-zero cache.
-const spkv_cache& cache_or_none(const spkv_cache* c) {
-  static const spkv_cache none = {};
-  return c ? *c : none;
-}
-
-int sm_count() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
-  static std::mutex mu;
-  static int cached[64] = {0};
-  std::lock_guard<std::mutex> lock(mu);
-  if (dev < 0 || dev >= 64) return -1;
-  if (cached[dev] == 0) {
-    int n = 0;
-    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return -1;
-    cached[dev] = n;
-  }
-  return cached[dev];
+  return spkv::cache_ok(c);
 }
 
 }  // namespace

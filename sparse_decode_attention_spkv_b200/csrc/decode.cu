@@ -29,6 +29,7 @@
 #include <math.h>
 
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 
 namespace spkv {
@@ -505,23 +506,24 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// Control words at the front of the CUDA-core kernel's workspace: per-head arrival
+// counters [n_heads], work counter, finished-CTA counter.
+size_t ctrl_bytes_simple(int n_heads) { return ((size_t)(n_heads + 2) * 4 + 255) / 256 * 256; }
+
 template <typename E, int D, int G>
 cudaError_t run(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
                 const int32_t* t_pos, void* o, float* lse, void* ws, int num_sms,
                 cudaStream_t stream) {
   using S = Smem<E, D, G>;
   const size_t smem = sizeof(S);
-  static bool configured = false;  // attribute set once per process (same for all devices)
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<E, D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem((const void*)decode_kernel<E, D, G>, (int)smem);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   const int n_heads = p.B * p.Hkv;
   char* w = static_cast<char*>(ws);
   int* ctrl = reinterpret_cast<int*>(w);
-  const size_t ctrl_bytes = ((size_t)(n_heads + 2) * 4 + 255) / 256 * 256;
+  const size_t ctrl_bytes = ctrl_bytes_simple(n_heads);
   const int grid = num_sms;
   const size_t max_chunks = (size_t)grid * kUnitsPerCta + n_heads;
   float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
@@ -552,10 +554,14 @@ cudaError_t dispatch_g(const spkv_params& p, const spkv_cache& c, const spkv_rin
 
 }  // namespace
 
+size_t decode_ctrl_bytes(const spkv_params& p) {
+  return decode_tc_supported(p) ? decode_tc_ctrl_bytes(p) : ctrl_bytes_simple(p.B * p.Hkv);
+}
+
 size_t decode_workspace_bytes(const spkv_params& p, int num_sms) {
   const int n_heads = p.B * p.Hkv;
   const int G = p.Hq / p.Hkv;
-  const size_t ctrl_bytes = ((size_t)(n_heads + 2) * 4 + 255) / 256 * 256;
+  const size_t ctrl_bytes = ctrl_bytes_simple(n_heads);
   const size_t max_chunks = (size_t)num_sms * kUnitsPerCta + n_heads;
   const size_t ml_bytes = (max_chunks * G * 2 * 4 + 255) / 256 * 256;
   const size_t o_bytes = max_chunks * G * p.head_dim * 4;

@@ -14,6 +14,7 @@
 
 #include "../../include/spkv.h"
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 #include "trace.h"
 
@@ -24,35 +25,38 @@ namespace {
 constexpr size_t kNoAllocScratchBytes = (size_t)SPKV_NOALLOC_SCRATCH_BYTES;
 __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 std::mutex g_mu;
-void* g_scratch_ptr[kMaxDevices] = {};
-int g_sms[kMaxDevices] = {};
+struct ScratchRef {
+  unsigned long long ctx;  // context the address belongs to (0: slot unused)
+  void* ptr;
+};
+ScratchRef g_scratch[kMaxContexts] = {};
 
-// Device address of the scratch on the current device; looked up once per device
-// (the array's host-side name is not a device address).
-cudaError_t scratch_for_current_device(void** ptr, int* sms) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
+// Device address of the scratch in the current context.  The array's host-side name is
+// not a device address; its address is looked up once per context (set-up of the first
+// call in that context) and kept with the context's identifier, so a context created
+// after a device reset (where the module is loaded anew) looks it up again.
+cudaError_t scratch_for_current_context(void** ptr) {
+  unsigned long long ctx = 0;
+  cudaError_t e = spkv::current_context_id(&ctx);
   if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_decode_scratch);
-    if (e != cudaSuccess) return e;
-    int n = 0;
-    e = cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-    g_sms[dev] = n;
-  }
-  *ptr = g_scratch_ptr[dev];
-  *sms = g_sms[dev];
+  for (const ScratchRef& r : g_scratch)
+    if (r.ctx == ctx) {
+      *ptr = r.ptr;
+      return cudaSuccess;
+    }
+  void* p = nullptr;
+  e = cudaGetSymbolAddress(&p, g_decode_scratch);
+  if (e != cudaSuccess) return e;
+  // remember it (a full table is reused from the front: a stale entry only costs a lookup)
+  static int next = 0;
+  g_scratch[next] = ScratchRef{ctx, p};
+  next = (next + 1) % kMaxContexts;
+  *ptr = p;
   return cudaSuccess;
 }
-
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 }  // namespace
 
@@ -61,29 +65,23 @@ extern "C" int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* 
                                         const int32_t* t_pos, void* o, float* lse,
                                         spkv_stream_t stream) {
   SPKV_TRACE("spkv_decode_attn_noalloc");
-  if (!p || !c || !ring || !q || !t_pos || !o) return SPKV_ERR_ARG;
-  if (!c->K_pool || !c->V_pool || !c->pos_pool || !c->page_table || !c->count || !c->err_flag ||
-      c->page_rows != spkv::kPageRows || !ring->K_win || !ring->V_win || !ring->z_win)
-    return SPKV_ERR_ARG;
-  if (!aligned16(q) || !aligned16(o) || !aligned16(c->K_pool) || !aligned16(c->V_pool) ||
-      !aligned16(ring->K_win) || !aligned16(ring->V_win))
-    return SPKV_ERR_ARG;
-  if (p->B < 1 || p->Hkv < 1 || p->Hq % p->Hkv || p->window < 1 || p->window > 1024 ||
-      (p->head_dim != 64 && p->head_dim != 128) || (p->dtype != SPKV_F32 && p->dtype != SPKV_BF16))
-    return SPKV_ERR_ARG;
-  const int G = p->Hq / p->Hkv;
-  if (G != 1 && G != 2 && G != 4 && G != 8) return SPKV_ERR_ARG;
+  // the same argument rules as spkv_decode_attn (cache NULL: a window-only layer)
+  if (!spkv::params_ok(p) || (c && !spkv::cache_ok(c)) || !spkv::ring_ok(ring)) return SPKV_ERR_ARG;
+  if (!q || !t_pos || !o || !spkv::aligned16(q) || !spkv::aligned16(o)) return SPKV_ERR_ARG;
   if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
-  void* scratch = nullptr;
-  int sms = 0;
-  if (scratch_for_current_device(&scratch, &sms) != cudaSuccess) return SPKV_ERR_CUDA;
+  const int sms = spkv::sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
   const size_t need = spkv::decode_workspace_bytes(*p, sms);
   if (need > kNoAllocScratchBytes) return SPKV_ERR_UNSUPPORTED;  // beyond the fixed scratch
-  // the arrival and work counters at the front of the scratch must start at zero
-  const size_t ctrl = (((size_t)p->B * p->Hkv + 2) * 4 + 255) / 256 * 256;
+  void* scratch = nullptr;
+  if (scratch_for_current_context(&scratch) != cudaSuccess) return SPKV_ERR_CUDA;
+  // The array is shared by calls of every shape, and the counters a call needs at zero
+  // sit at shape-dependent offsets that another shape's call may have filled with plan
+  // words (or that an aborted call left set): clear the control region of the kernel
+  // that will run, on the stream, before it.
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (cudaMemsetAsync(scratch, 0, ctrl, s) != cudaSuccess) return SPKV_ERR_CUDA;
-  const cudaError_t e =
-      spkv::launch_decode(*p, *c, *ring, q, t_pos, o, lse, scratch, kNoAllocScratchBytes, sms, s);
+  if (cudaMemsetAsync(scratch, 0, spkv::decode_ctrl_bytes(*p), s) != cudaSuccess) return SPKV_ERR_CUDA;
+  const cudaError_t e = spkv::launch_decode(*p, spkv::cache_or_none(c), *ring, q, t_pos, o, lse,
+                                            scratch, kNoAllocScratchBytes, sms, s);
   return e == cudaSuccess ? SPKV_OK : SPKV_ERR_CUDA;
 }

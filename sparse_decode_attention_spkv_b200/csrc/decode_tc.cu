@@ -45,6 +45,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 
 namespace spkv {
@@ -754,12 +755,9 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
                    void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
   using S = TcDecSmem<D, G>;
   const size_t smem = sizeof(S) + 1024 + ((size_t)5 * p.B * p.Hkv + 1) * 4;
-  static int configured = 0;
-  if ((int)smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<D, G>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem((const void*)decode_tc_kernel<D, G>, (int)smem);
     if (e != cudaSuccess) return e;
-    configured = (int)smem;
   }
   const cuuint64_t es = 2;
   CUtensorMap tkp, tvp, tkr, tvr;
@@ -821,6 +819,8 @@ bool decode_tc_supported(const spkv_params& p) {
   return p.dtype == SPKV_BF16 && (p.head_dim == 64 || p.head_dim == 128) &&
          p.window % kTileR == 0 && p.B * p.Hkv <= kMaxHeadsT && encode_fn_t() != nullptr;
 }
+
+size_t decode_tc_ctrl_bytes(const spkv_params& p) { return ctrl_bytes_tc(p.B * p.Hkv); }
 
 size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms) {
   const int n_heads = p.B * p.Hkv;

@@ -45,6 +45,10 @@ cudaError_t launch_score_tc(const spkv_params& p, const void* h, int n_tok, cons
                             uint8_t* z_out, cudaStream_t stream);
 
 size_t decode_workspace_bytes(const spkv_params& p, int num_sms);
+// Bytes of counters at the front of the decode workspace, for the kernel launch_decode
+// picks for these parameters (the rest of the workspace needs no initialisation).
+size_t decode_ctrl_bytes(const spkv_params& p);
+size_t decode_tc_ctrl_bytes(const spkv_params& p);
 bool decode_tc_supported(const spkv_params& p);
 size_t decode_tc_workspace_bytes(const spkv_params& p, int num_sms);
 // k_new / v_new given: before-append mode (the ring holds rows t-w .. t-1, the new row

@@ -40,6 +40,7 @@
 #include <mutex>
 
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 #include "tc.cuh"
 
@@ -421,14 +422,7 @@ constexpr size_t kSmem = sizeof(TcSmem) + 1024;  // + alignment slack
 
 template <bool SOFT>
 cudaError_t configure() {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t err = cudaFuncSetAttribute(prefill_tc_kernel<SOFT>,
-                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmem);
-    if (err != cudaSuccess) return err;
-    configured = true;
-  }
-  return cudaSuccess;
+  return ensure_dynamic_smem((const void*)prefill_tc_kernel<SOFT>, (int)kSmem);
 }
 
 }  // namespace

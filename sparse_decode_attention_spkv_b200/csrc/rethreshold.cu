@@ -19,6 +19,7 @@
 //           pending utilities; the work counter is cleared.
 #include "append.cuh"
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 
 namespace spkv {
@@ -257,12 +258,9 @@ cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const 
   RethrWs ws = carve(workspace, n_heads, c.max_pages_per_head);
   rethr_plan<<<n_heads, kPlanThreads, 0, stream>>>(m, ws, tau_new);
   const size_t smem = (size_t)2 * kPageRows * row_bytes + (size_t)(n_heads + 1) * 4;
-  static int configured = 0;
-  if ((int)smem > configured) {
-    cudaError_t e = cudaFuncSetAttribute(rethr_move, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem((const void*)rethr_move, (int)smem);
     if (e != cudaSuccess) return e;
-    configured = (int)smem;
   }
   // as many CTAs per SM as shared memory allows (each streams one page at a time)
   int per_sm = (int)((216u << 10) / (smem + (2u << 10)));

@@ -11,6 +11,7 @@
 
 #include "append.cuh"
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 
 namespace cg = cooperative_groups;
@@ -305,12 +306,9 @@ cudaError_t launch_small(const spkv_params& p, const void* h, int n_tok, const v
   using T = typename E::T;
   const int units = (p.hid + kSmallRanks - 1) / kSmallRanks;
   const size_t smem = (size_t)NT * p.d_model * E::kSize + (size_t)units * NT * 4;
-  static int configured_smem = 0;
-  if ((int)smem > configured_smem) {
-    cudaError_t e = cudaFuncSetAttribute(score_small_kernel<E, NT, MODE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  {
+    cudaError_t e = ensure_dynamic_smem((const void*)score_small_kernel<E, NT, MODE>, (int)smem);
     if (e != cudaSuccess) return e;
-    configured_smem = (int)smem;
   }
   const int groups = (n_tok + NT - 1) / NT;
   return launch_pdl(score_small_kernel<E, NT, MODE>, dim3(groups * kSmallRanks),

@@ -19,6 +19,7 @@
 #include <cooperative_groups.h>
 
 #include "common.cuh"
+#include "host.h"
 #include "launch.h"
 #include "tc.cuh"
 
@@ -200,12 +201,9 @@ bool score_tc_supported(const spkv_params& p, int n_tok) {
 cudaError_t launch_score_tc(const spkv_params& p, const void* h, int n_tok, const void* W1,
                             const float* b1, const float* W2, const float* b2, float* u_out,
                             uint8_t* z_out, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(score_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kScoreTcSmem);
+  {
+    cudaError_t e = ensure_dynamic_smem((const void*)score_tc_kernel, (int)kScoreTcSmem);
     if (e != cudaSuccess) return e;
-    configured = true;
   }
   CUtensorMap th, tw;
   {

@@ -289,11 +289,13 @@ def spkv_prefill_attn(p, cache: Optional[Cache], ring: Ring, q, K_chunk, V_chunk
         _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _stream(stream)))
 
 
-def spkv_decode_attn_noalloc(p, cache: Cache, ring: Ring, q, t_pos, o, lse, stream=None):
+def spkv_decode_attn_noalloc(p, cache: Optional[Cache], ring: Ring, q, t_pos, o, lse,
+                             stream=None):
     """spkv_decode_attn for callers that cannot allocate a workspace: the scratch is a
-    fixed array inside the library (see include/spkv.h)."""
+    fixed array inside the library (see include/spkv.h).  cache None: a window-only
+    layer."""
     return _check("spkv_decode_attn_noalloc", lib.spkv_decode_attn_noalloc(
-        ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
+        ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(t_pos), _ptr(o),
         _ptr(lse), _stream(stream)))
 
 

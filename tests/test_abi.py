@@ -107,3 +107,28 @@ def test_argument_validation_without_gpu():
                                                 ctypes.byref(ring), 16, 16, 16, 16, 16, None,
                                                 16, 1 << 20, S.DECODE_STATE_SETTLED,
                                                 None) == S.ERR_UNSUPPORTED
+
+
+def test_noalloc_argument_checks_match_decode_attn():
+    """The no-allocation decode applies spkv_decode_attn's argument rules (host side,
+    before anything is enqueued): the same bad calls give the same status."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    good = S.make_params(2, 8, 2, 128, 256, 64, 128, 0.5, S.BF16)
+    nan_tau = S.make_params(2, 8, 2, 128, 256, 64, 128, float("nan"), S.BF16)
+    ring = S.spkv_ring(16, 16, 16, None)
+    ok_cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
+    bad_caches = [S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 0, 64, 4),   # no pages
+                  S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 0),   # no table
+                  S.spkv_cache(16, 16, 16, 16, 16, None, 16, 16, None, 4, 64, 4),  # count_prev
+                  S.spkv_cache(16, 16, 16, 16, 16, 16, None, 16, None, 4, 64, 4)]  # pool_top
+    calls = [(good, c, ring, 16, 16, 16) for c in bad_caches]
+    calls += [(nan_tau, ok_cache, ring, 16, 16, 16),     # NaN threshold
+              (good, ok_cache, ring, 8, 16, 16),         # misaligned query
+              (good, ok_cache, ring, 16, None, 16),      # no positions
+              (good, ok_cache, S.spkv_ring(16, 16, None, None), 16, 16, 16)]  # no gates
+    for p, c, r, q, t, o in calls:
+        a = S.lib.spkv_decode_attn(ctypes.byref(p), ctypes.byref(c), ctypes.byref(r), q, t, o, None,
+                                   16, 1 << 30, None)
+        b = S.lib.spkv_decode_attn_noalloc(ctypes.byref(p), ctypes.byref(c), ctypes.byref(r), q, t,
+                                           o, None, None)
+        assert a == b == S.ERR_ARG, (a, b)

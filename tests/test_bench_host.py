@@ -1,5 +1,6 @@
 """Host-side logic of bench.py (no GPU): the profile key that ties a committed ncu
 capture to the kernel code it was taken on, and the scaling of its traffic."""
+import json
 import os
 
 import bench
@@ -18,9 +19,9 @@ def test_code_hash_ignores_comments_and_blank_lines(tmp_path):
 def test_profiled_traffic_scales_with_the_launch(monkeypatch, tmp_path):
     prof = tmp_path / "profiles"
     prof.mkdir()
-    (prof / "decode_attn_decode32k.md").write_text(
-        "text\nbench-key source_hash=abc\nbench-key traffic_bytes_per_launch=1020\n"
-        "bench-key algorithmic_bytes_per_launch=1000\n")
+    (prof / "decode_attn_decode32k.json").write_text(json.dumps(
+        {"source_hash": "abc", "traffic_bytes_per_launch": 1020,
+         "algorithmic_bytes_per_launch": 1000}))
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     monkeypatch.setattr(bench, "_kernel_source_hash", lambda: "abc")
     assert abs(bench._profiled_traffic(2000.0) - 2040.0) < 1e-9
@@ -29,15 +30,10 @@ def test_profiled_traffic_scales_with_the_launch(monkeypatch, tmp_path):
 
 
 def test_committed_profile_key_is_well_formed():
-    path = os.path.join(bench.ROOT, "profiles", "decode_attn_decode32k.md")
-    keys = {}
-    with open(path) as f:
-        for line in f:
-            if line.startswith("bench-key "):
-                k, _, v = line[len("bench-key "):].strip().partition("=")
-                keys[k] = v
-    assert set(keys) == {"source_hash", "traffic_bytes_per_launch", "algorithmic_bytes_per_launch"}
-    assert float(keys["traffic_bytes_per_launch"]) >= float(keys["algorithmic_bytes_per_launch"])
+    with open(os.path.join(bench.ROOT, "profiles", "decode_attn_decode32k.json")) as f:
+        key = json.load(f)
+    assert {"source_hash", "traffic_bytes_per_launch", "algorithmic_bytes_per_launch"} <= set(key)
+    assert float(key["traffic_bytes_per_launch"]) >= float(key["algorithmic_bytes_per_launch"])
 
 
 def test_reference_arm_line(monkeypatch):
