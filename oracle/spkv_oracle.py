@@ -25,6 +25,9 @@ Learning When to Write by Predicting Future Utility" (arXiv 2605.14037):
 * ``soft_mask``        Eq. (6): additive score 0 inside the causal window,
                        c (alpha_s - 1) outside it (and -inf for s > t: causal).
 * ``soft_gated_attention``  Eq. (3) with the mask of Eq. (6), every key s <= t.
+* ``merge``            Eq. (3) over a key set split into disjoint slices: the
+                       softmax factorises, so the slices' outputs combine by their
+                       log-sum-exp weights (a sequence decoded slice by slice).
 
 Readings where the page is silent (each listed in the design notes):
 * f is one perceptron per layer, d_model -> hid -> Hkv, with a GELU (exact erf
@@ -137,6 +140,26 @@ def cache_rows(z_col: np.ndarray, upto: int) -> np.ndarray:
     s < upto whose gate is 1, in increasing order (its "index list")."""
     z_col = np.asarray(z_col, dtype=np.uint8)[:upto]
     return np.nonzero(z_col == 1)[0].astype(np.int32)
+
+
+def merge(o_parts, lse_parts):
+    """Eq. (3) over the disjoint union of slices S_1..S_n of a key set: with o_i the
+    attention output over S_i alone and lse_i = log sum_{s in S_i} e^{x_s},
+    lse = log sum_i e^{lse_i} and o = sum_i e^{lse_i - lse} o_i.
+
+    o_parts [n][..][d], lse_parts [n][..]; slices without keys (lse = -inf) count for
+    nothing; if all are empty, o = 0 and lse = -inf.  Returns (o, lse)."""
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    m = np.max(lse_parts, axis=0)
+    finite = np.isfinite(m)
+    m_safe = np.where(finite, m, 0.0)
+    wgt = np.where(np.isfinite(lse_parts), np.exp(lse_parts - m_safe), 0.0)
+    total = np.sum(wgt, axis=0)
+    lse = np.where(finite, m_safe + np.log(np.where(finite, total, 1.0)), -np.inf)
+    scale = np.where(finite, 1.0 / np.where(finite, total, 1.0), 0.0)
+    o = np.einsum("n...,n...d->...d", wgt * scale, o_parts)
+    return o, lse
 
 
 def rethreshold(cached_pos: np.ndarray, cached_u: np.ndarray, tau_new: float) -> np.ndarray:

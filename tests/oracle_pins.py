@@ -335,11 +335,47 @@ def pin_permutation_invariance():
         _close(np.array([l1]), np.array([l2]), 1e-12, "permuted keys: lse")
 
 
+def pin_merge_of_slices():
+    """Eq. (3) over a key set split into disjoint slices: merging the attention of each
+    slice alone (``merge``) gives the attention over the union (``attend`` on the whole
+    set), output and lse, for random splits into 1-4 slices, empty slices included; a
+    hand example with two one-key slices gives the two-key softmax."""
+    rng = np.random.default_rng(31)
+    for _ in range(100):
+        T, d = int(rng.integers(1, 50)), 8
+        q = rng.standard_normal(d) * 2.0
+        K = rng.standard_normal((T, d))
+        V = rng.standard_normal((T, d))
+        mask = rng.random(T) < 0.7
+        mask[int(rng.integers(T))] = True
+        n = int(rng.integers(1, 5))
+        part = rng.integers(0, n + 1, size=T)  # slice n never used when drawn: an extra empty one
+        o_full, l_full = O.attend(q, K, V, mask)
+        os_, ls_ = [], []
+        for i in range(n + 1):
+            sub = mask & (part == i)
+            if sub.any():
+                o_i, l_i = O.attend(q, K, V, sub)
+            else:
+                o_i, l_i = np.zeros(d), -np.inf
+            os_.append(o_i)
+            ls_.append(l_i)
+        o_m, l_m = O.merge(np.stack(os_), np.array(ls_))
+        _close(o_m, o_full, 1e-12, "merged slices: output")
+        _close(np.array([l_m]), np.array([l_full]), 1e-12, "merged slices: lse")
+    # two one-key slices: weights e^{x1} : e^{x2}
+    o_m, l_m = O.merge(np.array([[1.0, 0.0], [0.0, 1.0]]), np.array([0.0, math.log(3.0)]))
+    _close(o_m, np.array([0.25, 0.75]), 1e-15, "two one-key slices")
+    _close(np.array([l_m]), np.array([math.log(4.0)]), 1e-15, "two one-key slices: lse")
+    o_m, l_m = O.merge(np.zeros((2, 3)), np.array([-np.inf, -np.inf]))
+    assert np.all(o_m == 0.0) and l_m == -np.inf, "all slices empty"
+
+
 ALL_PINS = [
     pin_gelu_textbook, pin_gelu_library, pin_utility_zero_weights, pin_utility_hand_example,
     pin_utility_library, pin_gate_threshold, pin_gate_extremes, pin_keysets_golden,
     pin_two_key_softmax, pin_tau0_is_causal, pin_tau_gt1_is_sliding_window,
     pin_wide_window_is_causal, pin_dense_brute_force, pin_cache_rows, pin_rethreshold,
     pin_soft_gate_values, pin_soft_two_key_closed_form, pin_soft_special_cases,
-    pin_permutation_invariance,
+    pin_permutation_invariance, pin_merge_of_slices,
 ]

@@ -116,8 +116,23 @@ def _soft_gate_no_beta(u, tau, beta):
     return O.sigmoid(np.asarray(u, dtype=np.float64) - float(tau))
 
 
+def _merge_unweighted(o_parts, lse_parts):
+    o_parts = np.asarray(o_parts, dtype=np.float64)
+    lse_parts = np.asarray(lse_parts, dtype=np.float64)
+    live = np.isfinite(lse_parts)
+    o = np.sum(o_parts * live[..., None], axis=0) / np.maximum(np.sum(live, axis=0), 1)[..., None]
+    m = np.max(lse_parts, axis=0)
+    return o, np.where(np.isfinite(m), np.log(np.sum(np.exp(lse_parts), axis=0)), -np.inf)
+
+
+def _merge_lse_is_max(o_parts, lse_parts):
+    o, _ = _ORIG_MERGE(o_parts, lse_parts)
+    return o, np.max(np.asarray(lse_parts, dtype=np.float64), axis=0)
+
+
 _ORIG_ATTEND = O.attend
 _ORIG_LOGITS = O.utility_logits
+_ORIG_MERGE = O.merge
 
 MUTANTS = {
     "gelu_tanh_approximation": ("gelu", _gelu_tanh),
@@ -140,6 +155,8 @@ MUTANTS = {
     "soft_window_off_by_one": ("soft_mask", _soft_mask_window_off_by_one),
     "soft_bias_sign": ("soft_mask", _soft_mask_sign),
     "soft_not_causal": ("soft_mask", _soft_mask_acausal),
+    "merge_unweighted_mean": ("merge", _merge_unweighted),
+    "merge_lse_is_the_max": ("merge", _merge_lse_is_max),
 }
 
 
