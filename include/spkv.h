@@ -278,6 +278,50 @@ int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* cache
  * 128, window a multiple of 64), else 0.  Host only; enqueues nothing. */
 int spkv_decode_attn_before_append_supported(const spkv_params* p);
 
+/* Sequence split (decode over slices of one sequence's keys, combined afterwards).
+ *
+ * A sequence whose gated cache is spread over several caches (for instance over
+ * several GPUs: each holds the cache rows of a range of positions, one of them also
+ * the window) is decoded slice by slice and the slices' partials are combined.  The
+ * combination rests on Eq. (3) ("Self-Pruned Key-Value Attention", §2.1): the softmax
+ * over a disjoint union of key sets S_1..S_n factorises, so with o_i the attention
+ * output over S_i alone and lse_i the log of its sum of exponentials,
+ *   lse = log sum_i e^{lse_i},  o = sum_i e^{lse_i - lse} o_i
+ * is the attention over the whole set (the log-sum-exp merge that also combines the
+ * split-K chunks of one decode call). */
+
+/* flags of spkv_decode_attn_partial */
+#define SPKV_SLICE_WINDOW 1u /* this slice holds the window: the ring is read */
+
+/* a4 over one slice: for query t = t_pos[b] (as in spkv_decode_attn, after the step's
+ * update), the keys of this slice are the cache rows with position <= t - window and,
+ * with SPKV_SLICE_WINDOW, the window slots holding positions max(0, t-window+1)..t.
+ * Outputs (fp32): o_part [B][Hq][head_dim], the attention output over the slice's keys
+ * alone, and lse_part [B][Hq], the natural log of the slice's sum of exponentials of
+ * the scaled logits; a head with no key in the slice gets o_part = 0, lse_part = -inf.
+ * cache may be NULL for a slice that holds only the window; without SPKV_SLICE_WINDOW
+ * the cache is required and ring is ignored (may be NULL).  Each cache must hold
+ * distinct positions (the slices are disjoint), each in increasing order.  q
+ * [B][Hq][head_dim] dtype; workspace as for spkv_decode_attn
+ * (spkv_decode_workspace_bytes; calls sharing a workspace must not overlap).  Returns
+ * SPKV_ERR_UNSUPPORTED where spkv_decode_attn_partial_supported says 0. */
+int spkv_decode_attn_partial(const spkv_params* p, const spkv_cache* cache,
+                             const spkv_ring* ring, const void* q, const int32_t* t_pos,
+                             unsigned flags, float* o_part, float* lse_part, void* workspace,
+                             size_t ws_bytes, spkv_stream_t stream);
+
+/* 1 if spkv_decode_attn_partial runs for these parameters (bf16, head_dim 64 or 128,
+ * window a multiple of 64), else 0.  Host only. */
+int spkv_decode_attn_partial_supported(const spkv_params* p);
+
+/* a5 across slices: combine n_parts >= 1 slice partials of the same queries.
+ * o_parts [n_parts][B][Hq][head_dim] f32 and lse_parts [n_parts][B][Hq] f32 (as
+ * spkv_decode_attn_partial writes them; parts in any order) -> o [B][Hq][head_dim]
+ * dtype and lse [B][Hq] f32 natural log (may be NULL).  Parts with lse = -inf count
+ * for nothing; if every part is empty, o = 0 and lse = -inf. */
+int spkv_decode_merge(const spkv_params* p, int n_parts, const float* o_parts,
+                      const float* lse_parts, void* o, float* lse, spkv_stream_t stream);
+
 /* Size of the fixed device scratch used by spkv_decode_attn_noalloc (8 MiB).  Every
  * GPU on which the library is loaded keeps this much memory until the process exits. */
 #define SPKV_NOALLOC_SCRATCH_BYTES (8u << 20)

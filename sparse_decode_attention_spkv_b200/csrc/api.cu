@@ -214,6 +214,42 @@ int spkv_decode_attn_before_append(const spkv_params* p, const spkv_cache* c,
                                           (flags & SPKV_DECODE_STATE_SETTLED) != 0));
 }
 
+int spkv_decode_attn_partial(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
+                             const void* q, const int32_t* t_pos, unsigned flags, float* o_part,
+                             float* lse_part, void* workspace, size_t ws_bytes,
+                             spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_attn_partial");
+  if (!params_ok(p) || (flags & ~SPKV_SLICE_WINDOW)) return SPKV_ERR_ARG;
+  const bool window_on = (flags & SPKV_SLICE_WINDOW) != 0;
+  if (c && !cache_ok(p, c)) return SPKV_ERR_ARG;
+  if (window_on ? !ring_ok(ring) : !c) return SPKV_ERR_ARG;  // a slice holds something
+  if (!q || !t_pos || !o_part || !lse_part || !workspace) return SPKV_ERR_ARG;
+  if (!aligned16(q) || !aligned16(o_part)) return SPKV_ERR_ARG;
+  if ((size_t)p->B * p->Hkv > 2048) return SPKV_ERR_UNSUPPORTED;
+  if (!spkv::decode_tc_supported(*p)) return SPKV_ERR_UNSUPPORTED;
+  const int sms = sm_count();
+  if (sms <= 0) return SPKV_ERR_CUDA;
+  if (ws_bytes < spkv::decode_workspace_bytes(*p, sms)) return SPKV_ERR_ARG;
+  static const spkv_ring no_ring = {};
+  return status_of(spkv::launch_decode_partial(*p, cache_or_none(c), window_on ? *ring : no_ring,
+                                               q, t_pos, window_on, o_part, lse_part, workspace,
+                                               sms, static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_decode_attn_partial_supported(const spkv_params* p) {
+  return params_ok(p) && spkv::decode_tc_supported(*p) ? 1 : 0;
+}
+
+int spkv_decode_merge(const spkv_params* p, int n_parts, const float* o_parts,
+                      const float* lse_parts, void* o, float* lse, spkv_stream_t stream) {
+  SPKV_TRACE("spkv_decode_merge");
+  if (!params_ok(p) || n_parts < 1) return SPKV_ERR_ARG;
+  if (!o_parts || !lse_parts || !o) return SPKV_ERR_ARG;
+  if (!aligned16(o_parts) || !aligned16(o)) return SPKV_ERR_ARG;
+  return status_of(spkv::launch_decode_merge_parts(*p, n_parts, o_parts, lse_parts, o, lse,
+                                                   static_cast<cudaStream_t>(stream)));
+}
+
 size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* c) {
   if (!params_ok(p) || !cache_ok(p, c)) return 0;
   return spkv::rethreshold_workspace_bytes(*p, *c);

@@ -43,6 +43,7 @@
 #include <math.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "host.h"
@@ -214,20 +215,22 @@ __device__ __forceinline__ void fetch_pages(int (&pg)[kPgRegs], const ChunkDesc&
   }
 }
 
-template <int D, int G>
+template <int D, int G, bool F32OUT>
 __global__ void __launch_bounds__(kThreadsT, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tm_kp,
                      const __grid_constant__ CUtensorMap tm_vp,
                      const __grid_constant__ CUtensorMap tm_kr,
                      const __grid_constant__ CUtensorMap tm_vr, CacheView cache,
                      const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ t_pos,
-                     __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
+                     void* __restrict__ out_, float* __restrict__ lse_out,
                      int* __restrict__ ws_ctrl, float* __restrict__ ws_ml,
                      float* __restrict__ ws_o, int n_heads, int hkv, int window,
                      uint32_t* err, const __nv_bfloat16* __restrict__ k_new,
                      const __nv_bfloat16* __restrict__ v_new, const uint8_t* __restrict__ z_win,
-                     int early_plan) {
+                     int early_plan, int win_on) {
   using TB = TileBuf<D>;
+  using OutT = typename std::conditional<F32OUT, float, __nv_bfloat16>::type;
+  OutT* __restrict__ out = static_cast<OutT*>(out_);
   using S = TcDecSmem<D, G>;
   constexpr int NT_D = D / 8;     // n-tiles of 8 along head_dim
   constexpr int KS_D = D / 16;    // k-steps of 16 along head_dim
@@ -265,7 +268,7 @@ __global__ void __launch_bounds__(kThreadsT, 1)
     int nl, nw, hide = -1;
     if (!pre) {
       nl = cache_live_rows(cache, bh, t - window, window);
-      nw = t + 1 < window ? t + 1 : window;
+      nw = !win_on ? 0 : t + 1 < window ? t + 1 : window;
     } else {  // ring rows t-w .. t-1; row t - w (slot t mod w) counts if its gate is 1
       nl = cache_live_rows(cache, bh, t - window - 1, window + 1);
       nw = t < window ? t : window;
@@ -273,7 +276,11 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         hide = t % window;
     }
     int rows = ((nl + kTileR - 1) / kTileR) * kTileR + nw;
-    if (pre && rows == 0) rows = 1;  // one empty tile: its chunk carries the new row
+    // a head with no key here (before-append mode at t = 0, or a slice of a split
+    // sequence without rows for it) gets one empty tile: nothing is loaded or computed
+    // for it, and its chunk carries the new row or writes the empty partial (o = 0,
+    // lse = -inf)
+    if (rows == 0) rows = 1;
     s_live[bh] = nl;
     s_nw[bh] = nw;
     s_hide[bh] = hide;
@@ -386,10 +393,16 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           // the tile description must be in place before the phase can complete
           sm.info[s] = TileRef{cd.c, cd.bh, valid, k == cd.k1 - 1, qslot, hide};
           const bool first = k == cd.k0;
-          mbar_arrive_expect_tx(&sm.full[s], 2 * TB::kBytes + (first ? G * D * 2 : 0));
+          const uint32_t tx = (valid > 0 ? 2 * TB::kBytes : 0) + (first ? G * D * 2 : 0);
+          if (tx)
+            mbar_arrive_expect_tx(&sm.full[s], tx);
+          else
+            mbar_arrive(&sm.full[s]);
           if (first)
             bulk_g2s(sm.qbuf[qslot], q + (size_t)cd.bh * G * D, G * D * 2, &sm.full[s]);
-          if (from_cache) {
+          if (valid == 0) {
+            // the empty tile of a head without keys: nothing to load
+          } else if (from_cache) {
             const int page = sm.pages[(k - cd.k0) % kChunkPages];
 #pragma unroll
             for (int hf = 0; hf < TB::kHalves; ++hf) {
@@ -492,10 +505,15 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           }
           if (nch == 1) {
             const float inv = L > 0.f ? 1.f / L : 0.f;
-            uint2 pk;
-            pk.x = pack2(O.x * inv, O.y * inv);
-            pk.y = pack2(O.z * inv, O.w * inv);
-            *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+            if constexpr (F32OUT) {
+              *reinterpret_cast<float4*>(out + (hrow + g) * D + d) =
+                  make_float4(O.x * inv, O.y * inv, O.z * inv, O.w * inv);
+            } else {
+              uint2 pk;
+              pk.x = pack2(O.x * inv, O.y * inv);
+              pk.y = pack2(O.z * inv, O.w * inv);
+              *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+            }
           } else {
             *reinterpret_cast<float4*>(ws_o + ((size_t)c * G + g) * D + d) = O;
           }
@@ -545,59 +563,61 @@ __global__ void __launch_bounds__(kThreadsT, 1)
         m_run = -INFINITY;
         l_run = 0.f;
       }
-      const TB& tb = sm.st[s];
-      const uint32_t kbase = smem_u32(tb.k[0]);
-      const uint32_t vbase = smem_u32(tb.v[0]);
+      if (ti.valid > 0) {  // (an empty tile holds no data: nothing to compute)
+        const TB& tb = sm.st[s];
+        const uint32_t kbase = smem_u32(tb.k[0]);
+        const uint32_t vbase = smem_u32(tb.v[0]);
 
-      // S = Q K^T for keys row0 .. row0+15 (two n-tiles of 8)
-      float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
+        // S = Q K^T for keys row0 .. row0+15 (two n-tiles of 8)
+        float sa[4] = {0.f, 0.f, 0.f, 0.f}, sb[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int k = 0; k < KS_D; ++k) {
-        const int key = row0 + 8 * (mtx >> 1) + (lane & 7);
-        const int c16 = 2 * k + (mtx & 1);  // 16-byte chunk along d
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(kbase + (c16 >> 3) * TB::kHalfBytes + swz(key, c16 & 7), b0, b1, b2, b3);
-        mma16816(sa, qa[k][0], 0u, qa[k][1], 0u, b0, b1);
-        mma16816(sb, qa[k][0], 0u, qa[k][1], 0u, b2, b3);
-      }
-      float x[4];
-      const int r0 = row0 + qcol;
-      x[0] = r0 < ti.valid && r0 != ti.hide ? sa[0] * sc : -INFINITY;
-      x[1] = r0 + 1 < ti.valid && r0 + 1 != ti.hide ? sa[1] * sc : -INFINITY;
-      x[2] = r0 + 8 < ti.valid && r0 + 8 != ti.hide ? sb[0] * sc : -INFINITY;
-      x[3] = r0 + 9 < ti.valid && r0 + 9 != ti.hide ? sb[1] * sc : -INFINITY;
-      float rmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
-      rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
-      const bool need = rmax > m_run + kSlackT;
-      if (__any_sync(0xffffffffu, need)) {
-        const float mnew = need ? rmax : m_run;
-        const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
-#pragma unroll
-        for (int n = 0; n < NT_D; ++n) {
-          o[n][0] *= alpha;
-          o[n][1] *= alpha;
+        for (int k = 0; k < KS_D; ++k) {
+          const int key = row0 + 8 * (mtx >> 1) + (lane & 7);
+          const int c16 = 2 * k + (mtx & 1);  // 16-byte chunk along d
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4(kbase + (c16 >> 3) * TB::kHalfBytes + swz(key, c16 & 7), b0, b1, b2, b3);
+          mma16816(sa, qa[k][0], 0u, qa[k][1], 0u, b0, b1);
+          mma16816(sb, qa[k][0], 0u, qa[k][1], 0u, b2, b3);
         }
-        l_run *= alpha;
-        m_run = mnew;
-      }
-      float p[4];
+        float x[4];
+        const int r0 = row0 + qcol;
+        x[0] = r0 < ti.valid && r0 != ti.hide ? sa[0] * sc : -INFINITY;
+        x[1] = r0 + 1 < ti.valid && r0 + 1 != ti.hide ? sa[1] * sc : -INFINITY;
+        x[2] = r0 + 8 < ti.valid && r0 + 8 != ti.hide ? sb[0] * sc : -INFINITY;
+        x[3] = r0 + 9 < ti.valid && r0 + 9 != ti.hide ? sb[1] * sc : -INFINITY;
+        float rmax = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+        rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 1));
+        rmax = fmaxf(rmax, __shfl_xor_sync(0xffffffffu, rmax, 2));
+        const bool need = rmax > m_run + kSlackT;
+        if (__any_sync(0xffffffffu, need)) {
+          const float mnew = need ? rmax : m_run;
+          const float alpha = (m_run == -INFINITY) ? 0.f : exp2f(m_run - mnew);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        p[i] = x[i] == -INFINITY ? 0.f : exp2f(x[i] - m_run);
-        l_run += p[i];
-      }
-      // O += P V over the 16 keys
-      const uint32_t a0 = pack2(p[0], p[1]);
-      const uint32_t a2 = pack2(p[2], p[3]);
+          for (int n = 0; n < NT_D; ++n) {
+            o[n][0] *= alpha;
+            o[n][1] *= alpha;
+          }
+          l_run *= alpha;
+          m_run = mnew;
+        }
+        float p[4];
 #pragma unroll
-      for (int dnp = 0; dnp < NT_D / 2; ++dnp) {
-        const int key = row0 + 8 * (mtx & 1) + (lane & 7);
-        const int c16 = 2 * dnp + (mtx >> 1);
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(vbase + (c16 >> 3) * TB::kHalfBytes + swz(key, c16 & 7), b0, b1, b2, b3);
-        mma16816(o[2 * dnp], a0, 0u, a2, 0u, b0, b1);
-        mma16816(o[2 * dnp + 1], a0, 0u, a2, 0u, b2, b3);
+        for (int i = 0; i < 4; ++i) {
+          p[i] = x[i] == -INFINITY ? 0.f : exp2f(x[i] - m_run);
+          l_run += p[i];
+        }
+        // O += P V over the 16 keys
+        const uint32_t a0 = pack2(p[0], p[1]);
+        const uint32_t a2 = pack2(p[2], p[3]);
+#pragma unroll
+        for (int dnp = 0; dnp < NT_D / 2; ++dnp) {
+          const int key = row0 + 8 * (mtx & 1) + (lane & 7);
+          const int c16 = 2 * dnp + (mtx >> 1);
+          uint32_t b0, b1, b2, b3;
+          ldsm_x4_t(vbase + (c16 >> 3) * TB::kHalfBytes + swz(key, c16 & 7), b0, b1, b2, b3);
+          mma16816(o[2 * dnp], a0, 0u, a2, 0u, b0, b1);
+          mma16816(o[2 * dnp + 1], a0, 0u, a2, 0u, b2, b3);
+        }
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(&sm.empty[s]);
@@ -648,11 +668,13 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 // a programmatic dependent of the decode kernel: it waits for the decode grid to
 // complete before reading anything.  It also clears the work counter for the next
 // decode launch.
-template <int D, int G>
+template <int D, int G, bool F32OUT>
 __global__ void __launch_bounds__(kMergeThreads)
     decode_merge_kernel(int* __restrict__ ws_ctrl, const float* __restrict__ ws_ml,
-                        const float* __restrict__ ws_o, __nv_bfloat16* __restrict__ out,
+                        const float* __restrict__ ws_o, void* __restrict__ out_,
                         float* __restrict__ lse_out, int n_heads, int hkv) {
+  using OutT = typename std::conditional<F32OUT, float, __nv_bfloat16>::type;
+  OutT* __restrict__ out = static_cast<OutT*>(out_);
   // the next kernel may start launching now (its CTAs take SMs as the decode CTAs exit);
   // it waits for this grid before touching anything written here
   grid_dependents_launch();
@@ -710,10 +732,15 @@ __global__ void __launch_bounds__(kMergeThreads)
       M = mb;
     }
     const float inv = L > 0.f ? 1.f / L : 0.f;
-    uint2 pk;
-    pk.x = pack2(acc.x * inv, acc.y * inv);
-    pk.y = pack2(acc.z * inv, acc.w * inv);
-    *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+    if constexpr (F32OUT) {
+      *reinterpret_cast<float4*>(out + (hrow + g) * D + d) =
+          make_float4(acc.x * inv, acc.y * inv, acc.z * inv, acc.w * inv);
+    } else {
+      uint2 pk;
+      pk.x = pack2(acc.x * inv, acc.y * inv);
+      pk.y = pack2(acc.z * inv, acc.w * inv);
+      *reinterpret_cast<uint2*>(out + (hrow + g) * D + d) = pk;
+    }
     if (d == 0 && lse_out) lse_out[hrow + g] = L > 0.f ? (M + log2f(L)) * kLn2T : -INFINITY;
   }
 }
@@ -749,14 +776,15 @@ size_t max_chunks_tc(const spkv_params& p, int num_sms) {
   return (size_t)num_sms * kUnitsPerCta + (size_t)p.B * p.Hkv;
 }
 
-template <int D, int G>
+template <int D, int G, bool F32OUT>
 cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
                    const int32_t* t_pos, const void* k_new, const void* v_new, bool early_plan,
-                   void* o, float* lse, void* ws, int num_sms, cudaStream_t stream) {
+                   bool window_on, void* o, float* lse, void* ws, int num_sms,
+                   cudaStream_t stream) {
   using S = TcDecSmem<D, G>;
   const size_t smem = sizeof(S) + 1024 + ((size_t)5 * p.B * p.Hkv + 1) * 4;
   {
-    cudaError_t e = ensure_dynamic_smem((const void*)decode_tc_kernel<D, G>, (int)smem);
+    cudaError_t e = ensure_dynamic_smem((const void*)decode_tc_kernel<D, G, F32OUT>, (int)smem);
     if (e != cudaSuccess) return e;
   }
   const cuuint64_t es = 2;
@@ -768,7 +796,7 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
     if (!map_bf16(&tkp, c.K_pool, 2, dims, str, box) || !map_bf16(&tvp, c.V_pool, 2, dims, str, box))
       return cudaErrorInvalidValue;
   }
-  {
+  if (ring.K_win) {  // else a slice of a split sequence without the window: never read
     const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)p.window, (cuuint64_t)p.Hkv, (cuuint64_t)p.B};
     const cuuint64_t str[3] = {(cuuint64_t)D * es, (cuuint64_t)p.window * D * es,
                                (cuuint64_t)p.Hkv * p.window * D * es};
@@ -776,9 +804,13 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
     if (!map_bf16(&tkr, ring.K_win, 4, dims, str, box) || !map_bf16(&tvr, ring.V_win, 4, dims, str, box))
       return cudaErrorInvalidValue;
   }
+  if (!c.K_pool && !ring.K_win) return cudaErrorInvalidValue;
   if (!c.K_pool) {
     tkp = tkr;
     tvp = tvr;
+  } else if (!ring.K_win) {
+    tkr = tkp;
+    tvr = tvp;
   }
   const int n_heads = p.B * p.Hkv;
   char* w = static_cast<char*>(ws);
@@ -789,26 +821,27 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
   int* ctrl = reinterpret_cast<int*>(w);
   float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
   float* po = reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes);
-  cudaError_t e = launch_pdl(decode_tc_kernel<D, G>, dim3(num_sms), dim3(kThreadsT), smem, stream,
-                             tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q), t_pos,
-                             static_cast<__nv_bfloat16*>(o), lse, ctrl, ml, po, n_heads, p.Hkv,
-                             p.window, c.err_flag, static_cast<const __nv_bfloat16*>(k_new),
-                             static_cast<const __nv_bfloat16*>(v_new), ring.z_win, early_plan ? 1 : 0);
+  cudaError_t e = launch_pdl(decode_tc_kernel<D, G, F32OUT>, dim3(num_sms), dim3(kThreadsT), smem,
+                             stream, tkp, tvp, tkr, tvr, cv, static_cast<const __nv_bfloat16*>(q),
+                             t_pos, o, lse, ctrl, ml, po, n_heads, p.Hkv, p.window, c.err_flag,
+                             static_cast<const __nv_bfloat16*>(k_new),
+                             static_cast<const __nv_bfloat16*>(v_new), ring.z_win,
+                             early_plan ? 1 : 0, window_on ? 1 : 0);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_merge_kernel<D, G>, dim3(n_heads), dim3(kMergeThreads), 0, stream, ctrl,
-                    ml, po, static_cast<__nv_bfloat16*>(o), lse, n_heads, p.Hkv);
+  return launch_pdl(decode_merge_kernel<D, G, F32OUT>, dim3(n_heads), dim3(kMergeThreads), 0,
+                    stream, ctrl, ml, po, o, lse, n_heads, p.Hkv);
 }
 
-template <int D>
+template <int D, bool F32OUT>
 cudaError_t dispatch_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                         const void* q, const int32_t* t_pos, const void* k_new, const void* v_new,
-                        bool early_plan, void* o, float* lse, void* ws, int num_sms,
-                        cudaStream_t stream) {
+                        bool early_plan, bool window_on, void* o, float* lse, void* ws,
+                        int num_sms, cudaStream_t stream) {
   switch (p.Hq / p.Hkv) {
-    case 1: return run_tc<D, 1>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
-    case 2: return run_tc<D, 2>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
-    case 4: return run_tc<D, 4>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
-    case 8: return run_tc<D, 8>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, ws, num_sms, stream);
+    case 1: return run_tc<D, 1, F32OUT>(p, c, ring, q, t_pos, k_new, v_new, early_plan, window_on, o, lse, ws, num_sms, stream);
+    case 2: return run_tc<D, 2, F32OUT>(p, c, ring, q, t_pos, k_new, v_new, early_plan, window_on, o, lse, ws, num_sms, stream);
+    case 4: return run_tc<D, 4, F32OUT>(p, c, ring, q, t_pos, k_new, v_new, early_plan, window_on, o, lse, ws, num_sms, stream);
+    case 8: return run_tc<D, 8, F32OUT>(p, c, ring, q, t_pos, k_new, v_new, early_plan, window_on, o, lse, ws, num_sms, stream);
   }
   return cudaErrorInvalidValue;
 }
@@ -836,10 +869,21 @@ cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const sp
                              void* workspace, int num_sms, cudaStream_t stream,
                              const void* k_new, const void* v_new, bool early_plan) {
   if (p.head_dim == 128)
-    return dispatch_tc<128>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, workspace,
-                            num_sms, stream);
-  return dispatch_tc<64>(p, c, ring, q, t_pos, k_new, v_new, early_plan, o, lse, workspace,
-                         num_sms, stream);
+    return dispatch_tc<128, false>(p, c, ring, q, t_pos, k_new, v_new, early_plan, true, o, lse,
+                                   workspace, num_sms, stream);
+  return dispatch_tc<64, false>(p, c, ring, q, t_pos, k_new, v_new, early_plan, true, o, lse,
+                                workspace, num_sms, stream);
+}
+
+cudaError_t launch_decode_partial(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                                  const void* q, const int32_t* t_pos, bool window_on,
+                                  float* o_part, float* lse_part, void* workspace, int num_sms,
+                                  cudaStream_t stream) {
+  if (p.head_dim == 128)
+    return dispatch_tc<128, true>(p, c, ring, q, t_pos, nullptr, nullptr, false, window_on, o_part,
+                                  lse_part, workspace, num_sms, stream);
+  return dispatch_tc<64, true>(p, c, ring, q, t_pos, nullptr, nullptr, false, window_on, o_part,
+                               lse_part, workspace, num_sms, stream);
 }
 
 }  // namespace spkv

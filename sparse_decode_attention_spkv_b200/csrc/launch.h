@@ -58,6 +58,18 @@ cudaError_t launch_decode_tc(const spkv_params& p, const spkv_cache& c, const sp
                              void* workspace, int num_sms, cudaStream_t stream,
                              const void* k_new = nullptr, const void* v_new = nullptr,
                              bool early_plan = false);
+// Decode attention over one slice of a sequence's keys: the cache's rows with pos <=
+// t - w and, with window_on, the window; fp32 o_part normalised over the slice and its
+// lse (natural log), o = 0 and lse = -inf for a head without keys in the slice.
+// ring.K_win may be NULL when window_on is false.
+cudaError_t launch_decode_partial(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
+                                  const void* q, const int32_t* t_pos, bool window_on,
+                                  float* o_part, float* lse_part, void* workspace, int num_sms,
+                                  cudaStream_t stream);
+// Log-sum-exp combination of n_parts slice partials into one output per query head.
+cudaError_t launch_decode_merge_parts(const spkv_params& p, int n_parts, const float* o_parts,
+                                      const float* lse_parts, void* o, float* lse,
+                                      cudaStream_t stream);
 cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                           const void* q, const int32_t* t_pos, void* o, float* lse,
                           void* workspace, size_t ws_bytes, int num_sms, cudaStream_t stream);

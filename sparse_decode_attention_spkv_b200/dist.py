@@ -1,8 +1,10 @@
 """Process-group plumbing for running the hot path on several GPUs of one node.
 
-The SP-KV path has no exchange step: batch rows and key heads are independent, so
-N GPUs run N replicas (or disjoint batch shards) and only the timing is combined
-(max over ranks).  Backend "nccl" on GPUs, "gloo" for CPU tests.
+The SP-KV path has no exchange step between batch rows or key heads: they are
+independent, so N GPUs serve disjoint batch shards and only the timing is combined
+(max over ranks).  The one exchange is that of a sequence split by position across
+GPUs (``seqsplit``): every rank's decode partial is all-gathered before the merge.
+Backend "nccl" on GPUs, "gloo" for CPU tests.
 """
 from __future__ import annotations
 
@@ -55,6 +57,21 @@ def shard(n: int, world: int, rank: int) -> Tuple[int, int]:
     base, extra = divmod(n, world)
     start = rank * base + min(rank, extra)
     return start, base + (1 if rank < extra else 0)
+
+
+def all_gather_partials(o_part: torch.Tensor, lse_part: torch.Tensor, o_all: torch.Tensor,
+                        lse_all: torch.Tensor) -> None:
+    """Every rank's decode partial, in rank order: o_all[r] = rank r's o_part, lse_all[r] =
+    rank r's lse_part (fp32; o_all [world][...], lse_all [world][...]).  One collective:
+    both are packed into one buffer per rank."""
+    import torch.distributed as dist
+    world = o_all.shape[0]
+    n_o, n_l = o_part.numel(), lse_part.numel()
+    send = torch.cat([o_part.reshape(-1), lse_part.reshape(-1)])
+    recv = torch.empty((world, n_o + n_l), dtype=send.dtype, device=send.device)
+    dist.all_gather_into_tensor(recv.view(-1), send)
+    o_all.copy_(recv[:, :n_o].reshape(o_all.shape))
+    lse_all.copy_(recv[:, n_o:].reshape(lse_all.shape))
 
 
 def job_throughput(units_per_rank: float, world: int, elapsed_max_s: float) -> float:

@@ -3,7 +3,7 @@
     python -m sparse_decode_attention_spkv_b200.kernel_driver decode  [--layers 1] [--steps 3]
                                       [--decode-step attn-first|split|fused]
     python -m sparse_decode_attention_spkv_b200.kernel_driver score   [--tokens 8]
-    python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096]
+    python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096] [--source chunk|ring]
     python -m sparse_decode_attention_spkv_b200.kernel_driver prefill [--chunk 4096]
     python -m sparse_decode_attention_spkv_b200.kernel_driver rethreshold [--steps 2]
     python -m sparse_decode_attention_spkv_b200.kernel_driver soft [--seq 8192]
@@ -59,6 +59,24 @@ def run_score(args):
 
 
 def run_compact(args):
+    """--source chunk: one prefill16k chunk (batch 1, args.rows tokens, 8 key heads)
+    compacted from the chunk tensors, args.steps times (consecutive chunks);
+    --source ring: one serving bulk pass (batch 32, the 128 buffered tokens of every row,
+    8 key heads) compacted from the ring, args.steps times."""
+    if args.source == "ring":
+        wl = W.WORKLOADS["serving"]
+        n = wl.bulk
+        L = _layer(wl, (args.steps + 1) * n)
+        D.fill_normal(L.ring.K_win, wl.key(0, gen.T_K), wl.qkv_scale)
+        D.fill_normal(L.ring.V_win, wl.key(0, gen.T_V), wl.qkv_scale)
+        h = torch.empty((wl.B * n, wl.d_model), dtype=torch.bfloat16, device="cuda")
+        D.fill_normal(h, wl.key(0, gen.T_H), 1.0)
+        u, z = R.score(L, h, wl.B * n)
+        for i in range(args.steps):
+            src = torch.full((wl.B,), i * n, dtype=torch.int32, device="cuda")
+            S.spkv_write_compact(L.p, L.cache, L.ring, S.SRC_RING, None, None, z, u, src, n, n)
+        torch.cuda.synchronize()
+        return
     wl = W.WORKLOADS["prefill16k"]
     n = args.rows
     L = _layer(wl, 4 * n)
@@ -142,6 +160,7 @@ def main():
     ap.add_argument("--rows", type=int, default=4096)
     ap.add_argument("--chunk", type=int, default=4096)
     ap.add_argument("--seq", type=int, default=8192)
+    ap.add_argument("--source", default="chunk", choices=["chunk", "ring"])
     ap.add_argument("--decode-step", default="attn-first", choices=["attn-first", "split", "fused"])
     args = ap.parse_args()
     torch.cuda.set_device(0)

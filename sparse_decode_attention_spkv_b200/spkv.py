@@ -27,6 +27,7 @@ SRC_CHUNK, SRC_RING = 0, 1
 FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT = 1, 2, 4
 PAGE_ROWS = 64
 DECODE_STATE_SETTLED = 1
+SLICE_WINDOW = 1
 
 _vp = ctypes.c_void_p
 _i32 = ctypes.c_int
@@ -82,6 +83,10 @@ _sigs = {
                                         _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
     "spkv_decode_score": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _vp]),
+    "spkv_decode_attn_partial": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
+                                        ctypes.c_uint, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
+    "spkv_decode_attn_partial_supported": (_i32, [_P(spkv_params)]),
+    "spkv_decode_merge": (_i32, [_P(spkv_params), _i32, _vp, _vp, _vp, _vp, _vp]),
 }
 NOALLOC_SCRATCH_BYTES = 8 << 20
 for _name, (_res, _args) in _sigs.items():
@@ -325,3 +330,29 @@ def spkv_decode_score(p, ring: Ring, t_pos, h, W1, b1, W2, b2, u_out, z_out, str
     return _check("spkv_decode_score", lib.spkv_decode_score(
         ctypes.byref(p), ctypes.byref(ring.r), _ptr(t_pos), _ptr(h), _ptr(W1), _ptr(b1), _ptr(W2),
         _ptr(b2), _ptr(u_out), _ptr(z_out), _stream(stream)))
+
+
+def _ring_ref(ring: Optional[Ring]):
+    return ctypes.byref(ring.r) if ring is not None else None
+
+
+def spkv_decode_attn_partial(p, cache: Optional[Cache], ring: Optional[Ring], q, t_pos, flags,
+                             o_part, lse_part, workspace, stream=None):
+    """Decode attention over one slice of a split sequence (its cache rows, and the window
+    with flags SLICE_WINDOW): fp32 o_part [B][Hq][d] and lse_part [B][Hq].  See
+    include/spkv.h."""
+    return _check("spkv_decode_attn_partial", lib.spkv_decode_attn_partial(
+        ctypes.byref(p), _cache_ref(cache), _ring_ref(ring), _ptr(q), _ptr(t_pos), int(flags),
+        _ptr(o_part), _ptr(lse_part), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def spkv_decode_attn_partial_supported(p) -> bool:
+    return bool(lib.spkv_decode_attn_partial_supported(ctypes.byref(p)))
+
+
+def spkv_decode_merge(p, n_parts, o_parts, lse_parts, o, lse, stream=None):
+    """Log-sum-exp combination of slice partials o_parts [n][B][Hq][d], lse_parts [n][B][Hq]
+    (fp32) into o [B][Hq][d] and lse [B][Hq] (may be None)."""
+    return _check("spkv_decode_merge", lib.spkv_decode_merge(
+        ctypes.byref(p), int(n_parts), _ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse),
+        _stream(stream)))

@@ -20,10 +20,18 @@ import torch
 
 
 def build_decode_state(wl, layers, steps_total, device, compact_window: bool = False,
-                       chunk: int = 0, store_u: bool = False):
+                       chunk: int = 0, store_u: bool = False, row0: int = 0,
+                       pos_range=None, with_ring: bool = True):
     """Returns (params, [Layer], inputs) where inputs["h"|"q"|"k"|"v"][i][l] are step i's
     tensors of layer l and inputs["t"][i] the positions [B] of step i.  store_u keeps the
-    utilities of cached rows and pending window slots (for re-thresholding)."""
+    utilities of cached rows and pending window slots (for re-thresholding).
+
+    row0: the global index of batch row 0 (a rank serving rows row0 .. row0+B-1 of a
+    larger batch draws exactly those rows' inputs: every seeded stream is indexed by the
+    global row).  pos_range (lo, hi), per-row lists (hi None: no upper bound): only the
+    gated positions in [lo, hi) are written to the cache -- one slice of a sequence whose
+    cache is split by position; with_ring False leaves the ring unwritten (a slice that
+    does not hold the window)."""
     from sparse_decode_attention_spkv_b200 import runner as R
     from sparse_decode_attention_spkv_b200 import spkv as S
     from sparse_decode_attention_spkv_b200.inputs import device as D
@@ -45,6 +53,14 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
     # per row: positions below `limit` are compacted from the chunks
     limit = torch.tensor([c if compact_window else c - w for c in ctx], dtype=torch.int32,
                          device=device)
+    if pos_range is not None:  # a slice: positions outside [lo, hi) stay out of this cache
+        lo_l, hi_l = pos_range
+        lo_t = torch.tensor([int(x) for x in lo_l], dtype=torch.int32, device=device)
+        hi_t = torch.tensor([c + steps_total if h is None else int(h) for c, h in zip(ctx, hi_l)],
+                            dtype=torch.int32, device=device)
+        limit = torch.minimum(limit, hi_t)
+    else:
+        lo_t = torch.zeros(B, dtype=torch.int32, device=device)
     keep_table = W.load_biases()[wl.name]["keep_target"]
     Ls = []
     for l in range(layers):
@@ -62,16 +78,18 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
         for c0 in range(0, n_lim, chunk):
             n = min(chunk, n_lim - c0)
             for b in range(B):
-                D.fill_normal(h_c[b, :n], kh_, 1.0, offset=(b * Tt + c0) * Dm)
-                D.fill_normal(k_c[b, :n], kk_, wl.qkv_scale, offset=(b * Tt + c0) * Hkv * d)
-                D.fill_normal(v_c[b, :n], kv_, wl.qkv_scale, offset=(b * Tt + c0) * Hkv * d)
+                g = row0 + b
+                D.fill_normal(h_c[b, :n], kh_, 1.0, offset=(g * Tt + c0) * Dm)
+                D.fill_normal(k_c[b, :n], kk_, wl.qkv_scale, offset=(g * Tt + c0) * Hkv * d)
+                D.fill_normal(v_c[b, :n], kv_, wl.qkv_scale, offset=(g * Tt + c0) * Hkv * d)
             hc = h_c[:, :n].contiguous() if n < chunk else h_c
             kc = k_c[:, :n].contiguous() if n < chunk else k_c
             vc = v_c[:, :n].contiguous() if n < chunk else v_c
             u, z = R.score(L, hc, B * n)
             z = z.view(B, n, Hkv)
             pos = torch.arange(c0, c0 + n, dtype=torch.int32, device=device)
-            z.mul_((pos[None, :] < limit[:, None]).to(torch.uint8)[:, :, None])  # beyond a row's prefix
+            keep = (pos[None, :] < limit[:, None]) & (pos[None, :] >= lo_t[:, None])
+            z.mul_(keep.to(torch.uint8)[:, :, None])  # beyond a row's prefix or outside the slice
             src = torch.full((B,), c0, dtype=torch.int32, device=device)
             S.spkv_write_compact(p, L.cache, L.ring, S.SRC_CHUNK, kc, vc, z, u, src, n, n)
         # the ring: each row's last w tokens, gated (per-token) or marked as cached
@@ -80,12 +98,14 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
         hr = torch.empty((B, w, Dm), dtype=bf, device=device)
         for b in range(B):
             s0 = ctx[b] - w
-            D.fill_normal(hr[b], kh_, 1.0, offset=(b * Tt + s0) * Dm)
-            D.fill_normal(kr[b], kk_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
-            D.fill_normal(vr[b], kv_, wl.qkv_scale, offset=(b * Tt + s0) * Hkv * d)
-        ur, zr = R.score(L, hr, B * w)
-        src = torch.tensor([c - w for c in ctx], dtype=torch.int32, device=device)
-        S.spkv_ring_write(p, L.ring, kr, vr, zr, ur, w if compact_window else 0, src, w, w)
+            g = row0 + b
+            D.fill_normal(hr[b], kh_, 1.0, offset=(g * Tt + s0) * Dm)
+            D.fill_normal(kr[b], kk_, wl.qkv_scale, offset=(g * Tt + s0) * Hkv * d)
+            D.fill_normal(vr[b], kv_, wl.qkv_scale, offset=(g * Tt + s0) * Hkv * d)
+        if with_ring:
+            ur, zr = R.score(L, hr, B * w)
+            src = torch.tensor([c - w for c in ctx], dtype=torch.int32, device=device)
+            S.spkv_ring_write(p, L.ring, kr, vr, zr, ur, w if compact_window else 0, src, w, w)
         Ls.append(L)
     del h_c, k_c, v_c
     # per-step inputs [steps][layers][B][...]; row b's step i is position ctx[b] + i
@@ -97,10 +117,11 @@ def build_decode_state(wl, layers, steps_total, device, compact_window: bool = F
     for l in range(layers):
         for b in range(B):
             t0 = ctx[b]
-            D.fill_normal(h_s[l, b], wl.key(l, gen.T_H), 1.0, offset=(b * Tt + t0) * Dm)
-            D.fill_normal(q_s[l, b], wl.key(l, gen.T_Q), wl.qkv_scale, offset=(b * Tt + t0) * Hq * d)
-            D.fill_normal(k_s[l, b], wl.key(l, gen.T_K), wl.qkv_scale, offset=(b * Tt + t0) * Hkv * d)
-            D.fill_normal(v_s[l, b], wl.key(l, gen.T_V), wl.qkv_scale, offset=(b * Tt + t0) * Hkv * d)
+            g = row0 + b
+            D.fill_normal(h_s[l, b], wl.key(l, gen.T_H), 1.0, offset=(g * Tt + t0) * Dm)
+            D.fill_normal(q_s[l, b], wl.key(l, gen.T_Q), wl.qkv_scale, offset=(g * Tt + t0) * Hq * d)
+            D.fill_normal(k_s[l, b], wl.key(l, gen.T_K), wl.qkv_scale, offset=(g * Tt + t0) * Hkv * d)
+            D.fill_normal(v_s[l, b], wl.key(l, gen.T_V), wl.qkv_scale, offset=(g * Tt + t0) * Hkv * d)
     ctx_t = torch.tensor(ctx, dtype=torch.int32, device=device)
     inputs = {
         "h": h_s.permute(2, 0, 1, 3).contiguous(),

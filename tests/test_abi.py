@@ -132,3 +132,27 @@ def test_noalloc_argument_checks_match_decode_attn():
         b = S.lib.spkv_decode_attn_noalloc(ctypes.byref(p), ctypes.byref(c), ctypes.byref(r), q, t,
                                            o, None, None)
         assert a == b == S.ERR_ARG, (a, b)
+
+
+def test_sequence_split_argument_checks():
+    """Partial decode and merge of a split sequence: argument errors on the host."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    bf = S.make_params(2, 8, 2, 128, 256, 64, 128, 0.5, S.BF16)
+    f32 = S.make_params(2, 8, 2, 128, 256, 64, 128, 0.5, S.F32)
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
+    ring = S.spkv_ring(16, 16, 16, None)
+    part = S.lib.spkv_decode_attn_partial
+    r = ctypes.byref
+    assert part(r(bf), r(cache), r(ring), 16, 16, 2, 16, 16, 16, 1 << 30, None) == S.ERR_ARG  # flag
+    assert part(r(bf), None, None, 16, 16, 0, 16, 16, 16, 1 << 30, None) == S.ERR_ARG  # no keys
+    assert part(r(bf), None, None, 16, 16, S.SLICE_WINDOW, 16, 16, 16, 1 << 30,
+                None) == S.ERR_ARG  # window without a ring
+    assert part(r(bf), r(cache), None, 16, 16, 0, 16, None, 16, 1 << 30, None) == S.ERR_ARG  # lse
+    assert part(r(bf), r(cache), None, 16, 16, 0, 8, 16, 16, 1 << 30, None) == S.ERR_ARG  # align
+    assert part(r(f32), r(cache), None, 16, 16, 0, 16, 16, 16, 1 << 30,
+                None) == S.ERR_UNSUPPORTED
+    assert S.lib.spkv_decode_attn_partial_supported(r(f32)) == 0
+    merge = S.lib.spkv_decode_merge
+    assert merge(r(bf), 0, 16, 16, 16, None, None) == S.ERR_ARG      # no part
+    assert merge(r(bf), 2, None, 16, 16, None, None) == S.ERR_ARG
+    assert merge(r(bf), 2, 16, 16, 8, None, None) == S.ERR_ARG       # misaligned output
