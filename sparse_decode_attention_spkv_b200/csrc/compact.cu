@@ -19,6 +19,25 @@ namespace {
 
 CacheMut mut(const spkv_cache& c) { return cache_mut(c); }
 
+// Gates of rows [r0, r1) of one key head (stride hkv bytes), summed by the block: every
+// thread keeps 8 loads in flight per round.  The loads go to L2 (ld.global.cg): they may
+// run while the kernel that wrote the gates has only just finished.
+__device__ __forceinline__ int count_gates(const uint8_t* zb, int r0, int r1, int hkv) {
+  int kept = 0;
+  const int stride = blockDim.x;
+  for (int i0 = r0 + (int)threadIdx.x; i0 < r1; i0 += 8 * stride) {
+    int v[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = i0 + k * stride;
+      v[k] = i < r1 ? __ldcg(zb + (size_t)i * hkv) : 0;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; ++k) kept += v[k];
+  }
+  return kept;
+}
+
 __device__ __forceinline__ int block_sum(int v, int* red) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 #pragma unroll
@@ -33,21 +52,23 @@ __device__ __forceinline__ int block_sum(int v, int* red) {
 
 // One CTA per (batch row, key head): count this call's gated rows, extend the
 // head's page list (pages it still owns past its count, left by a re-threshold, first;
-// then new ones from the bump allocator), and publish count_prev / count.
+// then new ones from the bump allocator), and publish count_prev / count.  Launched as
+// a programmatic dependent: it waits for the kernel before it (which may have written
+// the gates or the cache), then lets the scatter start launching at once.
 __global__ void __launch_bounds__(256)
     compact_plan(CacheMut c, const uint8_t* __restrict__ z, int n_rows, int src_batch_rows,
                  int hkv) {
   __shared__ int red[8];
   __shared__ int s_have, s_need, s_free, s_first, s_grant;
+  grid_dependency_wait();
+  grid_dependents_launch();
   const int bh = blockIdx.x, b = bh / hkv, kh = bh % hkv;
   const uint8_t* zb = z + (size_t)b * src_batch_rows * hkv + kh;
   int32_t* table = c.page_table + (size_t)bh * c.max_pages;
-  int kept = 0;
-  for (int i = threadIdx.x; i < n_rows; i += blockDim.x) kept += zb[(size_t)i * hkv];
-  const int total = block_sum(kept, red);
+  const int total = block_sum(count_gates(zb, 0, n_rows, hkv), red);
   int old = 0, want = 0;
   if (threadIdx.x == 0) {
-    old = c.count[bh];
+    old = __ldcg(c.count + bh);
     const int cap = c.max_pages * kPageRows;
     want = old + total;
     if (want > cap) {
@@ -61,7 +82,7 @@ __global__ void __launch_bounds__(256)
   __syncthreads();
   // owned pages form a prefix of the table: find the first unowned entry we need
   for (int j = s_have + threadIdx.x; j < s_need; j += blockDim.x)
-    if (table[j] < 0) atomicMin(&s_free, j);
+    if (__ldcg(table + j) < 0) atomicMin(&s_free, j);
   __syncthreads();
   if (threadIdx.x == 0) {
     int need = s_need;
@@ -93,6 +114,10 @@ constexpr int kScatterThreads = 256;
 // grid (B*Hkv, tiles of 256 rows).  Each CTA counts the gated rows before its
 // tile (z is tiny), so tiles need no inter-CTA ordering; inside a tile, 256-row
 // rounds are ranked with a warp-ballot prefix sum and copied by lane groups.
+// Launched as a programmatic dependent of compact_plan: the prefix count (gates only,
+// which the plan does not write; the plan itself started after the gates' producer had
+// completed) runs while the plan works; the counts and page lists are read after the
+// wait for the plan.
 __global__ void __launch_bounds__(kScatterThreads)
     compact_scatter(CacheMut c, const char* __restrict__ Ksrc, const char* __restrict__ Vsrc,
                     const uint8_t* __restrict__ z, const float* __restrict__ u,
@@ -108,12 +133,11 @@ __global__ void __launch_bounds__(kScatterThreads)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const uint8_t* zb = z + (size_t)b * src_batch_rows * hkv + kh;
 
-  int before = 0;
-  for (int i = threadIdx.x; i < tile0; i += blockDim.x) before += zb[(size_t)i * hkv];
-  const int prefix = block_sum(before, red);
-  const int base = c.count_prev[bh];
-  const int limit = c.count[bh];
-  const int p0 = src_pos[b];
+  const int prefix = block_sum(count_gates(zb, 0, tile0, hkv), red);
+  grid_dependency_wait();  // the plan's counts and page lists
+  const int base = __ldcg(c.count_prev + bh);
+  const int limit = __ldcg(c.count + bh);
+  const int p0 = __ldcg(src_pos + b);
   int running = base + prefix;
 
   const int lpr = row_bytes >> 4;      // lanes per row
@@ -122,7 +146,7 @@ __global__ void __launch_bounds__(kScatterThreads)
 
   for (int r0 = tile0; r0 < tile0 + kScatterTile && r0 < n_rows; r0 += kScatterThreads) {
     const int i = r0 + threadIdx.x;
-    const int flag = (i < n_rows) ? zb[(size_t)i * hkv] : 0;
+    const int flag = (i < n_rows) ? __ldcg(zb + (size_t)i * hkv) : 0;
     const unsigned ball = __ballot_sync(0xffffffffu, flag);
     const int in_warp = __popc(ball & ((1u << lane) - 1u));
     if (lane == 0) warp_tot[warp] = __popc(ball);
@@ -142,7 +166,8 @@ __global__ void __launch_bounds__(kScatterThreads)
       const int src_i = list_src[e];
       const int dst = list_dst[e];
       if (dst >= limit) continue;  // dropped: capacity (flag already raised by the plan)
-      const int page = c.page_table[(size_t)bh * c.max_pages + (dst >> 6)];
+      const int page = __ldcg(c.page_table + (size_t)bh * c.max_pages + (dst >> 6));
+      if (!page_ok(page, c.num_pages, c.err)) continue;  // debug build: flagged, skipped
       const size_t drow = (size_t)page * kPageRows + (dst & 63);
       size_t srow;
       if (from_ring) {
@@ -225,14 +250,15 @@ cudaError_t launch_write_compact(const spkv_params& p, const spkv_cache& c, cons
   const int esize = p.dtype == SPKV_BF16 ? 2 : 4;
   const int row_bytes = p.head_dim * esize;
   CacheMut m = mut(c);
-  compact_plan<<<n_heads, 256, 0, stream>>>(m, z, n_rows, src_batch_rows, p.Hkv);
+  cudaError_t e = launch_pdl(compact_plan, dim3(n_heads), dim3(256), 0, stream, m, z, n_rows,
+                             src_batch_rows, p.Hkv);
+  if (e != cudaSuccess) return e;
   const char* Ks = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->K_win : K_src);
   const char* Vs = static_cast<const char*>(src_kind == SPKV_SRC_RING ? ring->V_win : V_src);
   dim3 grid(n_heads, (n_rows + kScatterTile - 1) / kScatterTile);
-  compact_scatter<<<grid, kScatterThreads, 0, stream>>>(m, Ks, Vs, z, u, src_pos, n_rows,
-                                                        src_batch_rows, p.Hkv, row_bytes,
-                                                        src_kind == SPKV_SRC_RING, p.window);
-  return cudaGetLastError();
+  return launch_pdl(compact_scatter, grid, dim3(kScatterThreads), 0, stream, m, Ks, Vs, z, u,
+                    src_pos, n_rows, src_batch_rows, p.Hkv, row_bytes,
+                    (int)(src_kind == SPKV_SRC_RING), p.window);
 }
 
 cudaError_t launch_decode_append(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
