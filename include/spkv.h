@@ -61,7 +61,8 @@ enum spkv_status {
   SPKV_ERR_CAPACITY = 2,    /* device-detected: pool or page table exhausted */
   SPKV_ERR_CUDA = 3,        /* a CUDA runtime call or a launch failed */
   SPKV_ERR_UNSUPPORTED = 4, /* valid but not built (shape/dtype combination) */
-  SPKV_ERR_TIMEOUT = 5      /* device-detected: a bounded wait gave up */
+  SPKV_ERR_TIMEOUT = 5,     /* device-detected: a bounded wait gave up */
+  SPKV_ERR_INDEX = 6        /* device-detected (debug build): an index check failed */
 };
 
 enum spkv_dtype { SPKV_F32 = 0, SPKV_BF16 = 1 };
@@ -75,6 +76,9 @@ enum spkv_src_kind {
 #define SPKV_FLAG_POOL_FULL 1u  /* no free page was left for an append */
 #define SPKV_FLAG_TABLE_FULL 2u /* a key head reached max_pages_per_head */
 #define SPKV_FLAG_TIMEOUT 4u    /* a bounded wait inside a kernel gave up */
+#define SPKV_FLAG_INDEX 8u      /* debug build (SPKV_DEBUG): a page number read from a page
+                                   table lay outside the pool, or a query position was
+                                   negative; the access was skipped or redirected */
 
 /* Shapes of one attention layer. */
 typedef struct spkv_params {
@@ -136,7 +140,7 @@ int spkv_cache_reset(const spkv_params* p, const spkv_cache* cache, const spkv_r
 
 /* Synchronise `stream`, copy err_flag to *flags_out (if not NULL) and return
  * SPKV_ERR_CAPACITY if a pool/table bit is set, SPKV_ERR_TIMEOUT if the timeout
- * bit is set, else SPKV_OK. */
+ * bit is set, SPKV_ERR_INDEX if the index bit is set, else SPKV_OK. */
 int spkv_cache_check(const spkv_cache* cache, spkv_stream_t stream, uint32_t* flags_out);
 
 /* a1 -- utility score and gate, Eqs. (1)-(2), fused:
@@ -385,6 +389,13 @@ size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* 
 int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                            float tau_new, void* workspace, size_t ws_bytes,
                            spkv_stream_t stream);
+
+/* Diagnostics, for testing failure reporting: the limit, in nanoseconds, of the bounded
+ * waits of spkv_cache_rethreshold's move kernel on the "page read" flags of other CTAs
+ * (default 2 s; 0 restores it).  A wait that runs out latches SPKV_FLAG_TIMEOUT and the
+ * rows bound for the unread page are not written.  Process-wide; applies to calls
+ * enqueued afterwards.  No other wait of the library is affected. */
+int spkv_debug_set_flag_wait_ns(unsigned long long ns);
 
 /* Bytes of workspace spkv_soft_attn needs (a per-key bias buffer). */
 size_t spkv_soft_attn_workspace_bytes(const spkv_params* p, int seq_len);

@@ -2,8 +2,9 @@
 
     python -m sparse_decode_attention_spkv_b200.build
 
-produces ``libspkv.so`` (the SP-KV kernels behind the C ABI of include/spkv.h) and
-``inputs/libspkv_inputs.so`` (the device side of the seeded input generator).
+produces ``libspkv.so`` (the SP-KV kernels behind the C ABI of include/spkv.h),
+``libspkv_debug.so`` (the same kernels built with SPKV_DEBUG: device-side index checks)
+and ``inputs/libspkv_inputs.so`` (the device side of the seeded input generator).
 Objects are cached under ``_build/`` and rebuilt when a source is newer.
 """
 from __future__ import annotations
@@ -21,8 +22,14 @@ FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "--expt-relaxe
          "-I", os.path.join(ROOT, "include")]
 
 LIBS = {
-    os.path.join(PKG, "libspkv.so"): sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu"))),
-    os.path.join(PKG, "inputs", "libspkv_inputs.so"): [os.path.join(PKG, "inputs", "inputs_gen.cu")],
+    # library: (sources, extra compiler flags, object directory)
+    os.path.join(PKG, "libspkv.so"): (sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu"))), [], ""),
+    # the same kernels with device-side checks of page-table entries and positions
+    # (SPKV_DEBUG: a failed check latches SPKV_FLAG_INDEX; nothing traps)
+    os.path.join(PKG, "libspkv_debug.so"): (sorted(glob.glob(os.path.join(PKG, "csrc", "*.cu"))),
+                                            ["-DSPKV_DEBUG"], "debug"),
+    os.path.join(PKG, "inputs", "libspkv_inputs.so"): ([os.path.join(PKG, "inputs", "inputs_gen.cu")],
+                                                      [], ""),
 }
 
 
@@ -43,19 +50,22 @@ def _run(cmd, verbose):
 
 
 def build(verbose: bool = False, ptxas_info: bool = False) -> list:
-    out_dir = os.path.join(ROOT, "_build")
-    os.makedirs(out_dir, exist_ok=True)
+    from concurrent.futures import ThreadPoolExecutor
     built = []
-    for lib, sources in LIBS.items():
-        objs = []
+    for lib, (sources, extra, sub) in LIBS.items():
+        out_dir = os.path.join(ROOT, "_build", sub)
+        os.makedirs(out_dir, exist_ok=True)
+        jobs, objs = [], []
         for src in sources:
             obj = os.path.join(out_dir, os.path.basename(src) + ".o")
             deps = [src] + _headers(os.path.dirname(src))
             stale = not os.path.exists(obj) or any(os.path.getmtime(d) > os.path.getmtime(obj) for d in deps)
             if stale or ptxas_info:
-                extra = ["-Xptxas", "-v"] if ptxas_info else []
-                _run([NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj], verbose or ptxas_info)
+                px = ["-Xptxas", "-v"] if ptxas_info else []
+                jobs.append([NVCC, *ARCH, *FLAGS, *extra, *px, "-c", src, "-o", obj])
             objs.append(obj)
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            list(ex.map(lambda c: _run(c, verbose or ptxas_info), jobs))
         if not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
             _run([NVCC, *ARCH, "-shared", "-o", lib, *objs, "-lcudart"], verbose)
         built.append(lib)

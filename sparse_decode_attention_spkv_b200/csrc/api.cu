@@ -37,6 +37,7 @@ const char* spkv_status_str(int status) {
     case SPKV_ERR_CUDA: return "CUDA error";
     case SPKV_ERR_UNSUPPORTED: return "unsupported shape or dtype";
     case SPKV_ERR_TIMEOUT: return "device wait timed out";
+    case SPKV_ERR_INDEX: return "device index check failed";
   }
   return "unknown status";
 }
@@ -72,6 +73,7 @@ int spkv_cache_check(const spkv_cache* c, spkv_stream_t stream, uint32_t* flags_
   if (flags_out) *flags_out = flags;
   if (flags & (SPKV_FLAG_POOL_FULL | SPKV_FLAG_TABLE_FULL)) return SPKV_ERR_CAPACITY;
   if (flags & SPKV_FLAG_TIMEOUT) return SPKV_ERR_TIMEOUT;
+  if (flags & SPKV_FLAG_INDEX) return SPKV_ERR_INDEX;
   return SPKV_OK;
 }
 
@@ -268,6 +270,11 @@ int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* c, const spkv
   if (sms <= 0) return SPKV_ERR_CUDA;
   return status_of(spkv::launch_rethreshold(*p, *c, ring, tau_new, workspace, sms,
                                             static_cast<cudaStream_t>(stream)));
+}
+
+int spkv_debug_set_flag_wait_ns(unsigned long long ns) {
+  spkv::set_flag_wait_ns(ns);
+  return SPKV_OK;
 }
 
 size_t spkv_soft_attn_workspace_bytes(const spkv_params* p, int seq_len) {

@@ -52,7 +52,7 @@ __device__ __forceinline__ int page_for_new_row(const CacheMut& c, int bh, int i
   }
   int32_t* slot = c.page_table + (size_t)bh * c.max_pages + (i >> 6);
   const int owned = *slot;
-  if (owned >= 0) return owned;
+  if (owned >= 0) return page_ok(owned, c.num_pages, c.err) ? owned : -1;
   const int pg = atomicAdd(c.pool_top, 1);
   if (pg >= c.num_pages) {
     atomicOr(c.err, SPKV_FLAG_POOL_FULL);
@@ -83,6 +83,7 @@ __device__ __forceinline__ void decode_append_warp(const CacheMut& c, const Ring
       page = __shfl_sync(0xffffffffu, page, 0);
     } else {
       page = c.page_table[(size_t)bh * c.max_pages + (i >> 6)];
+      if (!page_ok(page, c.num_pages, c.err)) page = -1;  // debug build: flagged, skipped
     }
     if (page >= 0) {
       const size_t drow = (size_t)page * kPageRows + (i & 63);
@@ -184,6 +185,8 @@ __device__ __forceinline__ void append_commit(const CacheMut& c, const RingMut& 
     if ((i & 63) == 0 && page < 0) {  // a page boundary with no page owned there yet
       if (lane == 0) page = page_for_new_row(c, bh, i);
       page = __shfl_sync(0xffffffffu, page, 0);
+    } else if (page >= 0 && !page_ok(page, c.num_pages, c.err)) {
+      page = -1;  // debug build: flagged, skipped
     }
     if (page >= 0) {
       const size_t drow = (size_t)page * kPageRows + (i & 63);

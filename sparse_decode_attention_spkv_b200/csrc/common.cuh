@@ -189,8 +189,46 @@ __device__ __forceinline__ void bulk_g2s(void* dst_smem, const void* src_gmem, u
       : "memory");
 }
 
+// Orders this thread's generic-proxy writes to shared memory before later async-proxy
+// reads of it (a TMA store, or a tensor-core operand).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+
+// ---- index checks of the debug build -----------------------------------------------------
+// Built with SPKV_DEBUG, every page number read from a page table is checked against the
+// pool (and query positions against 0) before it is used as an address: a failed check
+// latches SPKV_FLAG_INDEX in err_flag and the access is skipped or redirected to page 0
+// (the results are then wrong, and flagged).  Nothing traps.  Without SPKV_DEBUG the
+// checks compile away.
+#ifdef SPKV_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+
+__device__ __forceinline__ bool page_ok(int page, int num_pages, uint32_t* err) {
+  if constexpr (kDebugChecks) {
+    if ((unsigned)page >= (unsigned)num_pages) {
+      if (err) atomicOr(err, SPKV_FLAG_INDEX);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ int checked_position(int t, uint32_t* err) {
+  if constexpr (kDebugChecks) {
+    if (t < 0) {
+      if (err) atomicOr(err, SPKV_FLAG_INDEX);
+      return 0;
+    }
+  }
+  return t;
 }
 
 // ---- cache addressing ------------------------------------------------------------------
@@ -202,11 +240,21 @@ struct CacheView {
   const int32_t* page_table;
   const int32_t* count;
   int max_pages;
+  int num_pages;
+  uint32_t* err;
 };
 
-// Position of cache row i of head bh.
+inline CacheView cache_view(const spkv_cache& c) {
+  return CacheView{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool),
+                   c.pos_pool, c.page_table, c.count, c.max_pages_per_head, c.num_pages,
+                   c.err_flag};
+}
+
+// Position of cache row i of head bh (debug build: a bad page reads as "beyond every
+// limit").
 __device__ __forceinline__ int cache_pos(const CacheView& c, int bh, int i) {
   const int page = __ldcg(c.page_table + (size_t)bh * c.max_pages + (i >> 6));
+  if (!page_ok(page, c.num_pages, c.err)) return 0x7fffffff;
   return __ldcg(c.pos + (size_t)page * kPageRows + (i & 63));
 }
 

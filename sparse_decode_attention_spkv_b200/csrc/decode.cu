@@ -233,7 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const char* srcV;
           int valid;
           if (k * kTileRows < nlp) {
-            const int page = __ldg(cache.page_table + (size_t)bh * cache.max_pages + k);
+            int page = __ldg(cache.page_table + (size_t)bh * cache.max_pages + k);
+            if (!page_ok(page, cache.num_pages, err)) page = 0;  // debug build: flagged
             valid = min(kTileRows, nl - k * kTileRows);
             srcK = cache.K + (size_t)page * Gm::kTileBytes;
             srcV = cache.V + (size_t)page * Gm::kTileBytes;
@@ -529,8 +530,7 @@ cudaError_t run(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring
   float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
   const size_t ml_bytes = (max_chunks * G * 2 * 4 + 255) / 256 * 256;
   float* po = reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes);
-  CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
-               c.page_table, c.count, c.max_pages_per_head};
+  CacheView cv = cache_view(c);
   const float qscale = kLog2e / sqrtf((float)D);
   decode_kernel<E, D, G><<<grid, kThreads, smem, stream>>>(
       cv, static_cast<const char*>(ring.K_win), static_cast<const char*>(ring.V_win),

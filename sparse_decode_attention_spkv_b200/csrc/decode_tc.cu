@@ -264,13 +264,15 @@ __global__ void __launch_bounds__(kThreadsT, 1)
   int my_rows = 0;
   for (int bh = tid; bh < n_heads; bh += kThreadsT) {
     const int b = bh / hkv;
-    const int t = __ldcg(t_pos + b);
+    const int t = checked_position(__ldcg(t_pos + b), err);
     int nl, nw, hide = -1;
     if (!pre) {
       nl = cache_live_rows(cache, bh, t - window, window);
       nw = !win_on ? 0 : t + 1 < window ? t + 1 : window;
     } else {  // ring rows t-w .. t-1; row t - w (slot t mod w) counts if its gate is 1
-      nl = cache_live_rows(cache, bh, t - window - 1, window + 1);
+      // before the step's update the per-token schedule's cache holds positions up to
+      // t - w - 1 only (the entry point's precondition): every stored row is live
+      nl = cache.count ? __ldcg(cache.count + bh) : 0;
       nw = t < window ? t : window;
       if (t >= window && __ldcg(z_win + ((size_t)b * window + t % window) * hkv + bh % hkv) == 0)
         hide = t % window;
@@ -403,7 +405,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
           if (valid == 0) {
             // the empty tile of a head without keys: nothing to load
           } else if (from_cache) {
-            const int page = sm.pages[(k - cd.k0) % kChunkPages];
+            int page = sm.pages[(k - cd.k0) % kChunkPages];
+            if (!page_ok(page, cache.num_pages, err)) page = cache.num_pages;  // zero rows
 #pragma unroll
             for (int hf = 0; hf < TB::kHalves; ++hf) {
               tma2d(tb.k[hf], &tm_kp, hf * 64, page * kPageRows, &sm.full[s]);
@@ -816,8 +819,7 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
   char* w = static_cast<char*>(ws);
   const size_t ctrl_bytes = ctrl_bytes_tc(n_heads);
   const size_t ml_bytes = (max_chunks_tc(p, num_sms) * G * 2 * 4 + 255) / 256 * 256;
-  CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
-               c.page_table, c.count, c.max_pages_per_head};
+  CacheView cv = cache_view(c);
   int* ctrl = reinterpret_cast<int*>(w);
   float* ml = reinterpret_cast<float*>(w + ctrl_bytes);
   float* po = reinterpret_cast<float*>(w + ctrl_bytes + ml_bytes);

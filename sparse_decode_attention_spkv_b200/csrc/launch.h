@@ -80,6 +80,8 @@ cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const s
                               int chunk_start, int chunk_len, void* o, float* lse,
                               cudaStream_t stream);
 size_t rethreshold_workspace_bytes(const spkv_params& p, const spkv_cache& c);
+// Limit of the re-threshold move kernel's waits on page-read flags (0: default).
+void set_flag_wait_ns(unsigned long long ns);
 cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const spkv_ring* ring,
                                float tau_new, void* workspace, int num_sms, cudaStream_t stream);
 

@@ -69,7 +69,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     const char* vrow = nullptr;
     if (valid) {
       if (k < n_live) {
-        const int page = __ldg(cache.page_table + (size_t)bh * cache.max_pages + (k >> 6));
+        int page = __ldg(cache.page_table + (size_t)bh * cache.max_pages + (k >> 6));
+        if (!page_ok(page, cache.num_pages, cache.err)) page = 0;  // debug build: flagged
         const size_t r = (size_t)page * kPageRows + (k & 63);
         krow = cache.K + r * kRowBytes;
         vrow = cache.V + r * kRowBytes;
@@ -163,8 +164,7 @@ template <typename E, int D, int G>
 cudaError_t run(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring, const void* q,
                 const void* Kc, const void* Vc, int chunk_start, int chunk_len, void* o,
                 float* lse, cudaStream_t stream) {
-  CacheView cv{static_cast<const char*>(c.K_pool), static_cast<const char*>(c.V_pool), c.pos_pool,
-               c.page_table, c.count, c.max_pages_per_head};
+  CacheView cv = cache_view(c);
   dim3 grid(chunk_len, p.B * p.Hkv);
   prefill_simple_kernel<E, D, G><<<grid, kWarps * 32, 0, stream>>>(
       cv, static_cast<const char*>(ring.K_win), static_cast<const char*>(ring.V_win),

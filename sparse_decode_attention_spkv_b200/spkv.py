@@ -20,11 +20,12 @@ if not os.path.exists(_LIB_PATH):
     raise ImportError(f"{_LIB_PATH} is missing: build it with "
                       "`python -m sparse_decode_attention_spkv_b200.build`")
 lib = ctypes.CDLL(_LIB_PATH)
+DEBUG_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libspkv_debug.so")
 
-OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT = range(6)
+OK, ERR_ARG, ERR_CAPACITY, ERR_CUDA, ERR_UNSUPPORTED, ERR_TIMEOUT, ERR_INDEX = range(7)
 F32, BF16 = 0, 1
 SRC_CHUNK, SRC_RING = 0, 1
-FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT = 1, 2, 4
+FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT, FLAG_INDEX = 1, 2, 4, 8
 PAGE_ROWS = 64
 DECODE_STATE_SETTLED = 1
 SLICE_WINDOW = 1
@@ -87,12 +88,27 @@ _sigs = {
                                         ctypes.c_uint, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "spkv_decode_attn_partial_supported": (_i32, [_P(spkv_params)]),
     "spkv_decode_merge": (_i32, [_P(spkv_params), _i32, _vp, _vp, _vp, _vp, _vp]),
+    "spkv_debug_set_flag_wait_ns": (_i32, [ctypes.c_ulonglong]),
 }
 NOALLOC_SCRATCH_BYTES = 8 << 20
-for _name, (_res, _args) in _sigs.items():
-    _fn = getattr(lib, _name)
-    _fn.restype = _res
-    _fn.argtypes = _args
+
+
+def _bind(handle):
+    for _name, (_res, _args) in _sigs.items():
+        _fn = getattr(handle, _name)
+        _fn.restype = _res
+        _fn.argtypes = _args
+    return handle
+
+
+_bind(lib)
+
+
+def open_library(path: str):
+    """Another build of the same C ABI (e.g. the debug build, libspkv_debug.so, whose
+    kernels check page-table entries and positions), with the same signatures.  Assign
+    it to ``spkv.lib`` to route the functions below through it."""
+    return _bind(ctypes.CDLL(path))
 
 
 class SpkvError(RuntimeError):
@@ -356,3 +372,9 @@ def spkv_decode_merge(p, n_parts, o_parts, lse_parts, o, lse, stream=None):
     return _check("spkv_decode_merge", lib.spkv_decode_merge(
         ctypes.byref(p), int(n_parts), _ptr(o_parts), _ptr(lse_parts), _ptr(o), _ptr(lse),
         _stream(stream)))
+
+
+def spkv_debug_set_flag_wait_ns(ns: int):
+    """Limit of the re-threshold move kernel's page-flag waits (0: the default); for
+    testing failure reporting (see include/spkv.h)."""
+    return _check("spkv_debug_set_flag_wait_ns", lib.spkv_debug_set_flag_wait_ns(int(ns)))
