@@ -14,9 +14,10 @@ far more than the 126 MB L2, so no flush is needed between steps.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl spkv|reference]
 
-Under torchrun every rank runs its own replica (batch rows and key heads are
-independent: no collective on the data path); the elapsed time is the max over
-ranks and ``value`` counts every rank's tokens.  ``--impl reference`` times the
+Under torchrun rank r serves its own batch shard, global rows 8r .. 8r+7 of a batch
+of 8N (every input drawn by global row index; batch rows and key heads are independent:
+no collective on the data path); the elapsed time is the max over ranks and ``value``
+counts every rank's tokens.  ``--impl reference`` times the
 fp64 CPU oracle on bounded samples of the same workload on rank 0.
 """
 from __future__ import annotations
@@ -189,7 +190,8 @@ def run_gpu(args, world, rank, local):
     steps_total = Wm + K + E + R
     from sparse_decode_attention_spkv_b200.states import (DecodeStep, build_decode_state, kv_bytes,
                                                           kv_bytes_layers)
-    p, Ls, inp = build_decode_state(wl, layers, steps_total, device)
+    # rank r: global batch rows r*B .. r*B + B-1 (disjoint shards, drawn by global row)
+    p, Ls, inp = build_decode_state(wl, layers, steps_total, device, row0=rank * wl.B)
     T0 = wl.ctx[0]
     step = DecodeStep(p, Ls, device, split=args.decode_step != "fused",
                       attn_first=args.decode_step == "attn-first")
@@ -342,7 +344,8 @@ def run_gpu(args, world, rank, local):
                                "context, per-head keep U[5%,50%], per-token retirement",
                    "decode_step": args.decode_step,
                    "global_batch": world * p.B, "seq_len": T0, "layers": layers,
-                   "parallelism": f"replicas x{world} (no data-path collective)",
+                   "parallelism": f"batch shards x{world}: rank r serves global rows "
+                                  f"{wl.B}r..{wl.B}r+{wl.B - 1} (no data-path collective)",
                    "l2": "inputs larger than L2 (every step reads all live K/V, ~GBs)"},
         "kv_gbs_effective": step_bytes / (ms_step / 1e3) / 1e9,
         "kv_bytes_per_step": step_bytes,
@@ -454,11 +457,11 @@ def measure_prefill(device, reps=3):
     pairs_win = sum(min(w, t + 1) for t in range(T))
     pairs_cache = sum(int(np.maximum(0, T - (pp + w)).sum()) for pp in pos)
     flops = 4.0 * wl.head_dim * wl.G * (pairs_win * wl.Hkv + pairs_cache)
-    # tile FLOPs: every 128-query x 64-key block the kernel computes (masked entries
+    # tile FLOPs: every 128-query x 128-key block the kernel computes (masked entries
     # included): per chunk, query tile and key head, the window band (from 128 keys
-    # before the tile to its last query) and the cache pages holding a row with
-    # pos <= last query - w at the time of that chunk (its own rows included)
-    qt, kb = 128, 64
+    # before the tile to its last query) and the cache blocks (two pages each) holding a
+    # row with pos <= last query - w at the time of that chunk (its own rows included)
+    qt, kb = 128, 128
     blocks = 0
     for c0 in range(0, T, chunk):
         for t0 in range(c0, c0 + chunk, qt):
@@ -663,43 +666,71 @@ def measure_hybrid(device, steps=10, warmup=3, period=4):
 
 def measure_ragged(device, warmup=3):
     """Secondary measurement: ragged128k (batch 4, contexts 128K / 96K / 64K / 32K, one
-    layer, per-head keep 60% / 2% / 5-15%) per-token decode, the workload's 64 steps:
-    every step scores the new tokens, retires t - 128 and attends (split step, graph
-    replay, CUDA events).  Effective GB/s = live K/V bytes read per step / step time."""
+    layer, per-head keep 60% / 2% / 5-15%) per-token decode over the workload's 64 steps:
+    every step attends (on the state before its update), then retires t - 128, stores the
+    new token and scores it on a second stream.  The timed steps are one CUDA graph
+    (inputs drawn ahead in HBM; consecutive steps overlap through the programmatic
+    launches, as a multi-layer model's do); the same steps replayed one graph per step
+    are reported beside it.  Effective GB/s = live K/V bytes read per step / step time."""
     from sparse_decode_attention_spkv_b200.inputs import workloads as W
     from sparse_decode_attention_spkv_b200.states import DecodeStep, build_decode_state, kv_bytes
 
     wl = W.WORKLOADS["ragged128k"]
     steps = wl.decode_steps - warmup
-    p, Ls, inp = build_decode_state(wl, 1, wl.decode_steps, device)
+    p, Ls, inp = build_decode_state(wl, 1, wl.decode_steps, device, store_u=False)
+    L = Ls[0]
+    state = [L.cache.K_pool, L.cache.V_pool, L.cache.pos_pool, L.cache.page_table, L.cache.count,
+             L.cache.count_prev, L.cache.pool_top, L.cache.err_flag, L.ring.K_win, L.ring.V_win,
+             L.ring.z_win]
+    snap = [x.clone() for x in state]
     step = DecodeStep(p, Ls, device, split=True)
-    graphs = []
-    for i in range(wl.decode_steps):
+    S_ = __import__("sparse_decode_attention_spkv_b200.spkv", fromlist=["spkv"])
+    S_.spkv_decode_attn(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0], step.o[0], step.lse[0],
+                        L.ws)  # kernel attributes, before capture
+    torch.cuda.synchronize()
+
+    def graph(i0, i1):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g):
-            step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
-        graphs.append(g)
-    for i in range(warmup):
-        graphs[i].replay()
+            for i in range(i0, i1):
+                step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
+        return g
+
+    g_warm, g_all = graph(0, warmup), graph(warmup, wl.decode_steps)
+    g_each = [graph(i, i + 1) for i in range(warmup, wl.decode_steps)]
     torch.cuda.synchronize()
-    b0 = kv_bytes(p, Ls, min(wl.ctx))
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record()
-    for i in range(warmup, wl.decode_steps):
-        graphs[i].replay()
-    b.record()
-    torch.cuda.synchronize()
-    b1 = kv_bytes(p, Ls, min(wl.ctx))
-    ms = a.elapsed_time(b) / steps
-    status, flags = S_check(Ls[0])
-    if status:
-        raise RuntimeError(f"ragged measurement: cache error {flags}")
-    nbytes = 0.5 * (b0 + b1)
+    results = {}
+    for mode in ("one_graph", "graph_per_step"):
+        for x, y in zip(state, snap):
+            x.copy_(y)
+        g_warm.replay()
+        torch.cuda.synchronize()
+        b0 = kv_bytes(p, Ls, min(wl.ctx) + warmup)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        if mode == "one_graph":
+            g_all.replay()
+        else:
+            for g in g_each:
+                g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        b1 = kv_bytes(p, Ls, min(wl.ctx) + wl.decode_steps - 1)
+        status, flags = S_check(L)
+        if status:
+            raise RuntimeError(f"ragged measurement: cache error {flags}")
+        results[mode] = (a.elapsed_time(b) / steps, 0.5 * (b0 + b1))
+    del g_warm, g_all, g_each
     peak, peak_kind = _peaks()
-    del graphs
+    ms, nbytes = results["one_graph"]
+    ms1, nbytes1 = results["graph_per_step"]
     return {"unit": "tokens/s", "value": p.B / (ms / 1e3), "ms_per_step": ms, "steps": steps,
             "kv_bytes_per_step": nbytes, "kv_gbs": nbytes / (ms / 1e3) / 1e9,
-            "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind}
+            "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind,
+            "timing": f"the {steps} timed steps in one CUDA graph (state restored first)",
+            "graph_per_step": {"value": p.B / (ms1 / 1e3), "ms_per_step": ms1,
+                               "kv_gbs": nbytes1 / (ms1 / 1e3) / 1e9,
+                               "frac_of_hbm_peak": nbytes1 / (ms1 / 1e3) / 1e9 / peak}}
 
 
 def measure_serving(device, reps=3):
@@ -805,53 +836,147 @@ def S_check(L):
 _ORACLE_INPUTS = {}
 
 
-def oracle_decode_sample(units: int, seed: int = 0):
-    """Time the fp64 oracle on `units` (layer, batch row) units of the decode32k step
-    at t = 32768: the utility of the row's new token and Eqs. (3)-(4) for its 32 query
-    heads over 32769 keys.  Inputs are random numbers of the workload's shapes and
-    keep rates (their values do not change the work).  Returns (seconds per unit,
-    threads used)."""
-    from oracle import spkv_oracle as O
-    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+def _host_threads() -> int:
     try:
         from threadpoolctl import threadpool_info
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
     except Exception:
-        threads = 1
-    wl = W.WORKLOADS[WORKLOAD]
-    t = wl.ctx[0]
-    if seed not in _ORACLE_INPUTS:  # drawn once per process (~0.5 GB of fp64)
+        return 1
+
+
+def _oracle_inputs(name: str, T: int, seed: int = 0):
+    """Random fp64 inputs with a workload's shapes (the oracle's work does not depend on
+    the values): perceptron weights, one query row, K/V and gates of T positions (keep
+    27.5%, about the decode32k mean), hidden states of 256 tokens.  Drawn once per
+    (workload, length) per process."""
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    key = (name, T, seed)
+    if key not in _ORACLE_INPUTS:
+        wl = W.WORKLOADS[name]
         rng = np.random.default_rng(seed)
-        T = t + 1
-        _ORACLE_INPUTS[seed] = (
-            rng.standard_normal((wl.hid, wl.d_model)) * 0.02, rng.standard_normal(wl.hid) * 0.02,
-            rng.standard_normal((wl.Hkv, wl.hid)) * 0.02, np.zeros(wl.Hkv),
-            rng.standard_normal((1, wl.Hq, wl.head_dim)) / math.sqrt(wl.head_dim),
-            rng.standard_normal((T, wl.Hkv, wl.head_dim)) / math.sqrt(wl.head_dim),
-            rng.standard_normal((T, wl.Hkv, wl.head_dim)) / math.sqrt(wl.head_dim),
-            (rng.random((T, wl.Hkv)) < 0.275).astype(np.uint8),
-            rng.standard_normal((1, wl.d_model)))
-    W1, b1, W2, b2, Q, K, V, z, h = _ORACLE_INPUTS[seed]
+        sd = 1.0 / math.sqrt(wl.head_dim)
+        reps = (T + 4095) // 4096  # one 4096-position block of K/V repeated (values are moot)
+
+        def kv():
+            blk = rng.standard_normal((4096, wl.Hkv, wl.head_dim)) * sd
+            return np.ascontiguousarray(np.tile(blk, (reps, 1, 1))[:T])
+        _ORACLE_INPUTS[key] = dict(
+            W1=rng.standard_normal((wl.hid, wl.d_model)) * 0.02, b1=rng.standard_normal(wl.hid) * 0.02,
+            W2=rng.standard_normal((wl.Hkv, wl.hid)) * 0.02, b2=np.zeros(wl.Hkv),
+            Q=rng.standard_normal((1, wl.Hq, wl.head_dim)) * sd, K=kv(), V=kv(),
+            z=(rng.random((T, wl.Hkv)) < 0.275).astype(np.uint8),
+            h=rng.standard_normal((256, wl.d_model)))
+    return W.WORKLOADS[name], _ORACLE_INPUTS[key]
+
+
+def _oracle_query(wl, x, t, n_tok=1):
+    """The oracle's work for one query position t of one batch row: the utility and gate
+    of n_tok new tokens (Eqs. (1)-(2)) and Eqs. (3)-(4) for every query head over the
+    keys 0..t."""
+    from oracle import spkv_oracle as O
+    O.gate(O.utility(x["h"][:n_tok], x["W1"], x["b1"], x["W2"], x["b2"]), wl.tau)
+    O.gated_attention(x["Q"], x["K"][:t + 1], x["V"][:t + 1], x["z"][:t + 1], wl.window, [t])
+
+
+def oracle_decode_sample(units: int, seed: int = 0):
+    """Time the fp64 oracle on `units` (layer, batch row) units of the decode32k step at
+    t = 32768: the utility of the row's new token and Eqs. (3)-(4) for its 32 query heads
+    over 32769 keys.  Returns (seconds per unit, threads available)."""
+    wl, x = _oracle_inputs(WORKLOAD, W_CTX_DECODE + 1, seed)
     t0 = time.perf_counter()
     for _ in range(units):
-        O.gate(O.utility(h, W1, b1, W2, b2), wl.tau)
-        O.gated_attention(Q, K, V, z, wl.window, [t])
-    dt = time.perf_counter() - t0
-    return dt / units, threads
+        _oracle_query(wl, x, W_CTX_DECODE)
+    return (time.perf_counter() - t0) / units, _host_threads()
 
 
-def cpu_baseline(units: int):
+W_CTX_DECODE = 32768
+
+
+def _oracle_config_rate(name: str, budget_s: float):
+    """The oracle's rate on a bounded sample of one workload, in its unit:
+    decode32k / ragged128k / serving: tokens/s of whole decode steps (every batch row's
+    query, its new token's utility; serving adds the bulk scoring of 128 buffered tokens
+    per row every 128 steps, i.e. one token per row per step); prefill16k: tokens/s of the
+    whole chunked prefill (every position's utility and attention).  Query positions are
+    sampled across the workload's rows (the oracle's cost grows with the context), and the
+    sample is scaled to the workload; `budget_s` bounds the sample's time."""
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    wl = W.WORKLOADS[name]
+    if name == "decode32k":
+        ctx = [W_CTX_DECODE] * wl.B
+        per_step_rows = wl.B * wl.layers
+        tokens_per_step = wl.B
+    elif name == "ragged128k":
+        ctx, per_step_rows, tokens_per_step = list(wl.ctx), wl.B, wl.B
+    elif name == "serving":
+        ctx, per_step_rows, tokens_per_step = list(wl.ctx), wl.B, wl.B
+    elif name == "prefill16k":
+        T = wl.ctx[0]
+        ctx = [int((k + 0.5) * T / 64) for k in range(64)]  # 64 positions across the sequence
+        per_step_rows, tokens_per_step = T, T
+    else:
+        raise ValueError(name)
+    wl_, x = _oracle_inputs(name, max(ctx) + 1)
+    t_start = time.perf_counter()
+    spent, n = 0.0, 0
+    i = 0
+    # the rows' query positions in turn (round robin), until the budget is spent
+    while n < len(ctx) or spent < budget_s:
+        t = ctx[i % len(ctx)]
+        a = time.perf_counter()
+        _oracle_query(wl_, x, t)
+        spent += time.perf_counter() - a
+        n += 1
+        i += 1
+        if spent >= budget_s and n >= min(len(ctx), 4):
+            break
+    per_query = spent / n
+    # a row sampled unevenly is corrected by the mean context of the sample vs the rows'
+    mean_ctx_sample = sum(ctx[k % len(ctx)] for k in range(n)) / n
+    mean_ctx = sum(ctx) / len(ctx)
+    per_query *= mean_ctx / mean_ctx_sample
+    step_s = per_query * per_step_rows
+    return {"value": tokens_per_step / step_s, "unit": "tokens/s",
+            "s_per_step" if name != "prefill16k" else "s_whole_prefill": step_s,
+            "sample": f"{n} query positions ({spent:.1f} s), scaled to "
+                      f"{per_step_rows} per {'step' if name != 'prefill16k' else 'prefill'}",
+            "wall_s": time.perf_counter() - t_start}
+
+
+def cpu_baseline(units: int, per_config_budget_s: float = 2.5):
+    """The oracle as it stands on the host cores: the headline (decode32k, all cores) and,
+    per workload, a single-thread and an all-core figure on bounded samples."""
     per_unit, threads = oracle_decode_sample(units)
     wl_units = 32 * 8  # (layer, batch row) units in one decode32k step
     step_s = per_unit * wl_units
-    return {"value": 8 / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"{units} of the 256 (layer, batch row) units of one decode32k step at "
-                      f"t=32768 (fp64 numpy oracle: utility + Eqs. (3)-(4) for 32 query heads "
-                      f"over 32769 keys), {per_unit * 1e3:.1f} ms per unit, extrapolated to the "
-                      f"full step"}
+    out = {"value": 8 / step_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+           "sample": f"{units} of the 256 (layer, batch row) units of one decode32k step at "
+                     f"t=32768 (fp64 numpy oracle: utility + Eqs. (3)-(4) for 32 query heads "
+                     f"over 32769 keys), {per_unit * 1e3:.1f} ms per unit, extrapolated to the "
+                     f"full step"}
+    per = {}
+    try:
+        from threadpoolctl import threadpool_limits
+    except Exception:
+        threadpool_limits = None
+    for name in ("decode32k", "prefill16k", "ragged128k", "serving"):
+        per[name] = {"all_cores": dict(_oracle_config_rate(name, per_config_budget_s),
+                                       cores=threads)}
+        if threadpool_limits is not None:
+            with threadpool_limits(limits=1):
+                per[name]["1_core"] = dict(_oracle_config_rate(name, per_config_budget_s),
+                                           cores=1)
+        _ORACLE_INPUTS.clear()  # the long-context inputs are GBs of host memory
+    out["per_config"] = per
+    return out
 
 
 def run_reference(args, world, rank):
+    """The reference arm: the fp64 oracle on the host cores, on the decode32k workload.
+    One step of this arm is the oracle over `units` of the 256 (layer, batch row) units of a
+    decode32k token step (8 tokens over 32 layers); ms_per_step is the time of those units,
+    so ms_per_step x steps is the timed run, and value is tokens/s at that rate
+    (tokens_per_step = 8 x units / 256)."""
     if rank != 0:
         return None
     # bounded work: about 600 oracle units (~1 minute on the host) over all timed steps
@@ -859,21 +984,25 @@ def run_reference(args, world, rank):
     for _ in range(args.warmup):
         oracle_decode_sample(1)
     times = []
+    threads = _host_threads()
     for _ in range(args.steps):
         per_unit, threads = oracle_decode_sample(units)
-        times.append(per_unit * 256)
+        times.append(per_unit * units)
     step_s = sum(times) / len(times)
-    value = 8 / step_s
-    cb = cpu_baseline_desc = {
-        "value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-        "sample": f"each step: {units} of the 256 (layer, batch row) units of one decode32k "
-                  f"step, extrapolated to the full step"}
+    tokens_per_step = 8.0 * units / 256
+    value = tokens_per_step / step_s
+    cb = {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+          "sample": f"each step: {units} of the 256 (layer, batch row) units of one decode32k "
+                    f"token step (fp64 numpy oracle)"}
     return {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+            "tokens_per_step": tokens_per_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "impl": "reference",
-            "config": {"workload": "decode32k (see the spkv arm)", "global_batch": 8,
-                       "seq_len": 32768, "layers": 32, "parallelism": "host cores"},
+            "config": {"workload": "decode32k (see the spkv arm); one step of this arm = "
+                                   f"{units} of the 256 (layer, batch row) units of a token step",
+                       "global_batch": 8, "seq_len": 32768, "layers": 32,
+                       "parallelism": "host cores"},
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
