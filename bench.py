@@ -427,7 +427,8 @@ def measure_prefill(device, reps=3):
                                  chunk)
             if evs:
                 evs[i][0].record()
-            S.spkv_prefill_attn(p, L.cache, L.ring, qs[i], ks[i], vs[i], i * chunk, chunk, o, lse)
+            S.spkv_prefill_attn(p, L.cache, L.ring, qs[i], ks[i], vs[i], i * chunk, chunk, o, lse,
+                                L.pf_ws)
             if evs:
                 evs[i][1].record()
             S.spkv_ring_write(p, L.ring, ks[i], vs[i], z, u, chunk, src[i], chunk, chunk)

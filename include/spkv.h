@@ -356,6 +356,9 @@ int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* cache,
                              const spkv_ring* ring, const void* q, const int32_t* t_pos,
                              void* o, float* lse, spkv_stream_t stream);
 
+/* Bytes of the optional workspace of spkv_prefill_attn (a tile counter). */
+#define SPKV_PREFILL_WORKSPACE_BYTES 256
+
 /* a6 -- gated prefill attention, Eqs. (3)-(4), for the chunk of queries at
  * positions chunk_start .. chunk_start+chunk_len-1 of every batch row.  Keys:
  * the window, from K_chunk/V_chunk (positions >= chunk_start) and from the ring
@@ -364,14 +367,21 @@ int spkv_decode_attn_noalloc(const spkv_params* p, const spkv_cache* cache,
  * this chunk; those are used only by queries they have left the window of).
  * q [B][chunk_len][Hq][head_dim]; K_chunk, V_chunk [B][chunk_len][Hkv][head_dim];
  * o [B][chunk_len][Hq][head_dim]; lse [B][chunk_len][Hq] f32 (may be NULL).  cache
- * may be NULL for a window-only layer. */
+ * may be NULL for a window-only layer.
+ * workspace: NULL, or at least SPKV_PREFILL_WORKSPACE_BYTES (ws_bytes) of 16-byte
+ * aligned device memory, zero-filled once before its first use; the library leaves it
+ * zeroed after every call.  With it, the tensor-core path hands out its 128-query tiles
+ * heaviest first to whichever CTA is free (cache densities differ per key head, so no
+ * fixed order balances them); without it, a fixed order is used.  Calls sharing a
+ * workspace must not overlap. */
 int spkv_prefill_attn(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                       const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
-                      int chunk_len, void* o, float* lse, spkv_stream_t stream);
+                      int chunk_len, void* o, float* lse, void* workspace, size_t ws_bytes,
+                      spkv_stream_t stream);
 
 /* Bytes of workspace spkv_cache_rethreshold needs for this cache geometry.  The
  * workspace must be zero-filled once before its first use; the library leaves its
- * work counter at zero after every call.  Calls sharing a workspace must not overlap. */
+ * counters at zero after every call.  Calls sharing a workspace must not overlap. */
 size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* cache);
 
 /* Post-hoc re-threshold ("Self-Pruned Key-Value Attention", §3.3: at inference the
@@ -385,7 +395,8 @@ size_t spkv_rethreshold_workspace_bytes(const spkv_params* p, const spkv_cache* 
  * becomes z = 1[u_win >= tau_new] (NaN slots: 0), so the tokens still in the window
  * retire under the new threshold; later scoring should be given tau_new in p.
  * Requires cache->u_pool.  Three kernels (plan, move, finish); a bounded wait inside
- * the move kernel that gives up latches SPKV_FLAG_TIMEOUT and skips its writes. */
+ * the move kernel that gives up latches SPKV_FLAG_TIMEOUT and skips the writes of its
+ * page, and the call's later waits then give up at once (those pages are skipped too). */
 int spkv_cache_rethreshold(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                            float tau_new, void* workspace, size_t ws_bytes,
                            spkv_stream_t stream);

@@ -299,15 +299,18 @@ int spkv_soft_attn(const spkv_params* p, const void* q, const void* K, const voi
 
 int spkv_prefill_attn(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                       const void* q, const void* K_chunk, const void* V_chunk, int chunk_start,
-                      int chunk_len, void* o, float* lse, spkv_stream_t stream) {
+                      int chunk_len, void* o, float* lse, void* workspace, size_t ws_bytes,
+                      spkv_stream_t stream) {
   SPKV_TRACE("spkv_prefill_attn");
   if (!params_ok(p) || (c && !cache_ok(p, c)) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (chunk_start < 0 || chunk_len < 0) return SPKV_ERR_ARG;
   if (chunk_len == 0) return SPKV_OK;
   if (!q || !K_chunk || !V_chunk || !o) return SPKV_ERR_ARG;
   if (!aligned16(q) || !aligned16(K_chunk) || !aligned16(V_chunk) || !aligned16(o)) return SPKV_ERR_ARG;
+  if (workspace && (!aligned16(workspace) || ws_bytes < SPKV_PREFILL_WORKSPACE_BYTES)) return SPKV_ERR_ARG;
   return status_of(spkv::launch_prefill(*p, cache_or_none(c), *ring, q, K_chunk, V_chunk, chunk_start,
-                                        chunk_len, o, lse, static_cast<cudaStream_t>(stream)));
+                                        chunk_len, o, lse, static_cast<int*>(workspace),
+                                        static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"

@@ -77,7 +77,7 @@ cudaError_t launch_decode(const spkv_params& p, const spkv_cache& c, const spkv_
 bool prefill_tc_supported(const spkv_params& p, const spkv_cache& c, int chunk_start, int chunk_len);
 cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                               const void* q, const void* K_chunk, const void* V_chunk,
-                              int chunk_start, int chunk_len, void* o, float* lse,
+                              int chunk_start, int chunk_len, void* o, float* lse, int* sched,
                               cudaStream_t stream);
 size_t rethreshold_workspace_bytes(const spkv_params& p, const spkv_cache& c);
 // Limit of the re-threshold move kernel's waits on page-read flags (0: default).
@@ -87,7 +87,7 @@ cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const 
 
 cudaError_t launch_prefill(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                            const void* q, const void* K_chunk, const void* V_chunk,
-                           int chunk_start, int chunk_len, void* o, float* lse,
+                           int chunk_start, int chunk_len, void* o, float* lse, int* sched,
                            cudaStream_t stream);
 
 bool soft_tc_supported(const spkv_params& p, int seq_len);

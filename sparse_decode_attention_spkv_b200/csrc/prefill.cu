@@ -191,10 +191,11 @@ cudaError_t dispatch_g(const spkv_params& p, const spkv_cache& c, const spkv_rin
 
 cudaError_t launch_prefill(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                            const void* q, const void* K_chunk, const void* V_chunk,
-                           int chunk_start, int chunk_len, void* o, float* lse,
+                           int chunk_start, int chunk_len, void* o, float* lse, int* sched,
                            cudaStream_t stream) {
   if (prefill_tc_supported(p, c, chunk_start, chunk_len))
-    return launch_prefill_tc(p, c, ring, q, K_chunk, V_chunk, chunk_start, chunk_len, o, lse, stream);
+    return launch_prefill_tc(p, c, ring, q, K_chunk, V_chunk, chunk_start, chunk_len, o, lse, sched,
+                             stream);
   if (p.dtype == SPKV_BF16) {
     if (p.head_dim == 128) return dispatch_g<BF16, 128>(p, c, ring, q, K_chunk, V_chunk, chunk_start, chunk_len, o, lse, stream);
     if (p.head_dim == 64) return dispatch_g<BF16, 64>(p, c, ring, q, K_chunk, V_chunk, chunk_start, chunk_len, o, lse, stream);

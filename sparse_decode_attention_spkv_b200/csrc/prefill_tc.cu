@@ -57,11 +57,12 @@ constexpr int kQT = 128;          // queries per CTA and head
 constexpr int kKB = 128;          // keys per block
 constexpr int kHD = 128;          // head_dim
 constexpr int kWin = 128;         // window of this path
-constexpr int kSlots = 5;         // K/V ring: K(j) is item 2j, V(j) item 2j+1, slot = item % kSlots
+constexpr int kSlots = 4;         // K/V ring: K(j) is item 2j, V(j) item 2j+1, slot = item % kSlots
 constexpr int kAux = 2;           // side-data slots
 constexpr int kThr = 384;
 constexpr int kSoftWarps = 8;
 constexpr int kPlanReaders = 1 + 1 + kSoftWarps;  // producer, MMA thread, softmax warps
+constexpr int kTileReaders = kPlanReaders;        // the same roles read the tile slots
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kSlack = 8.f;
@@ -72,6 +73,7 @@ constexpr uint32_t kColO0 = 0, kColO1 = 128, kColS = 256;  // S of head h at kCo
 struct __align__(1024) TcSmem {
   char q[2][2][kQT * 128];   // [head][d half], 128B-swizzled rows
   char kv[kSlots][2][kHalf];  // [slot][d half]: K or V of one block
+  char ostage[kSoftWarps][32 * 128];  // per softmax warp: 32 output rows x 64 columns (bf16)
   int aux[kAux][kKB];         // per block: cache positions, or soft-mask biases
   uint64_t q_full, q_empty;
   uint64_t kv_full[kSlots], kv_empty[kSlots];
@@ -80,6 +82,8 @@ struct __align__(1024) TcSmem {
   uint64_t p_full[2];
   uint64_t o_full[2];
   uint64_t plan_ready[2], plan_free[2];  // plan slot of tile n: n % 2
+  uint64_t tile_ready[2], tile_free[2];  // tile slot of tile n: n % 2
+  int tile[2];                           // tile index, -1: no more tiles
   uint32_t tmem_base;
   int plan[2][4];  // nc (cache blocks), nfull (rows visible to the whole tile), nrows, -
   int red[2][4];
@@ -211,7 +215,8 @@ __global__ void __launch_bounds__(kThr, 1)
                       const __grid_constant__ CUtensorMap tm_vr, CacheView cache, int num_pages,
                       __nv_bfloat16* __restrict__ out, float* __restrict__ lse_out,
                       int chunk_start, int chunk_len, int hkv, int G, int n_qt, int n_hp,
-                      int n_bh, uint32_t* err, const float* __restrict__ soft_bias) {
+                      int n_bh, uint32_t* err, const float* __restrict__ soft_bias,
+                      int* __restrict__ sched) {
   extern __shared__ __align__(1024) char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;  // 128B-swizzle atoms
   TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw + pad);
@@ -238,6 +243,8 @@ __global__ void __launch_bounds__(kThr, 1)
       mbar_init(&sm.o_full[h], 1);
       mbar_init(&sm.plan_ready[h], 1);
       mbar_init(&sm.plan_free[h], kPlanReaders);
+      mbar_init(&sm.tile_ready[h], 1);
+      mbar_init(&sm.tile_free[h], kTileReaders);
     }
     fence_mbar_init();
   }
@@ -251,6 +258,12 @@ __global__ void __launch_bounds__(kThr, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
+  // tile n of this CTA from tile slot n % 2 (-1: none left); every reader role reads it
+  // once (a warp: all lanes, then lane 0 frees it)
+  auto read_tile = [&](int n) -> int {
+    mbar_wait(&sm.tile_ready[n & 1], (n >> 1) & 1, err);
+    return sm.tile[n & 1];
+  };
 
   // Every role walks the same tiles of this CTA.  Blocks are numbered across tiles (g):
   // the K/V ring, the side-data ring and the S/P barriers run on g; tile n (of this
@@ -261,7 +274,9 @@ __global__ void __launch_bounds__(kThr, 1)
     // 32 blocks at a time; lane 0 issues every copy.
     int g = 0;
     for (int n = 0;; ++n) {
-      const int ti = tile_index(n, cta, grid, n_tiles);
+      const int ti = read_tile(n);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tile_free[n & 1]);
       if (ti < 0) break;
       const Tile tl = tile_of(ti, n_qt, n_hp, n_bh);
       const int bh = tl.bh, b = bh / hkv, kh = bh % hkv;
@@ -393,12 +408,14 @@ __global__ void __launch_bounds__(kThr, 1)
       };
       int g = 0;
       for (int n = 0;; ++n) {
-        const int ti = tile_index(n, cta, grid, n_tiles);
+        const int ti = read_tile(n);
+        mbar_arrive(&sm.tile_free[n & 1]);
         if (ti < 0) break;
         const Tile tl = tile_of(ti, n_qt, n_hp, n_bh);
         const int t0 = chunk_start + tl.qt * kQT;
         const int nw = t0 >= kWin ? 2 : 1;
         int J = SOFT ? nw + (t0 >= kWin ? t0 / kKB - 1 : 0) : -1;
+        bool q_released = false;
         // S(0) of this tile: after its Q has landed (the S region it writes held the
         // previous tile's last P, whose PV was issued before: MMAs run in order)
         mbar_wait(&sm.q_full, n & 1, err);
@@ -425,32 +442,62 @@ __global__ void __launch_bounds__(kThr, 1)
             mbar_wait(&sm.kv_full[ks], kph, err);
             tc_fence_after();
             issue_s(0, ks);
+          } else {
+            mma_commit(&sm.o_full[0]);  // head 0's epilogue overlaps head 1's last PV
           }
           mbar_wait(&sm.p_full[1], g & 1, err);
           tc_fence_after();
           issue_pv(1, vs, j > 0);
           mma_commit(&sm.kv_empty[vs]);
           if (!more) {
-            mma_commit(&sm.q_empty);  // every S of this tile has been issued: Q may go
+            if (!q_released) mma_commit(&sm.q_empty);
+            mma_commit(&sm.o_full[1]);
             ++g;
             break;
           }
           issue_s(1, ks);
           mma_commit(&sm.kv_empty[ks]);
+          if (!q_released && J >= 0 && j + 2 >= J) {
+            // block j + 1 is the tile's last: its S was the last read of this Q, so the
+            // next tile's Q can load while these blocks' softmax and PV run
+            mma_commit(&sm.q_empty);
+            q_released = true;
+          }
         }
-        mma_commit(&sm.o_full[0]);
-        mma_commit(&sm.o_full[1]);
       }
     }
   } else if (warp < 4) {
-    // ------------------------------ cache plan -----------------------------------
-    // For tile n into plan slot n % 2, one tile ahead of its readers: the number of
-    // cache blocks, the rows visible to every query of the tile, the head's row count.
-    if constexpr (!SOFT) {
+    // --------------------------- tile scheduler, cache plan ------------------------
+    // Thread 64 hands out this CTA's tiles through tile slot n % 2, one tile ahead of
+    // their readers.  With a schedule counter (sched), the first tile of CTA c is tile
+    // c and every later one the next unclaimed tile of the launch (tiles go heaviest
+    // first, so the CTAs that finish early take the light ones); without it, the
+    // fixed order of tile_index.  The last CTA to run out of tiles zeroes the counter
+    // for the next launch.
+    // Warps 2-3 then write, for tile n into plan slot n % 2, the number of cache
+    // blocks, the rows visible to every query of the tile and the head's row count.
+    {
       const int pt = tid - 64;  // 0..63
       for (int n = 0;; ++n) {
-        const int ti = tile_index(n, cta, grid, n_tiles);
+        if (pt == 0) {
+          if (n >= 2) mbar_wait(&sm.tile_free[n & 1], ((n >> 1) - 1) & 1, err);
+          int ti = sched ? (n == 0 ? cta : grid + atomicAdd(sched, 1)) : tile_index(n, cta, grid, n_tiles);
+          if (ti >= n_tiles) ti = -1;
+          sm.tile[n & 1] = ti;
+          mbar_arrive(&sm.tile_ready[n & 1]);
+          if (ti < 0 && sched) {
+            __threadfence();  // this CTA's claims precede its count
+            if (atomicAdd(sched + 1, 1) == grid - 1) {  // every CTA has stopped claiming
+              __threadfence();
+              sched[0] = 0;
+              sched[1] = 0;
+            }
+          }
+        }
+        named_bar_sync(1, 64);
+        const int ti = sm.tile[n & 1];  // rewritten only after both plan warps pass the next barrier
         if (ti < 0) break;
+        if constexpr (SOFT) continue;
         const Tile tl = tile_of(ti, n_qt, n_hp, n_bh);
         const int bh = tl.bh;
         const int t0 = chunk_start + tl.qt * kQT;
@@ -517,7 +564,9 @@ __global__ void __launch_bounds__(kThr, 1)
     const float c = kLog2e * rsqrtf((float)kHD);
     int g = 0;
     for (int n = 0;; ++n) {
-      const int ti = tile_index(n, cta, grid, n_tiles);
+      const int ti = read_tile(n);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.tile_free[n & 1]);
       if (ti < 0) break;
       const Tile tl = tile_of(ti, n_qt, n_hp, n_bh);
       const int bh = tl.bh, b = bh / hkv, kh = bh % hkv;
@@ -601,22 +650,36 @@ __global__ void __launch_bounds__(kThr, 1)
       tc_fence_after();
       const int hg = kh * G + 2 * tl.hp + hh;
       const size_t row_out = ((size_t)b * chunk_len + (t - chunk_start)) * Hq + hg;
-      __nv_bfloat16* dst = out + row_out * kHD;
       const float inv = l > 0.f ? 1.f / l : 0.f;
+      // O / l to bf16 through this warp's staging tile, 64 columns at a time: lane r
+      // writes its row's eight 16-byte pieces (piece c at slot c ^ (r & 7), so that each
+      // group of 8 lanes covers all banks), then every store covers 4 whole 128-byte
+      // row pieces of the output (rows are Hq * head_dim apart)
+      char* stg = sm.ostage[warp - 4];
+      const size_t row_w = row_out - (size_t)lane * Hq;  // the warp's first query row
 #pragma unroll
-      for (int cc = 0; cc < kHD; cc += 32) {
-        uint32_t o[32];
-        tmem_ld32(lane_addr + colO + cc, o);
+      for (int pass = 0; pass < 2; ++pass) {
+        uint32_t o[64];
+        tmem_ld32(lane_addr + colO + pass * 64, o);
+        tmem_ld32(lane_addr + colO + pass * 64 + 32, o + 32);
         tmem_wait_ld();
 #pragma unroll
-        for (int v4 = 0; v4 < 4; ++v4) {
+        for (int pc = 0; pc < 8; ++pc) {
           uint4 pkt;
-          pkt.x = pack_bf16(__uint_as_float(o[v4 * 8 + 0]) * inv, __uint_as_float(o[v4 * 8 + 1]) * inv);
-          pkt.y = pack_bf16(__uint_as_float(o[v4 * 8 + 2]) * inv, __uint_as_float(o[v4 * 8 + 3]) * inv);
-          pkt.z = pack_bf16(__uint_as_float(o[v4 * 8 + 4]) * inv, __uint_as_float(o[v4 * 8 + 5]) * inv);
-          pkt.w = pack_bf16(__uint_as_float(o[v4 * 8 + 6]) * inv, __uint_as_float(o[v4 * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(dst + cc + v4 * 8) = pkt;
+          pkt.x = pack_bf16(__uint_as_float(o[pc * 8 + 0]) * inv, __uint_as_float(o[pc * 8 + 1]) * inv);
+          pkt.y = pack_bf16(__uint_as_float(o[pc * 8 + 2]) * inv, __uint_as_float(o[pc * 8 + 3]) * inv);
+          pkt.z = pack_bf16(__uint_as_float(o[pc * 8 + 4]) * inv, __uint_as_float(o[pc * 8 + 5]) * inv);
+          pkt.w = pack_bf16(__uint_as_float(o[pc * 8 + 6]) * inv, __uint_as_float(o[pc * 8 + 7]) * inv);
+          *reinterpret_cast<uint4*>(stg + lane * 128 + ((pc ^ (lane & 7)) << 4)) = pkt;
         }
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const int rr = k * 4 + (lane >> 3), pc = lane & 7;
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rr * 128 + ((pc ^ (rr & 7)) << 4));
+          *reinterpret_cast<uint4*>(out + (row_w + (size_t)rr * Hq) * kHD + pass * 64 + pc * 8) = v;
+        }
+        __syncwarp();  // the tile is refilled by the next pass
       }
       if (lse_out) lse_out[row_out] = l > 0.f ? (m + log2f(l)) * kLn2 : -INFINITY;
     }
@@ -650,7 +713,7 @@ bool prefill_tc_supported(const spkv_params& p, const spkv_cache& c, int chunk_s
 
 cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& ring,
                               const void* q, const void* K_chunk, const void* V_chunk,
-                              int chunk_start, int chunk_len, void* o, float* lse,
+                              int chunk_start, int chunk_len, void* o, float* lse, int* sched,
                               cudaStream_t stream) {
   const int G = p.Hq / p.Hkv;
   const cuuint64_t e = 2;  // bytes per element
@@ -695,7 +758,7 @@ cudaError_t launch_prefill_tc(const spkv_params& p, const spkv_cache& c, const s
   prefill_tc_kernel<false><<<n_tiles < sms ? n_tiles : sms, kThr, kSmem, stream>>>(
       tq, tkc, tvc, tkp, tvp, tkr, tvr, cv, c.K_pool ? c.num_pages : 0,
       static_cast<__nv_bfloat16*>(o), lse, chunk_start, chunk_len, p.Hkv, G, n_qt, n_hp, n_bh,
-      c.err_flag, nullptr);
+      c.err_flag, nullptr, sched);
   return cudaGetLastError();
 }
 
@@ -734,7 +797,7 @@ cudaError_t launch_soft_tc(const spkv_params& p, const void* q, const void* K, c
   // the cache and ring maps are not read in this mode: the sequence maps stand in
   prefill_tc_kernel<true><<<n_tiles < sms ? n_tiles : sms, kThr, kSmem, stream>>>(
       tq, tk, tv, tk, tv, tk, tv, cv, 0, static_cast<__nv_bfloat16*>(o), lse, 0, seq_len, p.Hkv,
-      G, n_qt, n_hp, n_bh, err, bias);
+      G, n_qt, n_hp, n_bh, err, bias, nullptr);
   return cudaGetLastError();
 }
 

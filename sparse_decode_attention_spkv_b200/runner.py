@@ -38,6 +38,7 @@ class Layer:
     cache: Optional[S.Cache]
     ring: S.Ring
     ws: torch.Tensor
+    pf_ws: Optional[torch.Tensor] = None  # tile counter of the prefill attention
 
     @property
     def local(self) -> bool:
@@ -49,7 +50,7 @@ class Layer:
         no utility perceptron, no cache."""
         ring = S.Ring.allocate(p, device)
         ws = S.alloc_decode_workspace(p, None, device)
-        return Layer(p, None, None, None, None, None, ring, ws)
+        return Layer(p, None, None, None, None, None, ring, ws, S.alloc_prefill_workspace(device))
 
     @staticmethod
     def create(p: S.spkv_params, W1, b1, W2, b2, num_pages: int, max_pages_per_head: int,
@@ -59,7 +60,7 @@ class Layer:
         cache = S.Cache.allocate(p, num_pages, max_pages_per_head, device, store_u=store_u)
         ring = S.Ring.allocate(p, device, store_u=store_u)
         ws = S.alloc_decode_workspace(p, cache, device)
-        layer = Layer(p, W1, b1, W2, b2, cache, ring, ws)
+        layer = Layer(p, W1, b1, W2, b2, cache, ring, ws, S.alloc_prefill_workspace(device))
         S.spkv_cache_reset(p, cache, ring)
         return layer
 
@@ -101,7 +102,7 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
     if layer.local:  # window only: attend, then keep the chunk's last rows in the ring
         o = torch.empty_like(q)
         lse = torch.empty((B, Tc, p.Hq), dtype=torch.float32, device=dev)
-        S.spkv_prefill_attn(p, None, layer.ring, q, k, v, chunk_start, Tc, o, lse)
+        S.spkv_prefill_attn(p, None, layer.ring, q, k, v, chunk_start, Tc, o, lse, layer.pf_ws)
         S.spkv_ring_write(p, layer.ring, k, v, None, None, Tc, src_pos, Tc, Tc)
         return o, lse, None, None
     u, z = score(layer, h, B * Tc)
@@ -110,7 +111,7 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
                              Tc)
     o = torch.empty_like(q)
     lse = torch.empty((B, Tc, p.Hq), dtype=torch.float32, device=dev)
-    S.spkv_prefill_attn(p, layer.cache, layer.ring, q, k, v, chunk_start, Tc, o, lse)
+    S.spkv_prefill_attn(p, layer.cache, layer.ring, q, k, v, chunk_start, Tc, o, lse, layer.pf_ws)
     S.spkv_ring_write(p, layer.ring, k, v, z, u, n_compact, src_pos, Tc, Tc)
     return o, lse, u.view(B, Tc, p.Hkv), z.view(B, Tc, p.Hkv)
 

@@ -77,7 +77,7 @@ _sigs = {
                                               ctypes.c_uint, _vp]),
     "spkv_decode_attn_before_append_supported": (_i32, [_P(spkv_params)]),
     "spkv_prefill_attn": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp, _vp, _i32,
-                                 _i32, _vp, _vp, _vp]),
+                                 _i32, _vp, _vp, _vp, ctypes.c_size_t, _vp]),
     "spkv_decode_attn_noalloc": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
                                         _vp, _vp, _vp]),
     "spkv_decode_score_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
@@ -91,6 +91,7 @@ _sigs = {
     "spkv_debug_set_flag_wait_ns": (_i32, [ctypes.c_ulonglong]),
 }
 NOALLOC_SCRATCH_BYTES = 8 << 20
+PREFILL_WORKSPACE_BYTES = 256
 
 
 def _bind(handle):
@@ -302,12 +303,20 @@ def spkv_decode_attn_before_append_supported(p) -> bool:
     return bool(lib.spkv_decode_attn_before_append_supported(ctypes.byref(p)))
 
 
+def alloc_prefill_workspace(device="cuda") -> torch.Tensor:
+    """The optional tile-counter workspace of spkv_prefill_attn (zero-filled)."""
+    return torch.zeros(PREFILL_WORKSPACE_BYTES, dtype=torch.uint8, device=device)
+
+
 def spkv_prefill_attn(p, cache: Optional[Cache], ring: Ring, q, K_chunk, V_chunk, chunk_start,
-                      chunk_len, o, lse, stream=None):
-    """cache None: a window-only layer."""
+                      chunk_len, o, lse, workspace=None, stream=None):
+    """cache None: a window-only layer.  workspace: None (fixed tile order) or a tensor
+    from alloc_prefill_workspace (tiles handed out to free CTAs)."""
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     return _check("spkv_prefill_attn", lib.spkv_prefill_attn(
         ctypes.byref(p), _cache_ref(cache), ctypes.byref(ring.r), _ptr(q), _ptr(K_chunk),
-        _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _stream(stream)))
+        _ptr(V_chunk), chunk_start, chunk_len, _ptr(o), _ptr(lse), _ptr(workspace), ws_bytes,
+        _stream(stream)))
 
 
 def spkv_decode_attn_noalloc(p, cache: Optional[Cache], ring: Ring, q, t_pos, o, lse,

@@ -60,7 +60,7 @@ def test_argument_validation_without_gpu():
     assert S.lib.spkv_decode_attn(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
                                   None, None, None, None, None, 0, None) == S.ERR_ARG
     assert S.lib.spkv_prefill_attn(ctypes.byref(good), ctypes.byref(cache), ctypes.byref(ring),
-                                   None, None, None, 0, 16, None, None, None) == S.ERR_ARG
+                                   None, None, None, 0, 16, None, None, None, 0, None) == S.ERR_ARG
     # misaligned pool pointer
     cache = S.spkv_cache(8, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
     assert S.lib.spkv_cache_reset(ctypes.byref(good), ctypes.byref(cache), None, None) == S.ERR_ARG
@@ -156,3 +156,19 @@ def test_sequence_split_argument_checks():
     assert merge(r(bf), 0, 16, 16, 16, None, None) == S.ERR_ARG      # no part
     assert merge(r(bf), 2, None, 16, 16, None, None) == S.ERR_ARG
     assert merge(r(bf), 2, 16, 16, 8, None, None) == S.ERR_ARG       # misaligned output
+
+
+def test_prefill_workspace_checks():
+    """The optional tile-counter workspace of the prefill attention: too small or
+    misaligned is an argument error, found before anything is launched."""
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    bf = S.make_params(2, 8, 2, 128, 256, 64, 128, 0.5, S.BF16)
+    cache = S.spkv_cache(16, 16, 16, 16, 16, 16, 16, 16, None, 4, 64, 4)
+    ring = S.spkv_ring(16, 16, 16, None)
+    pre = S.lib.spkv_prefill_attn
+    r = ctypes.byref
+    n = S.PREFILL_WORKSPACE_BYTES
+    assert pre(r(bf), r(cache), r(ring), 16, 16, 16, 0, 128, 16, None, 16, n - 1, None) == S.ERR_ARG
+    assert pre(r(bf), r(cache), r(ring), 16, 16, 16, 0, 128, 16, None, 8, n, None) == S.ERR_ARG
+    # an empty chunk is a no-op whatever the workspace
+    assert pre(r(bf), r(cache), r(ring), 16, 16, 16, 0, 0, 16, None, 8, 0, None) == S.OK

@@ -155,6 +155,10 @@ PREFILL_CASES = {
                                         keep="u05_50"), 1152, 384),
     "tc_g4_dense_pages": (W.small_case("decode32k", cid=54, B=1, Hq=8, Hkv=2, d_model=128, hid=32,
                                        ctx=[1536], decode_steps=0, layers=1, keep="spread"), 1536, 768),
+    # more 128-query tiles (8 x 2 head pairs x 16 key heads = 256 per chunk) than SMs: the
+    # persistent CTAs take several tiles each, from the tile counter
+    "tc_g4_many_tiles": (W.small_case("decode32k", cid=55, B=4, Hq=16, Hkv=4, d_model=128, hid=32,
+                                      ctx=[2048], decode_steps=0, layers=1, keep="u05_50"), 2048, 1024),
 }
 
 
@@ -179,6 +183,31 @@ def test_chunked_prefill_matches_oracle(name):
         o_ref, _ = O.gated_attention(q[b], k[b], v[b], z_ref[b], wl.window, np.arange(T))
         C.check_attn(o_gpu[b], o_ref, wl.dtype, f"{name} b={b}")
     _lists_equal(layer, z_ref, T)
+
+
+def test_prefill_tile_order_leaves_results_unchanged():
+    """Tiles handed out by the counter (workspace given) or in the fixed order (no
+    workspace): each tile's arithmetic is the same, so the outputs agree bit for bit;
+    the counter is back at zero after every call."""
+    wl, T, chunk = PREFILL_CASES["tc_g4_many_tiles"]
+    outs = {}
+    for mode in ("counter", "fixed"):
+        layer, _ = _layer(wl, T)
+        if mode == "fixed":
+            layer.pf_ws = None
+        h, q, k, v = _rows(wl, T)
+        res = []
+        for c0 in range(0, T, chunk):
+            o, lse, _, _ = R.prefill_chunk(layer, C.dev(h[:, c0:c0 + chunk], wl.dtype),
+                                           C.dev(q[:, c0:c0 + chunk], wl.dtype),
+                                           C.dev(k[:, c0:c0 + chunk], wl.dtype),
+                                           C.dev(v[:, c0:c0 + chunk], wl.dtype), c0)
+            res.append((o.clone(), lse.clone()))
+            if layer.pf_ws is not None:
+                assert int(layer.pf_ws.count_nonzero()) == 0
+        outs[mode] = res
+    for (o1, l1), (o2, l2) in zip(outs["counter"], outs["fixed"]):
+        assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
 def _decode_run(wl, T0, steps, layer_rows, retire=True, bulk=0, fused=True):
