@@ -7,15 +7,15 @@
 // order.  This is done in place, inside each head's own pages:
 //   plan    one CTA per head: rows kept per page (u >= tau'), exclusive prefix over
 //           the head's pages, read flags of its pages cleared;
-//   move    persistent CTAs take pages in order from a global counter.  A CTA copies
-//           its page (K, V, pos, u) into shared memory, publishes "page read", then
-//           writes the page's kept rows to their new places, while its next page is
-//           already being read into a second buffer.  A kept row only moves
-//           towards the front, so its new place lies in this page or in an earlier
-//           page of the same head; before writing into an earlier page the CTA waits
-//           (bounded) until that page has been read.  A page's flag is raised before
-//           its CTA waits on anything, and pages are taken in increasing order by
-//           running CTAs, so every wait ends.
+//   move    persistent CTAs take pages in order from a global counter; each CTA runs a
+//           few independent pipelines (two page buffers, one agent lane that claims,
+//           copies, raises the page's "page read" flag and checks those of the pages
+//           it writes into, four writer warps), so that one page is read while the
+//           previous one is written.  A kept row only moves towards the front, so its
+//           new place lies in this page or in an earlier page of the same head; rows
+//           are written into an earlier page only once that page has been read
+//           (bounded wait).  A page's flag is raised before anything is waited on for
+//           it, and pages are taken in increasing order, so every wait ends.
 //   finish  counts become the kept counts; the ring's gates are recomputed from the
 //           pending utilities; the work counter is cleared.
 #include <atomic>
@@ -32,11 +32,10 @@ namespace {
 std::atomic<unsigned long long> g_flag_wait_ns{0};
 
 constexpr int kPlanThreads = 256;
-constexpr int kMoveThreads = 128;
 constexpr int kMaxHeadsR = 2048;
 
 struct RethrWs {
-  int* ctr;      // [4]: work counter
+  int* ctr;      // [4]: work counter, "a wait gave up"
   int* pref;     // [heads][max_pages + 1] kept rows before each page
   int* flag;     // [heads][max_pages] page read
 };
@@ -74,6 +73,7 @@ __device__ __forceinline__ int block_scan_excl(int v, int* red, int& total) {
 __global__ void __launch_bounds__(kPlanThreads)
     rethr_plan(CacheMut c, RethrWs ws, float tau) {
   __shared__ int red[kPlanThreads / 32];
+  grid_dependents_launch();
   const int bh = blockIdx.x;
   const int n = c.count[bh];
   const int np = (n + kPageRows - 1) / kPageRows;
@@ -88,7 +88,7 @@ __global__ void __launch_bounds__(kPlanThreads)
       if (!page_ok(page, c.num_pages, c.err)) page = 0;  // debug build: flagged
       const int rows = min(kPageRows, n - j * kPageRows);
       const float4* u4 = reinterpret_cast<const float4*>(c.u + (size_t)page * kPageRows);
-#pragma unroll 4
+#pragma unroll
       for (int i = 0; i < kPageRows / 4; ++i) {
         const float4 v = u4[i];
         kept += (4 * i + 0 < rows && v.x >= tau) + (4 * i + 1 < rows && v.y >= tau) +
@@ -104,171 +104,252 @@ __global__ void __launch_bounds__(kPlanThreads)
   if (threadIdx.x == 0) pref[np] = carry;
 }
 
-// Persistent: pages of all heads in order (head-major), claimed from ws.ctr[0].  Two
-// page buffers: while a page's kept rows are written out, the next claimed page is
-// already being read.  Progress: pages are claimed in increasing order, a page's flag
-// is raised as soon as its read lands (before its CTA waits on anything), and a page only
-// waits for earlier pages of its head; every page below the lowest claimed page whose
-// flag is still down is flagged, so the CTA holding that page (current, or next after a
-// current page whose waits all end) raises its flag.
+// Persistent; pages in page-major order (item i is page i / n_heads of head
+// i % n_heads, skipped where the head has fewer pages), claimed from ws.ctr[0] kBatch
+// items at a time, so that the earlier pages a page writes into (about page j / 2 of
+// its head, for half the rows kept) were claimed long before and have been read.  A CTA
+// runs kPipes independent pipelines, each with two page buffers (K, V, positions,
+// utilities), one agent lane and kWriters writer warps.  The agent, for its pages in turn
+// (page k of the pipeline in buffer k % 2):
+//   waits until the writer has emptied the buffer (page k - 2) and starts the copies
+//   of page k, claimed earlier with its page-table entry and prefix looked up;
+//   looks up the (at most two) pages the page's rows can land in (destinations lie in
+//   [base, base + rows)), loads their "read" flags and claims page k + 1 while the
+//   copies are in flight;
+//   once they land raises page k's "read" flag, then waits (bounded) until the
+//   destination pages that are earlier pages of the head have been read.
+// The writers take the buffers in turn, place the kept rows and write them out, so
+// that page k + 1 is read while page k is written.
+// Ordering: a page's copies have completed (its mbarrier phase) before its flag is
+// stored, and stores into a page are issued only after its flag has been seen, so no
+// store can reach a page before its reads; no fence is needed.
+// Progress: pages are claimed in increasing order; a pipeline holds its pages in that
+// order and a page waits only on lower pages.  Take the lowest claimed page M whose
+// flag is down: the pages its pipeline holds before M are lower, so flagged, their
+// waits are on still lower pages (all flagged), and their writes need nothing from
+// elsewhere; so the agent reaches M, its buffer frees, its copies start, and its flag
+// is raised when they land.
+constexpr int kPipes = 3;
+constexpr int kBatch = 4;  // items per claim
+constexpr int kWriters = 4;  // writer warps per pipeline
+// warps: writer wi of pipeline s is warp wi * kPipes + s; the agent of s is warp
+// kWriters * kPipes + s
+constexpr int kMoveThreads = 32 * (kWriters + 1) * kPipes;
+
 struct MoveItem {
-  int item;  // >= total: none
+  int item;  // >= total: no more pages for this pipeline
   int bh, j, page, rows, base;
+  int dpage[2];  // pool pages of the head's pages base / 64 and base / 64 + 1 (or -1)
 };
+
+__device__ __forceinline__ int load_relaxed(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ void store_relaxed(int* p, int v) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
 
 __global__ void __launch_bounds__(kMoveThreads)
     rethr_move(CacheMut c, RethrWs ws, float tau, int n_heads, int row_bytes,
                unsigned long long wait_ns) {
-  extern __shared__ __align__(16) char smem[];
+  extern __shared__ __align__(128) char smem[];
   const uint32_t page_bytes = (uint32_t)kPageRows * row_bytes;
-  char* buf[2] = {smem, smem + 2 * (size_t)page_bytes};  // [K page][V page] x 2
-  int* s_base = reinterpret_cast<int*>(smem + 4 * (size_t)page_bytes);  // [n_heads + 1]
-  __shared__ int s_pos[2][kPageRows];
-  __shared__ float s_u[2][kPageRows];
-  __shared__ int s_dst[kPageRows];  // new row index, or -1
-  __shared__ MoveItem s_it[2];
-  __shared__ int s_ok, s_wc[2];
-  __shared__ __align__(8) uint64_t bar[2];
+  const uint32_t buf_bytes = 2 * page_bytes + 2 * kPageRows * 4;  // K, V, pos, u
+  int* s_np = reinterpret_cast<int*>(smem + 2 * kPipes * (size_t)buf_bytes);  // [n_heads] pages
+  __shared__ MoveItem s_it[kPipes][2];
+  __shared__ int s_src[kPipes][2][kPageRows], s_dst[kPipes][2][kPageRows];  // kept rows: from, to
+  __shared__ int s_maxp;
+  __shared__ int s_ok[kPipes][2];
+  __shared__ __align__(8) uint64_t full[kPipes][2], ready[kPipes][2], empty[kPipes][2];
+  __shared__ __align__(8) uint64_t lists[kPipes][2];  // writer 0 has written the row lists
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
+  grid_dependents_launch();
   if (tid == 0) {
-    mbar_init(&bar[0], 1);
-    mbar_init(&bar[1], 1);
+    for (int s = 0; s < kPipes; ++s)
+      for (int b = 0; b < 2; ++b) {
+        mbar_init(&full[s][b], 1);
+        mbar_init(&ready[s][b], 1);
+        mbar_init(&empty[s][b], kWriters);
+        mbar_init(&lists[s][b], 1);
+      }
     fence_mbar_init();
   }
-  // pages per head, prefix over heads
-  {
-    __shared__ int red[kMoveThreads / 32];
-    int carry = 0;
-    for (int h0 = 0; h0 < n_heads; h0 += kMoveThreads) {
-      const int h = h0 + tid;
-      const int np = h < n_heads ? (c.count[h] + kPageRows - 1) / kPageRows : 0;
-      int tot = 0;
-      const int ex = block_scan_excl(np, red, tot);
-      if (h < n_heads) s_base[h] = carry + ex;
-      carry += tot;
-    }
-    if (tid == 0) s_base[n_heads] = carry;
+  // pages per head and their maximum (counts are not written by the plan kernel)
+  if (tid == 0) s_maxp = 0;
+  __syncthreads();
+  for (int h = tid; h < n_heads; h += kMoveThreads) {
+    const int np = (c.count[h] + kPageRows - 1) / kPageRows;
+    s_np[h] = np;
+    atomicMax(&s_maxp, np);
   }
   __syncthreads();
-  const int total = s_base[n_heads];
+  grid_dependency_wait();  // prefix sums and cleared flags of the plan kernel
+  const int total = n_heads * s_maxp;  // items, holes included
+  const int s = warp % kPipes;
+  auto buf = [&](int b) { return smem + (size_t)(2 * s + b) * buf_bytes; };
 
-  // thread 0: claim the next page and start reading it into buffer b (K, V by bulk copy;
-  // positions and utilities by the first 64 threads after the item is published)
-  auto claim = [&](int b) {
-    MoveItem it;
-    it.item = atomicAdd(ws.ctr, 1);
-    it.bh = it.j = it.page = it.rows = it.base = 0;
-    if (it.item < total) {
-      int lo = 0, hi = n_heads - 1;
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_base[mid] <= it.item) lo = mid; else hi = mid - 1;
+  if (warp >= kWriters * kPipes) {
+    // ------------------------------ agent of pipeline s -----------------------------
+    if (lane != 0) return;
+    // the next page of this pipeline: the next item of its batch that is a page (a new
+    // batch when the batch is used up), with its page-table entry and destination base
+    int bnext = 0, bend = 0;
+    auto claim = [&]() {
+      MoveItem it;
+      it.bh = it.j = it.page = it.rows = it.base = 0;
+      it.dpage[0] = it.dpage[1] = -1;
+      while (true) {
+        if (bnext == bend) {
+          bnext = atomicAdd(ws.ctr, kBatch);
+          bend = bnext + kBatch;
+        }
+        it.item = bnext++;
+        if (it.item >= total) return it;
+        it.bh = it.item % n_heads;
+        it.j = it.item / n_heads;
+        if (it.j < s_np[it.bh]) break;
       }
-      it.bh = lo;
-      it.j = it.item - s_base[lo];
-      it.rows = min(kPageRows, c.count[lo] - it.j * kPageRows);
+      const int lo = it.bh;
+      const int n = c.count[lo];
       it.page = c.page_table[(size_t)lo * c.max_pages + it.j];
-      if (!page_ok(it.page, c.num_pages, c.err)) it.page = 0;  // debug build: flagged
       it.base = ws.pref[(size_t)lo * (c.max_pages + 1) + it.j];
-      mbar_arrive_expect_tx(&bar[b], 2 * page_bytes);
-      bulk_g2s(buf[b], c.K + (size_t)it.page * page_bytes, page_bytes, &bar[b]);
-      bulk_g2s(buf[b] + page_bytes, c.V + (size_t)it.page * page_bytes, page_bytes, &bar[b]);
-    }
-    s_it[b] = it;
-  };
-  if (tid == 0) claim(0);
-  __syncthreads();
-  for (int round = 0;; ++round) {
-    const int cur = round & 1;
-    const MoveItem it = s_it[cur];
-    if (it.item >= total) break;
-    if (tid < kPageRows) {
-      s_pos[cur][tid] = c.pos[(size_t)it.page * kPageRows + tid];
-      s_u[cur][tid] = c.u[(size_t)it.page * kPageRows + tid];
-    }
-    if (tid == 0) claim(cur ^ 1);  // the next page's read overlaps this page's writes
-    mbar_wait(&bar[cur], (round >> 1) & 1, c.err);
-    __syncthreads();
-    int* flag = ws.flag + (size_t)it.bh * c.max_pages;
-    if (tid == 0) {
-      __threadfence();
-      atomicExch(flag + it.j, 1);  // this page has been read
-    }
-    // new places of the kept rows: rows 0-31 by warp 0, rows 32-63 by warp 1
-    bool keep = false;
-    unsigned ball = 0;
-    if (warp < 2) {
-      const int r = warp * 32 + lane;
-      keep = r < it.rows && s_u[cur][r] >= tau;
-      ball = __ballot_sync(0xffffffffu, keep);
-      if (lane == 0) s_wc[warp] = __popc(ball);
-    }
-    __syncthreads();
-    if (warp < 2) {
-      const int r = warp * 32 + lane;
-      s_dst[r] = keep ? it.base + (warp ? s_wc[0] : 0) + __popc(ball & ((1u << lane) - 1u)) : -1;
-    }
-    __syncthreads();
-    const int kept = s_wc[0] + s_wc[1];
-    // wait until every earlier page we write into has been read
-    if (tid == 0) {
+      it.rows = min(kPageRows, n - it.j * kPageRows);
+      if (!page_ok(it.page, c.num_pages, c.err)) it.page = 0;  // debug build: flagged
+      return it;
+    };
+    MoveItem nxt = claim();
+    for (int k = 0;; ++k) {
+      const int b = k & 1;
+      if (k >= 2 && !mbar_wait(&empty[s][b], ((k >> 1) - 1) & 1, c.err)) return;
+      if (nxt.item >= total) {
+        s_it[s][b].item = total;  // the end marker
+        mbar_arrive(&ready[s][b]);
+        return;
+      }
+      MoveItem it = nxt;
+      char* st = buf(b);
+      mbar_arrive_expect_tx(&full[s][b], buf_bytes);
+      bulk_g2s(st, c.K + (size_t)it.page * page_bytes, page_bytes, &full[s][b]);
+      bulk_g2s(st + page_bytes, c.V + (size_t)it.page * page_bytes, page_bytes, &full[s][b]);
+      bulk_g2s(st + 2 * page_bytes, c.pos + (size_t)it.page * kPageRows, kPageRows * 4, &full[s][b]);
+      bulk_g2s(st + 2 * page_bytes + kPageRows * 4, c.u + (size_t)it.page * kPageRows,
+               kPageRows * 4, &full[s][b]);
+      // while the copies are in flight: destination pages, their flags, the next claim
+      const int32_t* table = c.page_table + (size_t)it.bh * c.max_pages;
+      int* flag = ws.flag + (size_t)it.bh * c.max_pages;
+      const int d0 = it.base / kPageRows;
+      const int dl = (it.base + it.rows - 1) / kPageRows;  // <= it.j
+      const int dw = min(dl, it.j - 1);                     // last earlier page written into
+      it.dpage[0] = table[d0];
+      if (dl > d0) it.dpage[1] = table[d0 + 1];
+      int f0 = dw >= d0 ? load_relaxed(flag + d0) : 1;
+      int f1 = dw > d0 ? load_relaxed(flag + d0 + 1) : 1;
+      nxt = claim();
+      if (!mbar_wait(&full[s][b], (k >> 1) & 1, c.err)) return;
+      store_relaxed(flag + it.j, 1);  // this page has been read
       int ok = 1;
-      if (kept > 0) {
-        const int d0 = it.base / kPageRows, d1 = (it.base + kept - 1) / kPageRows;
-        for (int d = d0; d <= d1 && ok; ++d) {
-          if (d >= it.j) break;
-          if (atomicAdd(flag + d, 0) != 0) continue;
-          const uint64_t t0 = global_ns();
-          while (atomicAdd(flag + d, 0) == 0) {
-            if (global_ns() - t0 > wait_ns) {
-              atomicOr(c.err, SPKV_FLAG_TIMEOUT);
-              ok = 0;
-              break;
-            }
+      if (!(f0 && f1)) {
+        const uint64_t t0 = global_ns();
+        while (true) {
+          if (!f0) f0 = load_relaxed(flag + d0);
+          if (!f1) f1 = load_relaxed(flag + d0 + 1);
+          if (f0 && f1) break;
+          // once any wait of this call has given up, the others give up at once, so
+          // that a call with a lost page ends after one wait limit
+          if (global_ns() - t0 > wait_ns || load_relaxed(ws.ctr + 1) != 0) {
+            atomicOr(c.err, SPKV_FLAG_TIMEOUT);
+            atomicExch(ws.ctr + 1, 1);
+            ok = 0;
+            break;
           }
         }
-        __threadfence();
       }
-      s_ok = ok;
+      s_it[s][b] = it;
+      s_ok[s][b] = ok;
+      mbar_arrive(&ready[s][b]);  // release: s_it and s_ok are visible to the writer
     }
-    __syncthreads();
-    const int32_t* table = c.page_table + (size_t)it.bh * c.max_pages;
-    if (s_ok && kept > 0) {
-      const char* kbuf = buf[cur];
-      const char* vbuf = buf[cur] + page_bytes;
-      const int lpr = row_bytes >> 4;  // 16-byte pieces per row
-      for (int e = tid; e < kPageRows * lpr; e += kMoveThreads) {
-        const int r = e / lpr, off = (e % lpr) * 16;
-        const int dst = s_dst[r];
-        if (dst < 0) continue;
-        const int dpage = table[dst / kPageRows];
-        if (!page_ok(dpage, c.num_pages, c.err)) continue;  // debug build: flagged, skipped
-        const size_t drow = (size_t)dpage * kPageRows + (dst % kPageRows);
-        *reinterpret_cast<uint4*>(c.K + drow * row_bytes + off) =
-            *reinterpret_cast<const uint4*>(kbuf + (size_t)r * row_bytes + off);
-        *reinterpret_cast<uint4*>(c.V + drow * row_bytes + off) =
-            *reinterpret_cast<const uint4*>(vbuf + (size_t)r * row_bytes + off);
-      }
-      if (tid < kPageRows && s_dst[tid] >= 0) {
-        const int dst = s_dst[tid];
-        const int dpage = table[dst / kPageRows];
-        if (page_ok(dpage, c.num_pages, c.err)) {
-          const size_t drow = (size_t)dpage * kPageRows + (dst % kPageRows);
-          c.pos[drow] = s_pos[cur][tid];
-          c.u[drow] = s_u[cur][tid];
-        }
-      }
-    }
-    __syncthreads();  // this buffer is refilled two pages from now
   }
-  // a page claimed past the end was never read: nothing in flight
+  // ------------------------------ writers of pipeline s -----------------------------
+  const int wi = warp / kPipes;  // 0: also places the rows and writes positions, utilities
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int k = 0;; ++k) {
+    const int b = k & 1;
+    const uint32_t ph = (k >> 1) & 1;
+    if (!mbar_wait(&ready[s][b], ph, c.err)) return;
+    const MoveItem it = s_it[s][b];
+    if (it.item >= total) return;
+    if (!mbar_wait(&full[s][b], ph, c.err)) return;  // the copies' data, seen by this warp
+    const char* st = buf(b);
+    const int* s_pos = reinterpret_cast<const int*>(st + 2 * page_bytes);
+    const float* s_u = reinterpret_cast<const float*>(st + 2 * page_bytes + kPageRows * 4);
+    // rows lane and 32 + lane: kept?  new places in the head's row order
+    const bool k0 = lane < it.rows && s_u[lane] >= tau;
+    const bool k1 = 32 + lane < it.rows && s_u[32 + lane] >= tau;
+    const unsigned b0 = __ballot_sync(0xffffffffu, k0), b1 = __ballot_sync(0xffffffffu, k1);
+    const int d0 = it.base / kPageRows;
+    auto drow_of = [&](int dst) {
+      const int dpage = dst / kPageRows == d0 ? it.dpage[0] : it.dpage[1];
+      return page_ok(dpage, c.num_pages, c.err) ? dpage * kPageRows + dst % kPageRows : -1;
+    };
+    const int dr0 = k0 ? drow_of(it.base + __popc(b0 & lt)) : -1;
+    const int dr1 = k1 ? drow_of(it.base + __popc(b0) + __popc(b1 & lt)) : -1;
+    // the kept rows in order: where from (row of the page), where to (row of the pool)
+    if (wi == 0) {
+      if (k0) {
+        s_src[s][b][__popc(b0 & lt)] = lane;
+        s_dst[s][b][__popc(b0 & lt)] = dr0;
+      }
+      if (k1) {
+        s_src[s][b][__popc(b0) + __popc(b1 & lt)] = 32 + lane;
+        s_dst[s][b][__popc(b0) + __popc(b1 & lt)] = dr1;
+      }
+    }
+    if (wi == 0) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&lists[s][b]);
+    } else if (!mbar_wait(&lists[s][b], ph, c.err)) {
+      return;
+    }
+    if (s_ok[s][b]) {
+      // (kept row, 16-byte piece) pairs over the lanes: K pieces, then V pieces of a row
+      const int lpr = row_bytes >> 4;               // pieces per row, a power of two
+      const int sh = __ffs(2 * lpr) - 1;             // log2 of the pieces of K and V
+      const int n_e = (__popc(b0) + __popc(b1)) << sh;
+#pragma unroll 4
+      for (int e = wi * 32 + lane; e < n_e; e += 32 * kWriters) {
+        const int kr = e >> sh, pc = e & (2 * lpr - 1);
+        const int drow = s_dst[s][b][kr];
+        if (drow < 0) continue;
+        const int kv = pc >= lpr, off = (pc - kv * lpr) * 16;
+        char* dbase = kv ? c.V : c.K;
+        *reinterpret_cast<uint4*>(dbase + (size_t)drow * row_bytes + off) =
+            *reinterpret_cast<const uint4*>(st + kv * page_bytes + (size_t)s_src[s][b][kr] * row_bytes + off);
+      }
+      if (wi == 0 && dr0 >= 0) {
+        c.pos[dr0] = s_pos[lane];
+        c.u[dr0] = s_u[lane];
+      }
+      if (wi == 0 && dr1 >= 0) {
+        c.pos[dr1] = s_pos[32 + lane];
+        c.u[dr1] = s_u[32 + lane];
+      }
+    }
+    // this warp is done with the buffer (and its row lists, rewritten for page k + 2,
+    // which is issued only after both warps have arrived here)
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s][b]);
+  }
 }
 
 // Counts, ring gates, work counter.
 __global__ void __launch_bounds__(256)
     rethr_finish(CacheMut c, RethrWs ws, RingMut r, float tau, int n_heads, int ring_entries) {
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  grid_dependency_wait();  // every page has been moved
   if (i < n_heads) {
     const int n = c.count[i];
     const int np = (n + kPageRows - 1) / kPageRows;
@@ -277,7 +358,7 @@ __global__ void __launch_bounds__(256)
     c.count_prev[i] = kept;
   }
   if (r.u && i < ring_entries) r.z[i] = r.u[i] >= tau ? 1 : 0;
-  if (i == 0) ws.ctr[0] = 0;
+  if (i == 0) ws.ctr[0] = ws.ctr[1] = 0;
 }
 
 }  // namespace
@@ -298,21 +379,29 @@ cudaError_t launch_rethreshold(const spkv_params& p, const spkv_cache& c, const 
   CacheMut m = cache_mut(c);
   RethrWs ws = carve(workspace, n_heads, c.max_pages_per_head);
   rethr_plan<<<n_heads, kPlanThreads, 0, stream>>>(m, ws, tau_new);
-  const size_t smem = (size_t)4 * kPageRows * row_bytes + (size_t)(n_heads + 1) * 4;
+  const size_t smem = (size_t)2 * kPipes * (2 * kPageRows * row_bytes + 2 * kPageRows * 4) +
+                      ((size_t)n_heads * 4 + 15) / 16 * 16;
   {
     cudaError_t e = ensure_dynamic_smem((const void*)rethr_move, (int)smem);
     if (e != cudaSuccess) return e;
   }
-  // as many CTAs per SM as shared memory allows (each has two pages in flight)
-  int per_sm = (int)((216u << 10) / (smem + (2u << 10)));
+  int per_sm = 0;
+  {
+    cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, rethr_move,
+                                                                  kMoveThreads, smem);
+    if (e != cudaSuccess) return e;
+  }
   per_sm = per_sm < 1 ? 1 : (per_sm > 8 ? 8 : per_sm);
   const unsigned long long w = g_flag_wait_ns.load();
-  rethr_move<<<num_sms * per_sm, kMoveThreads, smem, stream>>>(m, ws, tau_new, n_heads, row_bytes,
-                                                               w ? w : kWaitLimitNs);
+  cudaError_t e = launch_pdl(rethr_move, dim3(num_sms * per_sm), dim3(kMoveThreads), smem, stream,
+                             m, ws, tau_new, n_heads, row_bytes, w ? w : kWaitLimitNs);
+  if (e != cudaSuccess) return e;
   RingMut r = ring ? ring_mut(*ring) : RingMut{nullptr, nullptr, nullptr, nullptr};
   const int ring_entries = ring ? p.B * p.window * p.Hkv : 0;
   const int n = n_heads > ring_entries ? n_heads : ring_entries;
-  rethr_finish<<<(n + 255) / 256, 256, 0, stream>>>(m, ws, r, tau_new, n_heads, ring_entries);
+  e = launch_pdl(rethr_finish, dim3((n + 255) / 256), dim3(256), 0, stream, m, ws, r, tau_new,
+                 n_heads, ring_entries);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 
