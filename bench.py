@@ -665,11 +665,13 @@ def measure_hybrid(device, steps=10, warmup=3, period=4):
             "launches_per_step": per_glob * n_glob + per_loc * (n_layers - n_glob)}
 
 
-def measure_ragged(device, warmup=3):
+def measure_ragged(device, warmup=3, one_stream=True):
     """Secondary measurement: ragged128k (batch 4, contexts 128K / 96K / 64K / 32K, one
     layer, per-head keep 60% / 2% / 5-15%) per-token decode over the workload's 64 steps:
-    every step attends (on the state before its update), then retires t - 128, stores the
-    new token and scores it on a second stream.  The timed steps are one CUDA graph
+    every step attends (on the state before its update), then scores the new token,
+    retires t - 128 and stores the new token (one_stream: one fused launch on the same
+    stream, as a single layer's next attention needs the update anyway; else the
+    retirement and the scoring on a second stream).  The timed steps are one CUDA graph
     (inputs drawn ahead in HBM; consecutive steps overlap through the programmatic
     launches, as a multi-layer model's do); the same steps replayed one graph per step
     are reported beside it.  Effective GB/s = live K/V bytes read per step / step time."""
@@ -684,7 +686,7 @@ def measure_ragged(device, warmup=3):
              L.cache.count_prev, L.cache.pool_top, L.cache.err_flag, L.ring.K_win, L.ring.V_win,
              L.ring.z_win]
     snap = [x.clone() for x in state]
-    step = DecodeStep(p, Ls, device, split=True)
+    step = DecodeStep(p, Ls, device, split=not one_stream, attn_first=True)
     S_ = __import__("sparse_decode_attention_spkv_b200.spkv", fromlist=["spkv"])
     S_.spkv_decode_attn(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0], step.o[0], step.lse[0],
                         L.ws)  # kernel attributes, before capture
@@ -729,6 +731,8 @@ def measure_ragged(device, warmup=3):
             "kv_bytes_per_step": nbytes, "kv_gbs": nbytes / (ms / 1e3) / 1e9,
             "frac_of_hbm_peak": nbytes / (ms / 1e3) / 1e9 / peak, "peak_kind": peak_kind,
             "timing": f"the {steps} timed steps in one CUDA graph (state restored first)",
+            "step": "attention, then fused score + update on one stream" if one_stream else
+                    "attention, then update and score on a second stream",
             "graph_per_step": {"value": p.B / (ms1 / 1e3), "ms_per_step": ms1,
                                "kv_gbs": nbytes1 / (ms1 / 1e3) / 1e9,
                                "frac_of_hbm_peak": nbytes1 / (ms1 / 1e3) / 1e9 / peak}}

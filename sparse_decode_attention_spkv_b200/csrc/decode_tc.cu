@@ -55,7 +55,7 @@ namespace {
 constexpr int kTileR = 64;           // rows per tile (one cache page)
 constexpr int kCons = 4;             // consumer warps, 16 rows each
 constexpr int kThreadsT = (kCons + 2) * 32;   // + producer + finisher
-constexpr int kMergeThreads = 128;
+constexpr int kMergeThreads = 512;
 constexpr int kConsThreads = kCons * 32;
 constexpr int kStagesT = 4;
 constexpr int kUnitsPerCta = 4;      // target chunks per CTA
@@ -690,50 +690,87 @@ __global__ void __launch_bounds__(kMergeThreads)
   if (nch <= 1) return;  // a single chunk wrote its output directly
   const size_t hrow = (size_t)bh * G;  // == (b * hkv + kh) * G
   constexpr int kVec = D / 4;
-  constexpr int kPairs = G * kVec;
-#pragma unroll
-  for (int pi = tid; pi < kPairs; pi += kMergeThreads) {
+  constexpr int kPairs = G * kVec;  // (query head, 4 columns) pairs of the head's output
+  // kSub threads per pair, each over every kSub-th chunk, combined through shared memory
+  constexpr int kSub = kPairs >= kMergeThreads ? 1 : kMergeThreads / kPairs;
+  constexpr int kSlotPairs = kPairs < kMergeThreads ? kPairs : kMergeThreads;
+  __shared__ float s_m[kSub][kSlotPairs], s_l[kSub][kSlotPairs];
+  __shared__ float4 s_o[kSub][kSlotPairs];
+  for (int p0 = 0; p0 < kPairs; p0 += kSlotPairs) {
+    const int sub = tid / kSlotPairs, pi = p0 + tid % kSlotPairs;
     const int g = pi / kVec, d = (pi % kVec) * 4;
     float M = -INFINITY, L = 0.f;
     float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int cb = 0; cb < nch; cb += kMergeBatch) {
-      float mv[kMergeBatch], lv[kMergeBatch];
-      float4 ov[kMergeBatch];
+    if (sub < kSub && pi < kPairs) {
+      for (int cb = sub; cb < nch; cb += kSub * kMergeBatch) {
+        float mv[kMergeBatch], lv[kMergeBatch];
+        float4 ov[kMergeBatch];
 #pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) {
-        const int c = cb + j;
-        if (c < nch) {
-          const size_t e = ((size_t)(c0 + c) * G + g);
-          mv[j] = __ldcg(ws_ml + e * 2);
-          lv[j] = __ldcg(ws_ml + e * 2 + 1);
-          ov[j] = __ldcg(reinterpret_cast<const float4*>(ws_o + e * D + d));
-        } else {
-          mv[j] = -INFINITY;
-          lv[j] = 0.f;
-          ov[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const int c = cb + j * kSub;
+          if (c < nch) {
+            const size_t e = ((size_t)(c0 + c) * G + g);
+            mv[j] = __ldcg(ws_ml + e * 2);
+            lv[j] = __ldcg(ws_ml + e * 2 + 1);
+            ov[j] = __ldcg(reinterpret_cast<const float4*>(ws_o + e * D + d));
+          } else {
+            mv[j] = -INFINITY;
+            lv[j] = 0.f;
+            ov[j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        float mb = M;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) mb = fmaxf(mb, mv[j]);
+        if (mb == -INFINITY) continue;
+        const float sc = M == -INFINITY ? 0.f : exp2f(M - mb);
+        acc.x *= sc;
+        acc.y *= sc;
+        acc.z *= sc;
+        acc.w *= sc;
+        L *= sc;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const float w = mv[j] == -INFINITY ? 0.f : exp2f(mv[j] - mb);
+          acc.x = fmaf(w, ov[j].x, acc.x);
+          acc.y = fmaf(w, ov[j].y, acc.y);
+          acc.z = fmaf(w, ov[j].z, acc.z);
+          acc.w = fmaf(w, ov[j].w, acc.w);
+          L = fmaf(w, lv[j], L);
+        }
+        M = mb;
+      }
+    }
+    if (kSub > 1) {
+      if (sub < kSub) {
+        s_m[sub][tid % kSlotPairs] = M;
+        s_l[sub][tid % kSlotPairs] = L;
+        s_o[sub][tid % kSlotPairs] = acc;
+      }
+      __syncthreads();
+      if (sub == 0) {  // the kSub partial sums of this pair
+        float mb = -INFINITY;
+#pragma unroll
+        for (int q = 0; q < kSub; ++q) mb = fmaxf(mb, s_m[q][tid]);
+        M = mb;
+        L = 0.f;
+        acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (mb != -INFINITY) {
+#pragma unroll
+          for (int q = 0; q < kSub; ++q) {
+            const float w = s_m[q][tid] == -INFINITY ? 0.f : exp2f(s_m[q][tid] - mb);
+            const float4 o = s_o[q][tid];
+            acc.x = fmaf(w, o.x, acc.x);
+            acc.y = fmaf(w, o.y, acc.y);
+            acc.z = fmaf(w, o.z, acc.z);
+            acc.w = fmaf(w, o.w, acc.w);
+            L = fmaf(w, s_l[q][tid], L);
+          }
         }
       }
-      float mb = M;
-#pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) mb = fmaxf(mb, mv[j]);
-      if (mb == -INFINITY) continue;
-      const float sc = M == -INFINITY ? 0.f : exp2f(M - mb);
-      acc.x *= sc;
-      acc.y *= sc;
-      acc.z *= sc;
-      acc.w *= sc;
-      L *= sc;
-#pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) {
-        const float w = mv[j] == -INFINITY ? 0.f : exp2f(mv[j] - mb);
-        acc.x = fmaf(w, ov[j].x, acc.x);
-        acc.y = fmaf(w, ov[j].y, acc.y);
-        acc.z = fmaf(w, ov[j].z, acc.z);
-        acc.w = fmaf(w, ov[j].w, acc.w);
-        L = fmaf(w, lv[j], L);
-      }
-      M = mb;
+      __syncthreads();  // the slots are reused by the next pairs
     }
+    if (sub != 0 || pi >= kPairs) continue;
     const float inv = L > 0.f ? 1.f / L : 0.f;
     if constexpr (F32OUT) {
       *reinterpret_cast<float4*>(out + (hrow + g) * D + d) =

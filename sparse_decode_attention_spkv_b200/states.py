@@ -151,15 +151,18 @@ class DecodeStep:
     With ``split`` and ``attn_first`` (the default where the kernels support it) the
     attention runs first, on the state before the step's update, and the retirement, ring
     write and scoring all run on the second stream: the attention of the next layer
-    follows the previous one directly."""
+    follows the previous one directly.  With ``attn_first`` alone, each layer's attention
+    (on the state before the update) is followed on the same stream by the fused score,
+    retirement and ring write: for a single layer, whose next attention needs the update
+    anyway, this saves the second stream's fork and join."""
 
     def __init__(self, p, layers, device, split: bool = False, attn_first=None):
         from sparse_decode_attention_spkv_b200 import spkv as S
         self.S, self.p, self.layers = S, p, layers
         if attn_first is None:
             attn_first = split and S.spkv_decode_attn_before_append_supported(p)
-        if attn_first and not split:
-            raise ValueError("attn_first needs split")
+        if attn_first and not S.spkv_decode_attn_before_append_supported(p):
+            raise ValueError("attention before the update is not built for these shapes")
         self.attn_first = bool(attn_first)
         n = len(layers)
         self.o = torch.empty((n, p.B, p.Hq, p.head_dim), dtype=torch.bfloat16, device=device)
@@ -190,6 +193,10 @@ class DecodeStep:
                                                  flags=S.DECODE_STATE_SETTLED)
                 if e is not None:
                     e[1].record()
+                if not self.split:  # score, retire t - w, store the new token: one launch
+                    S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2,
+                                               L.b2, k[l], v[l], self.u[l], self.z[l])
+                    continue
                 # retire t - w, store the new token (gate 0), then its gate: beside the
                 # following layers' attention
                 self.fork[l].record(main)

@@ -49,12 +49,14 @@ def _check_row(wl, L, b, t, o_gpu_b, z_new_b, nrows_retired):
 
 def _decode_one_step(wl, rows, order="fused"):
     """One decode step of a full-size state.  order "attn-first" is the bench's launch
-    configuration: attention on the state before the step's update (settled-state
-    flag), update and scoring on the second stream, the whole step captured in a CUDA
-    graph and replayed."""
+    configuration for several layers: attention on the state before the step's update
+    (settled-state flag), update and scoring on the second stream, the whole step
+    captured in a CUDA graph and replayed; "attn-first-one-stream" (the single-layer
+    configuration) follows the attention with the fused score and update on the same
+    stream, also captured."""
     p, Ls, inp = build_decode_state(wl, 1, 2, torch.device("cuda"))
-    step = DecodeStep(p, Ls, "cuda", split=order != "fused", attn_first=order == "attn-first")
-    if order == "attn-first":
+    step = DecodeStep(p, Ls, "cuda", split=order == "attn-first", attn_first=order != "fused")
+    if order != "fused":
         L = Ls[0]  # one eager attention (read-only) sets the kernel attributes before capture
         S.spkv_decode_attn_before_append(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0],
                                          inp["k"][0][0], inp["v"][0][0], step.o[0], step.lse[0],
@@ -89,6 +91,10 @@ def test_decode32k_attention_first_graph_full_size():
 
 def test_ragged128k_attention_first_graph_full_size():
     _decode_one_step(_one_layer("ragged128k"), rows=[0, 2], order="attn-first")
+
+
+def test_ragged128k_attention_first_one_stream_full_size():
+    _decode_one_step(_one_layer("ragged128k"), rows=[1, 3], order="attn-first-one-stream")
 
 
 def test_serving_buffered_full_size():
