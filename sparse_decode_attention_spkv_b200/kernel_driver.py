@@ -1,7 +1,8 @@
 """Run one kernel of the SP-KV path on a small, fixed configuration (for profilers).
 
     python -m sparse_decode_attention_spkv_b200.kernel_driver decode  [--layers 1] [--steps 3]
-                                      [--decode-step attn-first|split|fused]
+                                      [--decode-step attn-first|one-stream|split|fused]
+                                      [--workload decode32k|ragged128k]
     python -m sparse_decode_attention_spkv_b200.kernel_driver score   [--tokens 8]
     python -m sparse_decode_attention_spkv_b200.kernel_driver compact [--rows 4096] [--source chunk|ring]
     python -m sparse_decode_attention_spkv_b200.kernel_driver prefill [--chunk 4096]
@@ -9,7 +10,9 @@
     python -m sparse_decode_attention_spkv_b200.kernel_driver soft [--seq 8192]
 
 ``decode`` builds the decode32k state (batch 8, 32K context, ~300 MB of live K/V per
-layer, more than L2) for a few layers and runs eager decode steps; the others run
+layer, more than L2; or the ragged128k state, batch 4, contexts 128K..32K) for a few
+layers and runs eager decode steps (one-stream: attention first, then the fused score
+and update on the same stream); the others run
 their kernel a few times on decode32k / prefill16k shapes.  Prints nothing but a
 completion line: timings come from the profiler.
 """
@@ -39,10 +42,10 @@ def _layer(wl, rows_per_head, device="cuda"):
 
 def run_decode(args):
     from .states import DecodeStep, build_decode_state
-    wl = W.WORKLOADS["decode32k"]
+    wl = W.WORKLOADS[args.workload]
     p, Ls, inp = build_decode_state(wl, args.layers, args.steps, torch.device("cuda"))
-    step = DecodeStep(p, Ls, "cuda", split=args.decode_step != "fused",
-                      attn_first=args.decode_step == "attn-first")
+    step = DecodeStep(p, Ls, "cuda", split=args.decode_step in ("attn-first", "split"),
+                      attn_first=args.decode_step in ("attn-first", "one-stream"))
     for i in range(args.steps):
         step.launch(inp["h"][i], inp["q"][i], inp["k"][i], inp["v"][i], inp["t"][i])
     torch.cuda.synchronize()
@@ -161,7 +164,9 @@ def main():
     ap.add_argument("--chunk", type=int, default=4096)
     ap.add_argument("--seq", type=int, default=8192)
     ap.add_argument("--source", default="chunk", choices=["chunk", "ring"])
-    ap.add_argument("--decode-step", default="attn-first", choices=["attn-first", "split", "fused"])
+    ap.add_argument("--decode-step", default="attn-first",
+                    choices=["attn-first", "one-stream", "split", "fused"])
+    ap.add_argument("--workload", default="decode32k", choices=["decode32k", "ragged128k"])
     args = ap.parse_args()
     torch.cuda.set_device(0)
     {"decode": run_decode, "score": run_score, "compact": run_compact, "prefill": run_prefill,
