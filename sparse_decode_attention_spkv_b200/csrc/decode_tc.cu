@@ -55,7 +55,8 @@ namespace {
 constexpr int kTileR = 64;           // rows per tile (one cache page)
 constexpr int kCons = 4;             // consumer warps, 16 rows each
 constexpr int kThreadsT = (kCons + 2) * 32;   // + producer + finisher
-constexpr int kMergeThreads = 512;
+constexpr int kMergeThreads = 512;   // merge CTA when heads average many chunks
+constexpr int kMergeThreadsFew = 128;
 constexpr int kConsThreads = kCons * 32;
 constexpr int kStagesT = 4;
 constexpr int kUnitsPerCta = 4;      // target chunks per CTA
@@ -671,8 +672,8 @@ __global__ void __launch_bounds__(kThreadsT, 1)
 // a programmatic dependent of the decode kernel: it waits for the decode grid to
 // complete before reading anything.  It also clears the work counter for the next
 // decode launch.
-template <int D, int G, bool F32OUT>
-__global__ void __launch_bounds__(kMergeThreads)
+template <int D, int G, bool F32OUT, int MT>
+__global__ void __launch_bounds__(MT)
     decode_merge_kernel(int* __restrict__ ws_ctrl, const float* __restrict__ ws_ml,
                         const float* __restrict__ ws_o, void* __restrict__ out_,
                         float* __restrict__ lse_out, int n_heads, int hkv) {
@@ -692,8 +693,8 @@ __global__ void __launch_bounds__(kMergeThreads)
   constexpr int kVec = D / 4;
   constexpr int kPairs = G * kVec;  // (query head, 4 columns) pairs of the head's output
   // kSub threads per pair, each over every kSub-th chunk, combined through shared memory
-  constexpr int kSub = kPairs >= kMergeThreads ? 1 : kMergeThreads / kPairs;
-  constexpr int kSlotPairs = kPairs < kMergeThreads ? kPairs : kMergeThreads;
+  constexpr int kSub = kPairs >= MT ? 1 : MT / kPairs;
+  constexpr int kSlotPairs = kPairs < MT ? kPairs : MT;
   __shared__ float s_m[kSub][kSlotPairs], s_l[kSub][kSlotPairs];
   __shared__ float4 s_o[kSub][kSlotPairs];
   for (int p0 = 0; p0 < kPairs; p0 += kSlotPairs) {
@@ -867,8 +868,14 @@ cudaError_t run_tc(const spkv_params& p, const spkv_cache& c, const spkv_ring& r
                              static_cast<const __nv_bfloat16*>(v_new), ring.z_win,
                              early_plan ? 1 : 0, window_on ? 1 : 0);
   if (e != cudaSuccess) return e;
-  return launch_pdl(decode_merge_kernel<D, G, F32OUT>, dim3(n_heads), dim3(kMergeThreads), 0,
-                    stream, ctrl, ml, po, o, lse, n_heads, p.Hkv);
+  // about kUnitsPerCta chunks per SM are spread over the heads: a wide merge CTA (chunks
+  // over thread subsets) only when a head averages 16 or more, else a narrow one (its
+  // launch and barriers cost the next layer's decode less)
+  if (kUnitsPerCta * num_sms >= 16 * n_heads)
+    return launch_pdl(decode_merge_kernel<D, G, F32OUT, kMergeThreads>, dim3(n_heads),
+                      dim3(kMergeThreads), 0, stream, ctrl, ml, po, o, lse, n_heads, p.Hkv);
+  return launch_pdl(decode_merge_kernel<D, G, F32OUT, kMergeThreadsFew>, dim3(n_heads),
+                    dim3(kMergeThreadsFew), 0, stream, ctrl, ml, po, o, lse, n_heads, p.Hkv);
 }
 
 template <int D, bool F32OUT>
