@@ -378,8 +378,82 @@ def run_gpu(args, world, rank, local):
                       "soft_attn_16k": measure_soft(device),
                       "hybrid_3to1_decode32k": measure_hybrid(device),
                       "ragged128k": measure_ragged(device),
+                      "seqsplit_ragged128k": measure_seqsplit(device),
                       "serving_e2e": measure_serving(device)}
     return out
+
+
+def measure_seqsplit(device, reps=20):
+    """Secondary measurement: the sequence-split decode (f4) on one GPU.  The ragged128k
+    state (one layer) is cut by position into two slices (split_bounds: the first slice
+    the older rows, the second the newer rows and the window); each slice's attention
+    (spkv_decode_attn_partial, fp32 o and lse) and the merge of the two
+    (spkv_decode_merge) are timed against the unsplit attention of the same state
+    (spkv_decode_attn).  Every call reads its slice's live K/V from HBM (286 MB in all,
+    more than L2).  With one slice per GPU, a rank's share of a step is its slice's
+    partial, the exchange of B x Hq x (head_dim + 1) floats, and the merge; the exchange
+    is not measured here (one GPU)."""
+    from sparse_decode_attention_spkv_b200 import runner as R
+    from sparse_decode_attention_spkv_b200 import seqsplit as SS
+    from sparse_decode_attention_spkv_b200 import spkv as S
+    from sparse_decode_attention_spkv_b200.inputs import workloads as W
+    from sparse_decode_attention_spkv_b200.states import build_decode_state, kv_bytes
+
+    wl = W.small_case("ragged128k", layers=1)
+    (lo0, hi0), (lo1, hi1) = SS.split_bounds(wl.ctx, 2, wl.window)
+    p, (LA,), inp = build_decode_state(wl, 1, 1, device, pos_range=(lo0, hi0), with_ring=False)
+    _, (LB,), _ = build_decode_state(wl, 1, 1, device, pos_range=(lo1, hi1))
+    _, (LF,), _ = build_decode_state(wl, 1, 1, device)
+    t = inp["t"][0]
+    h, q, k, v = inp["h"][0][0], inp["q"][0][0], inp["k"][0][0], inp["v"][0][0]
+    R.decode_step(LF, t, h, q, k, v)  # the step's update; then only attention is timed
+    u_t, z_t = R.score(LB, h, p.B)
+    S.spkv_decode_append(p, LB.cache, LB.ring, t, k, v, z_t, u_t, 1)
+    sls = [SS.SliceDecode(p, LA.cache, None, False, device),
+           SS.SliceDecode(p, LB.cache, LB.ring, True, device)]
+    o = torch.empty_like(q)
+    lse = torch.empty((p.B, p.Hq), dtype=torch.float32, device=device)
+    o_parts = torch.empty((2, p.B, p.Hq, p.head_dim), dtype=torch.float32, device=device)
+    lse_parts = torch.empty((2, p.B, p.Hq), dtype=torch.float32, device=device)
+
+    def timed(fn):
+        # the calls captured in one CUDA graph, so that the figure is device time, not the
+        # host's launch rate (a merge is far shorter than a call from Python)
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps
+
+    unsplit = timed(lambda: S.spkv_decode_attn(p, LF.cache, LF.ring, q, t, o, lse, LF.ws))
+    part = [timed(lambda i=i: S.spkv_decode_attn_partial(p, sls[i].cache, sls[i].ring, q, t,
+                                                         sls[i].flags, o_parts[i], lse_parts[i],
+                                                         sls[i].ws)) for i in range(2)]
+    merge = timed(lambda: S.spkv_decode_merge(p, 2, o_parts, lse_parts, o, lse))
+    both = timed(lambda: SS.merge_local(p, sls, q, t, o, lse))
+    for L in (LA, LB, LF):
+        status, flags = S.spkv_cache_check(L.cache)
+        if status != S.OK:
+            raise RuntimeError(f"seqsplit measurement: cache error {flags}")
+    nbytes = kv_bytes(p, [LF], int(t.min().item()))
+    peak, peak_kind = _peaks()
+    return {"unit": "ms", "unsplit_ms": unsplit, "slice_ms": part, "merge_ms": merge,
+            "two_slices_one_gpu_ms": both, "per_rank_compute_ms": max(part) + merge,
+            "kv_bytes": nbytes, "unsplit_frac_of_hbm_peak": nbytes / (unsplit / 1e3) / 1e9 / peak,
+            "peak_kind": peak_kind, "slices": [[lo0, hi0], [lo1, hi1]],
+            "how": f"{reps} calls per figure captured in one CUDA graph, CUDA events around a "
+                   f"replay; inputs larger than L2"}
 
 
 def measure_prefill(device, reps=3):
