@@ -1,8 +1,9 @@
 // prefill_tc.cu -- a6 on the 5th-generation tensor cores (tcgen05 + TMEM + TMA).
 //
 // "Self-Pruned Key-Value Attention" (arXiv 2605.14037), §2.1, Eqs. (3)-(4), for a
-// chunk of queries.  One CTA owns 128 consecutive query positions t0 .. t0+127 of two
-// query heads of one key head.  Its key set is, in 128-key blocks:
+// chunk of queries.  Persistent CTAs (one per SM) take tiles: 128 consecutive query
+// positions t0 .. t0+127 of two query heads of one key head, heaviest tiles first.  A
+// tile's key set is, in 128-key blocks:
 //   * the causal window band first: the block t0-128 .. t0-1 (from the ring for
 //     positions before the chunk, else from the chunk's K/V; visible to query t0+r
 //     for keys i > r of the block) and the block t0 .. t0+127 (keys i <= r);
@@ -12,7 +13,8 @@
 //     (pos <= t-w), and rows beyond are never touched: the dead key blocks of the
 //     causal mask are simply absent.
 // The window blocks need no plan, so their loads and MMAs start at once while two
-// otherwise idle warps find the cache extent (a few dependent global reads).
+// otherwise idle warps find the cache extent (a few dependent global reads), one tile
+// ahead.
 //
 // Both contractions are dense tensor-core tiles: S = Q K^T (M=128 queries, N=128 keys,
 // K=128) and O += P V (M=128, N=128, K=128 keys), bf16 operands, fp32 accumulators in
@@ -22,19 +24,24 @@
 // head's softmax runs, the tensor cores do the other head's PV and next S.  The commit
 // that signals S(j+1) also covers PV(j) (a commit tracks every earlier MMA of the
 // thread), so a softmax that must rescale O (its running maximum grew by more than 8)
-// does it in TMEM at once, with no further wait.
+// does it in TMEM at once, with no further wait.  A tile's Q is released once its
+// last S is issued, so the next tile's Q loads while the last blocks finish; the
+// output is written through a shared-memory staging tile per softmax warp, so every
+// store covers whole 128-byte pieces of output rows.
 //
 // Warp roles (384 threads):
-//   warp 0      TMA producer: Q once; per block K (+ positions) and V, through one ring
-//               of five 32 KB slots (K(j+2) may load while PV(j) runs);
+//   warp 0      TMA producer: Q per tile; per block K (+ positions) and V, through one
+//               ring of four 32 KB slots;
 //   warp 1      TMEM allocation and the single MMA-issuing thread;
-//   warps 2-3   the cache plan (extent and fully visible rows of the tile);
+//   warps 2-3   the tile scheduler (thread 64) and the cache plan (extent and fully
+//               visible rows of the tile);
 //   warps 4-7   softmax of head 0 (one query row per thread, TMEM lanes 0..127);
 //   warps 8-11  softmax of head 1.
-// Per-block side data (cache positions, or soft-mask biases) ride in a 4-slot ring of
-// their own, released by the softmax warps, so no barrier can run more than one phase
-// ahead of a waiter.  Softmax runs in the log2 domain.  Every mbarrier wait is bounded
-// (a stuck wait raises SPKV_FLAG_TIMEOUT).
+// Per-block side data (cache positions, or soft-mask biases) ride in a 2-slot ring of
+// their own, released by the softmax warps; tiles and cache plans pass through 2-slot
+// rings too, so no barrier can run more than one phase ahead of a waiter.  Softmax runs
+// in the log2 domain.  Every mbarrier wait is bounded (a stuck wait raises
+// SPKV_FLAG_TIMEOUT).
 //
 // The same kernel (SOFT = true) computes the soft-gated attention used at training
 // time (§2.1, "soft relaxation", Eqs. (5)-(6)): every key s <= t of the sequence,

@@ -7,7 +7,7 @@
 // order.  This is done in place, inside each head's own pages:
 //   plan    one CTA per head: rows kept per page (u >= tau'), exclusive prefix over
 //           the head's pages, read flags of its pages cleared;
-//   move    persistent CTAs take pages in order from a global counter; each CTA runs a
+//   move    persistent CTAs take pages, page-major, from a global counter; each CTA runs a
 //           few independent pipelines (two page buffers, one agent lane that claims,
 //           copies, raises the page's "page read" flag and checks those of the pages
 //           it writes into, four writer warps), so that one page is read while the
@@ -17,7 +17,7 @@
 //           (bounded wait).  A page's flag is raised before anything is waited on for
 //           it, and pages are taken in increasing order, so every wait ends.
 //   finish  counts become the kept counts; the ring's gates are recomputed from the
-//           pending utilities; the work counter is cleared.
+//           pending utilities; the workspace counters are cleared.
 #include <atomic>
 
 #include "append.cuh"
@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kPlanThreads)
 // runs kPipes independent pipelines, each with two page buffers (K, V, positions,
 // utilities), one agent lane and kWriters writer warps.  The agent, for its pages in turn
 // (page k of the pipeline in buffer k % 2):
-//   waits until the writer has emptied the buffer (page k - 2) and starts the copies
+//   waits until the writers have emptied the buffer (page k - 2) and starts the copies
 //   of page k, claimed earlier with its page-table entry and prefix looked up;
 //   looks up the (at most two) pages the page's rows can land in (destinations lie in
 //   [base, base + rows)), loads their "read" flags and claims page k + 1 while the
