@@ -91,14 +91,19 @@ class ClockSampler:
 
     def __enter__(self):
         cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-               "-lms", "100"]
+               "-lms", "20"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
             self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
-        time.sleep(0.1)
+        # the timed region starts once the sampler is running (its first line is out)
+        t0 = time.time()
+        while self.proc is not None and time.time() - t0 < 3.0:
+            if os.path.getsize(self.out.name) > 0 or self.proc.poll() is not None:
+                break
+            time.sleep(0.01)
         return self
 
     def __exit__(self, *exc):
