@@ -765,7 +765,8 @@ def measure_ragged(device, warmup=3, one_stream=True):
              L.cache.count_prev, L.cache.pool_top, L.cache.err_flag, L.ring.K_win, L.ring.V_win,
              L.ring.z_win]
     snap = [x.clone() for x in state]
-    step = DecodeStep(p, Ls, device, split=not one_stream, attn_first=True)
+    step = DecodeStep(p, Ls, device, split=not one_stream, attn_first=True,
+                      inputs_settled=True)  # inputs drawn ahead in HBM
     S_ = __import__("sparse_decode_attention_spkv_b200.spkv", fromlist=["spkv"])
     S_.spkv_decode_attn(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0], step.o[0], step.lse[0],
                         L.ws)  # kernel attributes, before capture

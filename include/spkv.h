@@ -185,16 +185,23 @@ int spkv_decode_append(const spkv_params* p, const spkv_cache* cache, const spkv
                        const uint8_t* z_new, const float* u_new, int retire,
                        spkv_stream_t stream);
 
+/* Flag of spkv_decode_score_append: h was written by work that had completed before
+ * the kernel enqueued just before this call on `stream` started (e.g. the step's inputs,
+ * copied in ahead of the step).  The perceptron then runs while that kernel finishes;
+ * the ring and cache, which it may still read, are touched only after it ends. */
+#define SPKV_INPUTS_SETTLED 1u
+
 /* a1 + a2 + a3 fused for one per-token decode step: the same result as spkv_score on
  * the B new tokens (h [B][d_model], one per batch row, at positions t_pos) followed by
  * spkv_decode_append(..., z_new = z_out, u_new = u_out, retire = 1).  The warp that finishes the gate
  * of (batch row b, key head kh) also retires token t-window of (b, kh) and stores the
  * new token, so the step costs one launch.  u_out [B][Hkv] (may be NULL), z_out
- * [B][Hkv] as in spkv_score; k_new, v_new [B][Hkv][head_dim]. */
+ * [B][Hkv] as in spkv_score; k_new, v_new [B][Hkv][head_dim].  flags: 0 or
+ * SPKV_INPUTS_SETTLED (other bits: SPKV_ERR_ARG). */
 int spkv_decode_score_append(const spkv_params* p, const spkv_cache* cache, const spkv_ring* ring,
                              const int32_t* t_pos, const void* h, const void* W1, const float* b1,
                              const float* W2, const float* b2, const void* k_new,
-                             const void* v_new, float* u_out, uint8_t* z_out,
+                             const void* v_new, float* u_out, uint8_t* z_out, unsigned flags,
                              spkv_stream_t stream);
 
 /* a1 for one per-token decode step, kept off the attention's critical path: the

@@ -128,9 +128,10 @@ int spkv_decode_append(const spkv_params* p, const spkv_cache* c, const spkv_rin
 int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const spkv_ring* ring,
                              const int32_t* t_pos, const void* h, const void* W1, const float* b1,
                              const float* W2, const float* b2, const void* k_new,
-                             const void* v_new, float* u_out, uint8_t* z_out,
+                             const void* v_new, float* u_out, uint8_t* z_out, unsigned flags,
                              spkv_stream_t stream) {
   SPKV_TRACE("spkv_decode_score_append");
+  if (flags & ~SPKV_INPUTS_SETTLED) return SPKV_ERR_ARG;
   if (!params_ok(p) || !cache_ok(p, c) || !ring_ok(ring)) return SPKV_ERR_ARG;
   if (p->d_model < 1 || p->hid < 1) return SPKV_ERR_ARG;
   if (!t_pos || !h || !W1 || !b1 || !W2 || !b2 || !k_new || !v_new || !z_out) return SPKV_ERR_ARG;
@@ -138,7 +139,8 @@ int spkv_decode_score_append(const spkv_params* p, const spkv_cache* c, const sp
   if (ring->u_win && !u_out) return SPKV_ERR_ARG;
   if (!spkv::score_supported(*p)) return SPKV_ERR_UNSUPPORTED;
   return status_of(spkv::launch_score_append(*p, *c, *ring, t_pos, h, W1, b1, W2, b2, k_new, v_new,
-                                             u_out, z_out, static_cast<cudaStream_t>(stream)));
+                                             u_out, z_out, (flags & SPKV_INPUTS_SETTLED) != 0,
+                                             static_cast<cudaStream_t>(stream)));
 }
 
 int spkv_decode_score(const spkv_params* p, const spkv_ring* ring, const int32_t* t_pos,

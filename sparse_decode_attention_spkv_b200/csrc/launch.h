@@ -17,7 +17,7 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
                                 const int32_t* t_pos, const void* h, const void* W1,
                                 const float* b1, const float* W2, const float* b2,
                                 const void* k_new, const void* v_new, float* u_out,
-                                uint8_t* z_out, cudaStream_t stream);
+                                uint8_t* z_out, bool settled, cudaStream_t stream);
 
 cudaError_t launch_score_gates(const spkv_params& p, const spkv_ring& ring, const int32_t* t_pos,
                                const void* h, const void* W1, const float* b1, const float* W2,

@@ -156,6 +156,7 @@ struct SmallAppend {
   const char* v_new;
   int window;
   int row_bytes;
+  int settled;  // kScoreAppend: h was written before the preceding kernel started
 };
 
 // The gate (and, if the ring keeps them, the utility) of the token of batch row b at
@@ -404,13 +405,18 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
     b2v = __ldg(b2 + warp);
   }
   const float b1v = tid < 16 * kMmaTok ? __ldg(b1 + 16 * rank + tid / kMmaTok) : 0.f;
-  grid_dependency_wait();
-  grid_dependents_launch();
+  // with settled inputs the perceptron runs before the wait for the preceding kernel:
+  // only the ring and cache, which that kernel may still read, wait for it
+  const bool early = MODE == kScoreAppend && ap.settled;
+  if (!early) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+  }
 
   AppendPre pre;
   pre.t = -1;
   if constexpr (MODE == kScoreAppend) {
-    if (warp < hkv && my_n < nt) {
+    if (!early && warp < hkv && my_n < nt) {
       const int b = tok0 + my_n, bh = b * hkv + warp;
       pre = append_prefetch(ap.c, ap.r, bh, b, warp, __ldg(ap.t_pos + b), ap.k_new, ap.v_new, hkv,
                             ap.window, ap.row_bytes, lane, stage[warp]);
@@ -450,6 +456,17 @@ __global__ void __cluster_dims__(kMmaRanks, 1, 1) __launch_bounds__(kMmaThreads,
       cluster.map_shared_rank(&xs[0][0], dst)[(16 * rank + j) * kMmaTok + n] = x;
   }
   cluster.sync();  // every rank now holds all 128 x 8 GELU outputs; no remote access follows
+  if (early) {
+    grid_dependency_wait();
+    grid_dependents_launch();
+    if constexpr (MODE == kScoreAppend) {
+      if (warp < hkv && my_n < nt) {
+        const int b = tok0 + my_n, bh = b * hkv + warp;
+        pre = append_prefetch(ap.c, ap.r, bh, b, warp, __ldg(ap.t_pos + b), ap.k_new, ap.v_new,
+                              hkv, ap.window, ap.row_bytes, lane, stage[warp]);
+      }
+    }
+  }
 
   // second layer: token my_n, one warp per key head
   if (warp < hkv && my_n < nt) {
@@ -533,7 +550,7 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
                                 const int32_t* t_pos, const void* h, const void* W1,
                                 const float* b1, const float* W2, const float* b2,
                                 const void* k_new, const void* v_new, float* u_out,
-                                uint8_t* z_out, cudaStream_t stream) {
+                                uint8_t* z_out, bool settled, cudaStream_t stream) {
   const bool mma = mma_ok(p, p.B);
   if (!mma && !small_ok(p, p.B)) {  // many rows: the two steps as separate launches
     cudaError_t e = launch_score(p, h, p.B, W1, b1, W2, b2, u_out, z_out, stream);
@@ -544,7 +561,7 @@ cudaError_t launch_score_append(const spkv_params& p, const spkv_cache& c, const
   SmallAppend ap{cache_mut(c),
                  ring_mut(ring),
                  t_pos, static_cast<const char*>(k_new), static_cast<const char*>(v_new), p.window,
-                 p.head_dim * esize};
+                 p.head_dim * esize, settled ? 1 : 0};
   if (mma) return launch_mma<kScoreAppend>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
   return dispatch_small<kScoreAppend>(p, h, p.B, W1, b1, W2, b2, u_out, z_out, ap, stream);
 }

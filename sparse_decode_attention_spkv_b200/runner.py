@@ -118,7 +118,8 @@ def prefill_chunk(layer: Layer, h, q, k, v, chunk_start: int, n_compact: Optiona
 
 def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: bool = True,
                 o: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
-                fused: bool = True, score_stream=None, attn_first: bool = False):
+                fused: bool = True, score_stream=None, attn_first: bool = False,
+                score_flags: int = 0):
     """One decode step for every batch row at positions t_pos [B] (device int32).
 
     h_t [B][d_model] (ignored when retire is False: buffered scoring), q_t [B][Hq][d],
@@ -129,7 +130,8 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
     (spkv_decode_score); the caller joins that stream before the gates are needed.  With
     a ``score_stream`` and ``attn_first`` the attention runs first, on the state before
     the step's update (spkv_decode_attn_before_append, the new rows passed in), and the
-    update and the scoring both go to that stream.
+    update and the scoring both go to that stream.  ``score_flags`` go to the fused
+    launch (0 or spkv.INPUTS_SETTLED).
     Returns (o [B][Hq][d], lse [B][Hq], z_t or None)."""
     p = layer.p
     z_t = u_t = None
@@ -186,7 +188,7 @@ def decode_step(layer: Layer, t_pos: torch.Tensor, h_t, q_t, k_t, v_t, retire: b
         z_t = torch.empty((p.B, p.Hkv), dtype=torch.uint8, device=q_t.device)
         u_t = torch.empty((p.B, p.Hkv), dtype=torch.float32, device=q_t.device)
         S.spkv_decode_score_append(p, layer.cache, layer.ring, t_pos, h_t, layer.W1, layer.b1,
-                                   layer.W2, layer.b2, k_t, v_t, u_t, z_t)
+                                   layer.W2, layer.b2, k_t, v_t, u_t, z_t, flags=score_flags)
     else:
         if retire:
             u_t, z_t = score(layer, h_t, p.B)

@@ -28,6 +28,7 @@ SRC_CHUNK, SRC_RING = 0, 1
 FLAG_POOL_FULL, FLAG_TABLE_FULL, FLAG_TIMEOUT, FLAG_INDEX = 1, 2, 4, 8
 PAGE_ROWS = 64
 DECODE_STATE_SETTLED = 1
+INPUTS_SETTLED = 1
 SLICE_WINDOW = 1
 
 _vp = ctypes.c_void_p
@@ -81,7 +82,8 @@ _sigs = {
     "spkv_decode_attn_noalloc": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
                                         _vp, _vp, _vp]),
     "spkv_decode_score_append": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
-                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+                                        _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, ctypes.c_uint,
+                                        _vp]),
     "spkv_decode_score": (_i32, [_P(spkv_params), _P(spkv_ring), _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _vp, _vp]),
     "spkv_decode_attn_partial": (_i32, [_P(spkv_params), _P(spkv_cache), _P(spkv_ring), _vp, _vp,
@@ -330,11 +332,13 @@ def spkv_decode_attn_noalloc(p, cache: Optional[Cache], ring: Ring, q, t_pos, o,
 
 
 def spkv_decode_score_append(p, cache: Cache, ring: Ring, t_pos, h, W1, b1, W2, b2, k_new, v_new,
-                             u_out, z_out, stream=None):
+                             u_out, z_out, flags=0, stream=None):
+    """flags: 0 or INPUTS_SETTLED (h written before the preceding kernel started; see
+    include/spkv.h)."""
     return _check("spkv_decode_score_append", lib.spkv_decode_score_append(
         ctypes.byref(p), ctypes.byref(cache.c), ctypes.byref(ring.r), _ptr(t_pos), _ptr(h), _ptr(W1),
         _ptr(b1), _ptr(W2), _ptr(b2), _ptr(k_new), _ptr(v_new), _ptr(u_out), _ptr(z_out),
-        _stream(stream)))
+        int(flags), _stream(stream)))
 
 
 def spkv_soft_attn_workspace_bytes(p, seq_len: int) -> int:

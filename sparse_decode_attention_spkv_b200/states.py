@@ -154,11 +154,16 @@ class DecodeStep:
     follows the previous one directly.  With ``attn_first`` alone, each layer's attention
     (on the state before the update) is followed on the same stream by the fused score,
     retirement and ring write: for a single layer, whose next attention needs the update
-    anyway, this saves the second stream's fork and join."""
+    anyway, this saves the second stream's fork and join.  ``inputs_settled``: the hidden
+    states given to ``launch`` are written before the step begins (no kernel that writes
+    them can still be running), so the fused score may run its perceptron while the
+    attention finishes (SPKV_INPUTS_SETTLED)."""
 
-    def __init__(self, p, layers, device, split: bool = False, attn_first=None):
+    def __init__(self, p, layers, device, split: bool = False, attn_first=None,
+                 inputs_settled: bool = False):
         from sparse_decode_attention_spkv_b200 import spkv as S
         self.S, self.p, self.layers = S, p, layers
+        self.score_flags = S.INPUTS_SETTLED if inputs_settled else 0
         if attn_first is None:
             attn_first = split and S.spkv_decode_attn_before_append_supported(p)
         if attn_first and not S.spkv_decode_attn_before_append_supported(p):
@@ -195,7 +200,8 @@ class DecodeStep:
                     e[1].record()
                 if not self.split:  # score, retire t - w, store the new token: one launch
                     S.spkv_decode_score_append(p, L.cache, L.ring, t, h[l], L.W1, L.b1, L.W2,
-                                               L.b2, k[l], v[l], self.u[l], self.z[l])
+                                               L.b2, k[l], v[l], self.u[l], self.z[l],
+                                               flags=self.score_flags)
                     continue
                 # retire t - w, store the new token (gate 0), then its gate: beside the
                 # following layers' attention

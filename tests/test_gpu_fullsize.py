@@ -55,7 +55,8 @@ def _decode_one_step(wl, rows, order="fused"):
     configuration) follows the attention with the fused score and update on the same
     stream, also captured."""
     p, Ls, inp = build_decode_state(wl, 1, 2, torch.device("cuda"))
-    step = DecodeStep(p, Ls, "cuda", split=order == "attn-first", attn_first=order != "fused")
+    step = DecodeStep(p, Ls, "cuda", split=order == "attn-first", attn_first=order != "fused",
+                      inputs_settled=order == "attn-first-one-stream")  # inputs built ahead
     if order != "fused":
         L = Ls[0]  # one eager attention (read-only) sets the kernel attributes before capture
         S.spkv_decode_attn_before_append(p, L.cache, L.ring, inp["q"][0][0], inp["t"][0],

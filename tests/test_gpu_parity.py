@@ -320,6 +320,49 @@ def test_fused_and_separate_decode_steps_agree():
         assert np.array_equal(x, y)
 
 
+def test_fused_step_with_settled_inputs_is_unchanged():
+    """SPKV_INPUTS_SETTLED on the fused score + update (the tensor-core perceptron runs
+    before the wait for the preceding kernel; only the ring and cache wait) leaves the
+    step's gates, utilities, outputs and cache bit for bit as they are without it.  The
+    hidden states are copied in before each step, so they are settled."""
+    wl = W.small_case("decode32k", cid=58, B=4, ctx=[1100], decode_steps=24, layers=1,
+                      keep="fixed25")
+    T0, steps, w = wl.ctx[0], wl.decode_steps, wl.window
+    T = T0 + steps
+    W1, b1, W2, b2 = C.weights(wl)
+    p = _params(wl)
+    mp = R.pages_for(T)
+    layers = [R.Layer.create(p, C.dev(W1, wl.dtype), C.dev_f32(b1), C.dev_f32(W2), C.dev_f32(b2),
+                             num_pages=wl.B * wl.Hkv * mp, max_pages_per_head=mp, store_u=True)
+              for _ in range(2)]
+    h, q, k, v = _rows(wl, T)
+    for L in layers:
+        for c0 in range(0, T0, 512):
+            c1 = min(T0, c0 + 512)
+            R.prefill_chunk(L, C.dev(h[:, c0:c1], wl.dtype), C.dev(q[:, c0:c1], wl.dtype),
+                            C.dev(k[:, c0:c1], wl.dtype), C.dev(v[:, c0:c1], wl.dtype), c0,
+                            n_compact=max(0, min(c1, T0 - w) - c0))
+    for i in range(steps):
+        t = T0 + i
+        t_pos = torch.full((wl.B,), t, dtype=torch.int32, device="cuda")
+        res = []
+        for L, flags in zip(layers, (0, S.INPUTS_SETTLED)):
+            o, lse, z = R.decode_step(L, t_pos, C.dev(h[:, t], wl.dtype), C.dev(q[:, t], wl.dtype),
+                                      C.dev(k[:, t], wl.dtype), C.dev(v[:, t], wl.dtype),
+                                      score_flags=flags)
+            res.append((o.clone(), lse.clone(), z.clone()))
+        (oa, la, za), (ob, lb, zb) = res
+        assert torch.equal(za, zb) and torch.equal(oa, ob) and torch.equal(la, lb), f"step {i}"
+    torch.cuda.synchronize()
+    for L in layers:
+        assert S.spkv_cache_check(L.cache)[0] == S.OK
+    for x, y in zip(R.cache_lists(layers[0]), R.cache_lists(layers[1])):
+        assert np.array_equal(x, y)
+    for bh in range(wl.B * wl.Hkv):  # the stored rows, in list order
+        (ka, va), (kb, vb) = (R.cache_rows_kv(L, bh) for L in layers)
+        assert torch.equal(ka, kb) and torch.equal(va, vb), f"head {bh}"
+
+
 SPLIT_CASES = {
     # d_model 4096, hid 128: tensor-core score, gates stored by the score kernel
     "mma": W.small_case("decode32k", cid=55, B=4, ctx=[1100], decode_steps=140, layers=1,
