@@ -10,8 +10,9 @@
 //   * then the compacted cache, two 64-row pages per block, holding the rows with
 //     pos <= t0+127-w (gated-in keys of Eq. (4)); blocks whose rows all have
 //     pos <= t0-w need no mask, the last one or two are masked per query
-//     (pos <= t-w), and rows beyond are never touched: the dead key blocks of the
-//     causal mask are simply absent.
+//     (pos <= t-w: since rows are stored in position order, a prefix of the block
+//     whose length each query finds by bisection), and rows beyond are never
+//     touched: the dead key blocks of the causal mask are simply absent.
 // The window blocks need no plan, so their loads and MMAs start at once while two
 // otherwise idle warps find the cache extent (a few dependent global reads), one tile
 // ahead.
@@ -25,9 +26,11 @@
 // that signals S(j+1) also covers PV(j) (a commit tracks every earlier MMA of the
 // thread), so a softmax that must rescale O (its running maximum grew by more than 8)
 // does it in TMEM at once, with no further wait.  A tile's Q is released once its
-// last S is issued, so the next tile's Q loads while the last blocks finish; the
-// output is written through a shared-memory staging tile per softmax warp, so every
-// store covers whole 128-byte pieces of output rows.
+// last S is issued, so the next tile's Q loads while the last blocks finish, and head
+// 0's first S of the next tile is issued right after its last PV when that Q and the
+// first K block have landed (the heads stay staggered across tiles); the output is
+// written through a shared-memory staging tile per softmax warp, so every store covers
+// whole 128-byte pieces of output rows.
 //
 // Warp roles (384 threads):
 //   warp 0      TMA producer: Q per tile; per block K (+ positions) and V, through one
@@ -115,12 +118,25 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
+// Phase `parity` of an mbarrier completed?  (no waiting)
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Kinds of key block, each with its own straight-line softmax code.
 enum BlockKind : int {
   kOpen = 0,        // every key visible to every query (a cache block below the tile's limit)
   kKeysAfter = 1,   // window block [t0-128, t0): query r keeps keys i > r
   kKeysUpTo = 2,    // window block [t0, t0+128): query r keeps keys i <= r
-  kCacheMask = 3,   // cache block at the tile's limit: rows < count with pos <= t - w
+  kCacheMask = 3,   // cache block at the tile's limit: its first `vis` rows (pos <= t - w)
   kSoftFar = 4,     // soft mask, block outside every window: every key + its bias
   kSoftBefore = 5   // soft mask, block [t0-128, t0): keys i > r + 0, keys i <= r + bias
 };
@@ -134,10 +150,12 @@ struct RowStats {
 // One query row's softmax over one 128-key block: scores (raw q.k from TMEM) masked as
 // KIND says, row maximum, p = 2^(x c - m) packed to bf16 pairs in pk, and their sum.
 // The running maximum is raised only when a score exceeds it by more than kSlack.
+// r: the query's row in the tile; vis: visible rows of a kCacheMask block; aux: the
+// block's soft-mask biases.
 template <int KIND>
 __device__ __forceinline__ RowStats block_softmax(const uint32_t (&raw)[128], uint32_t (&pk)[64],
-                                                  float m, float c, int r, int row0, int nrows,
-                                                  int lim, const int* __restrict__ aux) {
+                                                  float m, float c, int r, int vis,
+                                                  const int* __restrict__ aux) {
   float x[128];
 #pragma unroll
   for (int i = 0; i < 128; ++i) {
@@ -149,7 +167,7 @@ __device__ __forceinline__ RowStats block_softmax(const uint32_t (&raw)[128], ui
     } else if constexpr (KIND == kKeysUpTo) {
       x[i] = i <= r ? sc : -INFINITY;
     } else if constexpr (KIND == kCacheMask) {
-      x[i] = (row0 + i < nrows && aux[i] <= lim) ? sc : -INFINITY;
+      x[i] = i < vis ? sc : -INFINITY;
     } else if constexpr (KIND == kSoftFar) {
       x[i] = sc + __int_as_float(aux[i]);
     } else {
@@ -414,23 +432,28 @@ __global__ void __launch_bounds__(kThr, 1)
         }
       };
       int g = 0;
+      int ti = read_tile(0);
+      mbar_arrive(&sm.tile_free[0]);
+      bool s0_issued = false;  // this tile's first S went out at the end of the previous one
       for (int n = 0;; ++n) {
-        const int ti = read_tile(n);
-        mbar_arrive(&sm.tile_free[n & 1]);
         if (ti < 0) break;
         const Tile tl = tile_of(ti, n_qt, n_hp, n_bh);
         const int t0 = chunk_start + tl.qt * kQT;
         const int nw = t0 >= kWin ? 2 : 1;
         int J = SOFT ? nw + (t0 >= kWin ? t0 / kKB - 1 : 0) : -1;
         bool q_released = false;
-        // S(0) of this tile: after its Q has landed (the S region it writes held the
-        // previous tile's last P, whose PV was issued before: MMAs run in order)
-        mbar_wait(&sm.q_full, n & 1, err);
-        mbar_wait(&sm.kv_full[(2 * g) % kSlots], ((2 * g) / kSlots) & 1, err);
-        tc_fence_after();
-        issue_s(0, (2 * g) % kSlots);
-        issue_s(1, (2 * g) % kSlots);
-        mma_commit(&sm.kv_empty[(2 * g) % kSlots]);
+        int ti_next = -2;  // the next tile, once read (-2: not yet)
+        if (!s0_issued) {
+          // S(0) of this tile: after its Q has landed (the S region it writes held the
+          // previous tile's last P, whose PV was issued before: MMAs run in order)
+          mbar_wait(&sm.q_full, n & 1, err);
+          mbar_wait(&sm.kv_full[(2 * g) % kSlots], ((2 * g) / kSlots) & 1, err);
+          tc_fence_after();
+          issue_s(0, (2 * g) % kSlots);
+          issue_s(1, (2 * g) % kSlots);
+          mma_commit(&sm.kv_empty[(2 * g) % kSlots]);
+        }
+        s0_issued = false;
         for (int j = 0;; ++j, ++g) {
           if (J < 0 && j + 1 >= nw) {  // the far blocks' count: from the plan
             const int ps = n & 1;
@@ -451,14 +474,37 @@ __global__ void __launch_bounds__(kThr, 1)
             issue_s(0, ks);
           } else {
             mma_commit(&sm.o_full[0]);  // head 0's epilogue overlaps head 1's last PV
+            if (!q_released) {
+              mma_commit(&sm.q_empty);
+              q_released = true;
+            }
+            // head 0's first S of the next tile goes out now if that tile, its Q and its
+            // first K are already in place (tested without waiting): head 0 then starts
+            // the next tile while head 1 finishes this one, and the two heads' softmax
+            // stay staggered across the boundary
+            const int n1 = n + 1;
+            const int ks1 = (2 * (g + 1)) % kSlots, kph1 = ((2 * (g + 1)) / kSlots) & 1;
+            if (mbar_test(&sm.tile_ready[n1 & 1], (n1 >> 1) & 1)) {
+              ti_next = sm.tile[n1 & 1];
+              mbar_arrive(&sm.tile_free[n1 & 1]);
+              if (ti_next >= 0 && mbar_test(&sm.q_full, n1 & 1) && mbar_test(&sm.kv_full[ks1], kph1)) {
+                tc_fence_after();
+                issue_s(0, ks1);
+                s0_issued = true;
+              }
+            }
           }
           mbar_wait(&sm.p_full[1], g & 1, err);
           tc_fence_after();
           issue_pv(1, vs, j > 0);
           mma_commit(&sm.kv_empty[vs]);
           if (!more) {
-            if (!q_released) mma_commit(&sm.q_empty);
             mma_commit(&sm.o_full[1]);
+            if (s0_issued) {
+              const int ks1 = (2 * (g + 1)) % kSlots;
+              issue_s(1, ks1);
+              mma_commit(&sm.kv_empty[ks1]);
+            }
             ++g;
             break;
           }
@@ -470,6 +516,12 @@ __global__ void __launch_bounds__(kThr, 1)
             mma_commit(&sm.q_empty);
             q_released = true;
           }
+        }
+        if (ti_next == -2) {
+          ti = read_tile(n + 1);
+          mbar_arrive(&sm.tile_free[(n + 1) & 1]);
+        } else {
+          ti = ti_next;
         }
       }
     }
@@ -612,16 +664,23 @@ __global__ void __launch_bounds__(kThr, 1)
         uint32_t pk[64];
         RowStats st;
         if (!far && nw == 2 && j == 0) {
-          st = SOFT ? block_softmax<kSoftBefore>(raw, pk, m, c, r, 0, 0, 0, aux)
-                    : block_softmax<kKeysAfter>(raw, pk, m, c, r, 0, 0, 0, aux);
+          st = SOFT ? block_softmax<kSoftBefore>(raw, pk, m, c, r, 0, aux)
+                    : block_softmax<kKeysAfter>(raw, pk, m, c, r, 0, aux);
         } else if (!far) {
-          st = block_softmax<kKeysUpTo>(raw, pk, m, c, r, 0, 0, 0, aux);
+          st = block_softmax<kKeysUpTo>(raw, pk, m, c, r, 0, aux);
         } else if (SOFT) {
-          st = block_softmax<kSoftFar>(raw, pk, m, c, r, 0, 0, 0, aux);
+          st = block_softmax<kSoftFar>(raw, pk, m, c, r, 0, aux);
         } else if (row0 + kKB <= nfull) {  // every row visible to every query of the tile
-          st = block_softmax<kOpen>(raw, pk, m, c, r, 0, 0, 0, aux);
+          st = block_softmax<kOpen>(raw, pk, m, c, r, 0, aux);
         } else {
-          st = block_softmax<kCacheMask>(raw, pk, m, c, r, row0, nrows, t - kWin, aux);
+          // cache positions ascend (rows are appended in position order), so the rows of
+          // this block that query t sees are its first vis, found by bisection
+          int vis = 0, hi = min(kKB, nrows - row0);
+          while (vis < hi) {
+            const int mid = (vis + hi) >> 1;
+            if (aux[mid] <= t - kWin) vis = mid + 1; else hi = mid;
+          }
+          st = block_softmax<kCacheMask>(raw, pk, m, c, r, vis, aux);
         }
         // the side data of this block have been read
         __syncwarp();
@@ -658,25 +717,28 @@ __global__ void __launch_bounds__(kThr, 1)
       const int hg = kh * G + 2 * tl.hp + hh;
       const size_t row_out = ((size_t)b * chunk_len + (t - chunk_start)) * Hq + hg;
       const float inv = l > 0.f ? 1.f / l : 0.f;
-      // O / l to bf16 through this warp's staging tile, 64 columns at a time: lane r
-      // writes its row's eight 16-byte pieces (piece c at slot c ^ (r & 7), so that each
-      // group of 8 lanes covers all banks), then every store covers 4 whole 128-byte
-      // row pieces of the output (rows are Hq * head_dim apart)
+      // O / l to bf16: the row's 128 columns come out of TMEM at once (one wait), then go
+      // through this warp's staging tile 64 columns at a time: lane r writes its row's
+      // eight 16-byte pieces (piece c at slot c ^ (r & 7), so that each group of 8 lanes
+      // covers all banks), then every store covers 4 whole 128-byte row pieces of the
+      // output (rows are Hq * head_dim apart)
       char* stg = sm.ostage[warp - 4];
       const size_t row_w = row_out - (size_t)lane * Hq;  // the warp's first query row
+      uint32_t o[kHD];
+#pragma unroll
+      for (int cc = 0; cc < kHD; cc += 32) tmem_ld32(lane_addr + colO + cc, o + cc);
+      tmem_wait_ld();
 #pragma unroll
       for (int pass = 0; pass < 2; ++pass) {
-        uint32_t o[64];
-        tmem_ld32(lane_addr + colO + pass * 64, o);
-        tmem_ld32(lane_addr + colO + pass * 64 + 32, o + 32);
-        tmem_wait_ld();
+        const uint32_t* oh = o + pass * 64;
 #pragma unroll
         for (int pc = 0; pc < 8; ++pc) {
+          const uint32_t* v = oh + pc * 8;
           uint4 pkt;
-          pkt.x = pack_bf16(__uint_as_float(o[pc * 8 + 0]) * inv, __uint_as_float(o[pc * 8 + 1]) * inv);
-          pkt.y = pack_bf16(__uint_as_float(o[pc * 8 + 2]) * inv, __uint_as_float(o[pc * 8 + 3]) * inv);
-          pkt.z = pack_bf16(__uint_as_float(o[pc * 8 + 4]) * inv, __uint_as_float(o[pc * 8 + 5]) * inv);
-          pkt.w = pack_bf16(__uint_as_float(o[pc * 8 + 6]) * inv, __uint_as_float(o[pc * 8 + 7]) * inv);
+          pkt.x = pack_bf16(__uint_as_float(v[0]) * inv, __uint_as_float(v[1]) * inv);
+          pkt.y = pack_bf16(__uint_as_float(v[2]) * inv, __uint_as_float(v[3]) * inv);
+          pkt.z = pack_bf16(__uint_as_float(v[4]) * inv, __uint_as_float(v[5]) * inv);
+          pkt.w = pack_bf16(__uint_as_float(v[6]) * inv, __uint_as_float(v[7]) * inv);
           *reinterpret_cast<uint4*>(stg + lane * 128 + ((pc ^ (lane & 7)) << 4)) = pkt;
         }
         __syncwarp();
